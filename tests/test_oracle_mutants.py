@@ -1,0 +1,65 @@
+"""Planted mistakes in the oracle: each plausible slip (a dropped term, a
+wrong tie rule, a wrong rounding, a wrong code table, a wrong summation
+order) is planted in a copy of the oracle's C source, built on the CPU, and
+must make at least one pin in test_oracle_pins fail."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle.build import CFLAGS
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sbl_oracle.c")
+
+MUTANTS = {
+    "tie_rule_higher_index": ("(kj == ki && j < i)", "(kj == ki && j > i)"),
+    "round_half_away": ("float q = nearbyintf(r);", "float q = roundf(r);"),
+    "sum_split_at_half": ("while (h * 2 < n) h *= 2;", "h = n / 2;"),
+    "gamma_over_dout_only": ("return (float)(s / (double)count);", "return (float)(s / (double)d_in);"),
+    "act_divide_form": ("float s = bf16_to_f32(row[k]) * r;", "float s = bf16_to_f32(row[k]) / a * 127.0f;"),
+    "act_scale_dropped": ("d[t] = a / 127.0f;", "d[t] = a;"),
+    "dequant_token_scale_dropped": ("float c = gamma * d[t];", "float c = gamma;"),
+    "dw_token_scale_dropped": ("(double)bf16_to_f32(dy[t * d_out + o]) * (double)d[t] *\n                         (double)q[t * d_in + k];",
+                               "(double)bf16_to_f32(dy[t * d_out + o]) *\n                         (double)q[t * d_in + k];"),
+    "dx_gamma_dropped": ("dx[t * d_in + k] = (double)gamma * s;", "dx[t * d_in + k] = s;"),
+    "mask_not_applied": ("weff[i] = (int8_t)(mask[i] ? wq[i] : 0);", "weff[i] = wq[i];"),
+    "sign_extension_codes": ("return (uint8_t)(v + 1);", "return (uint8_t)(v & 3);"),
+    "keep_rank_off_by_one": ("(rank < n ? 1 : 0)", "(rank < n - 1 ? 1 : 0)"),
+}
+
+PIN_CALLS = [
+    (pins.test_hand_row_6of8, ()),
+    (pins.test_abs_sum_pairwise_order, ()),
+    (pins.test_gamma_within_error_bound_of_exact_mean, ((128, 256),)),
+    (pins.test_ternarize_ties_and_clip, ()),
+    (pins.test_ternarize_matches_numpy_library_rounding, ()),
+    (pins.test_mask_brute_force_tiny, (6, 8)),
+    (pins.test_mask_degenerate_cases, ()),
+    (pins.test_pk2_roundtrip_and_padding, ()),
+    (pins.test_act_quant_invariants_and_zero_row, ()),
+    (pins.test_act_quant_matches_numpy_float32, ()),
+    (pins.test_output_matches_fp64_definition, ()),
+    (pins.test_backward_matches_numpy_fp64, ()),
+    (pins.test_nm_roundtrip, ()),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", *CFLAGS, "-o", str(lib), str(mut), "-lm"], check=True)
+    failed = []
+    with oracle.use_library(str(lib)):
+        for fn, args in PIN_CALLS:
+            try:
+                fn(*args)
+            except (AssertionError, IndexError, ValueError):
+                failed.append(fn.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"

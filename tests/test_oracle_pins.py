@@ -1,0 +1,401 @@
+"""Pins of the CPU oracle against things other than itself.
+
+The pages print no numeric worked example of the layer, so each oracle
+function is pinned by a hand-derived case (tests/golden), closed forms,
+invariants the definitions fix, special cases that reduce to an independent
+library routine (numpy / torch CPU), and brute force on tiny inputs.  Each
+test names the definition it pins: the Sparse-BitNet summary (arXiv
+2603.05168), section 3.4, and the BitNet b1.58 2B4T summary (arXiv
+2504.12285), section 3.4.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparsity_sbl_quantize_b200 import workloads as wl
+from conftest import load_golden
+
+
+def _floats(vals):
+    return np.array([float(v) for v in vals], dtype=np.float32)
+
+
+def _ints(vals):
+    return np.array([int(v, 0) for v in vals])
+
+
+def test_rounding_mode_is_nearest():
+    assert oracle.rounding_is_nearest()
+
+
+# ------------------------------------------------------------------ worked example
+
+def test_hand_row_6of8():
+    """Hand-derived row: gamma ("Step 1"), RoundClip ("Step 2"), 6:8 mask,
+    W_eff = W_q * M, 2-bit codes; see tests/golden/hand_row_6of8.txt."""
+    g = load_golden("hand_row_6of8.txt")
+    w = _floats(g["w"]).reshape(1, 8)
+    n, m = int(g["n"][0]), int(g["m"][0])
+    gam = oracle.gamma(w)
+    exact = Fraction(0)
+    for v in w.ravel():
+        exact += abs(Fraction(float(v)))
+    assert gam == np.float32(float(exact / 8))
+    assert abs(float(gam) - float(g["gamma"][0])) < 1e-7
+    wq = oracle.ternarize(w, gam)
+    np.testing.assert_array_equal(wq.ravel(), _ints(g["wq"]))
+    mask = oracle.nm_mask(w, n, m)
+    np.testing.assert_array_equal(mask.ravel(), _ints(g["mask"]))
+    weff = oracle.apply_mask(wq, mask)
+    np.testing.assert_array_equal(weff.ravel(), _ints(g["weff"]))
+    np.testing.assert_array_equal(oracle.pack_pk2(weff).ravel(), _ints(g["pk2"]))
+    vals, bm = oracle.pack_nm(weff, mask, n, m)
+    np.testing.assert_array_equal(vals.ravel(), _ints(g["nm_vals"]))
+    np.testing.assert_array_equal(bm.ravel(), _ints(g["nm_bitmap"]))
+
+
+# ------------------------------------------------------------------------ gamma
+
+def test_abs_sum_pairwise_order():
+    """Reading R1 (pairwise tree).  With a = 2**-53, 1 + a rounds back to 1
+    (tie to even), so a left-to-right sum of [1, a, a, a] is 1.0 while the tree
+    (1 + a) + (a + a) is 1 + 2**-52."""
+    a = 2.0 ** -53
+    assert oracle.abs_sum(np.array([1.0, a, a, a], dtype=np.float32)) == 1.0 + 2.0 ** -52
+    # eight leaves: ((1+a)+(a+a)) + ((a+a)+(a+a)) = 1 + 2**-52 + 2**-51
+    v = np.array([1.0] + [a] * 7, dtype=np.float32)
+    assert oracle.abs_sum(v) == 1.0 + 3 * 2.0 ** -52
+    # odd length: the tree over 3 leaves is (1 + a) + a = 1.0 (zero padding)
+    assert oracle.abs_sum(np.array([1.0, a, a], dtype=np.float32)) == 1.0
+    # five leaves split 4 + 1: ((a+a)+(a+a)) + 1 = 1 + 2**-51
+    assert oracle.abs_sum(np.array([a, a, a, a, 1.0], dtype=np.float32)) == 1.0 + 2.0 ** -51
+    # signs are dropped
+    assert oracle.abs_sum(np.array([-1.5, 2.0, -0.25], dtype=np.float32)) == 3.75
+
+
+def test_abs_sum_exact_for_dyadic_values():
+    """Sums of small dyadic values are exact in fp64 whatever the order."""
+    rng = np.random.default_rng(1)
+    v = (rng.integers(-1000, 1000, size=12345) / 64.0).astype(np.float32)
+    assert oracle.abs_sum(v) == sum(abs(Fraction(float(x))) for x in v)
+
+
+@pytest.mark.parametrize("shape", [(128, 256), (1000, 64), (37, 48)])
+def test_gamma_within_error_bound_of_exact_mean(shape):
+    """gamma = mean |W| ("Step 1" equation): the exact rational mean rounded to
+    fp32 and the oracle differ by at most one fp32 ulp (pairwise fp64 error is
+    ~log2(n) * 2**-53, far below half an fp32 ulp except at a tie)."""
+    w = wl.master_weights(*shape, seed=7)
+    exact = math.fsum(abs(float(x)) for x in w.ravel()) / w.size
+    gam = float(oracle.gamma(w))
+    ulp = np.spacing(np.float32(exact))
+    assert abs(gam - exact) <= float(ulp)
+    assert oracle.gamma(w) == np.float32(exact) or abs(gam - exact) <= 0.5 * float(ulp) + 1e-300
+
+
+def test_gamma_includes_masked_weights():
+    """"Composition Order": gamma is taken over all weights, masked ones too,
+    so it does not depend on n:m and equals the plain mean of |W|."""
+    w = wl.master_weights(64, 128, seed=3)
+    gam = oracle.gamma(w)
+    assert gam == np.float32(np.abs(w.astype(np.float64)).mean()) or \
+        abs(float(gam) - np.abs(w.astype(np.float64)).mean()) <= float(np.spacing(gam))
+
+
+def test_gamma_zero_matrix():
+    w = np.zeros((4, 16), dtype=np.float32)
+    assert oracle.gamma(w) == 0.0
+    assert not oracle.ternarize(w, 0.0).any()
+
+
+# -------------------------------------------------------------------- ternarise
+
+def test_ternarize_ties_and_clip():
+    """RoundClip at the rounding ties: |W|/gamma = 0.5 -> 0 (half-even),
+    1.5 -> 2 -> clip 1, 2.5 -> 2 -> clip 1; the row's mean |W| is exactly 1."""
+    v = [0.5, -0.5, 1.5, -1.5, 2.5, -2.5] + [0.75] * 8 + [0.5, 0.5]
+    w = np.array(v, dtype=np.float32).reshape(1, 16)
+    gam = oracle.gamma(w)
+    assert gam == 1.0
+    expect = [0, 0, 1, -1, 1, -1] + [1] * 8 + [0, 0]
+    np.testing.assert_array_equal(oracle.ternarize(w, gam).ravel(), expect)
+    # just above and below the 0.5 boundary
+    up = np.nextafter(np.float32(0.5), np.float32(1))
+    dn = np.nextafter(np.float32(0.5), np.float32(0))
+    np.testing.assert_array_equal(
+        oracle.ternarize(np.array([up, -up, dn, -dn, 0.0, -0.0], dtype=np.float32), 1.0),
+        [1, -1, 0, 0, 0, 0])
+
+
+def test_ternarize_matches_numpy_library_rounding():
+    """Special case reducing to library routines: numpy's IEEE float32 divide,
+    rint (half-even) and clip give the same W_q."""
+    w = wl.master_weights(300, 512, seed=11)
+    gam = oracle.gamma(w)
+    ref = np.clip(np.rint(w / np.float32(gam)), -1, 1).astype(np.int8)
+    np.testing.assert_array_equal(oracle.ternarize(w, gam), ref)
+
+
+def test_ternary_values_and_gaussian_zero_fraction():
+    """W_q in {-1, 0, 1}; for Gaussian W the zero fraction is
+    P(|Z| < 0.5 * sqrt(2/pi)) = erf(0.5/sqrt(pi)) ~= 0.3101 (closed form)."""
+    w = wl.master_weights(1024, 1024, seed=5)
+    wq = oracle.ternarize(w, oracle.gamma(w))
+    assert set(np.unique(wq).tolist()) <= {-1, 0, 1}
+    frac0 = float((wq == 0).mean())
+    expect = math.erf(0.5 / math.sqrt(math.pi))
+    assert abs(frac0 - expect) < 3e-3, (frac0, expect)
+
+
+# ------------------------------------------------------------------------- mask
+
+def _brute_mask_group(keys, n):
+    """Top-n by (key desc, index asc) via an exhaustive search over subsets."""
+    m = len(keys)
+    best = None
+    for subset in itertools.combinations(range(m), n):
+        # a valid top-n set dominates every outsider under the (key, -index) order
+        ok = all((keys[i], -i) > (keys[j], -j) for i in subset for j in range(m) if j not in subset)
+        if ok:
+            assert best is None
+            best = subset
+    out = np.zeros(m, dtype=np.uint8)
+    out[list(best)] = 1
+    return out
+
+
+@pytest.mark.parametrize("n,m", [(6, 8), (2, 4), (1, 4), (3, 8), (7, 8), (2, 8), (4, 8)])
+def test_mask_brute_force_tiny(n, m):
+    """"N:M Mask Generation": per group of m along d_in keep the n largest |W|;
+    brute force over subsets, with values drawn from a tiny set to force ties."""
+    rng = np.random.default_rng(n * 10 + m)
+    w = (rng.integers(-3, 4, size=(40, 4 * m)) * 0.25).astype(np.float32)
+    mask = oracle.nm_mask(w, n, m)
+    for r in range(w.shape[0]):
+        for g in range(4):
+            keys = [abs(float(x)) for x in w[r, g * m:(g + 1) * m]]
+            np.testing.assert_array_equal(mask[r, g * m:(g + 1) * m], _brute_mask_group(keys, n))
+
+
+@pytest.mark.parametrize("n,m", [(6, 8), (2, 4), (5, 8)])
+def test_mask_exactly_n_and_matches_stable_sort(n, m):
+    """Exactly n kept per group; equals numpy's stable argsort of -|W| (ties
+    to the lower index, the reading for ties)."""
+    w = wl.master_weights(200, 64 * m, seed=13)
+    mask = oracle.nm_mask(w, n, m)
+    groups = np.abs(w).reshape(-1, m)
+    assert (mask.reshape(-1, m).sum(axis=1) == n).all()
+    order = np.argsort(-groups, axis=1, kind="stable")
+    ref = np.zeros_like(groups, dtype=np.uint8)
+    np.put_along_axis(ref, order[:, :n], 1, axis=1)
+    np.testing.assert_array_equal(mask.reshape(-1, m), ref)
+
+
+def test_mask_degenerate_cases():
+    # all keys equal (including -0 vs +0): the first n positions are kept
+    w = np.array([[0.0, -0.0, 0.0, -0.0, 0.5, -0.5, 0.5, -0.5]], dtype=np.float32)
+    np.testing.assert_array_equal(oracle.nm_mask(w, 2, 4).ravel(), [1, 1, 0, 0, 1, 1, 0, 0])
+    # n == m keeps everything: the layer reduces to dense BitLinear
+    w = wl.master_weights(8, 64, seed=2)
+    assert oracle.nm_mask(w, 8, 8).all() and oracle.nm_mask(w, 4, 4).all()
+
+
+def test_nm_equal_m_is_dense_bitlinear():
+    """8:8 is dense BitLinear: W_eff == W_q."""
+    w = wl.master_weights(32, 64, seed=9)
+    layer = oracle.Layer(w, 8, 8)
+    np.testing.assert_array_equal(layer.weff, layer.wq)
+
+
+def test_mask_uses_master_not_quantized_weights():
+    """The mask ranks |W| of the master weights, not |W_q|: two weights that
+    both ternarise to +1 are still ordered by their master magnitude."""
+    w = np.array([[0.9, 0.8, 0.7, 0.6, 0.1, 0.2, 0.3, 0.4]], dtype=np.float32)
+    # all of the first four quantise to 1; 2:8 must keep the two largest masters
+    np.testing.assert_array_equal(oracle.nm_mask(w, 2, 8).ravel(), [1, 1, 0, 0, 0, 0, 0, 0])
+
+
+# ---------------------------------------------------------------------- packing
+
+def _decode_pk2(packed, d_in):
+    b = packed[:, : d_in // 4].astype(np.int16)
+    codes = np.stack([(b >> (2 * j)) & 3 for j in range(4)], axis=-1).reshape(packed.shape[0], d_in)
+    return (codes - 1).astype(np.int8)
+
+
+def test_pk2_roundtrip_and_padding():
+    w = wl.master_weights(16, 80, seed=4)  # 80/4 = 20 bytes -> padded to 32
+    layer = oracle.Layer(w, 6, 8)
+    pk = oracle.pack_pk2(layer.weff)
+    assert pk.shape == (16, 32)
+    np.testing.assert_array_equal(_decode_pk2(pk, 80), layer.weff)
+    assert (pk[:, 20:] == 0x55).all()
+    assert not ((pk[:, :20] >> 6) == 3).any()  # code 3 is never written
+
+
+def test_nm_roundtrip():
+    for n, m in [(6, 8), (2, 4), (3, 8)]:
+        w = wl.master_weights(12, 96, seed=n + m)
+        layer = oracle.Layer(w, n, m)
+        vals, bm = oracle.pack_nm(layer.weff, layer.mask, n, m)
+        for r in range(12):
+            bits = np.array([(bm[r, k // 8] >> (k % 8)) & 1 for k in range(96)])
+            np.testing.assert_array_equal(bits, layer.mask[r])
+            kept = np.nonzero(bits)[0]
+            codes = np.array([(vals[r, s // 4] >> (2 * (s % 4))) & 3 for s in range(len(kept))])
+            dec = np.zeros(96, dtype=np.int8)
+            dec[kept] = codes - 1
+            np.testing.assert_array_equal(dec, layer.weff[r])
+
+
+# ------------------------------------------------------------ activation quant
+
+def test_act_quant_invariants_and_zero_row():
+    """Per-token absmax ("Activation Quantization: Per-Token Absmax"): every
+    nonzero row reaches |q| = 127 exactly at its absmax, zero rows give q = 0
+    and d = 0, and |q| never exceeds 127."""
+    x = wl.activations(33, 256, seed=1, outlier_frac=0.01)
+    x[5] = 0
+    x[6] = 0x8000  # all -0.0
+    q, d = oracle.quantize_act(x)
+    xf = wl.bf16_bits_to_f32(x)
+    for t in range(33):
+        if np.abs(xf[t]).max() == 0:
+            assert not q[t].any() and d[t] == 0
+        else:
+            assert np.abs(q[t]).max() == 127
+            assert d[t] == np.float32(np.abs(xf[t]).max()) / np.float32(127)
+    assert np.abs(q.astype(np.int32)).max() <= 127
+
+
+def test_act_quant_matches_numpy_float32():
+    """Special case reducing to library routines: numpy float32 arithmetic of
+    x * fl(127 / a) with rint (half-even)."""
+    x = wl.activations(50, 320, seed=2)
+    xf = wl.bf16_bits_to_f32(x)
+    a = np.abs(xf).max(axis=1)
+    r = (np.float32(127) / a).astype(np.float32)
+    ref = np.clip(np.rint(xf * r[:, None]), -128, 127).astype(np.int8)
+    q, d = oracle.quantize_act(x)
+    np.testing.assert_array_equal(q, ref)
+    np.testing.assert_array_equal(d, (a / np.float32(127)).astype(np.float32))
+
+
+def test_act_quant_tiny_by_hand():
+    # x = [2, -1, 0.5, 0] -> a = 2, r = 63.5; q = [127, -63.5 -> -64 (half-even), 31.75 -> 32, 0]
+    x = wl.f32_to_bf16_bits(np.array([[2.0, -1.0, 0.5, 0.0]], dtype=np.float32))
+    q, d = oracle.quantize_act(x)
+    np.testing.assert_array_equal(q.ravel(), [127, -64, 32, 0])
+    assert d[0] == np.float32(2.0) / np.float32(127.0)
+
+
+# ---------------------------------------------------------------------- forward
+
+def test_gemm_acc_matches_numpy_int64():
+    w = wl.master_weights(96, 256, seed=6)
+    layer = oracle.Layer(w, 6, 8)
+    q, d = oracle.quantize_act(wl.activations(40, 256, seed=6))
+    acc = oracle.gemm_acc(q, layer.weff)
+    np.testing.assert_array_equal(acc, q.astype(np.int64) @ layer.weff.astype(np.int64).T)
+
+
+def test_gemm_acc_brute_force_tiny():
+    q = np.array([[1, -2, 3, 127]], dtype=np.int8)
+    weff = np.array([[1, 0, -1, 1], [-1, -1, -1, -1]], dtype=np.int8)
+    np.testing.assert_array_equal(oracle.gemm_acc(q, weff), [[1 - 3 + 127, -(1 - 2 + 3 + 127)]])
+
+
+def test_output_matches_fp64_definition():
+    """y = s * (W_eff x~) with s = gamma * max|x| / 127 ("The Full
+    Sparse-BitLinear Layer", forward step 5) within 1e-6 normwise of an fp64
+    numpy evaluation, and the bf16 output equals torch's CPU RNE rounding."""
+    w = wl.master_weights(128, 256, seed=0)
+    x = wl.activations(64, 256, seed=0, outlier_frac=0.01)
+    layer = oracle.Layer(w, 6, 8)
+    q, d, acc, y, yb = layer.forward(x)
+    ref = (q.astype(np.float64) * d.astype(np.float64)[:, None]) @ \
+          (float(layer.gamma) * layer.weff.astype(np.float64)).T
+    assert np.abs(y - ref).max() / np.abs(ref).max() < 1e-6
+    tb = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(yb, tb)
+
+
+# --------------------------------------------------------------------- backward
+
+def _setup_bwd(n, m, t=24, o=40, k=64, seed=8):
+    w = wl.master_weights(o, k, seed=seed)
+    x = wl.activations(t, k, seed=seed)
+    dy = wl.output_grad(t, o, seed=seed)
+    layer = oracle.Layer(w, n, m)
+    q, d = oracle.quantize_act(x)
+    return w, layer, q, d, dy
+
+
+def test_backward_matches_numpy_fp64():
+    """Dual STE ("dL/dW ~= dL/dW_eff"): dX = gamma dY W_eff, dW = dY^T X~."""
+    w, layer, q, d, dy = _setup_bwd(6, 8)
+    dx, dw = oracle.backward(dy, layer.weff, layer.gamma, q, d)
+    dyf = wl.bf16_bits_to_f32(dy).astype(np.float64)
+    np.testing.assert_allclose(dx, float(layer.gamma) * dyf @ layer.weff.astype(np.float64), rtol=1e-12, atol=1e-12)
+    xt = q.astype(np.float64) * d.astype(np.float64)[:, None]
+    np.testing.assert_allclose(dw, dyf.T @ xt, rtol=1e-12, atol=1e-12)
+
+
+def test_dual_ste_dw_independent_of_mask_and_dense_at_masked_positions():
+    """Dual STE passes the gradient through the mask as identity: dW is the
+    same for every n:m and is nonzero at masked positions too."""
+    dws = []
+    for n, m in [(8, 8), (6, 8), (2, 4), (3, 8)]:
+        w, layer, q, d, dy = _setup_bwd(n, m)
+        _, dw = oracle.backward(dy, layer.weff, layer.gamma, q, d, want_dx=False)
+        dws.append(dw)
+        masked = layer.mask == 0
+        if masked.any():
+            assert (np.abs(dw[masked]) > 0).mean() > 0.99
+    for dw in dws[1:]:
+        np.testing.assert_array_equal(dw, dws[0])
+
+
+def test_dx_at_n_equal_m_is_dense_bitlinear():
+    """At n = m the layer is dense BitLinear, so dX uses W_q itself."""
+    w, layer, q, d, dy = _setup_bwd(8, 8)
+    dx, _ = oracle.backward(dy, layer.wq, layer.gamma, q, d, want_dw=False)
+    dx2, _ = oracle.backward(dy, layer.weff, layer.gamma, q, d, want_dw=False)
+    np.testing.assert_array_equal(dx, dx2)
+
+
+def test_sampled_variants_agree_with_full():
+    w, layer, q, d, dy = _setup_bwd(6, 8, t=16, o=24, k=32)
+    dx, dw = oracle.backward(dy, layer.weff, layer.gamma, q, d)
+    acc = oracle.gemm_acc(q, layer.weff)
+    rng = np.random.default_rng(0)
+    it, io, ik = rng.integers(0, 16, 50), rng.integers(0, 24, 50), rng.integers(0, 32, 50)
+    np.testing.assert_array_equal(oracle.acc_samples(q, layer.weff, it, io), acc[it, io])
+    np.testing.assert_array_equal(oracle.dx_samples(dy, layer.weff, layer.gamma, it, ik), dx[it, ik])
+    np.testing.assert_array_equal(oracle.dw_samples(dy, q, d, io, ik), dw[io, ik])
+
+
+# -------------------------------------------------------- planted-mistake check
+
+def test_pins_catch_planted_mistakes():
+    """A plausible slip in the oracle's arithmetic (here re-implemented in
+    numpy with a dropped term / wrong tie rule / wrong rounding) fails the
+    same pins, which shows the pins have teeth."""
+    # wrong tie rule (higher index wins) fails the all-equal case
+    keys = np.zeros(8, dtype=np.float32)
+    wrong = np.zeros(8, dtype=np.uint8)
+    wrong[np.argsort(-keys, kind="stable")[::-1][:6]] = 1
+    assert not np.array_equal(wrong, oracle.nm_mask(keys.reshape(1, 8), 6, 8).ravel())
+    # round-half-away instead of half-even fails the 0.5 tie
+    assert np.float32(np.floor(0.5 + 0.5)) != oracle.ternarize(np.array([0.5], dtype=np.float32), 1.0)[0]
+    # sequential instead of pairwise summation fails the order pin
+    a = 2.0 ** -53
+    seq = 0.0
+    for v in [1.0, a, a, a]:
+        seq += v
+    assert seq != oracle.abs_sum(np.array([1.0, a, a, a], dtype=np.float32))
