@@ -1,0 +1,185 @@
+/*
+ * sbl.h -- C ABI of the B200 (sm_100a) Sparse-BitLinear library (libsbl.so).
+ *
+ * The layer follows the Sparse-BitNet summary (paper-graph-ui, arXiv
+ * 2603.05168), section 3.4, "The Full Sparse-BitLinear Layer: Forward and
+ * Backward Pass": fp32 master weights are masked (N:M by magnitude) and
+ * ternarised (absmean), activations are quantised to int8 per token, the
+ * masked ternary weights multiply the int8 activations with int32
+ * accumulation, one scalar per token restores the scale, and the backward is
+ * the Dual straight-through estimator.
+ *
+ * Conventions for every entry point:
+ *  - Every data pointer is a DEVICE pointer (cudaMalloc / PyTorch memory)
+ *    owned by the caller; the library never allocates, frees or keeps them.
+ *  - Row-major layouts.  O = out_features (d_out), K = in_features (d_in),
+ *    T = tokens.  Weights are [O, K]; activations are [T, K]; outputs [T, O].
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    only enqueues work on that stream and returns; none synchronises.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns an error status and enqueues nothing.
+ *  - Data pointers must be 16-byte aligned (SBL_ERR_ALIGNMENT otherwise).
+ *  - Inputs must be finite; results for NaN/Inf inputs are unspecified.
+ *  - The library needs an sm_100 device (B200); other devices get
+ *    SBL_ERR_DEVICE.
+ *  - A device-side wait that exceeds its time limit (it never should) makes
+ *    the kernel record a code readable with sbl_device_error() and return.
+ */
+#ifndef SBL_H
+#define SBL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SBL_OK = 0,
+    SBL_ERR_INVALID_ARG = 1,  /* null pointer, unknown enum value          */
+    SBL_ERR_SHAPE = 2,        /* sizes out of range or not divisible       */
+    SBL_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned          */
+    SBL_ERR_UNSUPPORTED = 4,  /* valid but not implemented (n:m, format)   */
+    SBL_ERR_WORKSPACE = 5,    /* workspace missing or too small            */
+    SBL_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed      */
+    SBL_ERR_DEVICE = 7        /* no sm_100 device current                  */
+} sbl_status;
+
+/* Packed weight formats (bit mask for sbl_quantize_mask_pack).
+ *  PK2   2-bit codes of W_eff, code = w + 1 ({-1,0,+1} -> {0,1,2}, following
+ *        the 2-bit packing of the BitNet b1.58 2B4T summary, "Inference
+ *        Implementation: GPU"); weight k of a row sits at bits 2*(k%4) of
+ *        byte k/4; rows are padded to a multiple of 16 bytes with 0x55
+ *        (zero weights).  Layout [O, sbl_packed_row_bytes(PK2)] uint8.
+ *  NM    compressed: per row, the 2-bit codes of the kept positions in
+ *        ascending order, four per byte LSB-first, padded to 16 bytes with
+ *        code 1 ([O, row_bytes(NM values)] uint8), plus a keep bitmap (bit
+ *        k%8 of byte k/8 set when position k is kept, padded with 0 bits to
+ *        16 bytes; [O, row_bytes(NM bitmap)] uint8).
+ *  I8    W_eff as int8 [O, K] (the GEMM operand).
+ *  BF16T W_eff transposed, bf16 [K, O] (the dX operand of the backward).  */
+typedef enum {
+    SBL_FMT_PK2 = 1,
+    SBL_FMT_NM = 2,
+    SBL_FMT_I8 = 4,
+    SBL_FMT_BF16T = 8
+} sbl_format;
+
+/* Which buffer of a format sbl_packed_row_bytes() describes. */
+typedef enum {
+    SBL_BUF_MAIN = 0,      /* PK2 / I8 / BF16T data, NM values */
+    SBL_BUF_NM_BITMAP = 1  /* NM keep bitmap                   */
+} sbl_buffer;
+
+/* Operations that take a workspace. */
+typedef enum {
+    SBL_OP_QUANTIZE_MASK_PACK = 0,
+    SBL_OP_BACKWARD = 1
+} sbl_op;
+
+/* A Sparse-BitLinear layer: W is [out_features, in_features]; the N:M mask
+ * keeps n of every m consecutive weights along in_features.
+ * Requirements: 1 <= n <= m, m in {4, 8}; in_features >= 16 and a multiple
+ * of 16 (and of m); out_features >= 16 and a multiple of 16. */
+typedef struct {
+    int32_t out_features;
+    int32_t in_features;
+    int32_t n;
+    int32_t m;
+} sbl_layer_desc;
+
+/* Device buffers of a packed layer.  Only the members a call uses must be
+ * non-null.  `gamma` is a device fp32 scalar written by
+ * sbl_quantize_mask_pack and read by the forward and backward. */
+typedef struct {
+    uint8_t *pk2;       /* SBL_FMT_PK2                                  */
+    uint8_t *nm_values; /* SBL_FMT_NM values                            */
+    uint8_t *nm_bitmap; /* SBL_FMT_NM keep bitmap                       */
+    int8_t *i8;         /* SBL_FMT_I8  [O, K]                           */
+    uint16_t *bf16t;    /* SBL_FMT_BF16T [K, O] bf16 bits               */
+    float *gamma;       /* device scalar                                */
+} sbl_packed;
+
+/* Human-readable text for a status code (static storage). */
+const char *sbl_status_string(sbl_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t sbl_version(void);
+
+/* Bytes per row of one buffer of a packed format (0 for an invalid
+ * descriptor).  The buffer holds out_features rows, or in_features rows for
+ * SBL_FMT_BF16T. */
+size_t sbl_packed_row_bytes(const sbl_layer_desc *desc, sbl_format fmt, sbl_buffer which);
+
+/* Workspace bytes an operation needs for `tokens` tokens (tokens is ignored
+ * by SBL_OP_QUANTIZE_MASK_PACK).  0 for an invalid descriptor. */
+size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op);
+
+/* Steps 2-4 of the forward ("compute mask from master weights", "ternary
+ * quantization of master weights", "apply mask to quantized weights"):
+ *   gamma = mean |W| over all O*K master weights (sum in fp64 over a
+ *           pairwise tree in flat row-major order, then rounded to fp32);
+ *   W_q   = clamp(round_half_even(fl32(W / gamma)), -1, 1)  (0 if gamma==0);
+ *   M     = per group of m along K, keep the n largest |W| (lower index
+ *           wins ties);
+ *   W_eff = W_q * M, written in every format whose bit is set in `formats`.
+ * W: [O, K] fp32 device.  out: the buffers of the requested formats plus
+ * `gamma` (always written).  workspace: device memory of at least
+ * sbl_workspace_bytes(desc, 0, SBL_OP_QUANTIZE_MASK_PACK) bytes, 256-byte
+ * aligned; its contents are scratch.  Two launches. */
+sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W,
+                                  uint32_t formats, const sbl_packed *out,
+                                  void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/* Step 1 of the forward, per-token absmax int8 quantisation (BitNet b1.58
+ * 2B4T summary, "Activation Quantization: Per-Token Absmax"; Sparse-BitNet
+ * summary, activation quantization equation):
+ *   a_t = max_k |x[t,k]|;  a_t == 0 -> q[t,:] = 0, d[t] = 0;  otherwise
+ *   q[t,k] = clamp(round_half_even(fl32(x[t,k] * fl32(127 / a_t))), -128, 127)
+ *   d[t]   = fl32(a_t / 127).
+ * X: [T, K] bf16 bits; Xq: [T, K] int8; d: [T] fp32.  K as for a layer
+ * (multiple of 16); T >= 0 (T == 0 enqueues nothing).  One launch. */
+sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K,
+                            int8_t *Xq, float *d, void *stream);
+
+/* Step 5 of the forward: acc[t,o] = sum_k W_eff[o,k] * Xq[t,k] (int32), and
+ *   Y[t,o] = fl32(fl32(acc) * fl32(gamma * d[t]))  (bf16 by RNE, or fp32).
+ * fmt selects the weight operand: SBL_FMT_I8 runs the tcgen05 int8 tensor
+ * core GEMM (any T); SBL_FMT_PK2 runs the decode kernel that streams the
+ * 2-bit codes (T <= 16).  Y: [T, O] bf16 bits (y_is_fp32 = 0) or fp32.
+ * acc_out: optional [T, O] int32 copy of the accumulators (NULL to skip).
+ * One launch. */
+sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d,
+                       int32_t T, const sbl_packed *w, sbl_format fmt,
+                       void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);
+
+/* Backward through the layer with the Dual straight-through estimator
+ * (Sparse-BitNet summary, "The Dual Straight-Through Estimator": the
+ * gradient passes through mask and quantiser as identity):
+ *   dX[t,k] = gamma * sum_o dY[t,o] * W_eff[o,k]        (bf16 or fp32 out)
+ *   dW[o,k] = sum_t dY[t,o] * d[t] * Xq[t,k]           (fp32, unmasked)
+ * dY: [T, O] bf16 bits; Xq, d: the forward's quantised activations; w must
+ * hold SBL_FMT_BF16T and gamma.  dX may be NULL (skips dX), dW may be NULL
+ * (skips dW).  Arithmetic: tensor cores with fp32 accumulation; dY and W_eff
+ * enter dX as bf16 (exact), dY*d[t] enters dW rounded to fp16 and Xq as fp16
+ * (exact).  Requires |dY * d| < 65504.  workspace: at least
+ * sbl_workspace_bytes(desc, T, SBL_OP_BACKWARD) bytes, 256-byte aligned. */
+sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY,
+                                 const int8_t *Xq, const float *d, int32_t T,
+                                 const sbl_packed *w, void *dX, int32_t dx_is_fp32,
+                                 float *dW, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/* Device error word of the current device: 0 when every kernel's bounded
+ * waits completed; otherwise a bit per kernel family that gave up a wait.
+ * Synchronises the device.  `clear` != 0 resets it to 0 afterwards. */
+sbl_status sbl_device_error(uint32_t *code, int32_t clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBL_H */

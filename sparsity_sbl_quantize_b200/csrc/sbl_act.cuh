@@ -1,0 +1,159 @@
+// sbl_act.cuh -- activation side of the Sparse-BitLinear layer on sm_100a.
+//   * per-token absmax int8 quantisation (BitNet b1.58 2B4T summary, section
+//     3.4, "Activation Quantization: Per-Token Absmax to 8-Bit Integers";
+//     Sparse-BitNet summary, activation quantization equation): one row of X
+//     is read once into registers, reduced to max|x|, then scaled, rounded
+//     half-to-even and stored as int8 with d_t = max|x| / 127;
+//   * the operand preparation of the Dual-STE backward: dY * d_t as fp16
+//     transposed to [O, T], and the int8 activations as fp16 transposed to
+//     [K, T], so both dW operands are K-major for the tensor cores.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "sbl_device.cuh"
+
+namespace sbl {
+
+constexpr int kActMaxChunks = 8;  // 16-byte chunks (8 bf16) per thread
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float r)
+{
+    int q[4] = {__float2int_rn(__fmul_rn(a, r)), __float2int_rn(__fmul_rn(b, r)),
+                __float2int_rn(__fmul_rn(c, r)), __float2int_rn(__fmul_rn(d, r))};
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int v = min(127, max(-128, q[i]));
+        w |= (static_cast<uint32_t>(v) & 0xffu) << (8 * i);
+    }
+    return w;
+}
+
+// RT threads per token row; 256 / RT rows per CTA (RT <= 256) or one row per
+// CTA of RT threads (RT > 256).  Thread i of a row owns the 16-byte chunks
+// i, i + RT, ... (at most kActMaxChunks), so loads and stores are coalesced.
+template <int RT>
+__global__ void __launch_bounds__(RT > 256 ? RT : 256)
+    act_quant_kernel(const uint16_t *__restrict__ X, int32_t T, int32_t K, int8_t *__restrict__ Xq,
+                     float *__restrict__ d)
+{
+    constexpr int kRowsPerCta = RT >= 256 ? 1 : 256 / RT;
+    constexpr int kWarpsPerRow = RT / 32 > 0 ? RT / 32 : 1;
+    __shared__ float red[kRowsPerCta][kWarpsPerRow];
+    const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + sub;
+    const bool active = row < T;
+    const int chunks = K / 8;
+
+    uint4 v[kActMaxChunks];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const int ci = lt + c * RT;
+        if (active && ci < chunks) {
+            v[c] = __ldg(reinterpret_cast<const uint4 *>(X + row * K) + ci);
+            const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (kWarpsPerRow > 1) {
+        if ((lt & 31) == 0) red[sub][lt >> 5] = amax;
+        __syncthreads();
+        amax = red[sub][0];
+#pragma unroll
+        for (int w = 1; w < kWarpsPerRow; ++w) amax = fmaxf(amax, red[sub][w]);
+    }
+    if (!active) return;
+    const bool zero = !(amax > 0.0f);
+    const float r = zero ? 0.0f : __fdiv_rn(127.0f, amax);
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const int ci = lt + c * RT;
+        if (ci < chunks) {
+            uint2 out = make_uint2(0u, 0u);
+            if (!zero) {
+                out.x = quant4(bf16_lo(v[c].x), bf16_hi(v[c].x), bf16_lo(v[c].y), bf16_hi(v[c].y), r);
+                out.y = quant4(bf16_lo(v[c].z), bf16_hi(v[c].z), bf16_lo(v[c].w), bf16_hi(v[c].w), r);
+            }
+            reinterpret_cast<uint2 *>(Xq + row * K)[ci] = out;
+        }
+    }
+    if (lt == 0) d[row] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
+}
+
+// out[c, r] = fp16(conv(in[r, c])) for r < rows, c < cols; out has row stride
+// ld_out >= rows, and out[c, r] = 0 for rows <= r < ld_out (padding).
+// Mode 0: in is bf16 bits, value = fl32(bf16 * scale[r]) rounded to fp16.
+// Mode 1: in is int8, value = fp16(in) (exact).
+// 64 x 64 tiles through shared memory; cols % 16 == 0.
+template <int MODE>
+__global__ void __launch_bounds__(256) transpose_to_f16_kernel(const void *__restrict__ in,
+                                                               int32_t rows, int32_t cols,
+                                                               const float *__restrict__ scale,
+                                                               __half *__restrict__ out,
+                                                               int64_t ld_out)
+{
+    __shared__ float tile[64][65];
+    const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+    // load: 64 rows x 64 columns, 16 consecutive columns per thread-quarter
+    for (int idx = threadIdx.x; idx < 64 * 4; idx += 256) {
+        const int r = idx >> 2, cq = (idx & 3) * 16;
+        const int gr = r0 + r, gc = c0 + cq;
+        float vals[16];
+        if (gr < rows && gc < cols) {
+            if (MODE == 0) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(in) +
+                                                                  static_cast<int64_t>(gr) * cols + gc);
+                const float s = scale[gr];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 q = __ldg(p + h);
+                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        vals[8 * h + 2 * i] = __fmul_rn(bf16_lo(w[i]), s);
+                        vals[8 * h + 2 * i + 1] = __fmul_rn(bf16_hi(w[i]), s);
+                    }
+                }
+            } else {
+                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(in) +
+                                                                       static_cast<int64_t>(gr) * cols + gc));
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    vals[i] = static_cast<float>(static_cast<int8_t>((w[i >> 2] >> (8 * (i & 3))) & 0xffu));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) vals[i] = 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) tile[r][cq + i] = vals[i];
+    }
+    __syncthreads();
+    // store: 64 output rows (columns of in) x 64 entries, 8 per thread-chunk
+    for (int idx = threadIdx.x; idx < 64 * 8; idx += 256) {
+        const int c = idx >> 3, rq = (idx & 7) * 8;
+        const int gc = c0 + c, gr = r0 + rq;
+        if (gc < cols && gr < ld_out) {
+            uint32_t w[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const __half2 h2 = __floats2half2_rn(tile[rq + 2 * p][c], tile[rq + 2 * p + 1][c]);
+                w[p] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            *reinterpret_cast<uint4 *>(out + static_cast<int64_t>(gc) * ld_out + gr) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+}  // namespace sbl

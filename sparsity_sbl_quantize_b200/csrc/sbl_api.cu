@@ -1,0 +1,462 @@
+// sbl_api.cu -- host side of libsbl.so: argument validation, tensor-map
+// encoding and kernel launches behind the C ABI declared in include/sbl.h.
+// The library allocates no device memory; every call only enqueues work on
+// the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "sbl.h"
+#include "sbl_act.cuh"
+#include "sbl_decode.cuh"
+#include "sbl_gemm.cuh"
+#include "sbl_pack.cuh"
+
+namespace sbl {
+
+__device__ uint32_t g_device_error;
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = 65536;
+
+struct DeviceInfo {
+    bool probed = false;
+    bool ok = false;
+    int num_sms = 0;
+    uint32_t *err = nullptr;
+};
+
+static std::mutex g_mutex;
+static DeviceInfo g_devices[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn g_encode = nullptr;
+
+// Probe the current device once: sm_100, SM count, error word address,
+// kernel attributes.
+static sbl_status current_device(DeviceInfo **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBL_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &di = g_devices[dev];
+    if (!di.probed) {
+        di.probed = true;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            return SBL_ERR_DEVICE;
+        }
+        if (major != 10 || minor != 0) return SBL_ERR_DEVICE;
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&di.err), g_device_error) != cudaSuccess)
+            return SBL_ERR_CUDA;
+        if (cudaFuncSetAttribute(gemm_kernel<kKindI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 200 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 200 * 1024) != cudaSuccess)
+            return SBL_ERR_CUDA;
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                                 &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return SBL_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        di.ok = true;
+    }
+    if (!di.ok) return SBL_ERR_DEVICE;
+    *out = &di;
+    return SBL_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+static sbl_status check_desc(const sbl_layer_desc *d)
+{
+    if (!d) return SBL_ERR_INVALID_ARG;
+    if (d->m != 4 && d->m != 8) return SBL_ERR_UNSUPPORTED;
+    if (d->n < 1 || d->n > d->m) return SBL_ERR_SHAPE;
+    if (d->in_features < 16 || d->in_features % 16 != 0 || d->in_features % d->m != 0 ||
+        d->in_features > kMaxDim)
+        return SBL_ERR_SHAPE;
+    if (d->out_features < 16 || d->out_features % 16 != 0 || d->out_features > kMaxDim)
+        return SBL_ERR_SHAPE;
+    const int64_t count = static_cast<int64_t>(d->out_features) * d->in_features;
+    if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
+    return SBL_OK;
+}
+
+static sbl_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? SBL_OK : SBL_ERR_CUDA;
+}
+
+// 2-D K-major tensor map with the 128-byte swizzle: rows x inner elements,
+// box = 128 bytes of K x box_rows rows.
+static bool encode_kmajor(CUtensorMap *map, const void *base, CUtensorMapDataType dt, int elem_bytes,
+                          int64_t inner, int64_t rows, int64_t row_stride_bytes, int box_rows)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes / elem_bytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int KIND>
+static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_bytes, const void *B,
+                              int64_t ldb_bytes, int32_t M, int32_t N, int32_t K, GemmArgs args,
+                              cudaStream_t stream)
+{
+    const int eb = (KIND == kKindI8) ? 1 : 2;
+    const CUtensorMapDataType dt = (KIND == kKindI8)    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : (KIND == kKindF16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap ta, tb;
+    if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
+    if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, kBN)) return SBL_ERR_CUDA;
+    args.M = M;
+    args.N = N;
+    args.K = K;
+    args.tiles_m = static_cast<int32_t>((M + kBM - 1) / kBM);
+    args.tiles_n = static_cast<int32_t>((N + kBN - 1) / kBN);
+    args.k_blocks = static_cast<int32_t>((static_cast<int64_t>(K) * eb + kBKBytes - 1) / kBKBytes);
+    args.err = di->err;
+    const int tiles = args.tiles_m * args.tiles_n;
+    const int grid = tiles < di->num_sms ? tiles : di->num_sms;
+    gemm_kernel<KIND><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, args);
+    return launch_status();
+}
+
+}  // namespace sbl
+
+using namespace sbl;
+
+extern "C" {
+
+const char *sbl_status_string(sbl_status s)
+{
+    switch (s) {
+    case SBL_OK: return "ok";
+    case SBL_ERR_INVALID_ARG: return "invalid argument (null pointer or unknown enum)";
+    case SBL_ERR_SHAPE: return "unsupported or inconsistent sizes";
+    case SBL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SBL_ERR_UNSUPPORTED: return "valid but unsupported configuration";
+    case SBL_ERR_WORKSPACE: return "workspace missing or too small";
+    case SBL_ERR_CUDA: return "CUDA runtime error";
+    case SBL_ERR_DEVICE: return "no sm_100 (B200) device current";
+    }
+    return "unknown status";
+}
+
+int32_t sbl_version(void) { return 100; }
+
+size_t sbl_packed_row_bytes(const sbl_layer_desc *desc, sbl_format fmt, sbl_buffer which)
+{
+    if (check_desc(desc) != SBL_OK) return 0;
+    const int64_t K = desc->in_features, O = desc->out_features;
+    switch (fmt) {
+    case SBL_FMT_PK2: return which == SBL_BUF_MAIN ? static_cast<size_t>(round_up(K / 4, 16)) : 0;
+    case SBL_FMT_NM:
+        if (which == SBL_BUF_MAIN) return static_cast<size_t>(round_up((K / desc->m * desc->n + 3) / 4, 16));
+        return static_cast<size_t>(round_up(K / 8, 16));
+    case SBL_FMT_I8: return which == SBL_BUF_MAIN ? static_cast<size_t>(K) : 0;
+    case SBL_FMT_BF16T: return which == SBL_BUF_MAIN ? static_cast<size_t>(2 * O) : 0;
+    }
+    return 0;
+}
+
+size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op)
+{
+    if (check_desc(desc) != SBL_OK) return 0;
+    if (op == SBL_OP_QUANTIZE_MASK_PACK) return static_cast<size_t>(round_up(sizeof(GammaWorkspace), 256));
+    if (op == SBL_OP_BACKWARD) {
+        if (tokens < 0) return 0;
+        const int64_t tp = round_up(tokens > 0 ? tokens : 1, 64);
+        return static_cast<size_t>(round_up(static_cast<int64_t>(desc->out_features) * tp * 2, 256) +
+                                   round_up(static_cast<int64_t>(desc->in_features) * tp * 2, 256));
+    }
+    return 0;
+}
+
+sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, uint32_t formats,
+                                  const sbl_packed *out, void *workspace, size_t workspace_bytes,
+                                  void *stream_p)
+{
+    sbl_status st = check_desc(desc);
+    if (st != SBL_OK) return st;
+    if (!W || !out || !out->gamma) return SBL_ERR_INVALID_ARG;
+    const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T;
+    if (formats & ~known) return SBL_ERR_INVALID_ARG;
+    if ((formats & SBL_FMT_PK2) && !out->pk2) return SBL_ERR_INVALID_ARG;
+    if ((formats & SBL_FMT_NM) && (!out->nm_values || !out->nm_bitmap)) return SBL_ERR_INVALID_ARG;
+    if ((formats & SBL_FMT_I8) && !out->i8) return SBL_ERR_INVALID_ARG;
+    if (formats & SBL_FMT_BF16T) {
+        if (!out->bf16t) return SBL_ERR_INVALID_ARG;
+        if (!(formats & SBL_FMT_I8)) return SBL_ERR_UNSUPPORTED;  // transposed from the int8 copy
+    }
+    if (!aligned16(W) || !aligned16(out->gamma) || ((formats & SBL_FMT_PK2) && !aligned16(out->pk2)) ||
+        ((formats & SBL_FMT_NM) && (!aligned16(out->nm_values) || !aligned16(out->nm_bitmap))) ||
+        ((formats & SBL_FMT_I8) && !aligned16(out->i8)) ||
+        ((formats & SBL_FMT_BF16T) && !aligned16(out->bf16t)))
+        return SBL_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < sbl_workspace_bytes(desc, 0, SBL_OP_QUANTIZE_MASK_PACK))
+        return SBL_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+
+    const int32_t O = desc->out_features, K = desc->in_features;
+    const int64_t count = static_cast<int64_t>(O) * K;
+    GammaWorkspace *ws = static_cast<GammaWorkspace *>(workspace);
+    if (cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+    const int gblocks = static_cast<int>((count + kGammaBlock - 1) / kGammaBlock);
+    gamma_kernel<<<gblocks, 256, 0, stream>>>(W, count, ws, out->gamma);
+    if ((st = launch_status()) != SBL_OK) return st;
+
+    PackOut po;
+    memset(&po, 0, sizeof(po));
+    if (formats & SBL_FMT_PK2) {
+        po.pk2 = out->pk2;
+        po.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_PK2, SBL_BUF_MAIN));
+    }
+    if (formats & SBL_FMT_I8) po.i8 = out->i8;
+    if (formats & SBL_FMT_NM) {
+        po.nm_values = out->nm_values;
+        po.nm_values_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_MAIN));
+        po.nm_bitmap = out->nm_bitmap;
+        po.nm_bitmap_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP));
+        if (cudaMemsetAsync(po.nm_values, 0x55, static_cast<size_t>(O) * po.nm_values_stride, stream) != cudaSuccess ||
+            cudaMemsetAsync(po.nm_bitmap, 0, static_cast<size_t>(O) * po.nm_bitmap_stride, stream) != cudaSuccess)
+            return SBL_ERR_CUDA;
+    }
+    if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM)) {
+        const int64_t groups = count / desc->m;
+        int64_t per_cta = (groups + static_cast<int64_t>(di->num_sms) * 8 - 1) / (static_cast<int64_t>(di->num_sms) * 8);
+        per_cta = round_up(per_cta < 256 ? 256 : per_cta, 256);
+        const int grid = static_cast<int>((groups + per_cta - 1) / per_cta);
+        if (desc->m == 8)
+            pack_kernel<8><<<grid, 256, 0, stream>>>(W, O, K, desc->n, ws, po, per_cta);
+        else
+            pack_kernel<4><<<grid, 256, 0, stream>>>(W, O, K, desc->n, ws, po, per_cta);
+        if ((st = launch_status()) != SBL_OK) return st;
+    }
+    if (formats & SBL_FMT_BF16T) {
+        dim3 grid((K + 63) / 64, (O + 63) / 64);
+        transpose_i8_to_bf16_kernel<<<grid, 256, 0, stream>>>(out->i8, O, K, out->bf16t);
+        if ((st = launch_status()) != SBL_OK) return st;
+    }
+    return SBL_OK;
+}
+
+sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq, float *d, void *stream_p)
+{
+    if (T < 0 || K < 16 || K % 16 != 0 || K > kMaxDim) return SBL_ERR_SHAPE;
+    if (T == 0) return SBL_OK;
+    if (!X || !Xq || !d) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xq) || !aligned16(d)) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    const int chunks = K / 8;
+    int rt = 32;
+    while (rt * kActMaxChunks < chunks) rt *= 2;
+    switch (rt) {
+#define SBL_ACT_CASE(R)                                                                     \
+    case R: {                                                                              \
+        constexpr int rows = R >= 256 ? 1 : 256 / R;                                       \
+        act_quant_kernel<R><<<(T + rows - 1) / rows, R > 256 ? R : 256, 0, stream>>>(X, T, K, Xq, d); \
+        break;                                                                             \
+    }
+        SBL_ACT_CASE(32)
+        SBL_ACT_CASE(64)
+        SBL_ACT_CASE(128)
+        SBL_ACT_CASE(256)
+        SBL_ACT_CASE(512)
+        SBL_ACT_CASE(1024)
+#undef SBL_ACT_CASE
+    default: return SBL_ERR_SHAPE;
+    }
+    return launch_status();
+}
+
+sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
+                       const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32,
+                       int32_t *acc_out, void *stream_p)
+{
+    sbl_status st = check_desc(desc);
+    if (st != SBL_OK) return st;
+    if (T < 0) return SBL_ERR_SHAPE;
+    if (T == 0) return SBL_OK;
+    if (!Xq || !d || !w || !Y || !w->gamma) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(Xq) || !aligned16(d) || !aligned16(Y) || !aligned16(w->gamma) ||
+        (acc_out && !aligned16(acc_out)))
+        return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    const int32_t O = desc->out_features, K = desc->in_features;
+
+    if (fmt == SBL_FMT_I8) {
+        if (!w->i8) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(w->i8)) return SBL_ERR_ALIGNMENT;
+        GemmArgs a;
+        memset(&a, 0, sizeof(a));
+        a.out = Y;
+        a.ldo = O;
+        a.out_fp32 = y_is_fp32 ? 1 : 0;
+        a.acc_out = acc_out;
+        a.gamma = w->gamma;
+        a.row_scale = d;
+        return launch_gemm<kKindI8>(di, Xq, K, w->i8, K, T, O, K, a, stream);
+    }
+    if (fmt == SBL_FMT_PK2) {
+        if (!w->pk2) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(w->pk2)) return SBL_ERR_ALIGNMENT;
+        if (T > kDecMaxTokens || K % kDecKUnit != 0) return SBL_ERR_UNSUPPORTED;
+        DecodeArgs a;
+        memset(&a, 0, sizeof(a));
+        a.pk2 = w->pk2;
+        a.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_PK2, SBL_BUF_MAIN));
+        a.xq = Xq;
+        a.d = d;
+        a.gamma = w->gamma;
+        a.out = Y;
+        a.out_fp32 = y_is_fp32 ? 1 : 0;
+        a.acc_out = acc_out;
+        a.T = T;
+        a.K = K;
+        a.O = O;
+        a.units = K / kDecKUnit;
+        a.err = di->err;
+        const int row_blocks = (O + kDecRows - 1) / kDecRows;
+        int cl = 1;
+        while (cl < 8 && row_blocks * cl < di->num_sms && a.units / (2 * cl) >= 1) cl *= 2;
+        a.cluster = cl;
+        a.max_slice = ((a.units + cl - 1) / cl) * kDecKUnit;
+        int ws = a.max_slice / 4;                 // bytes per packed row slice
+        if (((ws / 16) & 1) == 0) ws += 16;       // odd multiple of 16: conflict-free rows
+        a.w_stride = ws;
+        int as = a.max_slice;
+        if (((as / 16) & 1) == 0) as += 16;
+        a.a_stride = as;
+        const size_t smem = static_cast<size_t>(kDecRows) * ws + static_cast<size_t>(kDecMaxTokens) * as +
+                            static_cast<size_t>(kDecRows) * kDecMaxTokens * 4 + kDecMaxTokens * 4 + 16;
+        if (smem > 200 * 1024) return SBL_ERR_UNSUPPORTED;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(static_cast<unsigned>(row_blocks * cl));
+        cfg.blockDim = dim3(kDecThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = (T <= 8) ? cudaLaunchKernelEx(&cfg, decode_kernel<1>, a)
+                                 : cudaLaunchKernelEx(&cfg, decode_kernel<2>, a);
+        return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
+    }
+    return SBL_ERR_UNSUPPORTED;
+}
+
+sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq,
+                                 const float *d, int32_t T, const sbl_packed *w, void *dX,
+                                 int32_t dx_is_fp32, float *dW, void *workspace, size_t workspace_bytes,
+                                 void *stream_p)
+{
+    sbl_status st = check_desc(desc);
+    if (st != SBL_OK) return st;
+    if (T < 0) return SBL_ERR_SHAPE;
+    if (!dY || !w || (!dX && !dW)) return SBL_ERR_INVALID_ARG;
+    if (dX && (!w->bf16t || !w->gamma)) return SBL_ERR_INVALID_ARG;
+    if (dW && (!Xq || !d)) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(dY) || (dX && (!aligned16(dX) || !aligned16(w->bf16t) || !aligned16(w->gamma))) ||
+        (dW && (!aligned16(dW) || !aligned16(Xq) || !aligned16(d))))
+        return SBL_ERR_ALIGNMENT;
+    if (dW && (!workspace || workspace_bytes < sbl_workspace_bytes(desc, T, SBL_OP_BACKWARD)))
+        return SBL_ERR_WORKSPACE;
+    if (dW && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    const int32_t O = desc->out_features, K = desc->in_features;
+
+    if (dW && T == 0) {
+        if (cudaMemsetAsync(dW, 0, static_cast<size_t>(O) * K * 4, stream) != cudaSuccess) return SBL_ERR_CUDA;
+    }
+    if (T == 0) return SBL_OK;
+
+    if (dX) {
+        // dX[T, K] = gamma * dY[T, O] . W_eff[O, K]; B operand = W_eff^T [K, O] (K-major over O)
+        GemmArgs a;
+        memset(&a, 0, sizeof(a));
+        a.out = dX;
+        a.ldo = K;
+        a.out_fp32 = dx_is_fp32 ? 1 : 0;
+        a.gamma = w->gamma;
+        st = launch_gemm<kKindBF16>(di, dY, static_cast<int64_t>(O) * 2, w->bf16t, static_cast<int64_t>(O) * 2,
+                                    T, K, O, a, stream);
+        if (st != SBL_OK) return st;
+    }
+    if (dW) {
+        // dW[O, K] = sum_t (dY[t, o] * d_t) * q[t, k]: both operands transposed to
+        // [*, T_pad] fp16 so the reduction over tokens is K-major
+        const int64_t tp = round_up(T, 64);
+        __half *a_t = static_cast<__half *>(workspace);
+        __half *b_t = reinterpret_cast<__half *>(static_cast<uint8_t *>(workspace) +
+                                                 round_up(static_cast<int64_t>(O) * tp * 2, 256));
+        dim3 ga((O + 63) / 64, static_cast<unsigned>(tp / 64));
+        transpose_to_f16_kernel<0><<<ga, 256, 0, stream>>>(dY, T, O, d, a_t, tp);
+        if ((st = launch_status()) != SBL_OK) return st;
+        dim3 gb((K + 63) / 64, static_cast<unsigned>(tp / 64));
+        transpose_to_f16_kernel<1><<<gb, 256, 0, stream>>>(Xq, T, K, nullptr, b_t, tp);
+        if ((st = launch_status()) != SBL_OK) return st;
+        GemmArgs a;
+        memset(&a, 0, sizeof(a));
+        a.out = dW;
+        a.ldo = K;
+        a.out_fp32 = 1;
+        st = launch_gemm<kKindF16>(di, a_t, tp * 2, b_t, tp * 2, O, K, static_cast<int32_t>(tp), a, stream);
+        if (st != SBL_OK) return st;
+    }
+    return SBL_OK;
+}
+
+sbl_status sbl_device_error(uint32_t *code, int32_t clear)
+{
+    if (!code) return SBL_ERR_INVALID_ARG;
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SBL_ERR_CUDA;
+    if (cudaMemcpy(code, di->err, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return SBL_ERR_CUDA;
+    if (clear && cudaMemset(di->err, 0, sizeof(uint32_t)) != cudaSuccess) return SBL_ERR_CUDA;
+    return SBL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,297 @@
+// sbl_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for sm_100a.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]        (A, B K-major in global memory)
+//
+// Forward of the Sparse-BitLinear layer ("The Full Sparse-BitLinear Layer",
+// forward step 5 of the Sparse-BitNet summary): A = int8 activations [T, K],
+// B = int8 W_eff [O, K], int32 accumulators in tensor memory, then the
+// epilogue y = fl32(fl32(acc) * fl32(gamma * d_t)).  The same kernel with
+// 16-bit operands and fp32 accumulation runs the two GEMMs of the Dual-STE
+// backward.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA loads into a 4-stage shared
+// memory ring; warp 1 owns the tensor memory (512 columns = two 128 x 256
+// fp32/int32 accumulators) and lane 0 issues the MMAs; warps 2-5 drain the
+// accumulators (tcgen05.ld) and store the outputs, overlapping the next
+// tile's MMAs.  Every wait is time-bounded (see sbl_device.cuh).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "sbl_device.cuh"
+
+namespace sbl {
+
+enum GemmKind : int { kKindI8 = 0, kKindF16 = 1, kKindBF16 = 2 };
+
+constexpr int kBM = 128;                 // tile rows (A rows, TMEM lanes)
+constexpr int kBN = 256;                 // tile columns (B rows, TMEM columns)
+constexpr int kBKBytes = 128;            // K bytes per stage (one 128-byte swizzle row)
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBKBytes;  // 16 KiB
+constexpr int kBBytes = kBN * kBKBytes;  // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 2 * kBN;       // double-buffered accumulator
+constexpr int kGemmThreads = 192;
+constexpr int kGroupM = 8;               // tile raster: groups of 8 row tiles
+constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 256 /*barriers*/;
+
+struct GemmArgs {
+    int32_t M, N, K;        // K in elements
+    int32_t tiles_m, tiles_n;
+    int32_t k_blocks;       // ceil(K bytes / 128)
+    void *out;              // [M, ldo] fp32 or bf16
+    int64_t ldo;            // elements
+    int32_t out_fp32;
+    int32_t *acc_out;       // optional raw accumulators [M, ldo] (int32 / fp32 bits)
+    const float *gamma;     // device scalar (nullptr: 1)
+    const float *row_scale; // per-row d_t (nullptr: none)
+    uint32_t *err;
+};
+
+template <int KIND>
+__device__ __forceinline__ constexpr uint32_t gemm_idesc()
+{
+    // D format (bits 4-5), A/B formats (7-9, 10-12), K-major A and B (bits 15,
+    // 16 = 0), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+    uint32_t d = 0;
+    if (KIND == kKindI8) d |= (2u << 4) | (1u << 7) | (1u << 10);       // s32 <- s8 x s8
+    else if (KIND == kKindF16) d |= (1u << 4);                          // f32 <- f16 x f16
+    else d |= (1u << 4) | (1u << 7) | (1u << 10);                       // f32 <- bf16 x bf16
+    d |= static_cast<uint32_t>(kBN >> 3) << 17;
+    d |= static_cast<uint32_t>(kBM >> 4) << 24;
+    return d;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &tm, int &tn)
+{
+    const int per_group = kGroupM * tiles_n;
+    const int group = tile / per_group;
+    const int first_m = group * kGroupM;
+    const int gm = min(tiles_m - first_m, kGroupM);
+    const int r = tile - group * per_group;
+    tm = first_m + r % gm;
+    tn = r / gm;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw);
+    const uint32_t a_base = base;
+    const uint32_t b_base = base + kStages * kABytes;
+    const uint32_t bar_base = base + kStages * kStageBytes;
+    // barrier addresses: full[s], empty[s], tfull[2], tempty[2], drain
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
+    auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * kStages + a); };
+    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kStages + 2 + a); };
+    const uint32_t drain_bar = bar_base + 8u * (2 * kStages + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kStages * kStageBytes + 128);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = args.tiles_m * args.tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 4 * 32);
+        }
+        mbar_init(drain_bar, 1);
+        fence_barrier_init();
+        tma_prefetch_map(&tmA);
+        tma_prefetch_map(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // Roles run as whole warps: every lane waits on the barriers (warp-uniform
+    // outcome through __all_sync), lane 0 issues the TMA / MMA instructions.
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        uint32_t issued_mask = 0;
+        uint32_t issued_phase[kStages];
+        for (int s = 0; s < kStages; ++s) issued_phase[s] = 0;
+        constexpr int kElemsPerBlock = (KIND == kKindI8) ? 128 : 64;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            int tm, tn;
+            tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+            for (int kb = 0; kb < args.k_blocks; ++kb) {
+                const bool ready = mbar_wait(empty_bar(stage), phase ^ 1u, args.err, kErrGemmProducer);
+                if (!__all_sync(0xffffffffu, ready)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+                    tma_load_2d(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, tm * kBM,
+                                full_bar(stage));
+                    tma_load_2d(b_base + stage * kBBytes, &tmB, kb * kElemsPerBlock, tn * kBN,
+                                full_bar(stage));
+                }
+                __syncwarp();
+                issued_mask |= 1u << stage;
+                issued_phase[stage] = phase;
+                if (++stage == kStages) stage = 0, phase ^= 1u;
+            }
+        }
+        if (!ok) {
+            // let any load still in flight land before the CTA can exit
+            for (int s = 0; s < kStages; ++s)
+                if (issued_mask & (1u << s)) mbar_wait(full_bar(s), issued_phase[s], args.err, kErrGemmProducer);
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = gemm_idesc<KIND>();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int local = 0;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            const bool free_acc = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, args.err, kErrGemmMma);
+            if (!__all_sync(0xffffffffu, free_acc)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+            for (int kb = 0; kb < args.k_blocks; ++kb) {
+                const bool ready = mbar_wait(full_bar(stage), phase, args.err, kErrGemmMma);
+                if (!__all_sync(0xffffffffu, ready)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t adesc = smem_desc_k128(a_base + stage * kABytes);
+                    const uint64_t bdesc = smem_desc_k128(b_base + stage * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBKBytes / 32; ++kk) {
+                        // +32 bytes along K = +2 in the 16-byte address field
+                        const uint64_t step = static_cast<uint64_t>(2 * kk);
+                        if (KIND == kKindI8)
+                            mma_i8(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
+                        else
+                            mma_f16(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
+                    }
+                    tc_commit(empty_bar(stage));  // frees the stage once these MMAs finish
+                }
+                __syncwarp();
+                if (++stage == kStages) stage = 0, phase ^= 1u;
+            }
+            if (!ok) break;
+            if (lane == 0) tc_commit(tfull_bar(acc));  // accumulator ready for the epilogue
+            __syncwarp();
+        }
+        // every MMA issued above has completed before TMEM is released
+        if (lane == 0) tc_commit(drain_bar);
+        __syncwarp();
+        mbar_wait(drain_bar, 0, args.err, kErrGemmMma);
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (warps 2-5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int r = quarter * 32 + lane;
+        const float g = args.gamma ? *args.gamma : 1.0f;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            int tm, tn;
+            tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
+            if (!__all_sync(0xffffffffu, ready)) break;  // warp-uniform decision
+            tc_fence_after();
+            const int m = tm * kBM + r;
+            const bool row_ok = m < args.M;
+            float scale = g;
+            if (args.row_scale) scale = row_ok ? __fmul_rn(g, args.row_scale[m]) : 0.0f;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kBN);
+#pragma unroll 1
+            for (int j = 0; j < kBN / 32; ++j) {
+                uint32_t v[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + 32u * j, v);
+                tmem_wait_ld();
+                if (j == kBN / 32 - 1) {
+                    // all of this accumulator is in registers: hand TMEM back
+                    tc_fence_before();
+                    mbar_arrive(tempty_bar(acc));
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int n = tn * kBN + 32 * j + 16 * h;
+                        if (n < args.N) {  // N % 16 == 0
+                            float y[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float a = (KIND == kKindI8)
+                                                    ? __int2float_rn(static_cast<int32_t>(v[16 * h + i]))
+                                                    : __uint_as_float(v[16 * h + i]);
+                                y[i] = __fmul_rn(a, scale);
+                            }
+                            const int64_t off = static_cast<int64_t>(m) * args.ldo + n;
+                            if (args.out_fp32) {
+                                float4 *dst =
+                                    reinterpret_cast<float4 *>(static_cast<float *>(args.out) + off);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+                            } else {
+                                uint32_t p[8];
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
+                                    p[q] = *reinterpret_cast<const uint32_t *>(&b2);
+                                }
+                                uint4 *dst =
+                                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(args.out) + off);
+                                dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+                                dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+                            }
+                            if (args.acc_out) {
+                                uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + off);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    dst[q] = make_uint4(v[16 * h + 4 * q], v[16 * h + 4 * q + 1],
+                                                        v[16 * h + 4 * q + 2], v[16 * h + 4 * q + 3]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace sbl

@@ -1,0 +1,192 @@
+"""Python binding of libsbl.so (include/sbl.h): argument marshalling only.
+
+Every function keeps the C name and takes torch tensors that already live on
+the current CUDA device; the work runs in the library's sm_100a kernels on
+torch's current stream.  Importing this module loads ``libsbl.so`` from this
+directory and raises if it is missing -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsbl.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m sparsity_sbl_quantize_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+SBL_OK = 0
+SBL_FMT_PK2, SBL_FMT_NM, SBL_FMT_I8, SBL_FMT_BF16T = 1, 2, 4, 8
+SBL_BUF_MAIN, SBL_BUF_NM_BITMAP = 0, 1
+SBL_OP_QUANTIZE_MASK_PACK, SBL_OP_BACKWARD = 0, 1
+
+STATUS_NAMES = {0: "SBL_OK", 1: "SBL_ERR_INVALID_ARG", 2: "SBL_ERR_SHAPE", 3: "SBL_ERR_ALIGNMENT",
+                4: "SBL_ERR_UNSUPPORTED", 5: "SBL_ERR_WORKSPACE", 6: "SBL_ERR_CUDA",
+                7: "SBL_ERR_DEVICE"}
+
+
+class sbl_layer_desc(ctypes.Structure):
+    _fields_ = [("out_features", ctypes.c_int32), ("in_features", ctypes.c_int32),
+                ("n", ctypes.c_int32), ("m", ctypes.c_int32)]
+
+
+class sbl_packed(ctypes.Structure):
+    _fields_ = [("pk2", ctypes.c_void_p), ("nm_values", ctypes.c_void_p),
+                ("nm_bitmap", ctypes.c_void_p), ("i8", ctypes.c_void_p),
+                ("bf16t", ctypes.c_void_p), ("gamma", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_D = ctypes.POINTER(sbl_layer_desc)
+_W = ctypes.POINTER(sbl_packed)
+_i32, _u32, _sz = ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
+
+_lib.sbl_status_string.restype = ctypes.c_char_p
+_lib.sbl_status_string.argtypes = [ctypes.c_int]
+_lib.sbl_version.restype = _i32
+_lib.sbl_packed_row_bytes.restype = _sz
+_lib.sbl_packed_row_bytes.argtypes = [_D, ctypes.c_int, ctypes.c_int]
+_lib.sbl_workspace_bytes.restype = _sz
+_lib.sbl_workspace_bytes.argtypes = [_D, _i32, ctypes.c_int]
+_lib.sbl_quantize_mask_pack.restype = ctypes.c_int
+_lib.sbl_quantize_mask_pack.argtypes = [_D, _P, _u32, _W, _P, _sz, _P]
+_lib.sbl_quantize_act.restype = ctypes.c_int
+_lib.sbl_quantize_act.argtypes = [_P, _i32, _i32, _P, _P, _P]
+_lib.sbl_forward.restype = ctypes.c_int
+_lib.sbl_forward.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, _P]
+_lib.sbl_backward_dual_ste.restype = ctypes.c_int
+_lib.sbl_backward_dual_ste.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _sz, _P]
+_lib.sbl_device_error.restype = ctypes.c_int
+_lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
+
+EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
+            "sbl_quantize_mask_pack", "sbl_quantize_act", "sbl_forward", "sbl_backward_dual_ste",
+            "sbl_device_error"]
+
+
+class SblError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        msg = _lib.sbl_status_string(status).decode()
+        super().__init__(f"{call}: {STATUS_NAMES.get(status, status)} ({msg})")
+
+
+def _check(status: int, call: str):
+    if status != SBL_OK:
+        raise SblError(status, call)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def desc(out_features: int, in_features: int, n: int, m: int) -> sbl_layer_desc:
+    return sbl_layer_desc(out_features, in_features, n, m)
+
+
+@dataclass
+class Packed:
+    """Device buffers of one packed layer (torch tensors; None = absent)."""
+    gamma: torch.Tensor
+    pk2: Optional[torch.Tensor] = None
+    nm_values: Optional[torch.Tensor] = None
+    nm_bitmap: Optional[torch.Tensor] = None
+    i8: Optional[torch.Tensor] = None
+    bf16t: Optional[torch.Tensor] = None
+
+    def c(self) -> sbl_packed:
+        return sbl_packed(*[(t.data_ptr() if t is not None else None)
+                            for t in (self.pk2, self.nm_values, self.nm_bitmap, self.i8, self.bf16t,
+                                      self.gamma)])
+
+
+# ------------------------------------------------------------------ C calls
+
+def sbl_status_string(status: int) -> str:
+    return _lib.sbl_status_string(status).decode()
+
+
+def sbl_version() -> int:
+    return int(_lib.sbl_version())
+
+
+def sbl_packed_row_bytes(d: sbl_layer_desc, fmt: int, which: int = SBL_BUF_MAIN) -> int:
+    return int(_lib.sbl_packed_row_bytes(ctypes.byref(d), fmt, which))
+
+
+def sbl_workspace_bytes(d: sbl_layer_desc, tokens: int, op: int) -> int:
+    return int(_lib.sbl_workspace_bytes(ctypes.byref(d), tokens, op))
+
+
+def sbl_quantize_mask_pack(d: sbl_layer_desc, W: torch.Tensor, formats: int, out: Packed,
+                           workspace: torch.Tensor) -> None:
+    cp = out.c()
+    _check(_lib.sbl_quantize_mask_pack(ctypes.byref(d), _ptr(W), formats, ctypes.byref(cp),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream()), "sbl_quantize_mask_pack")
+
+
+def sbl_quantize_act(X: torch.Tensor, T: int, K: int, Xq: torch.Tensor, d: torch.Tensor) -> None:
+    _check(_lib.sbl_quantize_act(_ptr(X), T, K, _ptr(Xq), _ptr(d), _stream()), "sbl_quantize_act")
+
+
+def sbl_forward(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, w: Packed, fmt: int,
+                Y: torch.Tensor, y_is_fp32: bool = False, acc_out: Optional[torch.Tensor] = None) -> None:
+    cp = w.c()
+    _check(_lib.sbl_forward(ctypes.byref(dsc), _ptr(Xq), _ptr(d), T, ctypes.byref(cp), fmt, _ptr(Y),
+                            1 if y_is_fp32 else 0, _ptr(acc_out), _stream()), "sbl_forward")
+
+
+def sbl_backward_dual_ste(dsc: sbl_layer_desc, dY: torch.Tensor, Xq: Optional[torch.Tensor],
+                          d: Optional[torch.Tensor], T: int, w: Packed, dX: Optional[torch.Tensor],
+                          dx_is_fp32: bool, dW: Optional[torch.Tensor],
+                          workspace: Optional[torch.Tensor]) -> None:
+    cp = w.c()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.sbl_backward_dual_ste(ctypes.byref(dsc), _ptr(dY), _ptr(Xq), _ptr(d), T,
+                                      ctypes.byref(cp), _ptr(dX), 1 if dx_is_fp32 else 0, _ptr(dW),
+                                      _ptr(workspace), nbytes, _stream()), "sbl_backward_dual_ste")
+
+
+def sbl_device_error(clear: bool = False) -> int:
+    code = _u32(0)
+    _check(_lib.sbl_device_error(ctypes.byref(code), 1 if clear else 0), "sbl_device_error")
+    return int(code.value)
+
+
+# ------------------------------------------------- allocation helpers (torch)
+
+def alloc_packed(d: sbl_layer_desc, formats: int, device="cuda") -> Packed:
+    """Allocate (with torch) the buffers sbl_quantize_mask_pack writes."""
+    O, K = d.out_features, d.in_features
+    p = Packed(gamma=torch.empty(4, dtype=torch.float32, device=device))
+    if formats & SBL_FMT_PK2:
+        p.pk2 = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_PK2)), dtype=torch.uint8, device=device)
+    if formats & SBL_FMT_NM:
+        p.nm_values = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_NM)), dtype=torch.uint8, device=device)
+        p.nm_bitmap = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_NM, SBL_BUF_NM_BITMAP)),
+                                  dtype=torch.uint8, device=device)
+    if formats & SBL_FMT_I8:
+        p.i8 = torch.empty((O, K), dtype=torch.int8, device=device)
+    if formats & SBL_FMT_BF16T:
+        p.bf16t = torch.empty((K, O), dtype=torch.bfloat16, device=device)
+    return p
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Workspace as a 256-byte aligned torch buffer (torch's allocator aligns to 512)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/sbl.h declares, sizes its buffers like the oracle's
+formats, and rejects invalid arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "sbl.h")
+
+
+@pytest.fixture(scope="module")
+def sbl():
+    from sparsity_sbl_quantize_b200 import build
+    build.build()
+    from sparsity_sbl_quantize_b200 import sbl as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbl_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(sbl):
+    decl = declared_functions()
+    assert "sbl_forward" in decl and "sbl_quantize_mask_pack" in decl
+    lib = ctypes.CDLL(sbl.LIB_PATH)
+    for name in decl:
+        assert hasattr(lib, name), f"{name} declared in sbl.h but not exported"
+    assert sorted(sbl.EXPORTED) == decl
+
+
+def test_status_strings_and_version(sbl):
+    for code in range(8):
+        assert sbl.sbl_status_string(code)
+    assert sbl.sbl_version() >= 100
+
+
+@pytest.mark.parametrize("O,K,n,m", [(128, 256, 6, 8), (4864, 896, 2, 4), (2560, 6912, 2, 4),
+                                     (16, 16, 1, 4), (48, 80, 3, 8)])
+def test_row_bytes_match_oracle_formats(sbl, O, K, n, m):
+    import oracle
+    d = sbl.desc(O, K, n, m)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_PK2) == oracle.pk2_row_bytes(K)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_NM) == oracle.nm_value_row_bytes(K, n, m)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_NM, sbl.SBL_BUF_NM_BITMAP) == oracle.nm_bitmap_row_bytes(K)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_I8) == K
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_BF16T) == 2 * O
+
+
+@pytest.mark.parametrize("O,K,n,m", [(0, 256, 6, 8), (128, 250, 6, 8), (128, 256, 9, 8),
+                                     (128, 256, 0, 8), (128, 256, 3, 6), (20, 256, 2, 4),
+                                     (128, 8, 2, 4), (128, 131072, 2, 4)])
+def test_invalid_descriptors_are_rejected(sbl, O, K, n, m):
+    d = sbl.desc(O, K, n, m)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_PK2) == 0
+    assert sbl.sbl_workspace_bytes(d, 16, sbl.SBL_OP_BACKWARD) == 0
+
+
+def test_workspace_sizes(sbl):
+    d = sbl.desc(11008, 2048, 6, 8)
+    ws = sbl.sbl_workspace_bytes(d, 16384, sbl.SBL_OP_BACKWARD)
+    assert ws >= (11008 + 2048) * 16384 * 2
+    assert sbl.sbl_workspace_bytes(d, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK) >= 16384 * 8
+
+
+class _FakePtr:
+    """Stands in for a device tensor: only data_ptr() is read by the binding."""
+
+    def __init__(self, addr, nbytes=1 << 20):
+        self.addr, self.nbytes = addr, nbytes
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+def _raw(sbl, fn, *args):
+    return getattr(sbl._lib, fn)(*args)
+
+
+def test_validation_happens_before_any_device_access(sbl):
+    """Bad shapes, null pointers and misalignment return their status codes;
+    the device is only looked up after the arguments pass, so on a host
+    without a GPU a valid call reports SBL_ERR_DEVICE and launches nothing."""
+    good = 0x10000
+    P = ctypes.c_void_p
+    # act quant: shape, null, alignment, then device
+    assert _raw(sbl, "sbl_quantize_act", P(good), 4, 250, P(good), P(good), None) == 2
+    assert _raw(sbl, "sbl_quantize_act", None, 4, 256, P(good), P(good), None) == 1
+    assert _raw(sbl, "sbl_quantize_act", P(good + 4), 4, 256, P(good), P(good), None) == 3
+    assert _raw(sbl, "sbl_quantize_act", P(good), 0, 256, P(good), P(good), None) == 0  # T == 0: no-op
+    d = sbl.desc(128, 256, 6, 8)
+    w = sbl.sbl_packed(None, None, None, good, good, good)
+    st = _raw(sbl, "sbl_forward", ctypes.byref(d), P(good), P(good), 64, ctypes.byref(w),
+              sbl.SBL_FMT_I8, P(good), 0, None, None)
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if not has_gpu:
+        assert st == 7  # SBL_ERR_DEVICE: no launch was attempted
+    # unsupported forward format, bad n:m, missing workspace
+    assert _raw(sbl, "sbl_forward", ctypes.byref(d), P(good), P(good), 64, ctypes.byref(w),
+                sbl.SBL_FMT_NM, P(good), 0, None, None) in (4, 7)
+    bad = sbl.desc(128, 256, 3, 6)
+    assert _raw(sbl, "sbl_forward", ctypes.byref(bad), P(good), P(good), 64, ctypes.byref(w),
+                sbl.SBL_FMT_I8, P(good), 0, None, None) == 4
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d), P(good), sbl.SBL_FMT_I8,
+                ctypes.byref(w), None, 0, None) == 5
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d), P(good), 1 << 7,
+                ctypes.byref(w), P(good), 1 << 20, None) == 1
+    # BF16T needs the int8 copy in the same call
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d), P(good), sbl.SBL_FMT_BF16T,
+                ctypes.byref(w), P(good), 1 << 20, None) == 4
+    # decode path: more than 16 tokens is unsupported
+    wp = sbl.sbl_packed(good, None, None, None, None, good)
+    assert _raw(sbl, "sbl_forward", ctypes.byref(d), P(good), P(good), 17, ctypes.byref(wp),
+                sbl.SBL_FMT_PK2, P(good), 0, None, None) in (4, 7)

@@ -1,0 +1,255 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Integer stages (gamma, W_eff in every packed format, q, d, int32 accumulators)
+and the forward outputs must match bit for bit; the backward's fp32 results
+must be within 1e-3 normwise (max |gpu - ref| / max |ref|), the float
+tolerance the benchmark spec states.  Small cases compare every element and span
+several tiles with ragged tails; the full workload sizes compare all integer
+stages in full and the GEMM outputs at seeded sample coordinates.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparsity_sbl_quantize_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # the gpu marker deselects these on CPU hosts
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from gpu_case import (ALL_FORMATS, GpuLayer, bf16_dev, bits_of, forward, normwise,  # noqa: E402
+                      quantize_act, sbl_mod, to_dev)
+
+FWD_TOL = 1e-3  # only used where bit-exactness is not expected (backward)
+
+
+def check_pack(w, n, m, formats=ALL_FORMATS):
+    layer = GpuLayer(w, n, m, formats)
+    got = layer.host()
+    ref = oracle.Layer(w, n, m)
+    assert got["gamma"] == ref.gamma, (got["gamma"], ref.gamma)
+    if "i8" in got:
+        np.testing.assert_array_equal(got["i8"], ref.weff)
+    if "pk2" in got:
+        np.testing.assert_array_equal(got["pk2"], oracle.pack_pk2(ref.weff))
+    if "nm_values" in got:
+        vals, bm = oracle.pack_nm(ref.weff, ref.mask, n, m)
+        np.testing.assert_array_equal(got["nm_bitmap"], bm)
+        np.testing.assert_array_equal(got["nm_values"], vals)
+    if "bf16t" in got:
+        expect = np.where(ref.weff.T > 0, 0x3F80, np.where(ref.weff.T < 0, 0xBF80, 0)).astype(np.uint16)
+        np.testing.assert_array_equal(got["bf16t"], expect)
+    return layer, ref
+
+
+# ------------------------------------------------------------------- packing
+
+@pytest.mark.parametrize("O,K,n,m", [(128, 256, 6, 8), (48, 80, 6, 8), (64, 96, 2, 4), (32, 64, 1, 4),
+                                     (16, 16, 3, 4), (96, 160, 7, 8), (64, 128, 8, 8), (32, 64, 4, 4),
+                                     (80, 208, 3, 8), (528, 1040, 5, 8)])
+def test_pack_bit_exact(O, K, n, m):
+    check_pack(wl.master_weights(O, K, seed=O + K + n), n, m)
+
+
+def test_pack_gamma_multi_block_tree():
+    """> 16384 weights: several first-level partials plus the last-block tree,
+    with a count that is not a power of two."""
+    check_pack(wl.master_weights(1008, 1040, seed=21), 6, 8)
+
+
+def test_pack_ties_zero_and_signed_zero():
+    w = (np.random.default_rng(3).integers(-2, 3, size=(64, 128)) * 0.125).astype(np.float32)
+    w[5] = 0.0
+    w[6] = -0.0
+    check_pack(w, 6, 8)
+    check_pack(w, 2, 4)
+
+
+def test_pack_all_zero_matrix_gamma_zero():
+    layer, ref = check_pack(np.zeros((32, 64), dtype=np.float32), 6, 8)
+    assert ref.gamma == 0.0 and not layer.host()["i8"].any()
+
+
+def test_pack_rounding_boundaries():
+    """Weights at and next to the 0.5 * gamma rounding boundary (gamma = 1
+    exactly for these rows) hit the threshold test on both sides."""
+    base = np.array([0.5, -0.5, 1.5, -1.5, 2.5, -2.5] + [0.75] * 8 + [0.5, 0.5], dtype=np.float32)
+    up = np.nextafter(np.float32(0.5), np.float32(1))
+    dn = np.nextafter(np.float32(0.5), np.float32(0))
+    w = np.tile(base, (16, 4)).reshape(16, 64)
+    w[1, 0], w[2, 0], w[3, 0], w[4, 0] = up, -up, dn, -dn
+    check_pack(w, 8, 8)
+
+
+# -------------------------------------------------------------- activations
+
+@pytest.mark.parametrize("T,K", [(64, 256), (300, 1040), (1, 16), (7, 8960), (33, 11008), (5, 32768)])
+def test_act_quant_bit_exact(T, K):
+    x = wl.activations(T, K, seed=T + K, outlier_frac=0.01)
+    x[0] = 0  # an all-zero token
+    q, d = quantize_act(x)
+    qr, dr = oracle.quantize_act(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qr)
+    np.testing.assert_array_equal(d.cpu().numpy()[:T], dr)
+
+
+# ------------------------------------------------------------------- forward
+
+def run_forward_full_check(O, K, T, n, m, seed, fmt_name="I8", outliers=0.0):
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=seed)
+    x = wl.activations(T, K, seed=seed, outlier_frac=outliers)
+    layer = GpuLayer(w, n, m, 1 | 4)
+    ref = oracle.Layer(w, n, m)
+    q, d = quantize_act(x)
+    qr, dr, accr, yr, ybr = ref.forward(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qr)
+    fmt = sbl.SBL_FMT_I8 if fmt_name == "I8" else sbl.SBL_FMT_PK2
+    yb, acc = forward(layer, q, d, fmt)
+    np.testing.assert_array_equal(acc.cpu().numpy(), accr)
+    np.testing.assert_array_equal(bits_of(yb), ybr)
+    yf, _ = forward(layer, q, d, fmt, fp32=True, want_acc=False)
+    np.testing.assert_array_equal(yf.cpu().numpy(), yr)
+
+
+@pytest.mark.parametrize("O,K,T,n,m", [
+    (128, 256, 64, 6, 8),     # the single-layer workload shape
+    (528, 1040, 300, 6, 8),   # 3 x 3 tiles, ragged M, N and K
+    (256, 128, 128, 2, 4),    # exactly one tile
+    (16, 16, 1, 1, 4),        # minimum sizes
+    (784, 384, 257, 7, 8),
+    (512, 640, 1000, 2, 8),
+])
+def test_forward_gemm_bit_exact(O, K, T, n, m):
+    run_forward_full_check(O, K, T, n, m, seed=O + T)
+
+
+def test_forward_single_layer_workload_outliers():
+    wk = wl.WORKLOADS["single_256x128"]
+    lin = wk.linears[0]
+    n, m = wk.patterns[0]
+    run_forward_full_check(lin.d_out, lin.d_in, wk.tokens[0], n, m, seed=wk.seed, outliers=wk.outlier_frac)
+
+
+@pytest.mark.parametrize("O,K,T", [(256, 256, 1), (384, 640, 4), (528, 1088, 16), (6912, 2560, 16),
+                                   (2560, 6912, 1), (2560, 6912, 9), (16, 64, 3)])
+def test_forward_decode_pk2_bit_exact(O, K, T):
+    run_forward_full_check(O, K, T, 2, 4, seed=O + K + T, fmt_name="PK2")
+
+
+def test_forward_zero_tokens_is_noop():
+    sbl = sbl_mod()
+    layer = GpuLayer(wl.master_weights(32, 64, seed=1), 6, 8, 4)
+    q = torch.empty((0, 64), dtype=torch.int8, device="cuda")
+    d = torch.empty((1,), dtype=torch.float32, device="cuda")
+    y = torch.empty((1, 32), dtype=torch.bfloat16, device="cuda")
+    sbl.sbl_forward(layer.desc, q, d, 0, layer.packed, sbl.SBL_FMT_I8, y)
+
+
+def sampled_forward_check(O, K, T, n, m, seed, n_samples=2048):
+    """Full-size launch: integer stages in full, accumulators and outputs at
+    seeded sample coordinates through the oracle's sampled routine."""
+    w = wl.master_weights(O, K, seed=seed)
+    x = wl.activations(T, K, seed=seed)
+    layer = GpuLayer(w, n, m, 4)
+    ref = oracle.Layer(w, n, m)
+    got = layer.host()
+    assert got["gamma"] == ref.gamma
+    np.testing.assert_array_equal(got["i8"], ref.weff)
+    q, d = quantize_act(x)
+    qr, dr = oracle.quantize_act(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), qr)
+    np.testing.assert_array_equal(d.cpu().numpy(), dr)
+    yb, acc = forward(layer, q, d, layer.sbl.SBL_FMT_I8)
+    rng = np.random.default_rng(seed)
+    it, io = rng.integers(0, T, n_samples), rng.integers(0, O, n_samples)
+    it[:4], io[:4] = [0, T - 1, 0, T - 1], [0, 0, O - 1, O - 1]  # corners
+    acc_s = oracle.acc_samples(qr, ref.weff, it, io)
+    acc_g = acc.cpu().numpy()
+    np.testing.assert_array_equal(acc_g[it, io], acc_s)
+    _, yb_s = oracle.dequant(acc_s.astype(np.int32).reshape(-1, 1), ref.gamma, dr[it])
+    np.testing.assert_array_equal(bits_of(yb)[it, io], yb_s.ravel())
+
+
+@pytest.mark.parametrize("name", ["qwen05b_mlp", "qwen15b_decoder", "qwen3b_train"])
+def test_forward_full_workload_sizes_sampled(name):
+    wk = wl.WORKLOADS[name]
+    for li, lin in enumerate(wk.linears):
+        n, m = wk.patterns[li % len(wk.patterns)]
+        sampled_forward_check(lin.d_out, lin.d_in, wk.tokens[0], n, m, seed=wk.seed + li)
+
+
+def test_forward_sweep_patterns_full_width():
+    wk = wl.WORKLOADS["qwen15b_decoder"]
+    lin = wk.linears[4]  # gate 1536 -> 8960
+    for n, m in wk.patterns:
+        sampled_forward_check(lin.d_out, lin.d_in, 1024, n, m, seed=n * 8 + m, n_samples=512)
+
+
+def test_decode_workload_all_token_counts():
+    wk = wl.WORKLOADS["bitnet2b_decode"]
+    for lin in wk.linears:
+        for T in wk.tokens:
+            run_forward_full_check(lin.d_out, lin.d_in, T, 2, 4, seed=wk.seed + T, fmt_name="PK2")
+
+
+# ------------------------------------------------------------------ backward
+
+def run_backward(O, K, T, n, m, seed, dx_fp32=True):
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=seed)
+    x = wl.activations(T, K, seed=seed)
+    dy = wl.output_grad(T, O, seed=seed)
+    layer = GpuLayer(w, n, m, 4 | 8)
+    ref = oracle.Layer(w, n, m)
+    q, d = quantize_act(x)
+    dx = torch.empty((T, K), dtype=torch.float32 if dx_fp32 else torch.bfloat16, device="cuda")
+    dw = torch.empty((O, K), dtype=torch.float32, device="cuda")
+    ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(layer.desc, T, sbl.SBL_OP_BACKWARD))
+    sbl.sbl_backward_dual_ste(layer.desc, bf16_dev(dy), q, d, T, layer.packed, dx, dx_fp32, dw, ws)
+    torch.cuda.synchronize()
+    return layer, ref, x, dy, dx, dw
+
+
+@pytest.mark.parametrize("O,K,T,n,m", [(128, 256, 64, 6, 8), (528, 1040, 300, 6, 8), (256, 192, 70, 2, 4),
+                                       (64, 64, 1, 8, 8)])
+def test_backward_dual_ste_small(O, K, T, n, m):
+    layer, ref, x, dy, dx, dw = run_backward(O, K, T, n, m, seed=O + K)
+    qr, dr = oracle.quantize_act(x)
+    dxr, dwr = oracle.backward(dy, ref.weff, ref.gamma, qr, dr)
+    assert normwise(dx.cpu().numpy(), dxr) <= FWD_TOL
+    assert normwise(dw.cpu().numpy(), dwr) <= FWD_TOL
+    # Dual STE: the gradient reaches masked weights too
+    masked = ref.mask == 0
+    if masked.any():
+        assert (np.abs(dw.cpu().numpy()[masked]) > 0).mean() > 0.99
+
+
+def test_backward_bf16_dx():
+    layer, ref, x, dy, dx, dw = run_backward(256, 256, 128, 6, 8, seed=5, dx_fp32=False)
+    qr, dr = oracle.quantize_act(x)
+    dxr, _ = oracle.backward(dy, ref.weff, ref.gamma, qr, dr, want_dw=False)
+    dxg = bits_of(dx).astype(np.uint32) << 16
+    assert normwise(dxg.view(np.float32), dxr) <= 1e-2  # bf16 output rounding (2^-9)
+
+
+def test_backward_training_workload_sampled():
+    """The 3B training linears at full size: dX and dW at seeded samples."""
+    wk = wl.WORKLOADS["qwen3b_train"]
+    T = wk.tokens[0]
+    for li, lin in enumerate(wk.linears):
+        layer, ref, x, dy, dx, dw = run_backward(lin.d_out, lin.d_in, T, 6, 8, seed=wk.seed + li)
+        qr, dr = oracle.quantize_act(x)
+        rng = np.random.default_rng(li)
+        it, ik, io = rng.integers(0, T, 256), rng.integers(0, lin.d_in, 256), rng.integers(0, lin.d_out, 256)
+        dx_s = oracle.dx_samples(dy, ref.weff, ref.gamma, it, ik)
+        dw_s = oracle.dw_samples(dy, qr, dr, io, ik)
+        assert normwise(dx.cpu().numpy()[it, ik], dx_s) <= FWD_TOL
+        assert normwise(dw.cpu().numpy()[io, ik], dw_s) <= FWD_TOL
+
+
+def test_device_error_word_clear():
+    sbl = sbl_mod()
+    assert sbl.sbl_device_error(clear=True) == 0
