@@ -134,6 +134,31 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W,
                                   void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* Same result as sbl_quantize_mask_pack, but the caller passes no workspace
+ * and the library allocates nothing.  The paper has no counterpart; this
+ * entry point exists for callers that cannot obtain device memory at the
+ * call site: a plugin hosted by a framework that owns every device
+ * allocation and exposes no allocator to it, a runtime that partitions a
+ * fixed memory budget up front, or a latency-critical path that must not
+ * risk the implicit device synchronisation cudaMalloc/cudaFree may perform.
+ *
+ * Scratch: one file-scope static device array of SBL_NOALLOC_SCRATCH_BYTES
+ * (131328 bytes) per device that loads the library, held until the process
+ * exits.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress) with the device current; make that first call
+ * before any stream capture.  Every call on a device shares the array and
+ * the library resets the part that must start at zero on each call, so
+ * calls whose kernels overlap on the GPU (different streams, no ordering)
+ * race and may produce wrong results; order them on one stream.
+ * Limit: O * K <= 2^28 weights (the array holds 16384 fp64 partial sums of
+ * 16384 weights each), the same maximum as every entry point; larger layers
+ * return SBL_ERR_SHAPE.  Other arguments, formats and errors as for
+ * sbl_quantize_mask_pack. */
+#define SBL_NOALLOC_SCRATCH_BYTES 131328
+sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const float *W,
+                                          uint32_t formats, const sbl_packed *out,
+                                          void *stream);
+
 /* Step 1 of the forward, per-token absmax int8 quantisation (BitNet b1.58
  * 2B4T summary, "Activation Quantization: Per-Token Absmax"; Sparse-BitNet
  * summary, activation quantization equation):

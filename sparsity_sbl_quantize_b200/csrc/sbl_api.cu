@@ -447,6 +447,46 @@ sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY,
     return SBL_OK;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------ no-allocation variant --
+// File-scope scratch for sbl_quantize_mask_pack_noalloc: holds the gamma
+// partial sums, the finishing counter and the ternary threshold.  In host
+// code the symbol is only a handle; its device address comes from
+// cudaGetSymbolAddress, looked up once per device on the first call.
+namespace sbl {
+static_assert(SBL_NOALLOC_SCRATCH_BYTES >= sizeof(GammaWorkspace), "scratch too small");
+static_assert(SBL_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte granularity");
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SBL_NOALLOC_SCRATCH_BYTES];
+static std::mutex g_noalloc_mutex;
+static void *g_noalloc_ptr[kMaxDevices];
+}  // namespace sbl
+
+extern "C" {
+
+sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const float *W, uint32_t formats,
+                                          const sbl_packed *out, void *stream)
+{
+    sbl_status st = check_desc(desc);
+    if (st != SBL_OK) return st;
+    // the scratch holds kGammaMaxPartials partial sums of kGammaBlock weights
+    const int64_t count = static_cast<int64_t>(desc->out_features) * desc->in_features;
+    if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBL_ERR_DEVICE;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        if (!g_noalloc_ptr[dev]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SBL_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return sbl_quantize_mask_pack(desc, W, formats, out, scratch, SBL_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 sbl_status sbl_device_error(uint32_t *code, int32_t clear)
 {
     if (!code) return SBL_ERR_INVALID_ARG;

@@ -58,6 +58,8 @@ _lib.sbl_workspace_bytes.restype = _sz
 _lib.sbl_workspace_bytes.argtypes = [_D, _i32, ctypes.c_int]
 _lib.sbl_quantize_mask_pack.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack.argtypes = [_D, _P, _u32, _W, _P, _sz, _P]
+_lib.sbl_quantize_mask_pack_noalloc.restype = ctypes.c_int
+_lib.sbl_quantize_mask_pack_noalloc.argtypes = [_D, _P, _u32, _W, _P]
 _lib.sbl_quantize_act.restype = ctypes.c_int
 _lib.sbl_quantize_act.argtypes = [_P, _i32, _i32, _P, _P, _P]
 _lib.sbl_forward.restype = ctypes.c_int
@@ -68,7 +70,7 @@ _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
-            "sbl_quantize_mask_pack", "sbl_quantize_act", "sbl_forward", "sbl_backward_dual_ste",
+            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward", "sbl_backward_dual_ste",
             "sbl_device_error"]
 
 
@@ -138,6 +140,15 @@ def sbl_quantize_mask_pack(d: sbl_layer_desc, W: torch.Tensor, formats: int, out
     _check(_lib.sbl_quantize_mask_pack(ctypes.byref(d), _ptr(W), formats, ctypes.byref(cp),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream()), "sbl_quantize_mask_pack")
+
+
+def sbl_quantize_mask_pack_noalloc(d: sbl_layer_desc, W: torch.Tensor, formats: int, out: Packed) -> None:
+    """sbl_quantize_mask_pack without a caller workspace: for callers that
+    cannot obtain device memory where they call the layer (the library uses
+    its own static per-device scratch; calls must not overlap on the GPU)."""
+    cp = out.c()
+    _check(_lib.sbl_quantize_mask_pack_noalloc(ctypes.byref(d), _ptr(W), formats, ctypes.byref(cp),
+                                               _stream()), "sbl_quantize_mask_pack_noalloc")
 
 
 def sbl_quantize_act(X: torch.Tensor, T: int, K: int, Xq: torch.Tensor, d: torch.Tensor) -> None:
