@@ -143,18 +143,18 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W,
  * risk the implicit device synchronisation cudaMalloc/cudaFree may perform.
  *
  * Scratch: one file-scope static device array of SBL_NOALLOC_SCRATCH_BYTES
- * (131328 bytes) per device that loads the library, held until the process
+ * (262400 bytes) per device that loads the library, held until the process
  * exits.  The first call on a device looks up that array's device address
  * (cudaGetSymbolAddress) with the device current; make that first call
  * before any stream capture.  Every call on a device shares the array and
  * the library resets the part that must start at zero on each call, so
  * calls whose kernels overlap on the GPU (different streams, no ordering)
  * race and may produce wrong results; order them on one stream.
- * Limit: O * K <= 2^28 weights (the array holds 16384 fp64 partial sums of
- * 16384 weights each), the same maximum as every entry point; larger layers
+ * Limit: O * K <= 2^28 weights (the array holds 32768 fp64 partial sums of
+ * 8192 weights each), the same maximum as every entry point; larger layers
  * return SBL_ERR_SHAPE.  Other arguments, formats and errors as for
  * sbl_quantize_mask_pack. */
-#define SBL_NOALLOC_SCRATCH_BYTES 131328
+#define SBL_NOALLOC_SCRATCH_BYTES 262400
 sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const float *W,
                                           uint32_t formats, const sbl_packed *out,
                                           void *stream);
@@ -174,9 +174,14 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K,
  *   Y[t,o] = fl32(fl32(acc) * fl32(gamma * d[t]))  (bf16 by RNE, or fp32).
  * fmt selects the weight operand: SBL_FMT_I8 runs the tcgen05 int8 tensor
  * core GEMM (any T); SBL_FMT_PK2 runs the decode kernel that streams the
- * 2-bit codes (T <= 16).  Y: [T, O] bf16 bits (y_is_fp32 = 0) or fp32.
- * acc_out: optional [T, O] int32 copy of the accumulators (NULL to skip).
- * One launch. */
+ * 2-bit codes (T <= 16, K a multiple of 64).  Y: [T, O] bf16 bits
+ * (y_is_fp32 = 0) or fp32.  acc_out: optional [T, O] int32 copy of the
+ * accumulators (NULL to skip).  One launch.
+ * The SBL_FMT_PK2 kernel is launched with programmatic dependent launch: it
+ * starts copying w->pk2 before it waits for the previous kernel on the
+ * stream, so w->pk2 must not be written by a preceding kernel that triggers
+ * its dependents early (sbl_quantize_mask_pack never does).  Xq, d, gamma
+ * and Y are only touched after that wait. */
 sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d,
                        int32_t T, const sbl_packed *w, sbl_format fmt,
                        void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);

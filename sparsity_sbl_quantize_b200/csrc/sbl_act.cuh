@@ -46,6 +46,9 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
     __shared__ float red[kRowsPerCta][kWarpsPerRow];
     const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + sub;
+    // programmatic dependent launch: X may come from the previous kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const bool active = row < T;
     const int chunks = K / 8;
 

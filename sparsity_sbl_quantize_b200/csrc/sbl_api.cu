@@ -122,6 +122,22 @@ static bool encode_kmajor(CUtensorMap *map, const void *base, CUtensorMapDataTyp
     return r == CUDA_SUCCESS;
 }
 
+// Output tensor map for the epilogue's TMA stores: rows x cols of bf16 or
+// fp32 with row stride ld elements; box = 32 rows x 128 bytes, 128-byte swizzle.
+static bool encode_output(CUtensorMap *map, void *base, bool fp32, int64_t rows, int64_t cols, int64_t ld)
+{
+    const int eb = fp32 ? 4 : 2;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * eb)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), 32};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int KIND>
 static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_bytes, const void *B,
                               int64_t ldb_bytes, int32_t M, int32_t N, int32_t K, GemmArgs args,
@@ -131,9 +147,10 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     const CUtensorMapDataType dt = (KIND == kKindI8)    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                    : (KIND == kKindF16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ty;
     if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
     if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, kBN)) return SBL_ERR_CUDA;
+    if (!encode_output(&ty, args.out, args.out_fp32 != 0, M, N, args.ldo)) return SBL_ERR_CUDA;
     args.M = M;
     args.N = N;
     args.K = K;
@@ -143,7 +160,7 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     args.err = di->err;
     const int tiles = args.tiles_m * args.tiles_n;
     const int grid = tiles < di->num_sms ? tiles : di->num_sms;
-    gemm_kernel<KIND><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, args);
+    gemm_kernel<KIND><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, ty, args);
     return launch_status();
 }
 
@@ -230,35 +247,54 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
     const int64_t count = static_cast<int64_t>(O) * K;
     GammaWorkspace *ws = static_cast<GammaWorkspace *>(workspace);
     if (cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+
     const int gblocks = static_cast<int>((count + kGammaBlock - 1) / kGammaBlock);
     gamma_kernel<<<gblocks, 256, 0, stream>>>(W, count, ws, out->gamma);
     if ((st = launch_status()) != SBL_OK) return st;
 
-    PackOut po;
-    memset(&po, 0, sizeof(po));
+    PackArgs pa;
+    memset(&pa, 0, sizeof(pa));
+    pa.W = W;
+    pa.rows = O;
+    pa.cols = K;
+    pa.n = desc->n;
+    pa.count = count;
+    pa.inv_cols = ~0ull / static_cast<uint64_t>(K) + 1ull;  // ceil(2^64 / K)
+    pa.gamma = out->gamma;
     if (formats & SBL_FMT_PK2) {
-        po.pk2 = out->pk2;
-        po.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_PK2, SBL_BUF_MAIN));
+        pa.out.pk2 = out->pk2;
+        pa.out.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_PK2, SBL_BUF_MAIN));
     }
-    if (formats & SBL_FMT_I8) po.i8 = out->i8;
+    if (formats & SBL_FMT_I8) pa.out.i8 = out->i8;
     if (formats & SBL_FMT_NM) {
-        po.nm_values = out->nm_values;
-        po.nm_values_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_MAIN));
-        po.nm_bitmap = out->nm_bitmap;
-        po.nm_bitmap_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP));
-        if (cudaMemsetAsync(po.nm_values, 0x55, static_cast<size_t>(O) * po.nm_values_stride, stream) != cudaSuccess ||
-            cudaMemsetAsync(po.nm_bitmap, 0, static_cast<size_t>(O) * po.nm_bitmap_stride, stream) != cudaSuccess)
+        pa.out.nm_values = out->nm_values;
+        pa.out.nm_values_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_MAIN));
+        pa.out.nm_bitmap = out->nm_bitmap;
+        pa.out.nm_bitmap_stride =
+            static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP));
+        if (cudaMemsetAsync(pa.out.nm_values, 0x55, static_cast<size_t>(O) * pa.out.nm_values_stride,
+                            stream) != cudaSuccess ||
+            cudaMemsetAsync(pa.out.nm_bitmap, 0, static_cast<size_t>(O) * pa.out.nm_bitmap_stride, stream) !=
+                cudaSuccess)
             return SBL_ERR_CUDA;
     }
     if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM)) {
+        // programmatic dependent launch behind gamma_kernel (see pack_kernel)
+        const int64_t per_cta = 256 * (16 / desc->m);  // groups per CTA
         const int64_t groups = count / desc->m;
-        int64_t per_cta = (groups + static_cast<int64_t>(di->num_sms) * 8 - 1) / (static_cast<int64_t>(di->num_sms) * 8);
-        per_cta = round_up(per_cta < 256 ? 256 : per_cta, 256);
-        const int grid = static_cast<int>((groups + per_cta - 1) / per_cta);
-        if (desc->m == 8)
-            pack_kernel<8><<<grid, 256, 0, stream>>>(W, O, K, desc->n, ws, po, per_cta);
-        else
-            pack_kernel<4><<<grid, 256, 0, stream>>>(W, O, K, desc->n, ws, po, per_cta);
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(static_cast<unsigned>((groups + per_cta - 1) / per_cta));
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = (desc->m == 8) ? cudaLaunchKernelEx(&cfg, pack_kernel<8>, pa)
+                                             : cudaLaunchKernelEx(&cfg, pack_kernel<4>, pa);
+        if (e != cudaSuccess) return SBL_ERR_CUDA;
         if ((st = launch_status()) != SBL_OK) return st;
     }
     if (formats & SBL_FMT_BF16T) {
@@ -282,12 +318,23 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq,
     const int chunks = K / 8;
     int rt = 32;
     while (rt * kActMaxChunks < chunks) rt *= 2;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaSuccess;
     switch (rt) {
-#define SBL_ACT_CASE(R)                                                                     \
-    case R: {                                                                              \
-        constexpr int rows = R >= 256 ? 1 : 256 / R;                                       \
-        act_quant_kernel<R><<<(T + rows - 1) / rows, R > 256 ? R : 256, 0, stream>>>(X, T, K, Xq, d); \
-        break;                                                                             \
+#define SBL_ACT_CASE(R)                                                        \
+    case R: {                                                                 \
+        constexpr int rows = R >= 256 ? 1 : 256 / R;                          \
+        cfg.gridDim = dim3(static_cast<unsigned>((T + rows - 1) / rows));     \
+        cfg.blockDim = dim3(R > 256 ? R : 256);                               \
+        e = cudaLaunchKernelEx(&cfg, act_quant_kernel<R>, X, T, K, Xq, d);    \
+        break;                                                                \
     }
         SBL_ACT_CASE(32)
         SBL_ACT_CASE(64)
@@ -298,6 +345,7 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq,
 #undef SBL_ACT_CASE
     default: return SBL_ERR_SHAPE;
     }
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
     return launch_status();
 }
 
@@ -351,32 +399,43 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         a.units = K / kDecKUnit;
         a.err = di->err;
         const int row_blocks = (O + kDecRows - 1) / kDecRows;
+        // K split over a cluster of cl CTAs: enough CTAs to cover the SMs,
+        // and a slice small enough for shared memory
+        auto stride_of = [](int bytes) { return ((bytes / 16) & 1) == 0 ? bytes + 16 : bytes; };
+        auto smem_of = [&](int c) {
+            const int slice = ((a.units + c - 1) / c) * kDecKUnit;
+            return static_cast<size_t>(kDecRows) * stride_of(slice / 4) +
+                   static_cast<size_t>(kDecMaxTokens) * stride_of(slice) +
+                   static_cast<size_t>(kDecRows) * kDecMaxTokens * 4 + kDecMaxTokens * 4;
+        };
         int cl = 1;
-        while (cl < 8 && row_blocks * cl < di->num_sms && a.units / (2 * cl) >= 1) cl *= 2;
+        while (cl < 8 && a.units / (2 * cl) >= 1 &&
+               (row_blocks * cl < di->num_sms || smem_of(cl) > 96 * 1024 ||
+                ((a.units + cl - 1) / cl) * kDecKUnit > 1024))
+            cl *= 2;
         a.cluster = cl;
         a.max_slice = ((a.units + cl - 1) / cl) * kDecKUnit;
-        int ws = a.max_slice / 4;                 // bytes per packed row slice
-        if (((ws / 16) & 1) == 0) ws += 16;       // odd multiple of 16: conflict-free rows
-        a.w_stride = ws;
-        int as = a.max_slice;
-        if (((as / 16) & 1) == 0) as += 16;
-        a.a_stride = as;
-        const size_t smem = static_cast<size_t>(kDecRows) * ws + static_cast<size_t>(kDecMaxTokens) * as +
-                            static_cast<size_t>(kDecRows) * kDecMaxTokens * 4 + kDecMaxTokens * 4 + 16;
-        if (smem > 200 * 1024) return SBL_ERR_UNSUPPORTED;
+        a.w_stride = stride_of(a.max_slice / 4);  // odd multiple of 16: conflict-free rows
+        a.a_stride = stride_of(a.max_slice);
+        const size_t smem = smem_of(cl);
+        if (smem > 200 * 1024 || a.max_slice > 1024) return SBL_ERR_UNSUPPORTED;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3(static_cast<unsigned>(row_blocks * cl));
         cfg.blockDim = dim3(kDecThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        // programmatic dependent launch: the kernel streams its (read-only)
+        // packed weights before waiting on the previous kernel's outputs
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         cudaError_t e = (T <= 8) ? cudaLaunchKernelEx(&cfg, decode_kernel<1>, a)
                                  : cudaLaunchKernelEx(&cfg, decode_kernel<2>, a);
         return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;

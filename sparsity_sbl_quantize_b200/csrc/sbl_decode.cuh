@@ -49,12 +49,26 @@ struct DecodeArgs {
     uint32_t *err;
 };
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Programmatic dependent launch: let the next kernel on the stream start
+// launching, and wait for the previous kernel's results.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait_prior()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s)
@@ -101,41 +115,54 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs args)
     uint8_t *a_sm = w_sm + kDecRows * args.w_stride;                  // [16][a_stride]
     int32_t *part = reinterpret_cast<int32_t *>(a_sm + kDecMaxTokens * args.a_stride);  // [128][16]
     int32_t *colsum = part + kDecRows * kDecMaxTokens;                // [16]
-    uint64_t *bar = reinterpret_cast<uint64_t *>(colsum + kDecMaxTokens);
-    const uint32_t bar_a = smem_addr(bar);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // 1. weights: one bulk copy per row, all completing on one barrier
-    if (threadIdx.x == 0) {
-        mbar_init(bar_a, 1);
-        fence_barrier_init();
+    // 1. the packed weights of this slice (read-only for the whole decode
+    //    chain): 16-byte asynchronous copies from every thread, issued before
+    //    waiting on the previous kernel so the stream overlaps its tail
+    {
+        const int cpr = klen / 64;  // 16-byte chunks per packed row slice
+        const int total = rows_here * cpr;
+        for (int c = threadIdx.x; c < total; c += kDecThreads) {
+            const int r = c / cpr, q = c - r * cpr;
+            cp_async16(smem_addr(w_sm + r * args.w_stride + 16 * q),
+                       args.pk2 + static_cast<int64_t>(row0 + r) * args.pk2_stride + k0 / 4 + 16 * q);
+        }
     }
-    __syncthreads();
-    const uint32_t row_bytes = static_cast<uint32_t>(klen / 4);
-    if (warp == 0) {
-        if (lane == 0) mbar_arrive_expect_tx(bar_a, row_bytes * static_cast<uint32_t>(rows_here));
-        __syncwarp();
-        for (int r = lane; r < rows_here; r += 32)
-            bulk_load(smem_addr(w_sm + r * args.w_stride),
-                      args.pk2 + static_cast<int64_t>(row0 + r) * args.pk2_stride + k0 / 4, row_bytes,
-                      bar_a);
-    }
+    pdl_wait_prior();  // activations, scales and gamma come from earlier kernels
 
     // 2. activations of this K slice: 4x4 byte transpose per 16-byte group
-    //    (tokens >= T are zero), plus the per-token column sums
+    //    (tokens >= T are zero), plus the per-token column sums.  Each thread
+    //    issues all of its loads before transposing.
     const int tokens = NT * 8;
     const int groups = klen / 16;
-    for (int idx = threadIdx.x; idx < tokens * groups; idx += kDecThreads) {
-        const int t = idx / groups, gq = idx - t * groups;
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (t < args.T)
-            q = __ldg(reinterpret_cast<const uint4 *>(args.xq + static_cast<int64_t>(t) * args.K + k0) + gq);
-        const uint32_t t0 = prmt(q.x, q.y, 0x5140), t1 = prmt(q.z, q.w, 0x5140);
-        const uint32_t t2 = prmt(q.x, q.y, 0x7362), t3 = prmt(q.z, q.w, 0x7362);
-        *reinterpret_cast<uint4 *>(a_sm + t * args.a_stride + gq * 16) =
-            make_uint4(prmt(t0, t1, 0x5410), prmt(t0, t1, 0x7632), prmt(t2, t3, 0x5410),
-                       prmt(t2, t3, 0x7632));
+    {
+        constexpr int kMaxPer = (kDecMaxTokens * 1024 / 16 + kDecThreads - 1) / kDecThreads;  // slice <= 1024
+        const int total = tokens * groups;
+        uint4 q[kMaxPer];
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+            const int idx = threadIdx.x + i * kDecThreads;
+            q[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (idx < total) {
+                const int t = idx / groups, gq = idx - t * groups;
+                if (t < args.T)
+                    q[i] = __ldg(reinterpret_cast<const uint4 *>(args.xq + static_cast<int64_t>(t) * args.K + k0) + gq);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+            const int idx = threadIdx.x + i * kDecThreads;
+            if (idx < total) {
+                const int t = idx / groups, gq = idx - t * groups;
+                const uint32_t t0 = prmt(q[i].x, q[i].y, 0x5140), t1 = prmt(q[i].z, q[i].w, 0x5140);
+                const uint32_t t2 = prmt(q[i].x, q[i].y, 0x7362), t3 = prmt(q[i].z, q[i].w, 0x7362);
+                *reinterpret_cast<uint4 *>(a_sm + t * args.a_stride + gq * 16) =
+                    make_uint4(prmt(t0, t1, 0x5410), prmt(t0, t1, 0x7632), prmt(t2, t3, 0x5410),
+                               prmt(t2, t3, 0x7632));
+            }
+        }
     }
     __syncthreads();
     for (int t = warp; t < tokens; t += kDecThreads / 32) {
@@ -147,16 +174,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs args)
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) colsum[t] = s;
     }
-    const bool have_w = mbar_wait(bar_a, 0, args.err, kErrDecode);
+    cp_async_wait_all();
     __syncthreads();
+    // the weights are in shared memory: let the next kernel start streaming its own
+    pdl_launch_dependents();
 
     // 3. MMAs: warp w owns rows 16w .. 16w+15 of the block
     const int g = lane >> 2, tg = lane & 3;
     int32_t acc[NT][4];
 #pragma unroll
     for (int b = 0; b < NT; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0;
-    const bool all_w = __all_sync(0xffffffffu, have_w);
-    if (all_w) {
+    {
         const uint8_t *wr0 = w_sm + (16 * warp + g) * args.w_stride;
         const uint8_t *wr1 = wr0 + 8 * args.w_stride;
         const int sh = 2 * tg;
@@ -189,17 +217,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs args)
     }
     cluster.sync();
 
-    // 5. rank 0 adds the partials of all ranks in rank order and dequantises
-    if (rank == 0) {
+    // 5. every rank finishes a share of the (row, token) outputs: it adds the
+    //    partials of all ranks (integers: order-free) and dequantises
+    {
         const float gam = *args.gamma;
-        for (int idx = threadIdx.x; idx < kDecRows * args.T; idx += kDecThreads) {
+        const int items = kDecRows * args.T;
+        const int per = (items + nranks - 1) / nranks;
+        const int i0 = rank * per, i1 = min(items, i0 + per);
+        for (int idx = i0 + threadIdx.x; idx < i1; idx += kDecThreads) {
             const int t = idx / kDecRows, r = idx - t * kDecRows;
             if (r >= rows_here) continue;
-            int32_t s = 0;
-            for (int q = 0; q < nranks; ++q) {
-                const int32_t *rp = cluster.map_shared_rank(part, q);
-                s += rp[r * kDecMaxTokens + t];
-            }
+            int32_t v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)  // all remote loads in flight together
+                v[q] = (q < nranks) ? cluster.map_shared_rank(part, q)[r * kDecMaxTokens + t] : 0;
+            const int32_t s = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
             const int o = row0 + r;
             const int64_t off = static_cast<int64_t>(t) * args.O + o;
             const float c = __fmul_rn(gam, args.d[t]);
@@ -212,7 +244,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(DecodeArgs args)
             if (args.acc_out) args.acc_out[off] = s;
         }
     }
-    cluster.sync();  // keep every rank's shared memory alive until rank 0 is done
+    cluster.sync();  // keep every rank's shared memory alive until all reads are done
 }
 
 }  // namespace sbl

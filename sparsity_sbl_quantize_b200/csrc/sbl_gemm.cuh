@@ -35,7 +35,11 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kBN;       // double-buffered accumulator
 constexpr int kGemmThreads = 192;
 constexpr int kGroupM = 8;               // tile raster: groups of 8 row tiles
-constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 256 /*barriers*/;
+// Epilogue staging: per epilogue warp two 4 KiB buffers (32 rows x 128 bytes,
+// 128-byte swizzle) feeding TMA bulk tensor stores.
+constexpr int kEpiBufBytes = 32 * 128;
+constexpr int kEpiBytes = 4 * 2 * kEpiBufBytes;
+constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + 256 /*barriers*/;
 
 struct GemmArgs {
     int32_t M, N, K;        // K in elements
@@ -78,7 +82,7 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 template <int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                GemmArgs args)
+                const __grid_constant__ CUtensorMap tmY, GemmArgs args)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -86,14 +90,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t *base_ptr = smem_raw + (base - raw);
     const uint32_t a_base = base;
     const uint32_t b_base = base + kStages * kABytes;
-    const uint32_t bar_base = base + kStages * kStageBytes;
+    const uint32_t epi_base = base + kStages * kStageBytes;  // 1024-byte aligned
+    const uint32_t bar_base = epi_base + kEpiBytes;
     // barrier addresses: full[s], empty[s], tfull[2], tempty[2], drain
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
     auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * kStages + a); };
     auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kStages + 2 + a); };
     const uint32_t drain_bar = bar_base + 8u * (2 * kStages + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kStages * kStageBytes + 128);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kStages * kStageBytes + kEpiBytes + 128);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = args.tiles_m * args.tiles_n;
@@ -111,6 +116,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_barrier_init();
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmB);
+        tma_prefetch_map(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -211,10 +217,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (warps 2-5)
+        // Lane r of warp q drains TMEM row 32q + r, scales it, and writes it as
+        // 128-byte rows into a swizzled staging buffer that lane 0 stores with
+        // one TMA bulk tensor store per 32 x 128-byte block.
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int r = quarter * 32 + lane;
         const float g = args.gamma ? *args.gamma : 1.0f;
+        const uint32_t my_bufs = epi_base + static_cast<uint32_t>(quarter) * 2u * kEpiBufBytes;
+        constexpr int kColsPerStore = 64;  // bf16: 64 x 2 B; fp32: 2 stores of 32 x 4 B
         int local = 0;
+        int nbuf = 0;  // stores issued by this warp (selects the staging buffer)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
@@ -230,60 +242,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * kBN);
 #pragma unroll 1
-            for (int j = 0; j < kBN / 32; ++j) {
-                uint32_t v[32];
+            for (int j = 0; j < kBN / kColsPerStore; ++j) {
+                const int n0 = tn * kBN + kColsPerStore * j;
+                uint32_t v0[32], v1[32];
                 __syncwarp();
-                tmem_ld_32x32b_x32(t_row + 32u * j, v);
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerStore * j), v0);
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerStore * j + 32), v1);
                 tmem_wait_ld();
-                if (j == kBN / 32 - 1) {
+                if (j == kBN / kColsPerStore - 1) {
                     // all of this accumulator is in registers: hand TMEM back
                     tc_fence_before();
                     mbar_arrive(tempty_bar(acc));
                 }
-                if (row_ok) {
+                if (n0 >= args.N) continue;  // warp-uniform
+                float y[64];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int n = tn * kBN + 32 * j + 16 * h;
-                        if (n < args.N) {  // N % 16 == 0
-                            float y[16];
+                for (int i = 0; i < 32; ++i) {
+                    const float a0 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v0[i]))
+                                                       : __uint_as_float(v0[i]);
+                    const float a1 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v1[i]))
+                                                       : __uint_as_float(v1[i]);
+                    y[i] = __fmul_rn(a0, scale);
+                    y[32 + i] = __fmul_rn(a1, scale);
+                }
+                const int nparts = args.out_fp32 ? 2 : 1;  // 128-byte row blocks in this chunk
+                for (int part = 0; part < nparts; ++part) {
+                    const uint32_t buf = my_bufs + static_cast<uint32_t>(nbuf & 1) * kEpiBufBytes;
+                    // the store issued two blocks ago from this buffer has read it
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    uint32_t w[32];
+                    if (args.out_fp32) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float a = (KIND == kKindI8)
-                                                    ? __int2float_rn(static_cast<int32_t>(v[16 * h + i]))
-                                                    : __uint_as_float(v[16 * h + i]);
-                                y[i] = __fmul_rn(a, scale);
-                            }
-                            const int64_t off = static_cast<int64_t>(m) * args.ldo + n;
-                            if (args.out_fp32) {
-                                float4 *dst =
-                                    reinterpret_cast<float4 *>(static_cast<float *>(args.out) + off);
+                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(y[32 * part + i]);
+                    } else {
 #pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    dst[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
-                            } else {
-                                uint32_t p[8];
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
-                                    p[q] = *reinterpret_cast<const uint32_t *>(&b2);
-                                }
-                                uint4 *dst =
-                                    reinterpret_cast<uint4 *>(static_cast<uint16_t *>(args.out) + off);
-                                dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
-                                dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
-                            }
-                            if (args.acc_out) {
-                                uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + off);
-#pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    dst[q] = make_uint4(v[16 * h + 4 * q], v[16 * h + 4 * q + 1],
-                                                        v[16 * h + 4 * q + 2], v[16 * h + 4 * q + 3]);
-                            }
+                        for (int i = 0; i < 32; ++i) {
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+                            w[i] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
+                    }
+                    // row `lane`: 8 chunks of 16 bytes, chunk c at position c ^ (lane % 8)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t addr = buf + static_cast<uint32_t>(lane * 128 + ((c ^ (lane & 7)) * 16));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * c]),
+                                     "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int col = args.out_fp32 ? n0 + 32 * part : n0;
+                        tma_store_2d(&tmY, buf, col, tm * kBM + quarter * 32);
+                        bulk_commit_group();
+                    }
+                    ++nbuf;
+                }
+                if (args.acc_out && row_ok) {
+                    // raw accumulators for parity checks (direct stores)
+                    for (int h = 0; h < 4; ++h) {
+                        const int n = n0 + 16 * h;
+                        if (n >= args.N) break;
+                        uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + static_cast<int64_t>(m) * args.ldo + n);
+                        const uint32_t *src = (h < 2) ? v0 + 16 * h : v1 + 16 * (h - 2);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(src[4 * q], src[4 * q + 1], src[4 * q + 2], src[4 * q + 3]);
                     }
                 }
             }
         }
+        if (lane == 0) bulk_wait_group<0>();  // every store has landed before the CTA exits
+        __syncwarp();
     }
 
     __syncthreads();

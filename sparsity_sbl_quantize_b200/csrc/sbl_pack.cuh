@@ -13,15 +13,14 @@ namespace sbl {
 
 // Elements per first-level partial of the gamma tree (a tree node: the
 // partial of block j covers [j * kGammaBlock, (j + 1) * kGammaBlock)).
-constexpr int kGammaBlock = 16384;
-// Leaves of the second-level tree: 256 threads x 64 partials each.
-constexpr int kGammaMaxPartials = 16384;
+constexpr int kGammaBlock = 8192;
+// Leaves of the second-level tree: 256 threads x 128 partials each.
+constexpr int kGammaMaxPartials = 32768;
 
 struct GammaWorkspace {
     double partials[kGammaMaxPartials];
-    uint32_t counter;       // blocks finished (reset by the last block)
-    float threshold;        // smallest fp32 t with |w| >= t  <=>  W_q != 0
-    uint32_t pad[2];
+    uint32_t counter;       // blocks finished (zeroed by the host before each launch)
+    uint32_t pad[3];
 };
 
 // Pairwise sum of 16 consecutive leaves held by one thread.
@@ -49,89 +48,6 @@ __device__ __forceinline__ float ternary_threshold(float gamma)
     return f;
 }
 
-// One block per kGammaBlock elements, 256 threads; the last block to finish
-// combines the partials and writes gamma and the ternary threshold.
-// Requires count % 16 == 0 and count <= kGammaBlock * kGammaMaxPartials.
-__global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W, int64_t count,
-                                                    GammaWorkspace *ws, float *gamma_out)
-{
-    __shared__ double warp_sums[8];
-    __shared__ double thread_sums[256];
-    __shared__ int is_last;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kGammaBlock + warp * 2048;
-
-    double sub[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int64_t e = base + s * 512 + lane * 16;
-        double v[16];
-        if (e < count) {  // count % 16 == 0: the 16 leaves are all in range
-            const float4 *p = reinterpret_cast<const float4 *>(W + e);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 f = __ldg(p + q);
-                v[4 * q + 0] = fabs(static_cast<double>(f.x));
-                v[4 * q + 1] = fabs(static_cast<double>(f.y));
-                v[4 * q + 2] = fabs(static_cast<double>(f.z));
-                v[4 * q + 3] = fabs(static_cast<double>(f.w));
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.0;
-        }
-        double t = tree16(v);
-        // butterfly: after the step with offset `off`, lane 0 holds the tree
-        // over lanes [0, 2*off)
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
-        sub[s] = t;
-    }
-    if (lane == 0) warp_sums[warp] = (sub[0] + sub[1]) + (sub[2] + sub[3]);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const double b = ((warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3])) +
-                         ((warp_sums[4] + warp_sums[5]) + (warp_sums[6] + warp_sums[7]));
-        ws->partials[blockIdx.x] = b;
-        __threadfence();
-        const uint32_t prev = atomicAdd(&ws->counter, 1u);
-        is_last = (prev == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-
-    // Second level: thread i combines partials [64 i, 64 i + 64) (a tree node),
-    // then a shared-memory tree over the 256 thread sums.
-    const int nparts = static_cast<int>(gridDim.x);
-    double acc8[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        double v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int j = threadIdx.x * 64 + c * 8 + i;
-            v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
-        }
-        acc8[c] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-    }
-    thread_sums[threadIdx.x] = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
-                               ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-    __syncthreads();
-    for (int stride = 1; stride < 256; stride *= 2) {
-        const int i = threadIdx.x * 2 * stride;
-        if (i < 256) thread_sums[i] = thread_sums[i] + thread_sums[i + stride];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        const double mean = __ddiv_rn(thread_sums[0], static_cast<double>(count));
-        const float g = __double2float_rn(mean);
-        *gamma_out = g;
-        ws->threshold = ternary_threshold(g);
-        ws->counter = 0u;
-    }
-}
-
 // Packed output buffers of one pack launch.
 struct PackOut {
     uint8_t *pk2;
@@ -143,81 +59,163 @@ struct PackOut {
     int64_t nm_bitmap_stride;
 };
 
-// One thread per group of M consecutive weights of a row.  Each CTA takes a
-// contiguous range of groups, so row/column follow from one division per
-// thread plus increments.
-template <int M>
-__global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, int32_t rows,
-                                                   int32_t cols, int32_t n,
-                                                   const GammaWorkspace *__restrict__ ws,
-                                                   PackOut out, int64_t groups_per_cta)
-{
-    const float thr = ws->threshold;
-    const uint32_t thr_bits = __float_as_uint(thr);
-    const int32_t gpr = cols / M;  // groups per row
-    const int64_t total = static_cast<int64_t>(rows) * gpr;
-    const int64_t g_begin = static_cast<int64_t>(blockIdx.x) * groups_per_cta;
-    const int64_t g_end = min(total, g_begin + groups_per_cta);
-    int64_t g = g_begin + threadIdx.x;
-    if (g >= g_end) return;
-    int32_t row = static_cast<int32_t>(g / gpr);
-    int32_t gi = static_cast<int32_t>(g - static_cast<int64_t>(row) * gpr);
+struct PackArgs {
+    const float *W;
+    int32_t rows, cols, n;
+    int64_t count;         // rows * cols (a multiple of 16)
+    uint64_t inv_cols;     // ceil(2^64 / cols): row = umul64hi(e, inv_cols) exactly for e < 2^28
+    const float *gamma;    // written by gamma_kernel
+    PackOut out;
+};
 
-    for (; g < g_end; g += blockDim.x) {
-        const float *src = W + static_cast<int64_t>(row) * cols + static_cast<int64_t>(gi) * M;
-        uint32_t bits[M];
+// Pairwise tree of the 16 leaves held in four float4 (|.| in fp64).
+__device__ __forceinline__ double tree16_f4(const float4 &a, const float4 &b, const float4 &c,
+                                            const float4 &d)
+{
+    double v[16] = {fabs((double)a.x), fabs((double)a.y), fabs((double)a.z), fabs((double)a.w),
+                    fabs((double)b.x), fabs((double)b.y), fabs((double)b.z), fabs((double)b.w),
+                    fabs((double)c.x), fabs((double)c.y), fabs((double)c.z), fabs((double)c.w),
+                    fabs((double)d.x), fabs((double)d.y), fabs((double)d.z), fabs((double)d.w)};
+    return tree16(v);
+}
+
+// gamma: one CTA per tree node of kGammaBlock weights (thread t owns the 32
+// consecutive weights [node*8192 + 32t, +32): register tree, warp butterfly,
+// CTA tree); the last CTA to finish combines the node partials over the same
+// tree and writes gamma.  ws->counter must be zero at launch.
+__global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W, int64_t count,
+                                                    GammaWorkspace *ws, float *gamma_out)
+{
+    __shared__ double warp_sums[8];
+    __shared__ double thread_sums[256];
+    __shared__ int is_last;
+    // the pack kernel may launch now: it only streams W before waiting for us
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kGammaBlock + threadIdx.x * 32;
+    float4 f[8];
 #pragma unroll
-        for (int q = 0; q < M / 4; ++q) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(src) + q);
-            bits[4 * q + 0] = __float_as_uint(f.x);
-            bits[4 * q + 1] = __float_as_uint(f.y);
-            bits[4 * q + 2] = __float_as_uint(f.z);
-            bits[4 * q + 3] = __float_as_uint(f.w);
-        }
-        // |W| as ordered integers (sign bit cleared; -0 and +0 tie).
-        uint32_t key[M];
+    for (int q = 0; q < 8; ++q) {  // count % 4 == 0: a float4 is all in or all out
+        const int64_t e = e0 + 4 * q;
+        f[q] = (e < count) ? __ldg(reinterpret_cast<const float4 *>(W + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    double t = tree16_f4(f[0], f[1], f[2], f[3]) + tree16_f4(f[4], f[5], f[6], f[7]);
+    // butterfly: after the step with offset `off`, lane 0 holds the tree over
+    // lanes [0, 2*off)
 #pragma unroll
-        for (int i = 0; i < M; ++i) key[i] = bits[i] & 0x7fffffffu;
-        // rank_i = #{ j : key_j > key_i  or  (key_j == key_i and j < i) }
-        int rank[M];
+    for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) warp_sums[warp] = t;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ws->partials[blockIdx.x] = ((warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3])) +
+                                   ((warp_sums[4] + warp_sums[5]) + (warp_sums[6] + warp_sums[7]));
+        __threadfence();
+        const uint32_t prev = atomicAdd(&ws->counter, 1u);
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // Second level: thread i combines partials [128 i, 128 i + 128) (a tree
+    // node; zeros past the end), then a shared-memory tree over 256 sums.
+    const int nparts = static_cast<int>(gridDim.x);
+    double ts = 0.0;
+    if (threadIdx.x * 128 < nparts) {
+        double acc16[16];
 #pragma unroll
-        for (int i = 0; i < M; ++i) rank[i] = 0;
+        for (int c = 0; c < 16; ++c) {
+            double v[8];
 #pragma unroll
-        for (int i = 0; i < M; ++i)
-#pragma unroll
-            for (int j = i + 1; j < M; ++j) {
-                const int jb = key[j] > key[i];  // j beats i only if strictly larger
-                rank[i] += jb;
-                rank[j] += 1 - jb;
+            for (int i = 0; i < 8; ++i) {
+                const int j = threadIdx.x * 128 + c * 8 + i;
+                v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
             }
-        int8_t weff[M];
-        uint32_t keep_bits = 0;
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-            const bool keep = rank[i] < n;
-            const bool nz = key[i] >= thr_bits;  // |w| >= threshold (both non-negative)
-            const int8_t t = nz ? ((bits[i] >> 31) ? int8_t(-1) : int8_t(1)) : int8_t(0);
-            weff[i] = keep ? t : int8_t(0);
-            keep_bits |= (keep ? 1u : 0u) << i;
+            acc16[c] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
         }
-        const int64_t row64 = row;
-        if (out.i8) {
-            int8_t *dst = out.i8 + row64 * cols + static_cast<int64_t>(gi) * M;
-            uint32_t w0 = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w0 |= (static_cast<uint32_t>(weff[i]) & 0xffu) << (8 * i);
-            if constexpr (M == 8) {
-                uint32_t w1 = 0;
+        for (int w = 1; w < 16; w *= 2)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) w1 |= (static_cast<uint32_t>(weff[4 + i]) & 0xffu) << (8 * i);
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
-            } else {
-                *reinterpret_cast<uint32_t *>(dst) = w0;
-            }
+            for (int i = 0; i < 16; i += 2 * w) acc16[i] = acc16[i] + acc16[i + w];
+        ts = acc16[0];
+    }
+    thread_sums[threadIdx.x] = ts;
+    __syncthreads();
+    for (int stride = 1; stride < 256; stride *= 2) {
+        const int i = threadIdx.x * 2 * stride;
+        if (i < 256) thread_sums[i] = thread_sums[i] + thread_sums[i + stride];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double mean = __ddiv_rn(thread_sums[0], static_cast<double>(count));
+        *gamma_out = __double2float_rn(mean);
+    }
+}
+
+// Mask + ternarise one group of M weights given as fp32 bit patterns.
+// Returns W_eff as M bytes (int8, little-endian in w0/w1) and the keep mask.
+template <int M>
+__device__ __forceinline__ void eval_group(const uint32_t (&bits)[M], uint32_t thr_bits, int n,
+                                           uint32_t &w0, uint32_t &w1, uint32_t &keep_bits)
+{
+    // |W| as ordered integers (sign bit cleared; -0 and +0 tie).
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = bits[i] & 0x7fffffffu;
+    // rank_i = #{ j : key_j > key_i  or  (key_j == key_i and j < i) }
+    int rank[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) rank[i] = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int j = i + 1; j < M; ++j) {
+            if (key[j] > key[i]) ++rank[i];  // j beats i only if strictly larger
+            else ++rank[j];
         }
-        uint32_t codes = 0;  // 2-bit code w + 1 of weight i at bits 2i
+    keep_bits = 0;
+    uint32_t b[M];
 #pragma unroll
-        for (int i = 0; i < M; ++i) codes |= static_cast<uint32_t>(weff[i] + 1) << (2 * i);
+    for (int i = 0; i < M; ++i) {
+        const bool keep = rank[i] < n;
+        const bool nz = key[i] >= thr_bits;  // |w| >= threshold (both non-negative)
+        // sign byte: 0xff for negative, 0x01 for positive
+        const uint32_t sb = (static_cast<uint32_t>(static_cast<int32_t>(bits[i]) >> 31) | 1u) & 0xffu;
+        b[i] = (keep && nz) ? sb : 0u;
+        keep_bits |= (keep ? 1u : 0u) << i;
+    }
+    w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    w1 = 0;
+    if constexpr (M == 8) w1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+}
+
+// 2-bit codes (w + 1) of the M bytes of W_eff held in w0/w1, weight i at bits 2i.
+template <int M>
+__device__ __forceinline__ uint32_t codes_of(uint32_t w0, uint32_t w1)
+{
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        const uint32_t byte = ((i < 4 ? w0 : w1) >> (8 * (i & 3))) & 0xffu;
+        // 0x00 -> 1, 0x01 -> 2, 0xff -> 0
+        c |= ((byte + 1u) & 3u) << (2 * i);
+    }
+    return c;
+}
+
+template <int M>
+__device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int32_t gi, uint32_t w0,
+                                            uint32_t w1, uint32_t keep_bits)
+{
+    const PackOut &out = a.out;
+    const int32_t gpr = a.cols / M;
+    const int64_t row64 = row;
+    if (out.i8) {
+        int8_t *dst = out.i8 + row64 * a.cols + static_cast<int64_t>(gi) * M;
+        if constexpr (M == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
+        else *reinterpret_cast<uint32_t *>(dst) = w0;
+    }
+    if (out.pk2 || out.nm_values) {
+        const uint32_t codes = codes_of<M>(w0, w1);
         if (out.pk2) {
             uint8_t *prow = out.pk2 + row64 * out.pk2_stride;
             if constexpr (M == 8)
@@ -225,7 +223,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
             else
                 prow[gi] = static_cast<uint8_t>(codes);
             if (gi == gpr - 1)
-                for (int64_t b = cols / 4; b < out.pk2_stride; ++b) prow[b] = 0x55;
+                for (int64_t b = a.cols / 4; b < out.pk2_stride; ++b) prow[b] = 0x55;
         }
         if (out.nm_values) {
             // kept codes, ascending position, 2 bits each, at bit offset gi*2n
@@ -234,13 +232,13 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
 #pragma unroll
             for (int i = 0; i < M; ++i)
                 if (keep_bits & (1u << i)) {
-                    kc |= static_cast<uint32_t>(weff[i] + 1) << (2 * s);
+                    kc |= ((codes >> (2 * i)) & 3u) << (2 * s);
                     ++s;
                 }
             // the buffer was preset to 0x55 (code 1 everywhere): xor turns each
             // written slot's 01 into the code
-            const uint32_t delta = kc ^ (0x55555555u & ((1u << (2 * n)) - 1u));
-            const int64_t bit = static_cast<int64_t>(gi) * 2 * n;
+            const uint32_t delta = kc ^ (0x55555555u & ((1u << (2 * a.n)) - 1u));
+            const int64_t bit = static_cast<int64_t>(gi) * 2 * a.n;
             uint32_t *wrow = reinterpret_cast<uint32_t *>(out.nm_values + row64 * out.nm_values_stride);
             const int64_t wi = bit >> 5;
             const int sh = static_cast<int>(bit & 31);
@@ -256,10 +254,46 @@ __global__ void __launch_bounds__(256) pack_kernel(const float *__restrict__ W, 
                 atomicOr(reinterpret_cast<uint32_t *>(brow) + (bb >> 5), keep_bits << (bb & 31));
             }
         }
-        gi += blockDim.x;
-        while (gi >= gpr) {
-            gi -= gpr;
-            ++row;
+    }
+}
+
+// Mask + ternarise + pack: each thread owns kBatch groups (16 weights) of
+// the flat group index space.  Launched with programmatic dependent launch
+// right behind gamma_kernel: W is loaded before waiting (gamma_kernel does not
+// write it), gamma after.
+template <int M>
+__global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
+{
+    constexpr int kBatch = 16 / M;  // 2 groups of 8 or 4 groups of 4
+    const int64_t total_groups = a.count / M;
+    const int64_t gbase = (static_cast<int64_t>(blockIdx.x) * 256) * kBatch + threadIdx.x;
+    uint32_t bits[kBatch][M];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+        const int64_t g = gbase + 256 * b;
+        if (g < total_groups) {
+#pragma unroll
+            for (int q = 0; q < M / 4; ++q) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(a.W + g * M) + q);
+                bits[b][4 * q + 0] = __float_as_uint(v.x);
+                bits[b][4 * q + 1] = __float_as_uint(v.y);
+                bits[b][4 * q + 2] = __float_as_uint(v.z);
+                bits[b][4 * q + 3] = __float_as_uint(v.w);
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+        const int64_t g = gbase + 256 * b;
+        if (g < total_groups) {
+            const uint64_t e = static_cast<uint64_t>(g) * M;
+            const int32_t row = static_cast<int32_t>(__umul64hi(e, a.inv_cols));
+            const int32_t col = static_cast<int32_t>(e - static_cast<uint64_t>(row) * a.cols);
+            uint32_t w0, w1, keep_bits;
+            eval_group<M>(bits[b], thr_bits, a.n, w0, w1, keep_bits);
+            store_group<M>(a, row, col / M, w0, w1, keep_bits);
         }
     }
 }
