@@ -57,12 +57,18 @@ static sbl_status current_device(DeviceInfo **out)
         if (major != 10 || minor != 0) return SBL_ERR_DEVICE;
         if (cudaGetSymbolAddress(reinterpret_cast<void **>(&di.err), g_device_error) != cudaSuccess)
             return SBL_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm_kernel<kKindI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_kernel<kKindF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_kernel<kKindBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGemmSmemBytes) != cudaSuccess ||
+        if (cudaFuncSetAttribute(gemm_kernel<kKindI8, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindF16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindBF16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindI8, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  200 * 1024) != cudaSuccess ||
             cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -138,6 +144,42 @@ static bool encode_output(CUtensorMap *map, void *base, bool fp32, int64_t rows,
     return r == CUDA_SUCCESS;
 }
 
+// Tile width per shape: the persistent grid runs ceil(tiles / grid) rounds of
+// tiles whose MMA time is proportional to BN.  128-wide tiles move 30% more
+// operand bytes per MMA and ran slower at equal rounds on B200, so they are
+// taken only when they cut the column-rounds by at least 20%.
+static int choose_bn(int32_t M, int32_t N, int num_sms)
+{
+    auto rounds = [&](int bn) {
+        const int64_t tiles = static_cast<int64_t>((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
+        const int64_t grid = tiles < num_sms ? tiles : num_sms;
+        return ((tiles + grid - 1) / grid) * bn;
+    };
+    return 5 * rounds(128) <= 4 * rounds(256) ? 128 : 256;
+}
+
+template <int KIND, int BN>
+static sbl_status launch_gemm_bn(const DeviceInfo *di, const CUtensorMap &ta, const CUtensorMap &tb,
+                                 const CUtensorMap &ty, GemmArgs args, cudaStream_t stream)
+{
+    args.tiles_m = static_cast<int32_t>((args.M + kBM - 1) / kBM);
+    args.tiles_n = static_cast<int32_t>((args.N + BN - 1) / BN);
+    const int tiles = args.tiles_m * args.tiles_n;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < di->num_sms ? tiles : di->num_sms));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = GemmCfg<BN>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, ty, args) != cudaSuccess) return SBL_ERR_CUDA;
+    return launch_status();
+}
+
 template <int KIND>
 static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_bytes, const void *B,
                               int64_t ldb_bytes, int32_t M, int32_t N, int32_t K, GemmArgs args,
@@ -147,21 +189,18 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     const CUtensorMapDataType dt = (KIND == kKindI8)    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                    : (KIND == kKindF16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int bn = choose_bn(M, N, di->num_sms);
     CUtensorMap ta, tb, ty;
     if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
-    if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, kBN)) return SBL_ERR_CUDA;
+    if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, bn)) return SBL_ERR_CUDA;
     if (!encode_output(&ty, args.out, args.out_fp32 != 0, M, N, args.ldo)) return SBL_ERR_CUDA;
     args.M = M;
     args.N = N;
     args.K = K;
-    args.tiles_m = static_cast<int32_t>((M + kBM - 1) / kBM);
-    args.tiles_n = static_cast<int32_t>((N + kBN - 1) / kBN);
     args.k_blocks = static_cast<int32_t>((static_cast<int64_t>(K) * eb + kBKBytes - 1) / kBKBytes);
     args.err = di->err;
-    const int tiles = args.tiles_m * args.tiles_n;
-    const int grid = tiles < di->num_sms ? tiles : di->num_sms;
-    gemm_kernel<KIND><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, ty, args);
-    return launch_status();
+    return bn == 128 ? launch_gemm_bn<KIND, 128>(di, ta, tb, ty, args, stream)
+                     : launch_gemm_bn<KIND, 256>(di, ta, tb, ty, args, stream);
 }
 
 }  // namespace sbl
@@ -279,8 +318,9 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
             return SBL_ERR_CUDA;
     }
     if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM)) {
-        // programmatic dependent launch behind gamma_kernel (see pack_kernel)
-        const int64_t per_cta = 256 * (16 / desc->m);  // groups per CTA
+        // programmatic dependent launch behind gamma_kernel (see pack_kernel);
+        // a CTA covers 8 warps x 512 weights
+        const int64_t per_cta = 8 * 512 / desc->m;  // groups per CTA
         const int64_t groups = count / desc->m;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));

@@ -9,11 +9,17 @@
 // 16-bit operands and fp32 accumulation runs the two GEMMs of the Dual-STE
 // backward.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads into a 4-stage shared
-// memory ring; warp 1 owns the tensor memory (512 columns = two 128 x 256
-// fp32/int32 accumulators) and lane 0 issues the MMAs; warps 2-5 drain the
-// accumulators (tcgen05.ld) and store the outputs, overlapping the next
-// tile's MMAs.  Every wait is time-bounded (see sbl_device.cuh).
+// Tiles are 128 x BN (BN = 256 or 128).  Roles (320 threads): warp 0 issues
+// TMA loads into a shared-memory ring (4 stages of 48 KiB or 6 of 32 KiB);
+// warp 1 owns the tensor memory (all 512 columns: 2 accumulators of 256
+// columns or 4 of 128) and issues the MMAs from one lane; warps 2-9 drain
+// the accumulators (tcgen05.ld; two warps per 32-lane quarter, each half of
+// the columns), scale them and write the outputs through swizzled
+// shared-memory staging and TMA bulk tensor stores, overlapping the next
+// tiles' MMAs.  Every wait is time-bounded (see sbl_device.cuh).  The
+// kernel is launched with programmatic dependent launch: its prologue
+// overlaps the previous kernel, and it waits for that kernel before touching
+// global memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -26,20 +32,26 @@ namespace sbl {
 enum GemmKind : int { kKindI8 = 0, kKindF16 = 1, kKindBF16 = 2 };
 
 constexpr int kBM = 128;                 // tile rows (A rows, TMEM lanes)
-constexpr int kBN = 256;                 // tile columns (B rows, TMEM columns)
 constexpr int kBKBytes = 128;            // K bytes per stage (one 128-byte swizzle row)
-constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBKBytes;  // 16 KiB
-constexpr int kBBytes = kBN * kBKBytes;  // 32 KiB
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kTmemCols = 2 * kBN;       // double-buffered accumulator
-constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 512;           // the whole tensor memory of the SM
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 32 * (2 + kEpiWarps);
 constexpr int kGroupM = 8;               // tile raster: groups of 8 row tiles
-// Epilogue staging: per epilogue warp two 4 KiB buffers (32 rows x 128 bytes,
+// Epilogue staging: per epilogue warp one 4 KiB buffer (32 rows x 128 bytes,
 // 128-byte swizzle) feeding TMA bulk tensor stores.
 constexpr int kEpiBufBytes = 32 * 128;
-constexpr int kEpiBytes = 4 * 2 * kEpiBufBytes;
-constexpr int kGemmSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + 256 /*barriers*/;
+constexpr int kEpiBytes = kEpiWarps * kEpiBufBytes;
+
+template <int BN>
+struct GemmCfg {
+    static_assert(BN == 128 || BN == 256, "tile width");
+    static constexpr int kBBytes = BN * kBKBytes;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (192 * 1024) / kStageBytes;  // 4 (BN 256) or 6 (BN 128)
+    static constexpr int kNumAcc = kTmemCols / BN;              // 2 or 4 accumulators
+    static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + 256;
+};
 
 struct GemmArgs {
     int32_t M, N, K;        // K in elements
@@ -54,7 +66,7 @@ struct GemmArgs {
     uint32_t *err;
 };
 
-template <int KIND>
+template <int KIND, int BN>
 __device__ __forceinline__ constexpr uint32_t gemm_idesc()
 {
     // D format (bits 4-5), A/B formats (7-9, 10-12), K-major A and B (bits 15,
@@ -63,7 +75,7 @@ __device__ __forceinline__ constexpr uint32_t gemm_idesc()
     if (KIND == kKindI8) d |= (2u << 4) | (1u << 7) | (1u << 10);       // s32 <- s8 x s8
     else if (KIND == kKindF16) d |= (1u << 4);                          // f32 <- f16 x f16
     else d |= (1u << 4) | (1u << 7) | (1u << 10);                       // f32 <- bf16 x bf16
-    d |= static_cast<uint32_t>(kBN >> 3) << 17;
+    d |= static_cast<uint32_t>(BN >> 3) << 17;
     d |= static_cast<uint32_t>(kBM >> 4) << 24;
     return d;
 }
@@ -79,38 +91,42 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
     tn = r / gm;
 }
 
-template <int KIND>
+template <int KIND, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs args)
 {
+    using Cfg = GemmCfg<BN>;
+    constexpr int kStages = Cfg::kStages;
+    constexpr int kNumAcc = Cfg::kNumAcc;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw);
     const uint32_t a_base = base;
     const uint32_t b_base = base + kStages * kABytes;
-    const uint32_t epi_base = base + kStages * kStageBytes;  // 1024-byte aligned
+    const uint32_t epi_base = base + kStages * Cfg::kStageBytes;  // 1024-byte aligned
     const uint32_t bar_base = epi_base + kEpiBytes;
-    // barrier addresses: full[s], empty[s], tfull[2], tempty[2], drain
+    // barrier addresses: full[s], empty[s], tfull[a], tempty[a], drain
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
     auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * kStages + a); };
-    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kStages + 2 + a); };
-    const uint32_t drain_bar = bar_base + 8u * (2 * kStages + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kStages * kStageBytes + kEpiBytes + 128);
+    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kStages + kNumAcc + a); };
+    const uint32_t drain_bar = bar_base + 8u * (2 * kStages + 2 * kNumAcc);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (bar_base - base) + 224);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = args.tiles_m * args.tiles_n;
 
+    // ---------------------------------------------------------- prologue
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kNumAcc; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 4 * 32);
+            mbar_init(tempty_bar(a), kEpiWarps * 32);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -126,6 +142,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the previous kernel's outputs (our A operand, gamma, scales) are ready
+    // after this; our own dependents may start their prologue now
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // Roles run as whole warps: every lane waits on the barriers (warp-uniform
     // outcome through __all_sync), lane 0 issues the TMA / MMA instructions.
@@ -148,10 +168,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+                    mbar_arrive_expect_tx(full_bar(stage), Cfg::kStageBytes);
                     tma_load_2d(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, tm * kBM,
                                 full_bar(stage));
-                    tma_load_2d(b_base + stage * kBBytes, &tmB, kb * kElemsPerBlock, tn * kBN,
+                    tma_load_2d(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, tn * BN,
                                 full_bar(stage));
                 }
                 __syncwarp();
@@ -167,21 +187,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = gemm_idesc<KIND>();
+        constexpr uint32_t idesc = gemm_idesc<KIND, BN>();
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         int local = 0;
         for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
-            const int acc = local & 1;
-            const uint32_t acc_phase = (local >> 1) & 1;
+            const int acc = local % kNumAcc;
+            const uint32_t acc_phase = (local / kNumAcc) & 1;
             const bool free_acc = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, args.err, kErrGemmMma);
             if (!__all_sync(0xffffffffu, free_acc)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
             for (int kb = 0; kb < args.k_blocks; ++kb) {
                 const bool ready = mbar_wait(full_bar(stage), phase, args.err, kErrGemmMma);
                 if (!__all_sync(0xffffffffu, ready)) {
@@ -191,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_after();
                 if (lane == 0) {
                     const uint64_t adesc = smem_desc_k128(a_base + stage * kABytes);
-                    const uint64_t bdesc = smem_desc_k128(b_base + stage * kBBytes);
+                    const uint64_t bdesc = smem_desc_k128(b_base + stage * Cfg::kBBytes);
 #pragma unroll
                     for (int kk = 0; kk < kBKBytes / 32; ++kk) {
                         // +32 bytes along K = +2 in the 16-byte address field
@@ -216,72 +236,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait(drain_bar, 0, args.err, kErrGemmMma);
         __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue (warps 2-5)
-        // Lane r of warp q drains TMEM row 32q + r, scales it, and writes it as
-        // 128-byte rows into a swizzled staging buffer that lane 0 stores with
-        // one TMA bulk tensor store per 32 x 128-byte block.
+        // ---------------------------------------------------- epilogue (warps 2-9)
+        // Lane r of warp w drains TMEM row 32 (w % 4) + r over half of the
+        // columns ((w - 2) / 4), scales it, and writes it as 128-byte rows
+        // into a swizzled staging buffer that lane 0 stores with one TMA bulk
+        // tensor store per 32 x 128-byte block.
         const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
         const float g = args.gamma ? *args.gamma : 1.0f;
-        const uint32_t my_bufs = epi_base + static_cast<uint32_t>(quarter) * 2u * kEpiBufBytes;
-        constexpr int kColsPerStore = 64;  // bf16: 64 x 2 B; fp32: 2 stores of 32 x 4 B
+        const uint32_t buf = epi_base + static_cast<uint32_t>(warp - 2) * kEpiBufBytes;
+        constexpr int kColsPerChunk = 64;  // bf16: one 128-byte store; fp32: two
+        constexpr int kChunks = BN / kColsPerChunk / 2;  // per warp
         int local = 0;
-        int nbuf = 0;  // stores issued by this warp (selects the staging buffer)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
-            const int acc = local & 1;
-            const uint32_t acc_phase = (local >> 1) & 1;
+            const int acc = local % kNumAcc;
+            const uint32_t acc_phase = (local / kNumAcc) & 1;
             const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
             if (!__all_sync(0xffffffffu, ready)) break;  // warp-uniform decision
             tc_fence_after();
             const int m = tm * kBM + r;
             const bool row_ok = m < args.M;
+            const int row0 = tm * kBM + quarter * 32;  // first row of this warp's block
             float scale = g;
             if (args.row_scale) scale = row_ok ? __fmul_rn(g, args.row_scale[m]) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(acc * kBN);
+                                   static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
-            for (int j = 0; j < kBN / kColsPerStore; ++j) {
-                const int n0 = tn * kBN + kColsPerStore * j;
+            for (int jj = 0; jj < kChunks; ++jj) {
+                const int j = half * kChunks + jj;
+                const int n0 = tn * BN + kColsPerChunk * j;
                 uint32_t v0[32], v1[32];
                 __syncwarp();
-                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerStore * j), v0);
-                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerStore * j + 32), v1);
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerChunk * j), v0);
+                tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerChunk * j + 32), v1);
                 tmem_wait_ld();
-                if (j == kBN / kColsPerStore - 1) {
-                    // all of this accumulator is in registers: hand TMEM back
+                if (jj == kChunks - 1) {
+                    // all of this warp's share of the accumulator is in registers
                     tc_fence_before();
                     mbar_arrive(tempty_bar(acc));
                 }
-                if (n0 >= args.N) continue;  // warp-uniform
-                float y[64];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float a0 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v0[i]))
-                                                       : __uint_as_float(v0[i]);
-                    const float a1 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v1[i]))
-                                                       : __uint_as_float(v1[i]);
-                    y[i] = __fmul_rn(a0, scale);
-                    y[32 + i] = __fmul_rn(a1, scale);
-                }
+                if (n0 >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
                 const int nparts = args.out_fp32 ? 2 : 1;  // 128-byte row blocks in this chunk
                 for (int part = 0; part < nparts; ++part) {
-                    const uint32_t buf = my_bufs + static_cast<uint32_t>(nbuf & 1) * kEpiBufBytes;
-                    // the store issued two blocks ago from this buffer has read it
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
+                    const int col = args.out_fp32 ? n0 + 32 * part : n0;
+                    if (col >= args.N) break;  // warp-uniform
                     uint32_t w[32];
                     if (args.out_fp32) {
+                        const uint32_t *v = part ? v1 : v0;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(y[32 * part + i]);
+                        for (int i = 0; i < 32; ++i) {
+                            const float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[i]))
+                                                              : __uint_as_float(v[i]);
+                            w[i] = __float_as_uint(__fmul_rn(a, scale));
+                        }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+                            const uint32_t *v = (i < 16) ? v0 : v1;
+                            const int k = 2 * (i & 15);
+                            const float a0 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[k]))
+                                                               : __uint_as_float(v[k]);
+                            const float a1 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[k + 1]))
+                                                               : __uint_as_float(v[k + 1]);
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(a0, scale), __fmul_rn(a1, scale));
                             w[i] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
                     }
+                    // the previous store from this buffer has finished reading it
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
                     // row `lane`: 8 chunks of 16 bytes, chunk c at position c ^ (lane % 8)
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -293,11 +319,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        const int col = args.out_fp32 ? n0 + 32 * part : n0;
-                        tma_store_2d(&tmY, buf, col, tm * kBM + quarter * 32);
+                        tma_store_2d(&tmY, buf, col, row0);
                         bulk_commit_group();
                     }
-                    ++nbuf;
                 }
                 if (args.acc_out && row_ok) {
                     // raw accumulators for parity checks (direct stores)

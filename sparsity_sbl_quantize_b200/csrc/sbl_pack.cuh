@@ -23,16 +23,6 @@ struct GammaWorkspace {
     uint32_t pad[3];
 };
 
-// Pairwise sum of 16 consecutive leaves held by one thread.
-__device__ __forceinline__ double tree16(double (&v)[16])
-{
-#pragma unroll
-    for (int w = 1; w < 16; w *= 2)
-#pragma unroll
-        for (int i = 0; i < 16; i += 2 * w) v[i] = v[i] + v[i + w];
-    return v[0];
-}
-
 // Given gamma, the fp32 threshold T such that for every finite fp32 x
 //   clamp(rint_half_even(fl32(|x| / gamma)), 0, 1) == 1  <=>  |x| >= T.
 // fl32(q) > 0.5 exactly when q > 0.5 + 2^-25 (the midpoint to the next float
@@ -68,21 +58,13 @@ struct PackArgs {
     PackOut out;
 };
 
-// Pairwise tree of the 16 leaves held in four float4 (|.| in fp64).
-__device__ __forceinline__ double tree16_f4(const float4 &a, const float4 &b, const float4 &c,
-                                            const float4 &d)
-{
-    double v[16] = {fabs((double)a.x), fabs((double)a.y), fabs((double)a.z), fabs((double)a.w),
-                    fabs((double)b.x), fabs((double)b.y), fabs((double)b.z), fabs((double)b.w),
-                    fabs((double)c.x), fabs((double)c.y), fabs((double)c.z), fabs((double)c.w),
-                    fabs((double)d.x), fabs((double)d.y), fabs((double)d.z), fabs((double)d.w)};
-    return tree16(v);
-}
-
-// gamma: one CTA per tree node of kGammaBlock weights (thread t owns the 32
-// consecutive weights [node*8192 + 32t, +32): register tree, warp butterfly,
-// CTA tree); the last CTA to finish combines the node partials over the same
-// tree and writes gamma.  ws->counter must be zero at launch.
+// gamma: one CTA per tree node of kGammaBlock weights.  Warp w owns the 1024
+// consecutive weights [node*8192 + 1024w, +1024) as eight 128-weight chunks;
+// for chunk q lane l loads the float4 at 128q + 4l (coalesced), sums its four
+// leaves, and a butterfly over the lanes completes the chunk's tree; the eight
+// chunk sums, the eight warp sums and finally (in the last CTA to finish) the
+// node partials are combined over the same pairwise tree.  ws->counter must
+// be zero at launch.
 __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W, int64_t count,
                                                     GammaWorkspace *ws, float *gamma_out)
 {
@@ -92,18 +74,25 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
     // the pack kernel may launch now: it only streams W before waiting for us
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kGammaBlock + threadIdx.x * 32;
+    const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kGammaBlock + warp * 1024;
     float4 f[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {  // count % 4 == 0: a float4 is all in or all out
-        const int64_t e = e0 + 4 * q;
+        const int64_t e = wbase + 128 * q + 4 * lane;
         f[q] = (e < count) ? __ldg(reinterpret_cast<const float4 *>(W + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    double t = tree16_f4(f[0], f[1], f[2], f[3]) + tree16_f4(f[4], f[5], f[6], f[7]);
-    // butterfly: after the step with offset `off`, lane 0 holds the tree over
-    // lanes [0, 2*off)
+    double c[8];
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
+    for (int q = 0; q < 8; ++q)
+        c[q] = (fabs(static_cast<double>(f[q].x)) + fabs(static_cast<double>(f[q].y))) +
+               (fabs(static_cast<double>(f[q].z)) + fabs(static_cast<double>(f[q].w)));
+    // butterfly: after the step with offset `off`, every lane holds the tree
+    // over its aligned group of 2*off lanes (a + b == b + a exactly)
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c[q] = c[q] + __shfl_xor_sync(0xffffffffu, c[q], off);
+    const double t = ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
     if (lane == 0) warp_sums[warp] = t;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -116,37 +105,40 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    // Second level: thread i combines partials [128 i, 128 i + 128) (a tree
-    // node; zeros past the end), then a shared-memory tree over 256 sums.
+    // Second level, over the same tree: chunks of 2048 partials (tree nodes);
+    // in each chunk thread t loads [8t, 8t + 8) (all threads, loads in flight
+    // together), a shared-memory tree combines the 256 thread sums, and the
+    // <= 16 chunk sums finish pairwise (zeros past the end).
     const int nparts = static_cast<int>(gridDim.x);
-    double ts = 0.0;
-    if (threadIdx.x * 128 < nparts) {
-        double acc16[16];
+    __shared__ double chunk_sums[kGammaMaxPartials / 2048];
+    const int nchunks = (nparts + 2047) / 2048;
+    for (int c = 0; c < nchunks; ++c) {
+        double v[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            double v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int j = threadIdx.x * 128 + c * 8 + i;
-                v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
-            }
-            acc16[c] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+        for (int i = 0; i < 8; ++i) {
+            const int j = c * 2048 + threadIdx.x * 8 + i;
+            v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
         }
-#pragma unroll
-        for (int w = 1; w < 16; w *= 2)
-#pragma unroll
-            for (int i = 0; i < 16; i += 2 * w) acc16[i] = acc16[i] + acc16[i + w];
-        ts = acc16[0];
-    }
-    thread_sums[threadIdx.x] = ts;
-    __syncthreads();
-    for (int stride = 1; stride < 256; stride *= 2) {
-        const int i = threadIdx.x * 2 * stride;
-        if (i < 256) thread_sums[i] = thread_sums[i] + thread_sums[i + stride];
+        thread_sums[threadIdx.x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+        __syncthreads();
+        for (int stride = 1; stride < 256; stride *= 2) {
+            const int i = threadIdx.x * 2 * stride;
+            if (i < 256) thread_sums[i] = thread_sums[i] + thread_sums[i + stride];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) chunk_sums[c] = thread_sums[0];
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        const double mean = __ddiv_rn(thread_sums[0], static_cast<double>(count));
+        constexpr int kChunks = kGammaMaxPartials / 2048;
+        double cs[kChunks];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) cs[c] = (c < nchunks) ? chunk_sums[c] : 0.0;
+#pragma unroll
+        for (int w = 1; w < kChunks; w *= 2)
+#pragma unroll
+            for (int i = 0; i < kChunks; i += 2 * w) cs[i] = cs[i] + cs[i + w];
+        const double mean = __ddiv_rn(cs[0], static_cast<double>(count));
         *gamma_out = __double2float_rn(mean);
     }
 }
@@ -257,36 +249,62 @@ __device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int3
     }
 }
 
-// Mask + ternarise + pack: each thread owns kBatch groups (16 weights) of
-// the flat group index space.  Launched with programmatic dependent launch
-// right behind gamma_kernel: W is loaded before waiting (gamma_kernel does not
-// write it), gamma after.
+// Mask + ternarise + pack.  A warp covers 512 consecutive weights: lane l
+// loads the float4s l, l+32, l+64, l+96 of that span (coalesced).  For M = 4
+// each float4 is a group; for M = 8 the two halves of a group sit in lanes
+// 2i and 2i+1, and one exchange gives lane 2i the groups of float4 pairs
+// (0, 1) and lane 2i+1 those of (2, 3).  Launched with programmatic dependent
+// launch right behind gamma_kernel: W is loaded before waiting (gamma_kernel
+// does not write it), gamma after.
 template <int M>
 __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
 {
-    constexpr int kBatch = 16 / M;  // 2 groups of 8 or 4 groups of 4
-    const int64_t total_groups = a.count / M;
-    const int64_t gbase = (static_cast<int64_t>(blockIdx.x) * 256) * kBatch + threadIdx.x;
+    constexpr int kBatch = 16 / M;  // groups per thread: 2 of 8 or 4 of 4
+    const int lane = threadIdx.x & 31;
+    const int64_t span = (static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * 512;  // weights
+    float4 f[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t e = span + 4 * (lane + 32 * j);
+        f[j] = (e < a.count) ? __ldg(reinterpret_cast<const float4 *>(a.W + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     uint32_t bits[kBatch][M];
+    int64_t gidx[kBatch];
+    if constexpr (M == 4) {
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-        const int64_t g = gbase + 256 * b;
-        if (g < total_groups) {
+        for (int j = 0; j < 4; ++j) {
+            bits[j][0] = __float_as_uint(f[j].x), bits[j][1] = __float_as_uint(f[j].y);
+            bits[j][2] = __float_as_uint(f[j].z), bits[j][3] = __float_as_uint(f[j].w);
+            gidx[j] = span / 4 + lane + 32 * j;
+        }
+    } else {
+        // even lane: keeps j = 0, 1 (its first halves), receives the partner's
+        // halves of j = 0, 1; odd lane: keeps j = 2, 3 (second halves)
+        const bool odd = lane & 1;
 #pragma unroll
-            for (int q = 0; q < M / 4; ++q) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(a.W + g * M) + q);
-                bits[b][4 * q + 0] = __float_as_uint(v.x);
-                bits[b][4 * q + 1] = __float_as_uint(v.y);
-                bits[b][4 * q + 2] = __float_as_uint(v.z);
-                bits[b][4 * q + 3] = __float_as_uint(v.w);
-            }
+        for (int b = 0; b < 2; ++b) {
+            const float4 mine = odd ? f[2 + b] : f[b];
+            const float4 give = odd ? f[b] : f[2 + b];
+            float4 got;
+            got.x = __shfl_xor_sync(0xffffffffu, give.x, 1);
+            got.y = __shfl_xor_sync(0xffffffffu, give.y, 1);
+            got.z = __shfl_xor_sync(0xffffffffu, give.z, 1);
+            got.w = __shfl_xor_sync(0xffffffffu, give.w, 1);
+            const float4 lo = odd ? got : mine, hi = odd ? mine : got;
+            bits[b][0] = __float_as_uint(lo.x), bits[b][1] = __float_as_uint(lo.y);
+            bits[b][2] = __float_as_uint(lo.z), bits[b][3] = __float_as_uint(lo.w);
+            bits[b][4] = __float_as_uint(hi.x), bits[b][5] = __float_as_uint(hi.y);
+            bits[b][6] = __float_as_uint(hi.z), bits[b][7] = __float_as_uint(hi.w);
+            // float4 index lane + 32 j, j = b (even lane) or 2 + b (odd lane); group = that / 2
+            gidx[b] = span / 8 + ((lane & ~1) + 32 * (odd ? 2 + b : b)) / 2;
         }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
+    const int64_t total_groups = a.count / M;
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-        const int64_t g = gbase + 256 * b;
+        const int64_t g = gidx[b];
         if (g < total_groups) {
             const uint64_t e = static_cast<uint64_t>(g) * M;
             const int32_t row = static_cast<int32_t>(__umul64hi(e, a.inv_cols));
