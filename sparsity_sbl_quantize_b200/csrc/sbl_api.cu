@@ -319,8 +319,8 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
     }
     if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM)) {
         // programmatic dependent launch behind gamma_kernel (see pack_kernel);
-        // a CTA covers 8 warps x 512 weights
-        const int64_t per_cta = 8 * 512 / desc->m;  // groups per CTA
+        // a thread covers 16 weights
+        const int64_t per_cta = 256 * 16 / desc->m;  // groups per CTA
         const int64_t groups = count / desc->m;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));

@@ -254,14 +254,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
             const int acc = local % kNumAcc;
             const uint32_t acc_phase = (local / kNumAcc) & 1;
-            const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
-            if (!__all_sync(0xffffffffu, ready)) break;  // warp-uniform decision
-            tc_fence_after();
             const int m = tm * kBM + r;
             const bool row_ok = m < args.M;
             const int row0 = tm * kBM + quarter * 32;  // first row of this warp's block
+            // the token scale is loaded while the MMAs of this tile still run
+            const float d_m = (args.row_scale && row_ok) ? args.row_scale[m] : 0.0f;
+            const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
+            if (!__all_sync(0xffffffffu, ready)) break;  // warp-uniform decision
+            tc_fence_after();
             float scale = g;
-            if (args.row_scale) scale = row_ok ? __fmul_rn(g, args.row_scale[m]) : 0.0f;
+            if (args.row_scale) scale = row_ok ? __fmul_rn(g, d_m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
 #pragma unroll 1

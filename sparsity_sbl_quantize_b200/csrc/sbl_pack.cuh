@@ -143,16 +143,46 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
     }
 }
 
-// Mask + ternarise one group of M weights given as fp32 bit patterns.
-// Returns W_eff as M bytes (int8, little-endian in w0/w1) and the keep mask.
+// Keep mask of the n largest |W| of a group (lower index wins ties; keys are
+// |W| bit patterns, ordered like the magnitudes).  Rank counting is the
+// general case; when at most two weights are dropped (or at most two kept) a
+// scan for the extreme element is cheaper and gives the same set:
+//  * the element dropped first is the minimum under (key ascending, index
+//    descending) -- a scan from the highest index with a strict `<`;
+//  * the element kept first is the maximum under (key descending, index
+//    ascending) -- a scan from index 0 with a strict `>`.
 template <int M>
-__device__ __forceinline__ void eval_group(const uint32_t (&bits)[M], uint32_t thr_bits, int n,
-                                           uint32_t &w0, uint32_t &w1, uint32_t &keep_bits)
+__device__ __forceinline__ uint32_t keep_mask(const uint32_t (&key)[M], int n)
 {
-    // |W| as ordered integers (sign bit cleared; -0 and +0 tie).
-    uint32_t key[M];
+    constexpr uint32_t kAll = (1u << M) - 1u;
+    const int drop = M - n;
+    if (drop <= 2 || n <= 2) {
+        const bool by_drop = drop <= 2;
+        const int picks = by_drop ? drop : n;
+        uint32_t chosen = 0;
+        uint32_t k[M];
 #pragma unroll
-    for (int i = 0; i < M; ++i) key[i] = bits[i] & 0x7fffffffu;
+        for (int i = 0; i < M; ++i)  // both forms stay below 2^31, under the sentinel
+            k[i] = by_drop ? key[i] : 0x7fffffffu - key[i];  // max of key = min of (2^31 - 1 - key)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            if (p >= picks) break;
+            // minimum of k with ties to the higher index (drop) or the lower
+            // index (keep: the complement reverses the key order, not the index order)
+            int best = by_drop ? M - 1 : 0;
+            uint32_t kb = k[best];
+#pragma unroll
+            for (int t = 1; t < M; ++t) {
+                const int i = by_drop ? M - 1 - t : t;
+                if (k[i] < kb) { kb = k[i]; best = i; }
+            }
+            chosen |= 1u << best;
+#pragma unroll
+            for (int i = 0; i < M; ++i)
+                if (i == best) k[i] = 0xffffffffu;  // above every k: never picked again
+        }
+        return by_drop ? (kAll & ~chosen) : chosen;
+    }
     // rank_i = #{ j : key_j > key_i  or  (key_j == key_i and j < i) }
     int rank[M];
 #pragma unroll
@@ -164,16 +194,29 @@ __device__ __forceinline__ void eval_group(const uint32_t (&bits)[M], uint32_t t
             if (key[j] > key[i]) ++rank[i];  // j beats i only if strictly larger
             else ++rank[j];
         }
-    keep_bits = 0;
+    uint32_t keep = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i) keep |= (rank[i] < n ? 1u : 0u) << i;
+    return keep;
+}
+
+// Mask + ternarise one group of M weights given as fp32 bit patterns.
+// Returns W_eff as M bytes (int8, little-endian in w0/w1) and the keep mask.
+template <int M>
+__device__ __forceinline__ void eval_group(const uint32_t (&bits)[M], uint32_t thr_bits, int n,
+                                           uint32_t &w0, uint32_t &w1, uint32_t &keep_bits)
+{
+    // |W| as ordered integers (sign bit cleared; -0 and +0 tie).
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = bits[i] & 0x7fffffffu;
+    keep_bits = keep_mask<M>(key, n);
     uint32_t b[M];
 #pragma unroll
     for (int i = 0; i < M; ++i) {
-        const bool keep = rank[i] < n;
-        const bool nz = key[i] >= thr_bits;  // |w| >= threshold (both non-negative)
-        // sign byte: 0xff for negative, 0x01 for positive
-        const uint32_t sb = (static_cast<uint32_t>(static_cast<int32_t>(bits[i]) >> 31) | 1u) & 0xffu;
-        b[i] = (keep && nz) ? sb : 0u;
-        keep_bits |= (keep ? 1u : 0u) << i;
+        // |w| >= threshold (both non-negative) and kept -> 0x01 or 0xff by sign
+        const bool on = (key[i] >= thr_bits) && ((keep_bits >> i) & 1u);
+        b[i] = on ? ((bits[i] >> 31) ? 0xffu : 0x01u) : 0u;
     }
     w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
     w1 = 0;
@@ -249,70 +292,38 @@ __device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int3
     }
 }
 
-// Mask + ternarise + pack.  A warp covers 512 consecutive weights: lane l
-// loads the float4s l, l+32, l+64, l+96 of that span (coalesced).  For M = 4
-// each float4 is a group; for M = 8 the two halves of a group sit in lanes
-// 2i and 2i+1, and one exchange gives lane 2i the groups of float4 pairs
-// (0, 1) and lane 2i+1 those of (2, 3).  Launched with programmatic dependent
-// launch right behind gamma_kernel: W is loaded before waiting (gamma_kernel
-// does not write it), gamma after.
+// Mask + ternarise + pack: thread t of CTA c owns the 16 consecutive weights
+// (two groups of 8 or four of 4) starting at (256 c + t) * 16.  Launched with
+// programmatic dependent launch right behind gamma_kernel: W is loaded before
+// waiting (gamma_kernel does not write it), gamma after.
 template <int M>
 __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
 {
-    constexpr int kBatch = 16 / M;  // groups per thread: 2 of 8 or 4 of 4
-    const int lane = threadIdx.x & 31;
-    const int64_t span = (static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * 512;  // weights
+    constexpr int kBatch = 16 / M;  // groups per thread
+    const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 16;
     float4 f[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int64_t e = span + 4 * (lane + 32 * j);
-        f[j] = (e < a.count) ? __ldg(reinterpret_cast<const float4 *>(a.W + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    uint32_t bits[kBatch][M];
-    int64_t gidx[kBatch];
-    if constexpr (M == 4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            bits[j][0] = __float_as_uint(f[j].x), bits[j][1] = __float_as_uint(f[j].y);
-            bits[j][2] = __float_as_uint(f[j].z), bits[j][3] = __float_as_uint(f[j].w);
-            gidx[j] = span / 4 + lane + 32 * j;
-        }
-    } else {
-        // even lane: keeps j = 0, 1 (its first halves), receives the partner's
-        // halves of j = 0, 1; odd lane: keeps j = 2, 3 (second halves)
-        const bool odd = lane & 1;
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const float4 mine = odd ? f[2 + b] : f[b];
-            const float4 give = odd ? f[b] : f[2 + b];
-            float4 got;
-            got.x = __shfl_xor_sync(0xffffffffu, give.x, 1);
-            got.y = __shfl_xor_sync(0xffffffffu, give.y, 1);
-            got.z = __shfl_xor_sync(0xffffffffu, give.z, 1);
-            got.w = __shfl_xor_sync(0xffffffffu, give.w, 1);
-            const float4 lo = odd ? got : mine, hi = odd ? mine : got;
-            bits[b][0] = __float_as_uint(lo.x), bits[b][1] = __float_as_uint(lo.y);
-            bits[b][2] = __float_as_uint(lo.z), bits[b][3] = __float_as_uint(lo.w);
-            bits[b][4] = __float_as_uint(hi.x), bits[b][5] = __float_as_uint(hi.y);
-            bits[b][6] = __float_as_uint(hi.z), bits[b][7] = __float_as_uint(hi.w);
-            // float4 index lane + 32 j, j = b (even lane) or 2 + b (odd lane); group = that / 2
-            gidx[b] = span / 8 + ((lane & ~1) + 32 * (odd ? 2 + b : b)) / 2;
-        }
-    }
+    for (int j = 0; j < 4; ++j)  // count % 16 == 0: the 16 weights are all in or all out
+        f[j] = (e0 < a.count) ? __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (e0 >= a.count) return;
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
-    const int64_t total_groups = a.count / M;
+    const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
+    const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);  // 16 | K: same row
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-        const int64_t g = gidx[b];
-        if (g < total_groups) {
-            const uint64_t e = static_cast<uint64_t>(g) * M;
-            const int32_t row = static_cast<int32_t>(__umul64hi(e, a.inv_cols));
-            const int32_t col = static_cast<int32_t>(e - static_cast<uint64_t>(row) * a.cols);
-            uint32_t w0, w1, keep_bits;
-            eval_group<M>(bits[b], thr_bits, a.n, w0, w1, keep_bits);
-            store_group<M>(a, row, col / M, w0, w1, keep_bits);
+        uint32_t bits[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const int e = b * M + i;
+            const float4 &v = f[e >> 2];
+            const float x = (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
+            bits[i] = __float_as_uint(x);
         }
+        uint32_t w0, w1, keep_bits;
+        eval_group<M>(bits, thr_bits, a.n, w0, w1, keep_bits);
+        store_group<M>(a, row, col0 / M + b, w0, w1, keep_bits);
     }
 }
 

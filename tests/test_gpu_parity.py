@@ -59,12 +59,15 @@ def test_pack_gamma_multi_block_tree():
     check_pack(wl.master_weights(1008, 1040, seed=21), 6, 8)
 
 
-def test_pack_ties_zero_and_signed_zero():
+@pytest.mark.parametrize("n,m", [(6, 8), (2, 4), (2, 8), (1, 4), (3, 4), (7, 8), (5, 8), (3, 8), (1, 8), (4, 8)])
+def test_pack_ties_zero_and_signed_zero(n, m):
+    """Tie-heavy weights (few distinct magnitudes), all-zero and all -0.0 rows:
+    the kept set must follow the lower-index rule in every selection path."""
     w = (np.random.default_rng(3).integers(-2, 3, size=(64, 128)) * 0.125).astype(np.float32)
     w[5] = 0.0
     w[6] = -0.0
-    check_pack(w, 6, 8)
-    check_pack(w, 2, 4)
+    w[7, ::2] = -0.0
+    check_pack(w, n, m)
 
 
 def test_pack_all_zero_matrix_gamma_zero():
