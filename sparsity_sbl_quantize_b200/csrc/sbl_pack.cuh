@@ -69,7 +69,6 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
                                                     GammaWorkspace *ws, float *gamma_out)
 {
     __shared__ double warp_sums[8];
-    __shared__ double thread_sums[256];
     __shared__ int is_last;
     // the pack kernel may launch now: it only streams W before waiting for us
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -119,14 +118,14 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
             const int j = c * 2048 + threadIdx.x * 8 + i;
             v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
         }
-        thread_sums[threadIdx.x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+        double u = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) u = u + __shfl_xor_sync(0xffffffffu, u, off);
+        if (lane == 0) warp_sums[warp] = u;
         __syncthreads();
-        for (int stride = 1; stride < 256; stride *= 2) {
-            const int i = threadIdx.x * 2 * stride;
-            if (i < 256) thread_sums[i] = thread_sums[i] + thread_sums[i + stride];
-            __syncthreads();
-        }
-        if (threadIdx.x == 0) chunk_sums[c] = thread_sums[0];
+        if (threadIdx.x == 0)
+            chunk_sums[c] = ((warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3])) +
+                            ((warp_sums[4] + warp_sums[5]) + (warp_sums[6] + warp_sums[7]));
         __syncthreads();
     }
     if (threadIdx.x == 0) {
@@ -202,20 +201,17 @@ __device__ __forceinline__ uint32_t keep_mask(const uint32_t (&key)[M], int n)
 
 // Mask + ternarise one group of M weights given as fp32 bit patterns.
 // Returns W_eff as M bytes (int8, little-endian in w0/w1) and the keep mask.
+// Ternarise one group of M weights (fp32 bit patterns) under its keep mask.
+// Returns W_eff as M bytes (int8, little-endian in w0/w1).
 template <int M>
-__device__ __forceinline__ void eval_group(const uint32_t (&bits)[M], uint32_t thr_bits, int n,
-                                           uint32_t &w0, uint32_t &w1, uint32_t &keep_bits)
+__device__ __forceinline__ void ternarise_group(const uint32_t (&bits)[M], uint32_t keep_bits,
+                                                uint32_t thr_bits, uint32_t &w0, uint32_t &w1)
 {
-    // |W| as ordered integers (sign bit cleared; -0 and +0 tie).
-    uint32_t key[M];
-#pragma unroll
-    for (int i = 0; i < M; ++i) key[i] = bits[i] & 0x7fffffffu;
-    keep_bits = keep_mask<M>(key, n);
     uint32_t b[M];
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         // |w| >= threshold (both non-negative) and kept -> 0x01 or 0xff by sign
-        const bool on = (key[i] >= thr_bits) && ((keep_bits >> i) & 1u);
+        const bool on = ((bits[i] & 0x7fffffffu) >= thr_bits) && ((keep_bits >> i) & 1u);
         b[i] = on ? ((bits[i] >> 31) ? 0xffu : 0x01u) : 0u;
     }
     w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
@@ -294,36 +290,45 @@ __device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int3
 
 // Mask + ternarise + pack: thread t of CTA c owns the 16 consecutive weights
 // (two groups of 8 or four of 4) starting at (256 c + t) * 16.  Launched with
-// programmatic dependent launch right behind gamma_kernel: W is loaded before
-// waiting (gamma_kernel does not write it), gamma after.
+// programmatic dependent launch right behind gamma_kernel: W is loaded and the
+// N:M keep masks (which need only |W|) are computed before waiting for
+// gamma_kernel (which does not write W); gamma is read after.
 template <int M>
 __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
 {
     constexpr int kBatch = 16 / M;  // groups per thread
     const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 16;
-    float4 f[4];
+    const bool active = e0 < a.count;  // count % 16 == 0: the 16 weights are all in or all out
+    uint32_t bits[kBatch][M];
+    uint32_t keep[kBatch];
+    if (active) {
+        float4 f[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)  // count % 16 == 0: the 16 weights are all in or all out
-        f[j] = (e0 < a.count) ? __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 4; ++j) f[j] = __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j);
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            uint32_t key[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                const int e = b * M + i;
+                const float4 &v = f[e >> 2];
+                const float x = (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
+                bits[b][i] = __float_as_uint(x);
+                key[i] = bits[b][i] & 0x7fffffffu;  // |W| ordered as integers; -0 ties +0
+            }
+            keep[b] = keep_mask<M>(key, a.n);
+        }
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (e0 >= a.count) return;
+    if (!active) return;
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
     const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
     const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);  // 16 | K: same row
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-        uint32_t bits[M];
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-            const int e = b * M + i;
-            const float4 &v = f[e >> 2];
-            const float x = (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
-            bits[i] = __float_as_uint(x);
-        }
-        uint32_t w0, w1, keep_bits;
-        eval_group<M>(bits, thr_bits, a.n, w0, w1, keep_bits);
-        store_group<M>(a, row, col0 / M + b, w0, w1, keep_bits);
+        uint32_t w0, w1;
+        ternarise_group<M>(bits[b], keep[b], thr_bits, w0, w1);
+        store_group<M>(a, row, col0 / M + b, w0, w1, keep[b]);
     }
 }
 
