@@ -138,11 +138,13 @@ class Runner:
             key = (lin.d_in, "shared" if lin.d_in == wk.linears[0].d_in else li)
             if key not in inputs:
                 x = wl.activations(T, lin.d_in, seed=wk.seed, layer=li, outlier_frac=wk.outlier_frac)
+                # one int8 copy per N:M pattern, so the patterns' passes can overlap
                 inputs[key] = {"x_host": x, "x": torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device),
-                               "q": torch.empty((T, lin.d_in), dtype=torch.int8, device=device),
-                               "d": torch.empty((T,), dtype=torch.float32, device=device)}
+                               "q": {p: torch.empty((T, lin.d_in), dtype=torch.int8, device=device) for p in wk.patterns},
+                               "d": {p: torch.empty((T,), dtype=torch.float32, device=device) for p in wk.patterns}}
             self.layers.append({"lin": lin, "w_host": w, "w": torch.from_numpy(w).to(device), "inp": inputs[key],
-                                "y": torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=device)})
+                                "y": {p: torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=device)
+                                      for p in wk.patterns}})
         self.inputs = list(inputs.values())
         fmts = sbl.SBL_FMT_I8 | (sbl.SBL_FMT_BF16T if wk.mode == "train" else 0)
         self.fmts = fmts
@@ -153,7 +155,9 @@ class Runner:
                 dsc = sbl.desc(lin.d_out, lin.d_in, n, m)
                 L["packed"][(n, m)] = (dsc, sbl.alloc_packed(dsc, fmts))
             dsc0 = L["packed"][wk.patterns[0]][0]
-            L["ws"] = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc0, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+            # one gamma workspace per pattern: the patterns' passes run concurrently
+            L["ws"] = {p: sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc0, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+                       for p in wk.patterns}
             if wk.mode == "train":
                 L["dy"] = torch.from_numpy(wl.output_grad(T, lin.d_out, seed=wk.seed, layer=li).view(np.int16)
                                            ).view(torch.bfloat16).to(device)
@@ -161,38 +165,61 @@ class Runner:
                 L["dw"] = torch.empty((lin.d_out, lin.d_in), dtype=torch.float32, device=device)
                 L["bws"] = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc0, T, sbl.SBL_OP_BACKWARD))
         self.launches_per_step = 0
+        n_side = max(len(self.layers), 1)
+        self.streams = [[torch.cuda.Stream(device) for _ in range(1 + n_side)] for _ in wk.patterns]
 
     def step(self, timed=False):
-        """Enqueue one step.  With timed=True, external CUDA events bracket
-        every GEMM launch (they become event-record nodes under capture)."""
+        """Enqueue one step.  Untimed: the N:M patterns' passes are
+        independent and go to their own streams; inside a pass the linears'
+        packing and the inputs' quantisation fork onto side streams and join
+        before the GEMMs.  Timed: everything on the current stream, in order,
+        with external CUDA events bracketing every GEMM launch (event-record
+        nodes under capture), so each GEMM's interval is its own."""
         sbl, torch = self.sbl, self.torch
+        main = torch.cuda.current_stream()
         launches = 0
         self.kernel_events = []
-        for (n, m) in self.wk.patterns:
-            for L in self.layers:
-                dsc, p = L["packed"][(n, m)]
-                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"])
+        for pi, (n, m) in enumerate(self.wk.patterns):
+            streams = [main] * len(self.streams[pi]) if timed else self.streams[pi]
+            for st in streams:
+                if st is not main:
+                    st.wait_stream(main)
+            side = streams[1:]
+            for li, L in enumerate(self.layers):
+                with torch.cuda.stream(side[li % len(side)]):
+                    dsc, p = L["packed"][(n, m)]
+                    sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"][(n, m)])
                 launches += 2 + (1 if self.fmts & sbl.SBL_FMT_BF16T else 0)
-            for inp in self.inputs:
-                sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"], inp["d"])
+            for ii, inp in enumerate(self.inputs):
+                with torch.cuda.stream(side[(len(self.layers) + ii) % len(side)]):
+                    sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"][(n, m)], inp["d"][(n, m)])
                 launches += 1
-            for L in self.layers:
-                dsc, p = L["packed"][(n, m)]
-                inp = L["inp"]
-                if timed:
-                    e0 = torch.cuda.Event(enable_timing=True, external=True)
-                    e1 = torch.cuda.Event(enable_timing=True, external=True)
-                    e0.record()
-                sbl.sbl_forward(dsc, inp["q"], inp["d"], self.T, p, sbl.SBL_FMT_I8, L["y"])
-                launches += 1
-                if timed:
-                    e1.record()
-                    lin = L["lin"]
-                    self.kernel_events.append((e0, e1, 2.0 * self.T * lin.d_out * lin.d_in * n / m))
-                if self.wk.mode == "train":
-                    sbl.sbl_backward_dual_ste(dsc, L["dy"], inp["q"], inp["d"], self.T, p, L["dx"], False,
-                                              L["dw"], L["bws"])
-                    launches += 4
+            g_stream = streams[0]
+            for st in side:
+                if st is not g_stream:
+                    g_stream.wait_stream(st)
+            with torch.cuda.stream(g_stream):
+                for L in self.layers:
+                    dsc, p = L["packed"][(n, m)]
+                    inp = L["inp"]
+                    q, d = inp["q"][(n, m)], inp["d"][(n, m)]
+                    if timed:
+                        e0 = torch.cuda.Event(enable_timing=True, external=True)
+                        e1 = torch.cuda.Event(enable_timing=True, external=True)
+                        e0.record()
+                    sbl.sbl_forward(dsc, q, d, self.T, p, sbl.SBL_FMT_I8, L["y"][(n, m)])
+                    launches += 1
+                    if timed:
+                        e1.record()
+                        lin = L["lin"]
+                        self.kernel_events.append((e0, e1, 2.0 * self.T * lin.d_out * lin.d_in * n / m))
+                    if self.wk.mode == "train":
+                        sbl.sbl_backward_dual_ste(dsc, L["dy"], q, d, self.T, p, L["dx"], False,
+                                                  L["dw"], L["bws"])
+                        launches += 4
+        if not timed:
+            for streams in self.streams:
+                main.wait_stream(streams[0])
         self.launches_per_step = launches
 
     def capture(self, timed: bool):
@@ -216,11 +243,15 @@ class Runner:
         self.h_w = [torch.from_numpy(L["w_host"]).pin_memory() for L in self.layers]
         self.h_x = [torch.from_numpy(inp["x_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
                     for inp in self.inputs]
-        self.h_y = [torch.empty(L["y"].shape, dtype=torch.bfloat16).pin_memory() for L in self.layers]
+        self.h_y = [torch.empty(L["y"][self.wk.patterns[0]].shape, dtype=torch.bfloat16).pin_memory()
+                    for L in self.layers]
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_w + self.h_x) * len(self.wk.patterns)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_y) * len(self.wk.patterns)
 
     def step_e2e(self):
+        """The same step through the public API from host memory: every pass
+        copies its weights and activations in and its outputs back, one
+        stream, in order (what a caller without device-resident data does)."""
         sbl = self.sbl
         for (n, m) in self.wk.patterns:
             for L, hw in zip(self.layers, self.h_w):
@@ -229,13 +260,15 @@ class Runner:
                 inp["x"].copy_(hx, non_blocking=True)
             for L in self.layers:
                 dsc, p = L["packed"][(n, m)]
-                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"])
+                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"][(n, m)])
             for inp in self.inputs:
-                sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"], inp["d"])
+                sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"][(n, m)], inp["d"][(n, m)])
             for L, hy in zip(self.layers, self.h_y):
                 dsc, p = L["packed"][(n, m)]
-                sbl.sbl_forward(dsc, L["inp"]["q"], L["inp"]["d"], self.T, p, sbl.SBL_FMT_I8, L["y"])
-                hy.copy_(L["y"], non_blocking=True)
+                inp = L["inp"]
+                sbl.sbl_forward(dsc, inp["q"][(n, m)], inp["d"][(n, m)], self.T, p, sbl.SBL_FMT_I8,
+                                L["y"][(n, m)])
+                hy.copy_(L["y"][(n, m)], non_blocking=True)
         self.torch.cuda.current_stream().synchronize()
 
 
@@ -264,7 +297,7 @@ def run_ours(args, wk):
     torch.cuda.synchronize()
     assert sbl.sbl_device_error() == 0
     g = r.capture(timed=False)
-    g_k = r.capture(timed=True)  # same step with event nodes around each GEMM
+    g_k = r.capture(timed=True)  # same step on one stream, event nodes around each GEMM
     # clock soak: replay untimed for ~1 s so clocks reach their loaded state
     t_end = time.perf_counter() + 1.0
     while time.perf_counter() < t_end:
@@ -293,8 +326,8 @@ def run_ours(args, wk):
         s1.record()
         s1.synchronize()
         times.append(s0.elapsed_time(s1))
-    # timed region 2: the same steps with every GEMM launch bracketed by
-    # events (the roofline of the dominant kernel)
+    # timed region 2: the same steps serialised on one stream with every
+    # GEMM launch bracketed by events (the roofline of the dominant kernel)
     gemm_ms, gemm_ops = 0.0, 0.0
     for _ in range(max(1, args.steps // 4)):
         flush.zero_()
@@ -316,9 +349,19 @@ def run_ours(args, wk):
     achieved = gemm_ops / (gemm_ms * 1e-3) / 1e12
     int8_peak = pk["bf16_tflops"] * 2.0  # int8 dense = 2 x bf16 dense (4.5 / 2.25 PFLOP/s nominal)
 
+    # self-check: the graph (streams forked per pass) and the single-stream
+    # public-API path must give bit-identical outputs (every kernel is
+    # deterministic), so a scheduling race cannot go unnoticed
+    g.replay()
+    torch.cuda.synchronize()
+    graph_out = {(li, pat): L["y"][pat].clone() for li, L in enumerate(r.layers) for pat in wk.patterns}
     # end to end: host buffers, copies inside the timed region
     r.setup_e2e()
     r.step_e2e()
+    selfcheck = all(torch.equal(graph_out[(li, pat)], L["y"][pat])
+                    for li, L in enumerate(r.layers) for pat in wk.patterns)
+    if not selfcheck:
+        raise SystemExit("bench self-check failed: graph and single-stream outputs differ")
     if world > 1:
         dist.barrier()
     e_steps = max(2, min(args.steps, 5))
@@ -344,7 +387,9 @@ def run_ours(args, wk):
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (fp32 dequant, bf16 out)",
         "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32, X~N(0,1) bf16)",
-        "config": {"workload": wk.name, "tokens": r.T, "launch": "one CUDA graph per step",
+        "config": {"workload": wk.name, "tokens": r.T,
+                   "launch": "one CUDA graph per step; each N:M pass on its own stream, packing and "
+                             "activation quantisation of independent linears forked onto side streams",
                    "linears": [f"{l.name}:{l.d_in}->{l.d_out}" for l in wk.linears],
                    "patterns": [f"{n}:{m}" for n, m in wk.patterns], "mode": wk.mode,
                    "l2": "flushed between timed steps (512 MiB write outside the events)",
@@ -358,9 +403,10 @@ def run_ours(args, wk):
         "e2e": {"value": round(e_value, 3), "unit": "TOPS", "h2d_bytes_per_step": r.h2d,
                 "d2h_bytes_per_step": r.d2h},
         "gpu_launches": r.launches_per_step * args.steps,
-        "roofline_timing": "separate timed pass of the same graph with event nodes around each GEMM",
+        "roofline_timing": "separate timed pass: the same step serialised on one stream, event nodes around each GEMM",
         "clocks": clk,
         "device_error": err,
+        "selfcheck": "graph outputs bit-identical to the single-stream API path",
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
