@@ -266,6 +266,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (args.row_scale) scale = row_ok ? __fmul_rn(g, d_m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
+            if (!args.out_fp32) {
+                // bf16: drain this warp's share of the accumulator, converting
+                // each 64-column chunk to 32 packed words, hand TMEM back, and
+                // only then store -- the MMAs of the tile after next need not
+                // wait for the stores.
+                uint32_t packed[kChunks][32];
+#pragma unroll
+                for (int jj = 0; jj < kChunks; ++jj) {
+                    const int j = half * kChunks + jj;
+                    uint32_t v0[32], v1[32];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerChunk * j), v0);
+                    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(kColsPerChunk * j + 32), v1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t *v = (i < 16) ? v0 : v1;
+                        const int k = 2 * (i & 15);
+                        const float a0 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[k]))
+                                                           : __uint_as_float(v[k]);
+                        const float a1 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[k + 1]))
+                                                           : __uint_as_float(v[k + 1]);
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(a0, scale), __fmul_rn(a1, scale));
+                        packed[jj][i] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                    if (args.acc_out && row_ok) {
+                        // raw accumulators for parity checks (direct stores)
+                        const int n0 = tn * BN + kColsPerChunk * j;
+                        for (int h = 0; h < 4; ++h) {
+                            const int n = n0 + 16 * h;
+                            if (n >= args.N) break;
+                            uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + static_cast<int64_t>(m) * args.ldo + n);
+                            const uint32_t *src = (h < 2) ? v0 + 16 * h : v1 + 16 * (h - 2);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                dst[q] = make_uint4(src[4 * q], src[4 * q + 1], src[4 * q + 2], src[4 * q + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tempty_bar(acc));
+#pragma unroll
+                for (int jj = 0; jj < kChunks; ++jj) {
+                    const int j = half * kChunks + jj;
+                    const int col = tn * BN + kColsPerChunk * j;
+                    if (col >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
+                    // the previous store from this buffer has finished reading it
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
+                    // row `lane`: 8 chunks of 16 bytes, chunk c at position c ^ (lane % 8)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t addr = buf + static_cast<uint32_t>(lane * 128 + ((c ^ (lane & 7)) * 16));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[jj][4 * c]),
+                                     "r"(packed[jj][4 * c + 1]), "r"(packed[jj][4 * c + 2]), "r"(packed[jj][4 * c + 3])
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, buf, col, row0);
+                        bulk_commit_group();
+                    }
+                }
+                continue;
+            }
+            // fp32: chunk by chunk (the two 128-byte blocks of a chunk need all
+            // of its 64 registers), TMEM handed back after the last load
 #pragma unroll 1
             for (int jj = 0; jj < kChunks; ++jj) {
                 const int j = half * kChunks + jj;
