@@ -178,10 +178,14 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K,
  * (y_is_fp32 = 0) or fp32.  acc_out: optional [T, O] int32 copy of the
  * accumulators (NULL to skip).  One launch.
  * The SBL_FMT_PK2 kernel is launched with programmatic dependent launch: it
- * starts copying w->pk2 before it waits for the previous kernel on the
+ * starts loading w->pk2 before it waits for the previous kernel on the
  * stream, so w->pk2 must not be written by a preceding kernel that triggers
  * its dependents early (sbl_quantize_mask_pack never does).  Xq, d, gamma
- * and Y are only touched after that wait. */
+ * and Y are only touched after that wait.  It also lets the next kernel on
+ * the stream launch as soon as it starts: a kernel launched after it with
+ * programmatic stream serialization must wait for its grid dependencies
+ * (griddepcontrol.wait) before it reads Y or acc_out; kernels launched
+ * without that attribute see the usual stream order. */
 sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d,
                        int32_t T, const sbl_packed *w, sbl_format fmt,
                        void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);

@@ -68,11 +68,7 @@ static sbl_status current_device(DeviceInfo **out)
             cudaFuncSetAttribute(gemm_kernel<kKindF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 200 * 1024) != cudaSuccess ||
-            cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 200 * 1024) != cudaSuccess)
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess)
             return SBL_ERR_CUDA;
         if (!g_encode) {
             void *fn = nullptr;
@@ -206,6 +202,31 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
 }  // namespace sbl
 
 using namespace sbl;
+
+namespace {
+
+// Row groups (16 rows, 8 warps each) per decode CTA, for T <= 8 and T > 8.
+// One group measured fastest for both: two groups halve the activation
+// re-reads from L2 but lose more to fewer, larger CTAs.
+constexpr int kDecGroupsSmallT = 1;
+constexpr int kDecGroupsLargeT = 1;
+
+// cpw: chunks per warp per round, 1, 2, 4 or 8 (at most 4 with two row
+// groups, whose 512 threads get at most 128 registers each).
+template <int NT, int RG>
+cudaError_t launch_decode_nt(const cudaLaunchConfig_t &cfg, const DecodeArgs &a, int cpw)
+{
+    switch (cpw) {
+    case 1: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 1, RG>, a);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 2, RG>, a);
+    case 4: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, RG>, a);
+    default:
+        if constexpr (RG == 1) return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 8, RG>, a);
+        else return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, RG>, a);
+    }
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -436,48 +457,27 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         a.T = T;
         a.K = K;
         a.O = O;
-        a.units = K / kDecKUnit;
-        a.err = di->err;
-        const int row_blocks = (O + kDecRows - 1) / kDecRows;
-        // K split over a cluster of cl CTAs: enough CTAs to cover the SMs,
-        // and a slice small enough for shared memory
-        auto stride_of = [](int bytes) { return ((bytes / 16) & 1) == 0 ? bytes + 16 : bytes; };
-        auto smem_of = [&](int c) {
-            const int slice = ((a.units + c - 1) / c) * kDecKUnit;
-            return static_cast<size_t>(kDecRows) * stride_of(slice / 4) +
-                   static_cast<size_t>(kDecMaxTokens) * stride_of(slice) +
-                   static_cast<size_t>(kDecRows) * kDecMaxTokens * 4 + kDecMaxTokens * 4;
-        };
-        int cl = 1;
-        while (cl < 8 && a.units / (2 * cl) >= 1 &&
-               (row_blocks * cl < di->num_sms || smem_of(cl) > 96 * 1024 ||
-                ((a.units + cl - 1) / cl) * kDecKUnit > 1024))
-            cl *= 2;
-        a.cluster = cl;
-        a.max_slice = ((a.units + cl - 1) / cl) * kDecKUnit;
-        a.w_stride = stride_of(a.max_slice / 4);  // odd multiple of 16: conflict-free rows
-        a.a_stride = stride_of(a.max_slice);
-        const size_t smem = smem_of(cl);
-        if (smem > 200 * 1024 || a.max_slice > 1024) return SBL_ERR_UNSUPPORTED;
+        a.chunks = (K + kDecChunk - 1) / kDecChunk;
+        // chunks per warp per round: the whole row in one round up to
+        // K = 16384 (more rounds above)
+        const int need = (a.chunks + 7) / 8;
+        const int cpw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
+        const int rg = T <= 8 ? kDecGroupsSmallT : kDecGroupsLargeT;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(static_cast<unsigned>(row_blocks * cl));
-        cfg.blockDim = dim3(kDecThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.gridDim = dim3(static_cast<unsigned>((O + kDecRows * rg - 1) / (kDecRows * rg)));
+        cfg.blockDim = dim3(static_cast<unsigned>(256 * rg));
+        cfg.dynamicSmemBytes = 0;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        // programmatic dependent launch: the kernel streams its (read-only)
+        // programmatic dependent launch: the kernel loads its (read-only)
         // packed weights before waiting on the previous kernel's outputs
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 2;
-        cudaError_t e = (T <= 8) ? cudaLaunchKernelEx(&cfg, decode_kernel<1>, a)
-                                 : cudaLaunchKernelEx(&cfg, decode_kernel<2>, a);
+        cfg.numAttrs = 1;
+        const cudaError_t e = T <= 8 ? (rg == 1 ? launch_decode_nt<1, 1>(cfg, a, cpw) : launch_decode_nt<1, 2>(cfg, a, cpw))
+                                     : (rg == 1 ? launch_decode_nt<2, 1>(cfg, a, cpw) : launch_decode_nt<2, 2>(cfg, a, cpw));
         return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
     }
     return SBL_ERR_UNSUPPORTED;

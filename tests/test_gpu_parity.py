@@ -137,9 +137,17 @@ def test_forward_single_layer_workload_outliers():
 
 
 @pytest.mark.parametrize("O,K,T", [(256, 256, 1), (384, 640, 4), (528, 1088, 16), (6912, 2560, 16),
-                                   (2560, 6912, 1), (2560, 6912, 9), (16, 64, 3)])
+                                   (2560, 6912, 1), (2560, 6912, 9), (16, 64, 3),
+                                   (48, 11008, 7),    # 43 K chunks: eight per warp
+                                   (32, 16448, 16),   # two rounds of chunks, 64-weight last chunk
+                                   (16, 192, 8),      # one partial chunk
+                                   (48, 2560, 12)])   # a CTA of two 16-row groups, one past O
 def test_forward_decode_pk2_bit_exact(O, K, T):
     run_forward_full_check(O, K, T, 2, 4, seed=O + K + T, fmt_name="PK2")
+
+
+def test_forward_decode_pk2_six_of_eight():
+    run_forward_full_check(896, 4864, 5, 6, 8, seed=11, fmt_name="PK2")
 
 
 def test_forward_zero_tokens_is_noop():
