@@ -42,6 +42,12 @@ def _load():
         lib.sbl_oracle_nm_bitmap_row_bytes.restype = i64
         lib.sbl_oracle_nm_bitmap_row_bytes.argtypes = [i64]
         lib.sbl_oracle_pack_nm.argtypes = [p, p, i64, i64, i32, i32, p, p]
+        lib.sbl_oracle_sp24_value_row_bytes.restype = i64
+        lib.sbl_oracle_sp24_value_row_bytes.argtypes = [i64]
+        lib.sbl_oracle_sp24_meta_row_bytes.restype = i64
+        lib.sbl_oracle_sp24_meta_row_bytes.argtypes = [i64]
+        lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
+        lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
         lib.sbl_oracle_quantize_act.argtypes = [p, i64, i64, p, p]
         lib.sbl_oracle_gemm_acc.restype = i32
         lib.sbl_oracle_gemm_acc.argtypes = [p, p, i64, i64, i64, p]
@@ -163,6 +169,27 @@ def pack_nm(weff, mask, n: int, m: int):
     bm = np.empty((d_out, nm_bitmap_row_bytes(d_in)), dtype=np.uint8)
     _load().sbl_oracle_pack_nm(_ptr(weff), _ptr(mask), d_out, d_in, n, m, _ptr(vals), _ptr(bm))
     return vals, bm
+
+
+def sp24_value_row_bytes(d_in: int) -> int:
+    return int(_load().sbl_oracle_sp24_value_row_bytes(d_in))
+
+
+def sp24_meta_row_bytes(d_in: int) -> int:
+    return int(_load().sbl_oracle_sp24_meta_row_bytes(d_in))
+
+
+def pack_sp24(weff, mask):
+    """2:4-compressed values int8 [O, value_row_bytes] and metadata uint8
+    [O, meta_row_bytes]; raises ValueError when the mask is not 2:4."""
+    weff = _i8(weff)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    d_out, d_in = weff.shape
+    vals = np.empty((d_out, sp24_value_row_bytes(d_in)), dtype=np.int8)
+    meta = np.empty((d_out, sp24_meta_row_bytes(d_in)), dtype=np.uint8)
+    if _load().sbl_oracle_pack_sp24(_ptr(weff), _ptr(mask), d_out, d_in, _ptr(vals), _ptr(meta)) != 0:
+        raise ValueError("mask keeps more than two positions in a group of four")
+    return vals, meta
 
 
 def quantize_act(x_bf16_bits):

@@ -182,6 +182,57 @@ void sbl_oracle_pack_nm(const int8_t *weff, const uint8_t *mask, int64_t d_out,
     }
 }
 
+int64_t sbl_oracle_sp24_value_row_bytes(int64_t d_in) { return round_up(d_in / 2, 16); }
+
+int64_t sbl_oracle_sp24_meta_row_bytes(int64_t d_in) { return round_up(d_in / 8, 16); }
+
+/* SP24: W_eff as the 2:4-compressed operand of the sparse tensor-core MMA
+ * (two stored values per group of four positions plus their 2-bit indices).
+ * For group g of a row (positions 4g .. 4g+3) the two positions i0 < i1 are
+ * the group's kept positions, completed, when fewer than two are kept, with
+ * the smallest positions of the group that are not kept.  Values: int8
+ * W_eff at 4g+i0 and 4g+i1 in bytes 2g and 2g+1 of the value row.
+ * Metadata: the nibble i0 | (i1 << 2) at bits 4*(g%2) of byte g/2 of the
+ * metadata row.  Padding bytes are 0.  Returns -1 (writing nothing further)
+ * when a group keeps more than two positions: such a mask is not 2:4. */
+int sbl_oracle_pack_sp24(const int8_t *weff, const uint8_t *mask, int64_t d_out, int64_t d_in,
+                         int8_t *vals, uint8_t *meta)
+{
+    int64_t vb = sbl_oracle_sp24_value_row_bytes(d_in);
+    int64_t mb = sbl_oracle_sp24_meta_row_bytes(d_in);
+    for (int64_t o = 0; o < d_out; ++o) {
+        int8_t *vrow = vals + o * vb;
+        uint8_t *mrow = meta + o * mb;
+        for (int64_t b = 0; b < vb; ++b) vrow[b] = 0;
+        for (int64_t b = 0; b < mb; ++b) mrow[b] = 0;
+        for (int64_t g = 0; g < d_in / 4; ++g) {
+            int idx[2];
+            int count = 0;
+            for (int i = 0; i < 4; ++i) {
+                if (!mask[o * d_in + 4 * g + i]) continue;
+                if (count == 2) return -1;
+                idx[count++] = i;
+            }
+            /* complete with the smallest positions not kept */
+            for (int i = 0; i < 4 && count < 2; ++i) {
+                if (mask[o * d_in + 4 * g + i]) continue;
+                if (count == 1 && idx[0] == i) continue;
+                idx[count++] = i;
+            }
+            if (idx[0] > idx[1]) {
+                int t = idx[0];
+                idx[0] = idx[1];
+                idx[1] = t;
+            }
+            vrow[2 * g] = weff[o * d_in + 4 * g + idx[0]];
+            vrow[2 * g + 1] = weff[o * d_in + 4 * g + idx[1]];
+            unsigned nib = (unsigned)idx[0] | ((unsigned)idx[1] << 2);
+            mrow[g / 2] = (uint8_t)(mrow[g / 2] | (nib << (4 * (g % 2))));
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------- activation quantiser -- */
 
 static float bf16_to_f32(uint16_t b)

@@ -27,6 +27,11 @@ MUTANTS = {
     "mask_not_applied": ("weff[i] = (int8_t)(mask[i] ? wq[i] : 0);", "weff[i] = wq[i];"),
     "sign_extension_codes": ("return (uint8_t)(v + 1);", "return (uint8_t)(v & 3);"),
     "keep_rank_off_by_one": ("(rank < n ? 1 : 0)", "(rank < n - 1 ? 1 : 0)"),
+    "sp24_nibble_fields_swapped": ("unsigned nib = (unsigned)idx[0] | ((unsigned)idx[1] << 2);",
+                                   "unsigned nib = (unsigned)idx[1] | ((unsigned)idx[0] << 2);"),
+    "sp24_high_nibble_first": ("(nib << (4 * (g % 2)))", "(nib << (4 * (1 - g % 2)))"),
+    "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
+                           "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
 }
 
 PIN_CALLS = [
@@ -43,6 +48,9 @@ PIN_CALLS = [
     (pins.test_output_matches_fp64_definition, ()),
     (pins.test_backward_matches_numpy_fp64, ()),
     (pins.test_nm_roundtrip, ()),
+    (pins.test_sp24_hand_example, ()),
+    (pins.test_sp24_roundtrip, (2, 4)),
+    (pins.test_sp24_roundtrip, (1, 4)),
 ]
 
 

@@ -253,6 +253,62 @@ def test_nm_roundtrip():
             np.testing.assert_array_equal(dec, layer.weff[r])
 
 
+def _decode_sp24(vals, meta, d_in):
+    """Independent decompression of the SP24 operand: group g's nibble gives
+    the two positions of values 2g and 2g+1."""
+    out = np.zeros((vals.shape[0], d_in), dtype=np.int8)
+    for r in range(vals.shape[0]):
+        for g in range(d_in // 4):
+            nib = (int(meta[r, g // 2]) >> (4 * (g % 2))) & 0xF
+            i0, i1 = nib & 3, nib >> 2
+            assert i0 < i1, "positions must be distinct and ascending"
+            out[r, 4 * g + i0] = vals[r, 2 * g]
+            out[r, 4 * g + i1] = vals[r, 2 * g + 1]
+    return out
+
+
+def test_sp24_hand_example():
+    """Two groups by hand: positions {1, 3} kept -> nibble 1 | 3 << 2 = 0xD;
+    only position 2 kept -> completed with position 0 -> nibble 0 | 2 << 2 =
+    0x8; metadata byte 0x8D; values [W1, W3, W4, W6]; zero padding."""
+    weff = np.array([[0, 1, 0, -1, 0, 0, 1, 0] + [0] * 8], dtype=np.int8)
+    mask = np.array([[0, 1, 0, 1, 0, 0, 1, 0] + [1, 1, 0, 0] * 2], dtype=np.uint8)
+    vals, meta = oracle.pack_sp24(weff, mask)
+    assert vals.shape == (1, 16) and meta.shape == (1, 16)
+    np.testing.assert_array_equal(vals[0, :8], [1, -1, 0, 1, 0, 0, 0, 0])
+    np.testing.assert_array_equal(meta[0, :2], [0x8D, 0x44])
+    assert (vals[0, 8:] == 0).all() and (meta[0, 2:] == 0).all()
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (2, 8), (1, 8)])
+def test_sp24_roundtrip(n, m):
+    """Every 2:4-compatible mask (n <= 2 of 4, n <= 2 of 8) round-trips: the
+    decompressed operand equals W_eff, and each stored position is a kept
+    one unless the group keeps fewer than two."""
+    w = wl.master_weights(16, 96, seed=10 * n + m)
+    layer = oracle.Layer(w, n, m)
+    vals, meta = oracle.pack_sp24(layer.weff, layer.mask)
+    assert vals.shape == (16, oracle.sp24_value_row_bytes(96)) == (16, 48)
+    assert meta.shape == (16, oracle.sp24_meta_row_bytes(96)) == (16, 16)
+    np.testing.assert_array_equal(_decode_sp24(vals, meta, 96), layer.weff)
+    for r in range(16):
+        for g in range(24):
+            nib = (int(meta[r, g // 2]) >> (4 * (g % 2))) & 0xF
+            chosen = {nib & 3, nib >> 2}
+            kept = set(np.nonzero(layer.mask[r, 4 * g: 4 * g + 4])[0])
+            assert kept <= chosen
+            # completion uses the smallest positions not kept
+            fill = sorted(chosen - kept)
+            assert fill == sorted(set(range(4)) - kept)[: len(fill)]
+
+
+def test_sp24_rejects_masks_that_are_not_2of4():
+    w = wl.master_weights(16, 64, seed=3)
+    layer = oracle.Layer(w, 6, 8)
+    with pytest.raises(ValueError):
+        oracle.pack_sp24(layer.weff, layer.mask)
+
+
 # ------------------------------------------------------------ activation quant
 
 def test_act_quant_invariants_and_zero_row():
