@@ -59,18 +59,30 @@ typedef enum {
  *        k%8 of byte k/8 set when position k is kept, padded with 0 bits to
  *        16 bytes; [O, row_bytes(NM bitmap)] uint8).
  *  I8    W_eff as int8 [O, K] (the GEMM operand).
- *  BF16T W_eff transposed, bf16 [K, O] (the dX operand of the backward).  */
+ *  BF16T W_eff transposed, bf16 [K, O] (the dX operand of the backward).
+ *  SP24  W_eff as the operand of the 2:4 sparse tensor-core MMA, for masks
+ *        with at most two kept weights in every group of four (n <= 2,
+ *        m = 4 or 8; other n:m give SBL_ERR_UNSUPPORTED).  For group g of
+ *        a row (positions 4g .. 4g+3) two positions i0 < i1 are stored: the
+ *        kept ones, completed with the smallest positions not kept when
+ *        fewer than two are kept.  Values: int8 W_eff at 4g+i0 and 4g+i1 in
+ *        bytes 2g, 2g+1 ([O, row_bytes(SP24 main)] int8, row_bytes =
+ *        K/2 rounded up to 16).  Metadata: nibble i0 | (i1 << 2) at bits
+ *        4*(g%2) of byte g/2 ([O, row_bytes(SP24 meta)] uint8, K/8 rounded
+ *        up to 16).  Padding bytes are 0.  */
 typedef enum {
     SBL_FMT_PK2 = 1,
     SBL_FMT_NM = 2,
     SBL_FMT_I8 = 4,
-    SBL_FMT_BF16T = 8
+    SBL_FMT_BF16T = 8,
+    SBL_FMT_SP24 = 16
 } sbl_format;
 
 /* Which buffer of a format sbl_packed_row_bytes() describes. */
 typedef enum {
-    SBL_BUF_MAIN = 0,      /* PK2 / I8 / BF16T data, NM values */
-    SBL_BUF_NM_BITMAP = 1  /* NM keep bitmap                   */
+    SBL_BUF_MAIN = 0,       /* PK2 / I8 / BF16T data, NM / SP24 values */
+    SBL_BUF_NM_BITMAP = 1,  /* NM keep bitmap                          */
+    SBL_BUF_SP24_META = 2   /* SP24 position metadata                  */
 } sbl_buffer;
 
 /* Operations that take a workspace. */
@@ -100,6 +112,8 @@ typedef struct {
     int8_t *i8;         /* SBL_FMT_I8  [O, K]                           */
     uint16_t *bf16t;    /* SBL_FMT_BF16T [K, O] bf16 bits               */
     float *gamma;       /* device scalar                                */
+    int8_t *sp24_values; /* SBL_FMT_SP24 values                         */
+    uint8_t *sp24_meta;  /* SBL_FMT_SP24 position metadata              */
 } sbl_packed;
 
 /* Human-readable text for a status code (static storage). */

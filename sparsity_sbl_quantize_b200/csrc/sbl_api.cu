@@ -12,6 +12,7 @@
 #include "sbl.h"
 #include "sbl_act.cuh"
 #include "sbl_decode.cuh"
+#include "sbl_sp24.cuh"
 #include "sbl_gemm.cuh"
 #include "sbl_pack.cuh"
 
@@ -68,7 +69,9 @@ static sbl_status current_device(DeviceInfo **out)
             cudaFuncSetAttribute(gemm_kernel<kKindF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 GemmCfg<128>::kSmemBytes) != cudaSuccess)
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(sp24_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSpSmemBytes) != cudaSuccess)
             return SBL_ERR_CUDA;
         if (!g_encode) {
             void *fn = nullptr;
@@ -103,6 +106,11 @@ static sbl_status check_desc(const sbl_layer_desc *d)
     if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
     return SBL_OK;
 }
+
+// The SP24 operand needs at most two kept weights in every group of four:
+// n <= 2 with m = 4, or n <= 2 with m = 8 (each half of a group of eight then
+// keeps at most two).
+static bool sp24_fits(const sbl_layer_desc *d) { return d->n <= 2; }
 
 static sbl_status launch_status()
 {
@@ -199,6 +207,78 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
                      : launch_gemm_bn<KIND, 256>(di, ta, tb, ty, args, stream);
 }
 
+// 3-D view of the SP24 metadata [O, row_bytes] for the sparse GEMM: dims
+// (16 bytes, O rows, row_bytes / 16 chunks) with strides (row_bytes, 16), box
+// (16, 128, 2), so one load writes the [2][128][16] no-swizzle layout that
+// tcgen05.cp reads.
+static bool encode_sp24_meta(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes)
+{
+    cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(row_bytes / 16)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), 16};
+    cuuint32_t box[3] = {16, static_cast<cuuint32_t>(kSpBM), 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Output map of the sparse GEMM's stores: [rows, cols] bf16 or fp32, box 32
+// rows x 32 columns, no swizzle.
+static bool encode_output_32x32(CUtensorMap *map, void *base, bool fp32, int64_t rows, int64_t cols)
+{
+    const int eb = fp32 ? 4 : 2;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * eb)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static sbl_status launch_sp24(const DeviceInfo *di, int32_t O, int32_t K, int32_t T, const int8_t *Xq,
+                              const float *d, const sbl_packed *w, void *Y, bool y_fp32, int32_t *acc_out,
+                              cudaStream_t stream)
+{
+    const int64_t vstride = round_up(K / 2, 16), mstride = round_up(K / 8, 16);
+    CUtensorMap ta, tb, te, ty;
+    if (!encode_kmajor(&ta, w->sp24_values, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, O, vstride, kSpBM) ||
+        !encode_kmajor(&tb, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, K, kSpBN) ||
+        !encode_sp24_meta(&te, w->sp24_meta, O, mstride) || !encode_output_32x32(&ty, Y, y_fp32, T, O))
+        return SBL_ERR_CUDA;
+    Sp24Args a;
+    memset(&a, 0, sizeof(a));
+    a.O = O;
+    a.T = T;
+    a.K = K;
+    a.tiles_m = (O + kSpBM - 1) / kSpBM;
+    a.tiles_n = (T + kSpBN - 1) / kSpBN;
+    a.k_blocks = (K + kSpKLogical - 1) / kSpKLogical;
+    a.out = Y;
+    a.out_fp32 = y_fp32 ? 1 : 0;
+    a.acc_out = acc_out;
+    a.gamma = w->gamma;
+    a.d = d;
+    a.err = di->err;
+    const int tiles = a.tiles_m * a.tiles_n;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles < di->num_sms ? tiles : di->num_sms));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kSpSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, sp24_gemm_kernel, ta, tb, te, ty, a) != cudaSuccess) return SBL_ERR_CUDA;
+    return launch_status();
+}
+
 }  // namespace sbl
 
 using namespace sbl;
@@ -258,6 +338,10 @@ size_t sbl_packed_row_bytes(const sbl_layer_desc *desc, sbl_format fmt, sbl_buff
         return static_cast<size_t>(round_up(K / 8, 16));
     case SBL_FMT_I8: return which == SBL_BUF_MAIN ? static_cast<size_t>(K) : 0;
     case SBL_FMT_BF16T: return which == SBL_BUF_MAIN ? static_cast<size_t>(2 * O) : 0;
+    case SBL_FMT_SP24:
+        if (which == SBL_BUF_MAIN) return static_cast<size_t>(round_up(K / 2, 16));
+        if (which == SBL_BUF_SP24_META) return static_cast<size_t>(round_up(K / 8, 16));
+        return 0;
     }
     return 0;
 }
@@ -282,8 +366,13 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
     sbl_status st = check_desc(desc);
     if (st != SBL_OK) return st;
     if (!W || !out || !out->gamma) return SBL_ERR_INVALID_ARG;
-    const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T;
+    const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T | SBL_FMT_SP24;
     if (formats & ~known) return SBL_ERR_INVALID_ARG;
+    if (formats & SBL_FMT_SP24) {
+        if (!out->sp24_values || !out->sp24_meta) return SBL_ERR_INVALID_ARG;
+        if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
+        if (!aligned16(out->sp24_values) || !aligned16(out->sp24_meta)) return SBL_ERR_ALIGNMENT;
+    }
     if ((formats & SBL_FMT_PK2) && !out->pk2) return SBL_ERR_INVALID_ARG;
     if ((formats & SBL_FMT_NM) && (!out->nm_values || !out->nm_bitmap)) return SBL_ERR_INVALID_ARG;
     if ((formats & SBL_FMT_I8) && !out->i8) return SBL_ERR_INVALID_ARG;
@@ -338,7 +427,13 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
                 cudaSuccess)
             return SBL_ERR_CUDA;
     }
-    if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM)) {
+    if (formats & SBL_FMT_SP24) {
+        pa.out.sp24_values = out->sp24_values;
+        pa.out.sp24_values_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_SP24, SBL_BUF_MAIN));
+        pa.out.sp24_meta = out->sp24_meta;
+        pa.out.sp24_meta_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_SP24, SBL_BUF_SP24_META));
+    }
+    if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM | SBL_FMT_SP24)) {
         // programmatic dependent launch behind gamma_kernel (see pack_kernel);
         // a thread covers 16 weights
         const int64_t per_cta = 256 * 16 / desc->m;  // groups per CTA
@@ -439,6 +534,12 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         a.gamma = w->gamma;
         a.row_scale = d;
         return launch_gemm<kKindI8>(di, Xq, K, w->i8, K, T, O, K, a, stream);
+    }
+    if (fmt == SBL_FMT_SP24) {
+        if (!w->sp24_values || !w->sp24_meta) return SBL_ERR_INVALID_ARG;
+        if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
+        if (!aligned16(w->sp24_values) || !aligned16(w->sp24_meta)) return SBL_ERR_ALIGNMENT;
+        return launch_sp24(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
     }
     if (fmt == SBL_FMT_PK2) {
         if (!w->pk2) return SBL_ERR_INVALID_ARG;

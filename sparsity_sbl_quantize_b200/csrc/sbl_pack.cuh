@@ -47,6 +47,10 @@ struct PackOut {
     int64_t nm_values_stride;
     uint8_t *nm_bitmap;
     int64_t nm_bitmap_stride;
+    int8_t *sp24_values;
+    int64_t sp24_values_stride;
+    uint8_t *sp24_meta;
+    int64_t sp24_meta_stride;
 };
 
 struct PackArgs {
@@ -288,6 +292,22 @@ __device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int3
     }
 }
 
+// SP24 form of four-group q of a thread's 16 weights: the group's kept
+// positions (at most two) completed with its smallest positions not kept,
+// i0 < i1; values W_eff[i0], W_eff[i1] go to value bytes 2q, 2q+1 and the
+// nibble i0 | i1 << 2 to bits 4q of the thread's 16 metadata bits.
+__device__ __forceinline__ void sp24_group(uint32_t wbytes, uint32_t keep4, int q, uint32_t (&vals)[2],
+                                           uint32_t &meta)
+{
+    uint32_t sel = keep4 & 0xfu;
+    if (__popc(sel) < 2) sel |= ~sel & (sel + 1u);  // lowest position not yet chosen
+    if (__popc(sel) < 2) sel |= ~sel & (sel + 1u);
+    const uint32_t i0 = static_cast<uint32_t>(__ffs(sel) - 1), i1 = static_cast<uint32_t>(31 - __clz(sel));
+    const uint32_t v = ((wbytes >> (8 * i0)) & 0xffu) | (((wbytes >> (8 * i1)) & 0xffu) << 8);
+    vals[q >> 1] |= v << (16 * (q & 1));
+    meta |= (i0 | (i1 << 2)) << (4 * q);
+}
+
 // Mask + ternarise + pack: thread t of CTA c owns the 16 consecutive weights
 // (two groups of 8 or four of 4) starting at (256 c + t) * 16.  Launched with
 // programmatic dependent launch right behind gamma_kernel: W is loaded and the
@@ -324,11 +344,32 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
     const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
     const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);  // 16 | K: same row
+    uint32_t sp_vals[2] = {0u, 0u}, sp_meta = 0u;
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
         uint32_t w0, w1;
         ternarise_group<M>(bits[b], keep[b], thr_bits, w0, w1);
         store_group<M>(a, row, col0 / M + b, w0, w1, keep[b]);
+        if (a.out.sp24_values) {
+            if constexpr (M == 4) {
+                sp24_group(w0, keep[b], b, sp_vals, sp_meta);
+            } else {
+                sp24_group(w0, keep[b], 2 * b, sp_vals, sp_meta);
+                sp24_group(w1, keep[b] >> 4, 2 * b + 1, sp_vals, sp_meta);
+            }
+        }
+    }
+    if (a.out.sp24_values) {
+        // 8 value bytes and 16 metadata bits per thread; the thread that ends
+        // a row also zeroes the row padding
+        uint8_t *vrow = reinterpret_cast<uint8_t *>(a.out.sp24_values) + static_cast<int64_t>(row) * a.out.sp24_values_stride;
+        uint8_t *mrow = a.out.sp24_meta + static_cast<int64_t>(row) * a.out.sp24_meta_stride;
+        *reinterpret_cast<uint2 *>(vrow + col0 / 2) = make_uint2(sp_vals[0], sp_vals[1]);
+        *reinterpret_cast<uint16_t *>(mrow + col0 / 8) = static_cast<uint16_t>(sp_meta);
+        if (col0 + 16 == a.cols) {
+            for (int64_t b = a.cols / 2; b < a.out.sp24_values_stride; ++b) vrow[b] = 0;
+            for (int64_t b = a.cols / 8; b < a.out.sp24_meta_stride; ++b) mrow[b] = 0;
+        }
     }
 }
 

@@ -61,6 +61,9 @@ class GpuLayer:
             out["i8"] = p.i8.cpu().numpy()
         if p.bf16t is not None:
             out["bf16t"] = bits_of(p.bf16t)
+        if p.sp24_values is not None:
+            out["sp24_values"] = p.sp24_values.cpu().numpy()
+            out["sp24_meta"] = p.sp24_meta.cpu().numpy()
         return out
 
 

@@ -52,6 +52,8 @@ def test_row_bytes_match_oracle_formats(sbl, O, K, n, m):
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_NM, sbl.SBL_BUF_NM_BITMAP) == oracle.nm_bitmap_row_bytes(K)
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_I8) == K
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_BF16T) == 2 * O
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_SP24) == oracle.sp24_value_row_bytes(K)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_SP24, sbl.SBL_BUF_SP24_META) == oracle.sp24_meta_row_bytes(K)
 
 
 @pytest.mark.parametrize("O,K,n,m", [(0, 256, 6, 8), (128, 250, 6, 8), (128, 256, 9, 8),
@@ -129,3 +131,25 @@ def test_validation_happens_before_any_device_access(sbl):
     wp = sbl.sbl_packed(good, None, None, None, None, good)
     assert _raw(sbl, "sbl_forward", ctypes.byref(d), P(good), P(good), 17, ctypes.byref(wp),
                 sbl.SBL_FMT_PK2, P(good), 0, None, None) in (4, 7)
+
+
+def test_sp24_validation(sbl):
+    """The sparse MMA operand exists only for masks with at most two kept
+    weights per group of four (n <= 2): other n:m are unsupported in both the
+    pack and the forward; missing or misaligned buffers are rejected first."""
+    good = 0x10000
+    P = ctypes.c_void_p
+    ws = P(good)
+    d68 = sbl.desc(128, 256, 6, 8)
+    d24 = sbl.desc(128, 256, 2, 4)
+    w = sbl.sbl_packed(None, None, None, None, None, good, good, good)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d68), P(good), sbl.SBL_FMT_SP24,
+                ctypes.byref(w), ws, 1 << 20, None) == 4
+    assert _raw(sbl, "sbl_forward", ctypes.byref(d68), P(good), P(good), 64, ctypes.byref(w),
+                sbl.SBL_FMT_SP24, P(good), 0, None, None) in (4, 7)
+    nometa = sbl.sbl_packed(None, None, None, None, None, good, good, None)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_SP24,
+                ctypes.byref(nometa), ws, 1 << 20, None) == 1
+    skew = sbl.sbl_packed(None, None, None, None, None, good, good + 8, good)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_SP24,
+                ctypes.byref(skew), ws, 1 << 20, None) == 3

@@ -25,7 +25,12 @@ from gpu_case import (ALL_FORMATS, GpuLayer, bf16_dev, bits_of, forward, normwis
 FWD_TOL = 1e-3  # only used where bit-exactness is not expected (backward)
 
 
+SP24 = 16
+
+
 def check_pack(w, n, m, formats=ALL_FORMATS):
+    if n <= 2 and formats == ALL_FORMATS:
+        formats |= SP24  # the sparse MMA operand exists for 2:4-compatible masks
     layer = GpuLayer(w, n, m, formats)
     got = layer.host()
     ref = oracle.Layer(w, n, m)
@@ -41,6 +46,10 @@ def check_pack(w, n, m, formats=ALL_FORMATS):
     if "bf16t" in got:
         expect = np.where(ref.weff.T > 0, 0x3F80, np.where(ref.weff.T < 0, 0xBF80, 0)).astype(np.uint16)
         np.testing.assert_array_equal(got["bf16t"], expect)
+    if "sp24_values" in got:
+        vals, meta = oracle.pack_sp24(ref.weff, ref.mask)
+        np.testing.assert_array_equal(got["sp24_values"], vals)
+        np.testing.assert_array_equal(got["sp24_meta"], meta)
     return layer, ref
 
 
@@ -109,7 +118,9 @@ def run_forward_full_check(O, K, T, n, m, seed, fmt_name="I8", outliers=0.0):
     q, d = quantize_act(x)
     qr, dr, accr, yr, ybr = ref.forward(x)
     np.testing.assert_array_equal(q.cpu().numpy(), qr)
-    fmt = sbl.SBL_FMT_I8 if fmt_name == "I8" else sbl.SBL_FMT_PK2
+    fmt = {"I8": sbl.SBL_FMT_I8, "PK2": sbl.SBL_FMT_PK2, "SP24": sbl.SBL_FMT_SP24}[fmt_name]
+    if fmt_name == "SP24":
+        layer = GpuLayer(w, n, m, sbl.SBL_FMT_SP24)
     yb, acc = forward(layer, q, d, fmt)
     np.testing.assert_array_equal(acc.cpu().numpy(), accr)
     np.testing.assert_array_equal(bits_of(yb), ybr)
@@ -148,6 +159,40 @@ def test_forward_decode_pk2_bit_exact(O, K, T):
 
 def test_forward_decode_pk2_six_of_eight():
     run_forward_full_check(896, 4864, 5, 6, 8, seed=11, fmt_name="PK2")
+
+
+@pytest.mark.parametrize("O,K,T,n,m", [
+    (128, 256, 128, 2, 4),    # exactly one tile and one k-block
+    (528, 1040, 300, 2, 4),   # ragged O, T, and K (16 past the last 256 block)
+    (384, 1536, 520, 2, 8),   # 2:8 run on the 2:4 hardware path
+    (16, 16, 5, 1, 4),        # minimum sizes
+    (256, 896, 257, 1, 8),    # half k-block tail (896 = 3.5 x 256)
+    (4864, 896, 64, 2, 4),    # the MLP gate/up shape, short T
+])
+def test_forward_sp24_bit_exact(O, K, T, n, m):
+    run_forward_full_check(O, K, T, n, m, seed=O + K + T, fmt_name="SP24")
+
+
+def test_forward_sp24_matches_dense_path_full_size():
+    """The sparse and dense tensor-core paths compute the same integers: at
+    the MLP down-projection size (T = 4096) their accumulators and outputs
+    agree bit for bit, and sampled accumulators match the oracle."""
+    sbl = sbl_mod()
+    O, K, T = 896, 4864, 4096
+    w = wl.master_weights(O, K, seed=2)
+    x = wl.activations(T, K, seed=2)
+    layer = GpuLayer(w, 2, 4, sbl.SBL_FMT_I8 | sbl.SBL_FMT_SP24)
+    q, d = quantize_act(x)
+    yd, accd = forward(layer, q, d, sbl.SBL_FMT_I8)
+    ys, accs = forward(layer, q, d, sbl.SBL_FMT_SP24)
+    assert torch.equal(accd, accs)
+    np.testing.assert_array_equal(bits_of(yd), bits_of(ys))
+    ref = oracle.Layer(w, 2, 4)
+    qr, _ = oracle.quantize_act(x)
+    rng = np.random.default_rng(7)
+    it, io = rng.integers(0, T, 1024), rng.integers(0, O, 1024)
+    it[:2], io[:2] = [T - 1, 0], [O - 1, O - 1]
+    np.testing.assert_array_equal(accs.cpu().numpy()[it, io], oracle.acc_samples(qr, ref.weff, it, io))
 
 
 def test_forward_zero_tokens_is_noop():
