@@ -36,6 +36,68 @@ from sparsity_sbl_quantize_b200 import workloads as wl  # noqa: E402
 
 METRIC = "Sparse-BitLinear int8 TOPS (prefill/train) & decode GB/s, % of B200 roofline"
 L2_FLUSH_BYTES = 512 << 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+KERNEL_SOURCES = ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh", "sbl_decode.cuh", "sbl_api.cu")
+
+
+UNIT_BYTES = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1024, "MB": 1 << 20, "GB": 1 << 30}
+
+
+def record_traffic(csv_path: str, workload: str, kernel_regex: str, command: str) -> dict:
+    """Parse an ncu --csv metric list (dram__bytes_read.sum and
+    dram__bytes_write.sum per launch) and store the mean read+write bytes per
+    launch of the kernels matching kernel_regex for `workload`, tagged with
+    the current kernel-source hash."""
+    import csv
+    import re
+    pat = re.compile(kernel_regex)
+    per_launch = {}
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for row in csv.DictReader(lines):
+        if not pat.search(row["Kernel Name"]) or not row["Metric Name"].startswith("dram__bytes_"):
+            continue
+        val = float(row["Metric Value"].replace(",", "")) * UNIT_BYTES[row["Metric Unit"]]
+        per_launch[row["ID"]] = per_launch.get(row["ID"], 0.0) + val
+    if not per_launch:
+        raise SystemExit(f"no launches of {kernel_regex} with DRAM metrics in {csv_path}")
+    rec = {"kernel_regex": kernel_regex, "launches": len(per_launch),
+           "bytes_per_launch": round(sum(per_launch.values()) / len(per_launch)),
+           "kernel_source_sha256": kernel_source_hash(), "command": command}
+    data = {}
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+    data[workload] = rec
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return rec
+
+
+def kernel_source_hash() -> str:
+    """SHA-256 over the CUDA sources of the timed kernels: a stored DRAM
+    traffic figure is reported only while these are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparsity_sbl_quantize_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the roofline kernel, from the
+    ncu capture recorded in profiles/roofline_traffic.json, or None when there
+    is none for this workload or the kernels changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
 
 
 def parse():
@@ -46,6 +108,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen05b_mlp", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="store the mean DRAM bytes per roofline-kernel launch from an ncu --csv metric list "
+                         "(dram__bytes_read.sum, dram__bytes_write.sum) for --workload, then exit")
+    ap.add_argument("--traffic-command", default="", help="the ncu command that produced NCU_CSV (recorded)")
     return ap.parse_args()
 
 
@@ -164,9 +230,31 @@ class Runner:
                 L["dx"] = torch.empty((T, lin.d_in), dtype=torch.bfloat16, device=device)
                 L["dw"] = torch.empty((lin.d_out, lin.d_in), dtype=torch.float32, device=device)
                 L["bws"] = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc0, T, sbl.SBL_OP_BACKWARD))
+        self.choose_forward_formats()
         self.launches_per_step = 0
         n_side = max(len(self.layers), 1)
         self.streams = [[torch.cuda.Stream(device) for _ in range(1 + n_side)] for _ in wk.patterns]
+
+    def choose_forward_formats(self):
+        """Forward operand per (layer, pattern), as the library recommends for
+        the shape (sbl_forward_format): the int8 W_eff for the dense MMA or,
+        when the mask keeps at most two of every four weights and the GEMM is
+        large enough, the 2:4 compressed operand of the sparse MMA."""
+        sbl = self.sbl
+        self.fwd_fmt = {}
+        self.pack_fmts = {}
+        for (n, m) in self.wk.patterns:
+            for li, L in enumerate(self.layers):
+                dsc, _ = L["packed"][(n, m)]
+                fmt = sbl.SBL_FMT_I8 if self.wk.mode == "train" else sbl.sbl_forward_format(dsc, self.T)
+                self.fwd_fmt[(li, (n, m))] = fmt
+                self.pack_fmts[(li, (n, m))] = self.fmts if fmt == sbl.SBL_FMT_I8 else fmt
+                if fmt != sbl.SBL_FMT_I8:
+                    L["packed"][(n, m)] = (dsc, sbl.alloc_packed(dsc, fmt))
+
+    def formats_used(self):
+        names = {self.sbl.SBL_FMT_I8: "I8 (dense MMA)", self.sbl.SBL_FMT_SP24: "SP24 (2:4 sparse MMA)"}
+        return {f"{n}:{m}/linear{li}": names[f] for (li, (n, m)), f in sorted(self.fwd_fmt.items())}
 
     def step(self, timed=False):
         """Enqueue one step.  Untimed: the N:M patterns' passes are
@@ -188,7 +276,7 @@ class Runner:
             for li, L in enumerate(self.layers):
                 with torch.cuda.stream(side[li % len(side)]):
                     dsc, p = L["packed"][(n, m)]
-                    sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"][(n, m)])
+                    sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)])
                 launches += 2 + (1 if self.fmts & sbl.SBL_FMT_BF16T else 0)
             for ii, inp in enumerate(self.inputs):
                 with torch.cuda.stream(side[(len(self.layers) + ii) % len(side)]):
@@ -199,7 +287,7 @@ class Runner:
                 if st is not g_stream:
                     g_stream.wait_stream(st)
             with torch.cuda.stream(g_stream):
-                for L in self.layers:
+                for li, L in enumerate(self.layers):
                     dsc, p = L["packed"][(n, m)]
                     inp = L["inp"]
                     q, d = inp["q"][(n, m)], inp["d"][(n, m)]
@@ -207,7 +295,7 @@ class Runner:
                         e0 = torch.cuda.Event(enable_timing=True, external=True)
                         e1 = torch.cuda.Event(enable_timing=True, external=True)
                         e0.record()
-                    sbl.sbl_forward(dsc, q, d, self.T, p, sbl.SBL_FMT_I8, L["y"][(n, m)])
+                    sbl.sbl_forward(dsc, q, d, self.T, p, self.fwd_fmt[(li, (n, m))], L["y"][(n, m)])
                     launches += 1
                     if timed:
                         e1.record()
@@ -258,18 +346,27 @@ class Runner:
                 L["w"].copy_(hw, non_blocking=True)
             for inp, hx in zip(self.inputs, self.h_x):
                 inp["x"].copy_(hx, non_blocking=True)
-            for L in self.layers:
+            for li, L in enumerate(self.layers):
                 dsc, p = L["packed"][(n, m)]
-                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.fmts, p, L["ws"][(n, m)])
+                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)])
             for inp in self.inputs:
                 sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"][(n, m)], inp["d"][(n, m)])
-            for L, hy in zip(self.layers, self.h_y):
+            for li, (L, hy) in enumerate(zip(self.layers, self.h_y)):
                 dsc, p = L["packed"][(n, m)]
                 inp = L["inp"]
-                sbl.sbl_forward(dsc, inp["q"][(n, m)], inp["d"][(n, m)], self.T, p, sbl.SBL_FMT_I8,
+                sbl.sbl_forward(dsc, inp["q"][(n, m)], inp["d"][(n, m)], self.T, p, self.fwd_fmt[(li, (n, m))],
                                 L["y"][(n, m)])
                 hy.copy_(L["y"][(n, m)], non_blocking=True)
         self.torch.cuda.current_stream().synchronize()
+
+
+def gemm_kernel_names(r, sbl):
+    names = ["gemm_kernel<int8> (tcgen05 dense MMA, TMEM accumulators, TMA)"]
+    if any(f == sbl.SBL_FMT_SP24 for f in r.fwd_fmt.values()):
+        names.append("sp24_pair_kernel (tcgen05.mma.sp cta_group::2)")
+        if not any(f == sbl.SBL_FMT_I8 for f in r.fwd_fmt.values()):
+            names = names[1:]
+    return " + ".join(names)
 
 
 def run_ours(args, wk):
@@ -394,12 +491,15 @@ def run_ours(args, wk):
                    "patterns": [f"{n}:{m}" for n, m in wk.patterns], "mode": wk.mode,
                    "l2": "flushed between timed steps (512 MiB write outside the events)",
                    "parallelism": f"independent replicas x{world}",
-                   "dense_equivalent_tops": round(value * dense_factor(wk), 3)},
-        "roofline": {"kernel": "gemm_kernel<int8> (tcgen05, TMEM accumulators, TMA)", "bound": "tensor",
+                   "dense_equivalent_tops": round(value * dense_factor(wk), 3),
+                   "forward_formats": r.formats_used()},
+        "roofline": {"kernel": gemm_kernel_names(r, sbl), "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": round(int8_peak, 1), "unit": "TOPS",
                      "frac": round(achieved / int8_peak, 4),
                      "peak_note": f"int8 dense = 2 x {pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s",
-                     "traffic": None},
+                     "traffic": stored_traffic(wk.name),
+                     "traffic_note": "mean DRAM read+write bytes per GEMM launch of the step (ncu capture in "
+                                     "profiles/roofline_traffic.json; null when absent or stale)"},
         "e2e": {"value": round(e_value, 3), "unit": "TOPS", "h2d_bytes_per_step": r.h2d,
                 "d2h_bytes_per_step": r.d2h},
         "gpu_launches": r.launches_per_step * args.steps,
@@ -498,7 +598,10 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
                                         "per_token_count": {str(T): results[T] for T in wk.tokens},
                                         "l2": "rotating weight copies > 4x L2 inside one CUDA graph"},
         "roofline": {"kernel": "decode_kernel (PK2 stream, mma.sync u8 x s8)", "bound": "hbm", "achieved": round(gemv, 1),
-                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gemv / pk["hbm_gbs"], 4), "traffic": None},
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gemv / pk["hbm_gbs"], 4),
+                     "traffic": stored_traffic(wk.name),
+                     "traffic_note": "mean DRAM read+write bytes per decode launch (ncu capture in "
+                                     "profiles/roofline_traffic.json; null when absent or stale)"},
         "gpu_launches": None,
     }
     if rank == 0:
@@ -564,6 +667,10 @@ def run_reference(args, wk):
 def main():
     args = parse()
     wk = wl.WORKLOADS[args.workload]
+    if args.record_traffic:
+        regex = r"decode_kernel" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
+        print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command)))
+        return
     if args.impl == "reference":
         run_reference(args, wk)
     else:

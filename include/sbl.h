@@ -204,6 +204,17 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
                        int32_t T, const sbl_packed *w, sbl_format fmt,
                        void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);
 
+/* The forward operand format the library recommends for a layer and a
+ * token count: SBL_FMT_SP24 (2:4 sparse tensor-core MMA on CTA pairs) when
+ * the mask allows it (n <= 2) and the GEMM is large enough for the sparse
+ * MMA to pay: in_features >= 1024 and tokens * out_features >= 8192 * 1024;
+ * SBL_FMT_I8 (dense tensor-core MMA) otherwise.  On B200 the sparse kernel
+ * measured 1.1-1.4x the dense one on such shapes and 0.8x on shorter ones
+ * (short K or few output tiles), where the dense kernel's wider tiles and
+ * cheaper epilogue win.  Either format gives identical results.  Returns
+ * 0 for an invalid descriptor or tokens < 0. */
+sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens);
+
 /* Backward through the layer with the Dual straight-through estimator
  * (Sparse-BitNet summary, "The Dual Straight-Through Estimator": the
  * gradient passes through mask and quantiser as identity):

@@ -71,7 +71,11 @@ static sbl_status current_device(DeviceInfo **out)
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSpSmemBytes) != cudaSuccess)
+                                 kSpSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(sp24_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Sp24PairCfg<128>::kSmemBytes) != cudaSuccess)
             return SBL_ERR_CUDA;
         if (!g_encode) {
             void *fn = nullptr;
@@ -106,6 +110,9 @@ static sbl_status check_desc(const sbl_layer_desc *d)
     if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
     return SBL_OK;
 }
+
+// The sparse GEMM runs on CTA pairs (cta_group::2) when set.
+constexpr bool kSp24UsePairs = true;
 
 // The SP24 operand needs at most two kept weights in every group of four:
 // n <= 2 with m = 4, or n <= 2 with m = 8 (each half of a group of eight then
@@ -237,6 +244,68 @@ static bool encode_output_32x32(CUtensorMap *map, void *base, bool fp32, int64_t
                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Token-tile width of the CTA-pair sparse GEMM: the persistent grid of
+// num_sms / 2 pairs runs ceil(tiles / pairs) rounds, each costing about the
+// tile width plus a fixed part (pipeline fill, epilogue tail) worth 64
+// columns; the narrower tile wins only when it saves whole rounds.
+static int choose_pair_bn(int32_t O, int32_t T, int num_sms)
+{
+    const int pairs = num_sms / 2;
+    auto cost = [&](int bn) {
+        const int64_t tiles = static_cast<int64_t>((O + 255) / 256) * ((T + bn - 1) / bn);
+        const int64_t p = tiles < pairs ? tiles : pairs;
+        return ((tiles + p - 1) / p) * (bn + 64);
+    };
+    return cost(128) < cost(224) ? 128 : 224;
+}
+
+// The same GEMM on CTA pairs: 256 weight rows x BN tokens per cluster of two.
+template <int BN>
+static sbl_status launch_sp24_pair(const DeviceInfo *di, int32_t O, int32_t K, int32_t T, const int8_t *Xq,
+                                   const float *d, const sbl_packed *w, void *Y, bool y_fp32, int32_t *acc_out,
+                                   cudaStream_t stream)
+{
+    const int64_t vstride = round_up(K / 2, 16), mstride = round_up(K / 8, 16);
+    CUtensorMap ta, tb, te, ty;
+    if (!encode_kmajor(&ta, w->sp24_values, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, O, vstride, kSpBM) ||
+        !encode_kmajor(&tb, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, K, BN / 2) ||
+        !encode_sp24_meta(&te, w->sp24_meta, O, mstride) || !encode_output_32x32(&ty, Y, y_fp32, T, O))
+        return SBL_ERR_CUDA;
+    Sp24Args a;
+    memset(&a, 0, sizeof(a));
+    a.O = O;
+    a.T = T;
+    a.K = K;
+    a.tiles_m = (O + 255) / 256;
+    a.tiles_n = (T + BN - 1) / BN;
+    a.k_blocks = (K + kSpKLogical - 1) / kSpKLogical;
+    a.out = Y;
+    a.out_fp32 = y_fp32 ? 1 : 0;
+    a.acc_out = acc_out;
+    a.gamma = w->gamma;
+    a.d = d;
+    a.err = di->err;
+    const int tiles = a.tiles_m * a.tiles_n;
+    const int pairs = tiles < di->num_sms / 2 ? tiles : di->num_sms / 2;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = Sp24PairCfg<BN>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, sp24_pair_kernel<BN>, ta, tb, te, ty, a) != cudaSuccess) return SBL_ERR_CUDA;
+    return launch_status();
 }
 
 static sbl_status launch_sp24(const DeviceInfo *di, int32_t O, int32_t K, int32_t T, const int8_t *Xq,
@@ -539,6 +608,11 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         if (!w->sp24_values || !w->sp24_meta) return SBL_ERR_INVALID_ARG;
         if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
         if (!aligned16(w->sp24_values) || !aligned16(w->sp24_meta)) return SBL_ERR_ALIGNMENT;
+        if (kSp24UsePairs) {
+            return choose_pair_bn(O, T, di->num_sms) == 224
+                       ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream)
+                       : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
+        }
         return launch_sp24(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
     }
     if (fmt == SBL_FMT_PK2) {
@@ -582,6 +656,14 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
     }
     return SBL_ERR_UNSUPPORTED;
+}
+
+sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
+{
+    if (check_desc(desc) != SBL_OK || tokens < 0) return static_cast<sbl_format>(0);
+    if (!sp24_fits(desc)) return SBL_FMT_I8;
+    const int64_t outputs = static_cast<int64_t>(tokens) * desc->out_features;
+    return (desc->in_features >= 1024 && outputs >= 8192LL * 1024) ? SBL_FMT_SP24 : SBL_FMT_I8;
 }
 
 sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq,

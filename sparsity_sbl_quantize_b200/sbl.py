@@ -67,12 +67,14 @@ _lib.sbl_forward.restype = ctypes.c_int
 _lib.sbl_forward.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, _P]
 _lib.sbl_backward_dual_ste.restype = ctypes.c_int
 _lib.sbl_backward_dual_ste.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _sz, _P]
+_lib.sbl_forward_format.restype = ctypes.c_int
+_lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
-            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward", "sbl_backward_dual_ste",
-            "sbl_device_error"]
+            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
+            "sbl_forward_format", "sbl_backward_dual_ste", "sbl_device_error"]
 
 
 class SblError(RuntimeError):
@@ -183,6 +185,10 @@ def sbl_device_error(clear: bool = False) -> int:
 
 
 # ------------------------------------------------- allocation helpers (torch)
+
+def sbl_forward_format(d: sbl_layer_desc, tokens: int) -> int:
+    return int(_lib.sbl_forward_format(ctypes.byref(d), tokens))
+
 
 def alloc_packed(d: sbl_layer_desc, formats: int, device="cuda") -> Packed:
     """Allocate (with torch) the buffers sbl_quantize_mask_pack writes."""

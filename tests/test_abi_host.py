@@ -153,3 +153,17 @@ def test_sp24_validation(sbl):
     skew = sbl.sbl_packed(None, None, None, None, None, good, good + 8, good)
     assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_SP24,
                 ctypes.byref(skew), ws, 1 << 20, None) == 3
+
+
+def test_forward_format_recommendation(sbl):
+    """The recommended forward operand: the dense int8 MMA unless the mask
+    is 2:4-compatible (n <= 2) and the GEMM is long in K and large in T x O."""
+    F = sbl.sbl_forward_format
+    assert F(sbl.desc(4864, 896, 2, 4), 4096) == sbl.SBL_FMT_I8      # short K
+    assert F(sbl.desc(896, 4864, 2, 4), 4096) == sbl.SBL_FMT_I8      # few output tiles
+    assert F(sbl.desc(8960, 1536, 2, 4), 8192) == sbl.SBL_FMT_SP24
+    assert F(sbl.desc(1536, 8960, 2, 8), 8192) == sbl.SBL_FMT_SP24   # 2:8 runs as 2:4
+    assert F(sbl.desc(2048, 11008, 6, 8), 16384) == sbl.SBL_FMT_I8   # 6:8 is not 2:4
+    assert F(sbl.desc(2048, 11008, 3, 4), 16384) == sbl.SBL_FMT_I8
+    assert F(sbl.desc(20, 256, 2, 4), 64) == 0                       # invalid descriptor
+    assert F(sbl.desc(128, 256, 2, 4), -1) == 0

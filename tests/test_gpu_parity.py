@@ -173,12 +173,14 @@ def test_forward_sp24_bit_exact(O, K, T, n, m):
     run_forward_full_check(O, K, T, n, m, seed=O + K + T, fmt_name="SP24")
 
 
-def test_forward_sp24_matches_dense_path_full_size():
+@pytest.mark.parametrize("O,K,T", [(896, 4864, 4096),    # MLP down projection (128-token pair tiles)
+                                   (4864, 896, 4096),    # MLP gate/up (224-token pair tiles)
+                                   (2048, 1024, 4000)])  # 224-token tiles with a ragged last tile
+def test_forward_sp24_matches_dense_path_full_size(O, K, T):
     """The sparse and dense tensor-core paths compute the same integers: at
-    the MLP down-projection size (T = 4096) their accumulators and outputs
-    agree bit for bit, and sampled accumulators match the oracle."""
+    full workload sizes their accumulators and outputs agree bit for bit, and
+    sampled accumulators match the oracle."""
     sbl = sbl_mod()
-    O, K, T = 896, 4864, 4096
     w = wl.master_weights(O, K, seed=2)
     x = wl.activations(T, K, seed=2)
     layer = GpuLayer(w, 2, 4, sbl.SBL_FMT_I8 | sbl.SBL_FMT_SP24)
