@@ -37,7 +37,8 @@ from sparsity_sbl_quantize_b200 import workloads as wl  # noqa: E402
 METRIC = "Sparse-BitLinear int8 TOPS (prefill/train) & decode GB/s, % of B200 roofline"
 L2_FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
-KERNEL_SOURCES = ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh", "sbl_decode.cuh", "sbl_api.cu")
+# the device code of the roofline kernels (the GEMMs and the decode GEMV)
+KERNEL_SOURCES = ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh", "sbl_decode.cuh")
 
 
 UNIT_BYTES = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1024, "MB": 1 << 20, "GB": 1 << 30}

@@ -70,8 +70,6 @@ static sbl_status current_device(DeviceInfo **out)
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(sp24_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSpSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -110,9 +108,6 @@ static sbl_status check_desc(const sbl_layer_desc *d)
     if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
     return SBL_OK;
 }
-
-// The sparse GEMM runs on CTA pairs (cta_group::2) when set.
-constexpr bool kSp24UsePairs = true;
 
 // The SP24 operand needs at most two kept weights in every group of four:
 // n <= 2 with m = 4, or n <= 2 with m = 8 (each half of a group of eight then
@@ -308,46 +303,6 @@ static sbl_status launch_sp24_pair(const DeviceInfo *di, int32_t O, int32_t K, i
     return launch_status();
 }
 
-static sbl_status launch_sp24(const DeviceInfo *di, int32_t O, int32_t K, int32_t T, const int8_t *Xq,
-                              const float *d, const sbl_packed *w, void *Y, bool y_fp32, int32_t *acc_out,
-                              cudaStream_t stream)
-{
-    const int64_t vstride = round_up(K / 2, 16), mstride = round_up(K / 8, 16);
-    CUtensorMap ta, tb, te, ty;
-    if (!encode_kmajor(&ta, w->sp24_values, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, O, vstride, kSpBM) ||
-        !encode_kmajor(&tb, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, K, kSpBN) ||
-        !encode_sp24_meta(&te, w->sp24_meta, O, mstride) || !encode_output_32x32(&ty, Y, y_fp32, T, O))
-        return SBL_ERR_CUDA;
-    Sp24Args a;
-    memset(&a, 0, sizeof(a));
-    a.O = O;
-    a.T = T;
-    a.K = K;
-    a.tiles_m = (O + kSpBM - 1) / kSpBM;
-    a.tiles_n = (T + kSpBN - 1) / kSpBN;
-    a.k_blocks = (K + kSpKLogical - 1) / kSpKLogical;
-    a.out = Y;
-    a.out_fp32 = y_fp32 ? 1 : 0;
-    a.acc_out = acc_out;
-    a.gamma = w->gamma;
-    a.d = d;
-    a.err = di->err;
-    const int tiles = a.tiles_m * a.tiles_n;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles < di->num_sms ? tiles : di->num_sms));
-    cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = kSpSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, sp24_gemm_kernel, ta, tb, te, ty, a) != cudaSuccess) return SBL_ERR_CUDA;
-    return launch_status();
-}
-
 }  // namespace sbl
 
 using namespace sbl;
@@ -517,8 +472,11 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = (desc->m == 8) ? cudaLaunchKernelEx(&cfg, pack_kernel<8>, pa)
-                                             : cudaLaunchKernelEx(&cfg, pack_kernel<4>, pa);
+        const bool sp = (formats & SBL_FMT_SP24) != 0;
+        const cudaError_t e = (desc->m == 8) ? (sp ? cudaLaunchKernelEx(&cfg, pack_kernel<8, true>, pa)
+                                                   : cudaLaunchKernelEx(&cfg, pack_kernel<8, false>, pa))
+                                             : (sp ? cudaLaunchKernelEx(&cfg, pack_kernel<4, true>, pa)
+                                                   : cudaLaunchKernelEx(&cfg, pack_kernel<4, false>, pa));
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         if ((st = launch_status()) != SBL_OK) return st;
     }
@@ -608,12 +566,9 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         if (!w->sp24_values || !w->sp24_meta) return SBL_ERR_INVALID_ARG;
         if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
         if (!aligned16(w->sp24_values) || !aligned16(w->sp24_meta)) return SBL_ERR_ALIGNMENT;
-        if (kSp24UsePairs) {
-            return choose_pair_bn(O, T, di->num_sms) == 224
-                       ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream)
-                       : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
-        }
-        return launch_sp24(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
+        return choose_pair_bn(O, T, di->num_sms) == 224
+                   ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream)
+                   : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
     }
     if (fmt == SBL_FMT_PK2) {
         if (!w->pk2) return SBL_ERR_INVALID_ARG;

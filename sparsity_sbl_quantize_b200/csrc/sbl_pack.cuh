@@ -313,7 +313,9 @@ __device__ __forceinline__ void sp24_group(uint32_t wbytes, uint32_t keep4, int 
 // programmatic dependent launch right behind gamma_kernel: W is loaded and the
 // N:M keep masks (which need only |W|) are computed before waiting for
 // gamma_kernel (which does not write W); gamma is read after.
-template <int M>
+// SP24: also write the 2:4 sparse-MMA operand (a separate instantiation, so
+// the other formats' kernel carries none of its registers).
+template <int M, bool SP24>
 __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
 {
     constexpr int kBatch = 16 / M;  // groups per thread
@@ -350,7 +352,7 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
         uint32_t w0, w1;
         ternarise_group<M>(bits[b], keep[b], thr_bits, w0, w1);
         store_group<M>(a, row, col0 / M + b, w0, w1, keep[b]);
-        if (a.out.sp24_values) {
+        if constexpr (SP24) {
             if constexpr (M == 4) {
                 sp24_group(w0, keep[b], b, sp_vals, sp_meta);
             } else {
@@ -359,7 +361,7 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
             }
         }
     }
-    if (a.out.sp24_values) {
+    if constexpr (SP24) {
         // 8 value bytes and 16 metadata bits per thread; the thread that ends
         // a row also zeroes the row padding
         uint8_t *vrow = reinterpret_cast<uint8_t *>(a.out.sp24_values) + static_cast<int64_t>(row) * a.out.sp24_values_stride;

@@ -1,5 +1,5 @@
 // sbl_sp24.cuh -- the forward GEMM of the Sparse-BitLinear layer on the 2:4
-// sparse tensor cores of sm_100a (tcgen05.mma.sp, kind::i8).
+// sparse tensor cores of sm_100a (tcgen05.mma.sp, kind::i8), run by CTA pairs.
 //
 //   acc[t, o] = sum_k W_eff[o, k] * Xq[t, k]
 //   Y[t, o]   = fl32(fl32(acc[t, o]) * fl32(gamma * d_t))
@@ -11,24 +11,14 @@
 // positions) and the tensor core skips the zero half, so each MMA covers 64
 // logical K with the operand bytes of 32.
 //
-// The sparse operand is A, so here the tile is 128 weight rows (TMEM lanes)
-// x 128 tokens (TMEM columns), the transpose of the dense kernel's tile.
-// Per stage (256 logical K): A = 128 rows x 128 compressed bytes (TMA,
-// 128-byte swizzle), B = 128 tokens x 256 bytes (two 128-byte swizzled
-// boxes), E = the metadata, 128 rows x 32 bytes, loaded by TMA as a 3-D box
-// into the no-swizzle canonical layout ([2][128][16] bytes) and copied into
-// tensor memory with tcgen05.cp (lane = weight row; the 64 metadata bits of
-// one MMA fill two columns, nibble g at bits 4g).
-//
-// Roles (320 threads) as in the dense kernel: warp 0 TMA producer, warp 1
-// tensor-memory owner and MMA issuer (tcgen05.cp then four tcgen05.mma.sp per
-// stage, in issue order), warps 2-9 epilogue.  Tensor memory: three 128-column
-// accumulators and one 8-column metadata slot per stage.  The epilogue warp
-// of lanes 32q..32q+31 and columns 64h..64h+63 drains two 32 x 32 blocks:
-// thread = weight row o, its 32 registers = 32 tokens; it scales column t by
-// gamma * d_t (the token scales arrive by shuffle from one load per lane),
-// writes the block transposed ([t][o]) into shared memory and stores it with
-// one TMA bulk tensor store.  Every wait is time-bounded.
+// The sparse operand is A, so the tile is weight rows (TMEM lanes) x tokens
+// (TMEM columns), the transpose of the dense kernel's tile.  Per stage (256
+// logical K) a CTA loads A = 128 rows x 128 compressed bytes (TMA, 128-byte
+// swizzle), B = its share of the tokens x 256 bytes (two 128-byte swizzled
+// boxes) and E = the metadata, 128 rows x 32 bytes, by TMA as a 3-D box into
+// the no-swizzle canonical layout ([2][128][16] bytes) that tcgen05.cp copies
+// into tensor memory (lane = weight row; the 64 metadata bits of one MMA fill
+// two columns, nibble g at bits 4g).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -38,20 +28,12 @@
 
 namespace sbl {
 
-constexpr int kSpBM = 128;                       // weight rows per tile
-constexpr int kSpBN = 128;                       // tokens per tile
+constexpr int kSpBM = 128;                       // weight rows per CTA
 constexpr int kSpKLogical = 256;                 // logical K per stage
 constexpr int kSpABytes = kSpBM * 128;           // 128 compressed bytes per row
-constexpr int kSpBBoxBytes = kSpBN * 128;        // one 128-byte box of B
-constexpr int kSpBBytes = 2 * kSpBBoxBytes;      // 256 bytes per token row
 constexpr int kSpEBytes = kSpBM * 32;            // 32 metadata bytes per row
-constexpr int kSpStageBytes = kSpABytes + kSpBBytes + kSpEBytes;
-constexpr int kSpStages = 3;
-constexpr int kSpNumAcc = 3;
-constexpr int kSpMetaCol = kSpNumAcc * kSpBN;    // first metadata column (384)
 constexpr int kSpEpiBufBytes = 32 * 32 * 4;      // one 32 x 32 block, fp32 at most
 constexpr int kSpEpiBytes = kEpiWarps * kSpEpiBufBytes;
-constexpr int kSpSmemBytes = 1024 + kSpStages * kSpStageBytes + kSpEpiBytes + 256;
 
 struct Sp24Args {
     int32_t O, T, K;
@@ -64,288 +46,6 @@ struct Sp24Args {
     const float *d;            // [T]
     uint32_t *err;
 };
-
-__device__ __forceinline__ constexpr uint32_t sp24_idesc()
-{
-    // sparse (bit 2), selector 0, s32 accumulator (bits 4-5), s8 A and B
-    // (bits 7-9, 10-12), K-major A and B, N >> 3 (bits 17-22), M >> 4 (24-28)
-    return (1u << 2) | (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kSpBN >> 3) << 17) |
-           (static_cast<uint32_t>(kSpBM >> 4) << 24);
-}
-
-// D(tmem) (+)= A(smem, 2:4 compressed) * B(smem)^T with A's metadata in
-// tensor memory at e_tmem; int8 x int8 -> int32, 64 logical K.
-__device__ __forceinline__ void mma_sp_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
-                                          uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// 128 lanes x 256 bits from shared memory (no-swizzle canonical layout:
-// 8-row groups 128 bytes apart, the two 16-byte halves of a row 2048 bytes
-// apart) into tensor memory columns taddr .. taddr + 7.
-__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(2048u >> 4) << 16;  // leading byte offset: the two halves
-    d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: 8-row groups
-    d |= static_cast<uint64_t>(1u) << 46;          // descriptor version (sm_100)
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t c1,
-                                            int32_t c2, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
-        : "memory");
-}
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    sp24_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-                     Sp24Args args)
-{
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_addr(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t *base_ptr = smem_raw + (base - raw);
-    const uint32_t a_base = base;
-    const uint32_t b_base = a_base + kSpStages * kSpABytes;
-    const uint32_t e_base = b_base + kSpStages * kSpBBytes;
-    const uint32_t epi_base = e_base + kSpStages * kSpEBytes;
-    const uint32_t bar_base = epi_base + kSpEpiBytes;
-    auto full_bar = [&](int s) { return bar_base + 8u * s; };
-    auto empty_bar = [&](int s) { return bar_base + 8u * (kSpStages + s); };
-    auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * kSpStages + a); };
-    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kSpStages + kSpNumAcc + a); };
-    const uint32_t drain_bar = bar_base + 8u * (2 * kSpStages + 2 * kSpNumAcc);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (bar_base - base) + 224);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = args.tiles_m * args.tiles_n;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kSpStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
-        for (int a = 0; a < kSpNumAcc; ++a) {
-            mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), kEpiWarps * 32);
-        }
-        mbar_init(drain_bar, 1);
-        fence_barrier_init();
-        tma_prefetch_map(&tmA);
-        tma_prefetch_map(&tmB);
-        tma_prefetch_map(&tmE);
-        tma_prefetch_map(&tmY);
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
-        tmem_relinquish();
-        tc_fence_before();
-    }
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-    if (warp == 0) {
-        // ---------------------------------------------------- TMA producer
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        uint32_t issued_mask = 0;
-        uint32_t issued_phase[kSpStages];
-        for (int s = 0; s < kSpStages; ++s) issued_phase[s] = 0;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-            int tm, tn;
-            tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
-            for (int kb = 0; kb < args.k_blocks; ++kb) {
-                const bool ready = mbar_wait(empty_bar(stage), phase ^ 1u, args.err, kErrGemmProducer);
-                if (!__all_sync(0xffffffffu, ready)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    const uint32_t fb = full_bar(stage);
-                    mbar_arrive_expect_tx(fb, kSpStageBytes);
-                    // compressed values: 128 bytes = 256 logical K
-                    tma_load_2d(a_base + stage * kSpABytes, &tmA, kb * 128, tm * kSpBM, fb);
-                    // activations: two 128-byte boxes
-                    tma_load_2d(b_base + stage * kSpBBytes, &tmB, kb * kSpKLogical, tn * kSpBN, fb);
-                    tma_load_2d(b_base + stage * kSpBBytes + kSpBBoxBytes, &tmB, kb * kSpKLogical + 128,
-                                tn * kSpBN, fb);
-                    // metadata: 16-byte chunks 2kb and 2kb + 1 of 128 rows
-                    tma_load_3d(e_base + stage * kSpEBytes, &tmE, 0, tm * kSpBM, 2 * kb, fb);
-                }
-                __syncwarp();
-                issued_mask |= 1u << stage;
-                issued_phase[stage] = phase;
-                if (++stage == kSpStages) stage = 0, phase ^= 1u;
-            }
-        }
-        if (!ok) {
-            for (int s = 0; s < kSpStages; ++s)
-                if (issued_mask & (1u << s)) mbar_wait(full_bar(s), issued_phase[s], args.err, kErrGemmProducer);
-        }
-    } else if (warp == 1) {
-        // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = sp24_idesc();
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        int local = 0;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
-            const int acc = local % kSpNumAcc;
-            const uint32_t acc_phase = (local / kSpNumAcc) & 1;
-            const bool free_acc = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, args.err, kErrGemmMma);
-            if (!__all_sync(0xffffffffu, free_acc)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kSpBN);
-            for (int kb = 0; kb < args.k_blocks; ++kb) {
-                const bool ready = mbar_wait(full_bar(stage), phase, args.err, kErrGemmMma);
-                if (!__all_sync(0xffffffffu, ready)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(kSpMetaCol + 8 * stage);
-                    // metadata first: tcgen05.cp and tcgen05.mma from one
-                    // thread execute in issue order
-                    tmem_cp_128x256b(e_tmem, e_base + stage * kSpEBytes);
-                    const uint64_t adesc = smem_desc_k128(a_base + stage * kSpABytes);
-                    const uint32_t b_stage = b_base + stage * kSpBBytes;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // A: +32 compressed bytes per MMA (+2 in 16-byte units);
-                        // B: box j/2, +64 bytes for odd j; E: +2 columns
-                        const uint64_t bdesc = smem_desc_k128(b_stage + (j >> 1) * kSpBBoxBytes) +
-                                               static_cast<uint64_t>(4 * (j & 1));
-                        mma_sp_i8(d_tmem, adesc + static_cast<uint64_t>(2 * j), bdesc, e_tmem + 2u * j, idesc,
-                                  (kb | j) != 0);
-                    }
-                    tc_commit(empty_bar(stage));
-                }
-                __syncwarp();
-                if (++stage == kSpStages) stage = 0, phase ^= 1u;
-            }
-            if (!ok) break;
-            if (lane == 0) tc_commit(tfull_bar(acc));
-            __syncwarp();
-        }
-        if (lane == 0) tc_commit(drain_bar);
-        __syncwarp();
-        mbar_wait(drain_bar, 0, args.err, kErrGemmMma);
-        __syncwarp();
-    } else {
-        // ---------------------------------------------------- epilogue (warps 2-9)
-        const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const float g = *args.gamma;
-        const uint32_t buf = epi_base + static_cast<uint32_t>(warp - 2) * kSpEpiBufBytes;
-        int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            int tm, tn;
-            tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
-            const int acc = local % kSpNumAcc;
-            const uint32_t acc_phase = (local / kSpNumAcc) & 1;
-            const int o0 = tm * kSpBM + quarter * 32;  // first weight row of this warp's block
-            const int o = o0 + lane;
-            const int t_base = tn * kSpBN + half * 64;
-            // token scales of this warp's 64 columns, loaded while the MMAs run
-            float sc[2];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int t = t_base + 32 * c + lane;
-                sc[c] = t < args.T ? __fmul_rn(g, args.d[t]) : 0.0f;
-            }
-            const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
-            if (!__all_sync(0xffffffffu, ready)) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(acc * kSpBN + half * 64);
-            uint32_t v[2][32];
-            tmem_ld_32x32b_x32(t_row, v[0]);
-            tmem_ld_32x32b_x32(t_row + 32u, v[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(tempty_bar(acc));  // the accumulator is in registers
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int t0 = t_base + 32 * c;
-                if (t0 >= args.T || o0 >= args.O) continue;  // warp-uniform: block outside Y
-                if (args.acc_out && o < args.O) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (t0 + j < args.T)
-                            args.acc_out[static_cast<int64_t>(t0 + j) * args.O + o] = static_cast<int32_t>(v[c][j]);
-                }
-                // the previous store from this buffer has finished reading it
-                if (lane == 0) bulk_wait_group_read<0>();
-                __syncwarp();
-                if (args.out_fp32) {
-                    // row j of the block = token t0 + j, 32 fp32 weight rows
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float s = __shfl_sync(0xffffffffu, sc[c], j);
-                        const float y = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[c][j])), s);
-                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(buf + static_cast<uint32_t>(j * 128 + lane * 4)),
-                                     "f"(y)
-                                     : "memory");
-                    }
-                } else {
-                    // bf16: lanes 2i and 2i+1 swap one value so each writes a
-                    // word of two weight rows (even lane: token j, odd lane:
-                    // token j + 1)
-                    const bool odd = lane & 1;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const float s0 = __shfl_sync(0xffffffffu, sc[c], j);
-                        const float s1 = __shfl_sync(0xffffffffu, sc[c], j + 1);
-                        const float y0 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[c][j])), s0);
-                        const float y1 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[c][j + 1])), s1);
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? y0 : y1, 1);
-                        const __nv_bfloat162 b2 = odd ? __floats2bfloat162_rn(other, y1) : __floats2bfloat162_rn(y0, other);
-                        const int row = odd ? j + 1 : j;
-                        const uint32_t addr = buf + static_cast<uint32_t>(row * 64 + (lane & ~1) * 2);
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(*reinterpret_cast<const uint32_t *>(&b2))
-                                     : "memory");
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, buf, o0, t0);
-                    bulk_commit_group();
-                }
-            }
-        }
-        if (lane == 0) bulk_wait_group<0>();
-        __syncwarp();
-    }
-
-    __syncthreads();
-    if (warp == 1) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
-    }
-}
 
 // ------------------------------------------------------------ CTA pairs --
 // The same GEMM on CTA pairs (cta_group::2): a cluster of two CTAs computes a
