@@ -113,6 +113,8 @@ def parse():
                     help="store the mean DRAM bytes per roofline-kernel launch from an ncu --csv metric list "
                          "(dram__bytes_read.sum, dram__bytes_write.sum) for --workload, then exit")
     ap.add_argument("--traffic-command", default="", help="the ncu command that produced NCU_CSV (recorded)")
+    ap.add_argument("--ref-step-seconds", type=float, default=0.0,
+                    help="oracle time per reference-arm step (default: about 120 s over the whole run)")
     return ap.parse_args()
 
 
@@ -139,6 +141,29 @@ def algorithmic_ops(wk, tokens):
             if wk.mode == "train":
                 total += 4.0 * tokens * lin.d_out * lin.d_in
     return total
+
+
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(value: float, dist, world: int, device) -> float:
+    """The largest of every rank's value (a time): all ranks take part."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank processed
+    units_per_rank in at most max_ms (weak scaling)."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
+def barrier(dist, world: int):
+    if world > 1:
+        dist.barrier()
 
 
 # ------------------------------------------------------------------ clocks
@@ -437,13 +462,9 @@ def run_ours(args, wk):
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    total_ms = sum(times)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times), dist, world, device)
     ops_step = algorithmic_ops(wk, r.T)
-    value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(ops_step * args.steps, world, total_ms) / 1e12
     achieved = gemm_ops / (gemm_ms * 1e-3) / 1e12
     int8_peak = pk["bf16_tflops"] * 2.0  # int8 dense = 2 x bf16 dense (4.5 / 2.25 PFLOP/s nominal)
 
@@ -471,10 +492,8 @@ def run_ours(args, wk):
         r.step_e2e()
     e1.record()
     torch.cuda.synchronize()
-    e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e_value = ops_step * e_steps * world / (float(e_ms.item()) * 1e-3) / 1e12
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device)
+    e_value = whole_job_rate(ops_step * e_steps, world, e_ms) / 1e12
 
     err = sbl.sbl_device_error()
     cpu = None
@@ -531,6 +550,8 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
     launch streams its weights from HBM."""
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 128 << 20)
+    clocks = ClockSampler(str(getattr(props, "uuid", "")) or None)
+    clk = None
     results = {}
     n, m = wk.patterns[0]
     for T in wk.tokens:
@@ -574,37 +595,83 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
             for _ in range(max(3, args.warmup)):
                 g.replay()
             torch.cuda.synchronize()
+            barrier(dist, world)
+            if T == wk.tokens[-1] and mode == "gemv":
+                clocks.start()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             for _ in range(args.steps):
                 g.replay()
             e1.record()
             torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / args.steps
-            launches = sum(len(c) for _, _, c, *_ in layers)
+            if T == wk.tokens[-1] and mode == "gemv":
+                clk = clocks.stop()
+            ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / args.steps
+            launches = sum(len(c) * (2 if mode == "step" else 1) for _, _, c, *_ in layers)
             # algorithmic bytes: packed weights + the layer's input (int8 Xq for the
             # GEMV alone, bf16 X for the step) + bf16 Y + the token scales
             alg_bytes = sum(len(c) * (bw + T * lin.d_in * (1 if mode == "gemv" else 2) + T * lin.d_out * 2 + 4 * T)
                             for lin, _, c, _, _, _, _, bw in layers)
-            res[mode] = {"ms_per_graph": ms, "gemvs": launches, "gbs": alg_bytes / (ms * 1e-3) / 1e9}
+            res[mode] = {"ms_per_graph": ms, "launches": launches,
+                         "gbs": whole_job_rate(alg_bytes, world, ms) / 1e9}
+        # end to end through the public API: every step copies the tokens'
+        # activations in from pinned host memory and the outputs back
+        hx = [torch.empty(x.shape, dtype=torch.bfloat16).pin_memory() for _, _, _, x, *_ in layers]
+        hy = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for *_, y, _ in layers]
+        for h, (_, _, _, x, *_) in zip(hx, layers):
+            h.copy_(x)
+        e_steps = max(2, min(args.steps, 10))
+        barrier(dist, world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e_steps):
+            for (lin, dsc, copies, x, q, d, y, _), h_in, h_out in zip(layers, hx, hy):
+                x.copy_(h_in, non_blocking=True)
+                sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
+                sbl.sbl_forward(dsc, q, d, T, copies[0], sbl.SBL_FMT_PK2, y)
+                h_out.copy_(y, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / e_steps
+        e_bytes = sum(bw + T * lin.d_in * 2 + T * lin.d_out * 2 + 4 * T for lin, _, _, _, _, _, _, bw in layers)
+        res["e2e"] = {"ms_per_step": e_ms, "gbs": whole_job_rate(e_bytes, world, e_ms) / 1e9,
+                      "h2d_bytes_per_step": sum(h.numel() * 2 for h in hx),
+                      "d2h_bytes_per_step": sum(h.numel() * 2 for h in hy)}
         results[T] = res
     Tm = wk.tokens[-1]
     value = statistics.mean(results[T]["step"]["gbs"] for T in wk.tokens)
     gemv = results[Tm]["gemv"]["gbs"]
+    e2e = statistics.mean(results[T]["e2e"]["gbs"] for T in wk.tokens)
+    err = sbl.sbl_device_error()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_decode(wk)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(results[Tm]["step"]["ms_per_graph"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "2-bit ternary x int8 -> int32",
-        "data": "synthetic", "config": {"workload": wk.name, "tokens": wk.tokens,
-                                        "per_token_count": {str(T): results[T] for T in wk.tokens},
-                                        "l2": "rotating weight copies > 4x L2 inside one CUDA graph"},
+        "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32 packed once to 2:4 PK2, X~N(0,1) bf16)",
+        "config": {"workload": wk.name, "tokens": wk.tokens,
+                   "step": "per token count: act quant + GEMV of each linear, over rotating weight copies",
+                   "per_token_count": {str(T): results[T] for T in wk.tokens},
+                   "l2": "inputs larger than L2: rotating weight copies > 4x L2 inside one CUDA graph",
+                   "parallelism": f"independent replicas x{world}"},
         "roofline": {"kernel": "decode_kernel (PK2 stream, mma.sync u8 x s8)", "bound": "hbm", "achieved": round(gemv, 1),
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gemv / pk["hbm_gbs"], 4),
                      "traffic": stored_traffic(wk.name),
                      "traffic_note": "mean DRAM read+write bytes per decode launch (ncu capture in "
                                      "profiles/roofline_traffic.json; null when absent or stale)"},
-        "gpu_launches": None,
+        "e2e": {"value": round(e2e, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": results[Tm]["e2e"]["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": results[Tm]["e2e"]["d2h_bytes_per_step"]},
+        "gpu_launches": sum(results[T]["step"]["launches"] for T in wk.tokens) * args.steps,
+        "clocks": clk,
+        "device_error": err,
     }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if world > 1:
+        dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -641,26 +708,51 @@ def cpu_baseline(wk, budget_s=12.0):
                       f"pack {t_pack:.2f}s, forward {t_fwd:.2f}s"}
 
 
+def cpu_baseline_decode(wk, budget_s=10.0):
+    """The oracle's GEMV (GEMM + dequantisation from W_eff, T tokens of the
+    first linear) timed on one host core, in the decode metric's unit:
+    algorithmic bytes (2-bit weights + bf16 X + bf16 Y + scales) per second."""
+    import oracle
+    lin = wk.linears[0]
+    n, m = wk.patterns[0]
+    T = wk.tokens[-1]
+    layer = oracle.Layer(wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed), n, m)
+    x = wl.activations(T, lin.d_in, seed=wk.seed)
+    reps, t = 0, 0.0
+    t0 = time.perf_counter()
+    while t < budget_s and reps < 1000:
+        layer.forward(x)
+        reps += 1
+        t = time.perf_counter() - t0
+    alg = lin.d_out * lin.d_in / 4 + T * lin.d_in * 2 + T * lin.d_out * 2 + 4 * T
+    return {"value": alg * reps / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{lin.name} {lin.d_in}->{lin.d_out} at {n}:{m}, T={T}: {reps} GEMVs "
+                      f"(act quant + GEMM + dequant from W_eff) in {t:.1f}s"}
+
+
 def run_reference(args, wk):
-    """The oracle arm: the plain-C oracle timed on the host cores."""
+    """The oracle arm: the plain-C oracle timed on the host cores, in our
+    arm's metric and unit (TOPS, or GB/s for decode).  Under torchrun rank 0
+    alone runs and prints; the other ranks exit without work."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    budget = args.ref_step_seconds or max(2.0, 120.0 / max(1, args.steps + args.warmup))
     res = []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(wk, budget_s=budget)
+        r = cpu_baseline_decode(wk, budget) if wk.mode == "decode" else cpu_baseline(wk, budget_s=budget)
         if i >= args.warmup:
             res.append(r)
     value = statistics.mean(r["value"] for r in res)
+    unit = res[-1]["unit"]
     line = {
-        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8 x ternary -> int64 (plain C)", "data": "synthetic",
         "config": {"workload": wk.name}, "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": res[-1]["sample"]},
-        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": res[-1]["sample"]},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
