@@ -48,6 +48,11 @@ def _load():
         lib.sbl_oracle_sp24_meta_row_bytes.argtypes = [i64]
         lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
         lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
+        lib.sbl_oracle_mask_flips.restype = i64
+        lib.sbl_oracle_mask_flips.argtypes = [p, p, i64]
+        lib.sbl_oracle_near_zero.restype = i64
+        lib.sbl_oracle_near_zero.argtypes = [p, i64, f32]
+        lib.sbl_oracle_block_threshold.argtypes = [p, p, i64, i64, i32, p]
         lib.sbl_oracle_quantize_act.argtypes = [p, i64, i64, p, p]
         lib.sbl_oracle_gemm_acc.restype = i32
         lib.sbl_oracle_gemm_acc.argtypes = [p, p, i64, i64, i64, p]
@@ -190,6 +195,27 @@ def pack_sp24(weff, mask):
     if _load().sbl_oracle_pack_sp24(_ptr(weff), _ptr(mask), d_out, d_in, _ptr(vals), _ptr(meta)) != 0:
         raise ValueError("mask keeps more than two positions in a group of four")
     return vals, meta
+
+
+def mask_flips(mask_prev, mask) -> int:
+    a = np.ascontiguousarray(mask_prev, dtype=np.uint8)
+    b = np.ascontiguousarray(mask, dtype=np.uint8)
+    assert a.shape == b.shape
+    return int(_load().sbl_oracle_mask_flips(_ptr(a), _ptr(b), a.size))
+
+
+def near_zero(w, g) -> int:
+    w = _f32(w)
+    return int(_load().sbl_oracle_near_zero(_ptr(w), w.size, float(g)))
+
+
+def block_threshold(w, mask, m: int) -> np.ndarray:
+    w = _f32(w)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    d_out, d_in = w.shape
+    t = np.empty((d_out, d_in // m), dtype=np.float32)
+    _load().sbl_oracle_block_threshold(_ptr(w), _ptr(mask), d_out, d_in, m, _ptr(t))
+    return t
 
 
 def quantize_act(x_bf16_bits):

@@ -233,6 +233,56 @@ int sbl_oracle_pack_sp24(const int8_t *weff, const uint8_t *mask, int64_t d_out,
     return 0;
 }
 
+/* ------------------------------------------------------ mask statistics -- */
+
+/* Mask flip count between consecutive steps ([P1] "Dynamic Mask
+ * Recomputation at Every Training Step": the flip rate r_t measures how
+ * many mask positions change from one step to the next; r_t = flips / count
+ * is the rate).  Masks are one byte per position (0 or 1). */
+int64_t sbl_oracle_mask_flips(const uint8_t *mask_prev, const uint8_t *mask, int64_t count)
+{
+    int64_t flips = 0;
+    for (int64_t i = 0; i < count; ++i)
+        if ((mask_prev[i] != 0) != (mask[i] != 0)) flips++;
+    return flips;
+}
+
+/* Near-zero mass ([P1] "Polarization analysis": the fraction of weights
+ * whose normalized magnitude |W| / gamma falls below 0.5), as a count:
+ * #{ fl32(|w| / gamma) < 0.5 }; every weight counts when gamma == 0 (all
+ * weights are then 0 and quantise to 0). */
+int64_t sbl_oracle_near_zero(const float *w, int64_t count, float gamma)
+{
+    if (!(gamma > 0.0f)) return count;
+    int64_t c = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        float r = fabsf(w[i]) / gamma;
+        if (r < 0.5f) c++;
+    }
+    return c;
+}
+
+/* Per-block pruning threshold ([P1] "Magnitude stratification": the
+ * magnitude of the (N+1)-th largest weight in each block of M): for row o
+ * and group g, the largest |W| among the group's positions the mask drops,
+ * which is the (n+1)-th largest |W| of the group; 0 when n == m (nothing is
+ * dropped).  Output fp32 [d_out, d_in / m]. */
+void sbl_oracle_block_threshold(const float *w, const uint8_t *mask, int64_t d_out, int64_t d_in,
+                                int m, float *t)
+{
+    for (int64_t o = 0; o < d_out; ++o)
+        for (int64_t g = 0; g < d_in / m; ++g) {
+            float best = 0.0f;
+            for (int i = 0; i < m; ++i) {
+                int64_t k = o * d_in + g * m + i;
+                if (mask[k]) continue;
+                float a = fabsf(w[k]);
+                if (a > best) best = a;
+            }
+            t[o * (d_in / m) + g] = best;
+        }
+}
+
 /* ------------------------------------------------- activation quantiser -- */
 
 static float bf16_to_f32(uint16_t b)

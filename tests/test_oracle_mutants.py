@@ -30,6 +30,11 @@ MUTANTS = {
     "sp24_nibble_fields_swapped": ("unsigned nib = (unsigned)idx[0] | ((unsigned)idx[1] << 2);",
                                    "unsigned nib = (unsigned)idx[1] | ((unsigned)idx[0] << 2);"),
     "sp24_high_nibble_first": ("(nib << (4 * (g % 2)))", "(nib << (4 * (1 - g % 2)))"),
+    "flips_count_agreements": ("if ((mask_prev[i] != 0) != (mask[i] != 0)) flips++;",
+                               "if ((mask_prev[i] != 0) == (mask[i] != 0)) flips++;"),
+    "near_zero_inclusive": ("if (r < 0.5f) c++;", "if (r <= 0.5f) c++;"),
+    "threshold_from_kept": ("if (mask[k]) continue;\n                float a = fabsf(w[k]);",
+                            "if (!mask[k]) continue;\n                float a = fabsf(w[k]);"),
     "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
                            "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
 }
@@ -51,6 +56,9 @@ PIN_CALLS = [
     (pins.test_sp24_hand_example, ()),
     (pins.test_sp24_roundtrip, (2, 4)),
     (pins.test_sp24_roundtrip, (1, 4)),
+    (pins.test_mask_flips_matches_numpy_and_invariants, ()),
+    (pins.test_near_zero_matches_numpy_and_gaussian_closed_form, ()),
+    (pins.test_block_threshold_brute_force_and_hand_row, ()),
 ]
 
 

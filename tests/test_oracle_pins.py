@@ -309,6 +309,63 @@ def test_sp24_rejects_masks_that_are_not_2of4():
         oracle.pack_sp24(layer.weff, layer.mask)
 
 
+# ----------------------------------------------------------- mask statistics
+
+def test_mask_flips_matches_numpy_and_invariants():
+    """Flip count between consecutive masks ("Dynamic Mask Recomputation":
+    how many positions change): numpy's != count; 0 for equal masks; every
+    position for complementary masks."""
+    w0 = wl.master_weights(32, 128, seed=1)
+    w1 = w0 + 0.01 * wl.master_weights(32, 128, seed=2)  # a small update moves some positions
+    m0 = oracle.nm_mask(w0, 6, 8)
+    m1 = oracle.nm_mask(w1, 6, 8)
+    f = oracle.mask_flips(m0, m1)
+    assert f == int((m0 != m1).sum()) and 0 < f < m0.size
+    assert f % 2 == 0  # exactly n per group: every drop is matched by an entry
+    assert oracle.mask_flips(m0, m0) == 0
+    assert oracle.mask_flips(m0, 1 - m0) == m0.size
+
+
+def test_near_zero_matches_numpy_and_gaussian_closed_form():
+    """Near-zero mass ("Polarization analysis": |W|/gamma below 0.5) as a
+    count: numpy float32 division; for W ~ N(0, s) the fraction tends to
+    2 Phi(0.5 sqrt(2/pi)) - 1 = 0.3101 (gamma -> s sqrt(2/pi)); every weight
+    counts when gamma == 0."""
+    w = wl.master_weights(2048, 2048, seed=7)
+    g = oracle.gamma(w)
+    c = oracle.near_zero(w, g)
+    assert c == int((np.abs(w) / np.float32(g) < np.float32(0.5)).sum())
+    frac = c / w.size
+    expect = math.erf(0.5 * math.sqrt(2 / math.pi) / math.sqrt(2))
+    assert abs(frac - expect) < 1.5e-3, (frac, expect)
+    assert oracle.near_zero(np.zeros((4, 16), np.float32), 0.0) == 64
+    # exactly 0.5 gamma is not below 0.5; the next float down is
+    w2 = np.array([[0.5, np.nextafter(np.float32(0.5), np.float32(0)), 1.0, 0.25] * 4], dtype=np.float32)
+    assert oracle.near_zero(w2, 1.0) == 8
+
+
+def test_block_threshold_brute_force_and_hand_row():
+    """Per-block threshold ("Magnitude stratification": the (N+1)-th largest
+    |W| of each block): the golden 1x8 row at 6:8 drops 0.05 and 0.0, so
+    t = 0.05; brute force by sorting on tie-heavy groups; 0 when n == m;
+    never above a kept magnitude."""
+    row = np.array([[0.9, -0.1, 0.5, -0.7, 0.05, 0.3, -0.2, 0.0] + [0.0] * 8], dtype=np.float32)
+    mask = oracle.nm_mask(row, 6, 8)
+    assert oracle.block_threshold(row, mask, 8)[0, 0] == np.float32(0.05)
+    rng = np.random.default_rng(5)
+    for n, m in [(6, 8), (2, 4), (5, 8), (1, 4), (3, 8)]:
+        w = (rng.integers(-3, 4, size=(16, 64)) * 0.25).astype(np.float32)
+        mask = oracle.nm_mask(w, n, m)
+        t = oracle.block_threshold(w, mask, m)
+        a = np.abs(w).reshape(16, 64 // m, m)
+        expect = -np.sort(-a, axis=-1)[..., n]
+        np.testing.assert_array_equal(t, expect)
+        kept_min = np.where(mask.reshape(a.shape) == 1, a, np.inf).min(axis=-1)
+        assert (t <= kept_min).all()
+    w = wl.master_weights(8, 32, seed=3)
+    assert not oracle.block_threshold(w, oracle.nm_mask(w, 8, 8), 8).any()
+
+
 # ------------------------------------------------------------ activation quant
 
 def test_act_quant_invariants_and_zero_row():
