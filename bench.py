@@ -256,6 +256,16 @@ class Runner:
                 L["dx"] = torch.empty((T, lin.d_in), dtype=torch.bfloat16, device=device)
                 L["dw"] = torch.empty((lin.d_out, lin.d_in), dtype=torch.float32, device=device)
                 L["bws"] = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc0, T, sbl.SBL_OP_BACKWARD))
+                # re-mask statistics of every training step: this step's keep
+                # bitmap against the previous step's, near-zero count, thresholds
+                rb = sbl.keep_bitmap_bytes(dsc0)
+                n0, m0 = wk.patterns[0]
+                L["stats"] = {"prev": torch.zeros((lin.d_out, rb), dtype=torch.uint8, device=device),
+                              "keep": torch.zeros((lin.d_out, rb), dtype=torch.uint8, device=device),
+                              "flips": torch.zeros((1,), dtype=torch.int64, device=device),
+                              "near_zero": torch.zeros((1,), dtype=torch.int64, device=device),
+                              "threshold": torch.empty((lin.d_out, lin.d_in // m0), dtype=torch.float32,
+                                                       device=device)}
         self.choose_forward_formats()
         self.launches_per_step = 0
         n_side = max(len(self.layers), 1)
@@ -277,6 +287,22 @@ class Runner:
                 self.pack_fmts[(li, (n, m))] = self.fmts if fmt == sbl.SBL_FMT_I8 else fmt
                 if fmt != sbl.SBL_FMT_I8:
                     L["packed"][(n, m)] = (dsc, sbl.alloc_packed(dsc, fmt))
+
+    def stats_summary(self):
+        """The last step's re-mask statistics per linear (read after timing):
+        mask flip rate r_t against the step before, near-zero fraction, and
+        the mean per-group threshold over gamma."""
+        out = {}
+        for L in self.layers:
+            st = L["stats"]
+            lin = L["lin"]
+            count = lin.d_out * lin.d_in
+            dsc, p = L["packed"][self.wk.patterns[0]]
+            g = float(p.gamma[0].item())
+            out[lin.name] = {"flip_rate": int(st["flips"].item()) / count,
+                             "near_zero_fraction": int(st["near_zero"].item()) / count,
+                             "mean_threshold_over_gamma": float(st["threshold"].mean().item()) / g if g else None}
+        return out
 
     def formats_used(self):
         names = {self.sbl.SBL_FMT_I8: "I8 (dense MMA)", self.sbl.SBL_FMT_SP24: "SP24 (2:4 sparse MMA)"}
@@ -302,7 +328,16 @@ class Runner:
             for li, L in enumerate(self.layers):
                 with torch.cuda.stream(side[li % len(side)]):
                     dsc, p = L["packed"][(n, m)]
-                    sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)])
+                    if "stats" in L:
+                        st = L["stats"]
+                        sbl.sbl_quantize_mask_pack_stats(dsc, L["w"], self.pack_fmts[(li, (n, m))], p,
+                                                         L["ws"][(n, m)], prev_keep=st["prev"], keep=st["keep"],
+                                                         flips=st["flips"], near_zero=st["near_zero"],
+                                                         block_threshold=st["threshold"])
+                        st["prev"].copy_(st["keep"])  # the next step compares with this one
+                    else:
+                        sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p,
+                                                   L["ws"][(n, m)])
                 launches += 2 + (1 if self.fmts & sbl.SBL_FMT_BF16T else 0)
             for ii, inp in enumerate(self.inputs):
                 with torch.cuda.stream(side[(len(self.layers) + ii) % len(side)]):
@@ -374,7 +409,14 @@ class Runner:
                 inp["x"].copy_(hx, non_blocking=True)
             for li, L in enumerate(self.layers):
                 dsc, p = L["packed"][(n, m)]
-                sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)])
+                if "stats" in L:
+                    st = L["stats"]
+                    sbl.sbl_quantize_mask_pack_stats(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)],
+                                                     prev_keep=st["prev"], keep=st["keep"], flips=st["flips"],
+                                                     near_zero=st["near_zero"], block_threshold=st["threshold"])
+                    st["prev"].copy_(st["keep"])
+                else:
+                    sbl.sbl_quantize_mask_pack(dsc, L["w"], self.pack_fmts[(li, (n, m))], p, L["ws"][(n, m)])
             for inp in self.inputs:
                 sbl.sbl_quantize_act(inp["x"], self.T, inp["x"].shape[1], inp["q"][(n, m)], inp["d"][(n, m)])
             for li, (L, hy) in enumerate(zip(self.layers, self.h_y)):
@@ -512,7 +554,8 @@ def run_ours(args, wk):
                    "l2": "flushed between timed steps (512 MiB write outside the events)",
                    "parallelism": f"independent replicas x{world}",
                    "dense_equivalent_tops": round(value * dense_factor(wk), 3),
-                   "forward_formats": r.formats_used()},
+                   "forward_formats": r.formats_used(),
+                   **({"remask_statistics": r.stats_summary()} if wk.mode == "train" else {})},
         "roofline": {"kernel": gemm_kernel_names(r, sbl), "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": round(int8_peak, 1), "unit": "TOPS",
                      "frac": round(achieved / int8_peak, 4),

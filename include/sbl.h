@@ -148,6 +148,43 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W,
                                   void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* By-products of the re-mask step, each optional (NULL to skip), computed
+ * by the packing kernel from the values it already holds:
+ *  keep            this step's keep mask M as a bitmap, bit k%8 of byte k/8 of
+ *                  a row of round_up(K/8, 16) bytes ([O, that] uint8; the
+ *                  same layout as the SBL_FMT_NM bitmap, padding bits 0);
+ *  prev_keep       the previous step's bitmap in that layout (input; needed
+ *                  by flips);
+ *  flips           device uint64: the number of positions whose keep bit
+ *                  differs from prev_keep -- the mask flip count; the flip
+ *                  rate r_t of the Sparse-BitNet summary ("Dynamic Mask
+ *                  Recomputation at Every Training Step") is flips / (O K);
+ *  near_zero       device uint64: #{ w : fl32(|w| / gamma) < 0.5 } (all O K
+ *                  when gamma == 0) -- the near-zero mass of "Polarization
+ *                  analysis" times O K;
+ *  block_threshold fp32 [O, K/m]: per group, the magnitude of the (n+1)-th
+ *                  largest |w| (the largest |w| the mask drops; 0 when
+ *                  n == m) -- the per-block pruning threshold t of
+ *                  "Magnitude stratification".
+ * Counters are overwritten (not accumulated).  Alignment: 16 bytes for the
+ * arrays, 8 for the counters. */
+typedef struct {
+    const uint8_t *prev_keep;
+    uint8_t *keep;
+    unsigned long long *flips;
+    unsigned long long *near_zero;
+    float *block_threshold;
+} sbl_mask_stats;
+
+/* sbl_quantize_mask_pack plus the statistics requested in `stats` (NULL or
+ * all-NULL members: exactly sbl_quantize_mask_pack).  flips without
+ * prev_keep is SBL_ERR_INVALID_ARG.  formats may be 0 when only statistics
+ * are wanted. */
+sbl_status sbl_quantize_mask_pack_stats(const sbl_layer_desc *desc, const float *W,
+                                        uint32_t formats, const sbl_packed *out,
+                                        const sbl_mask_stats *stats, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
 /* Same result as sbl_quantize_mask_pack, but the caller passes no workspace
  * and the library allocates nothing.  The paper has no counterpart; this
  * entry point exists for callers that cannot obtain device memory at the

@@ -315,6 +315,15 @@ namespace {
 constexpr int kDecGroupsSmallT = 1;
 constexpr int kDecGroupsLargeT = 1;
 
+template <int M>
+cudaError_t launch_pack(const cudaLaunchConfig_t &cfg, const PackArgs &pa, bool sp24, bool stats)
+{
+    if (stats) return sp24 ? cudaLaunchKernelEx(&cfg, pack_kernel<M, true, true>, pa)
+                           : cudaLaunchKernelEx(&cfg, pack_kernel<M, false, true>, pa);
+    return sp24 ? cudaLaunchKernelEx(&cfg, pack_kernel<M, true, false>, pa)
+                : cudaLaunchKernelEx(&cfg, pack_kernel<M, false, false>, pa);
+}
+
 // cpw: chunks per warp per round, 1, 2, 4 or 8 (at most 4 with two row
 // groups, whose 512 threads get at most 128 registers each).
 template <int NT, int RG>
@@ -383,9 +392,12 @@ size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op
     return 0;
 }
 
-sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, uint32_t formats,
-                                  const sbl_packed *out, void *workspace, size_t workspace_bytes,
-                                  void *stream_p)
+}  // extern "C"
+
+// sbl_quantize_mask_pack with optional re-mask statistics (stats may be null).
+static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const float *W, uint32_t formats,
+                                          const sbl_packed *out, const sbl_mask_stats *stats, void *workspace,
+                                          size_t workspace_bytes, void *stream_p)
 {
     sbl_status st = check_desc(desc);
     if (st != SBL_OK) return st;
@@ -409,6 +421,14 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         ((formats & SBL_FMT_I8) && !aligned16(out->i8)) ||
         ((formats & SBL_FMT_BF16T) && !aligned16(out->bf16t)))
         return SBL_ERR_ALIGNMENT;
+    if (stats) {
+        if (stats->flips && !stats->prev_keep) return SBL_ERR_INVALID_ARG;  // nothing to compare with
+        if ((stats->prev_keep && !aligned16(stats->prev_keep)) || (stats->keep && !aligned16(stats->keep)) ||
+            (stats->flips && (reinterpret_cast<uintptr_t>(stats->flips) & 7u)) ||
+            (stats->near_zero && (reinterpret_cast<uintptr_t>(stats->near_zero) & 7u)) ||
+            (stats->block_threshold && !aligned16(stats->block_threshold)))
+            return SBL_ERR_ALIGNMENT;
+    }
     if (!workspace || workspace_bytes < sbl_workspace_bytes(desc, 0, SBL_OP_QUANTIZE_MASK_PACK))
         return SBL_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
@@ -420,6 +440,28 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
     const int64_t count = static_cast<int64_t>(O) * K;
     GammaWorkspace *ws = static_cast<GammaWorkspace *>(workspace);
     if (cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+    if (formats & SBL_FMT_NM) {
+        // presets the packing kernel edits in place (set before gamma_kernel,
+        // so the packing kernel follows gamma_kernel directly: a memset in
+        // between would break its programmatic dependent launch)
+        if (cudaMemsetAsync(out->nm_values, 0x55,
+                            static_cast<size_t>(O) * sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_MAIN),
+                            stream) != cudaSuccess ||
+            cudaMemsetAsync(out->nm_bitmap, 0,
+                            static_cast<size_t>(O) * sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP),
+                            stream) != cudaSuccess)
+            return SBL_ERR_CUDA;
+    }
+    if (stats) {
+        // before gamma_kernel, for the same reason
+        if ((stats->flips && cudaMemsetAsync(stats->flips, 0, sizeof(unsigned long long), stream) != cudaSuccess) ||
+            (stats->near_zero &&
+             cudaMemsetAsync(stats->near_zero, 0, sizeof(unsigned long long), stream) != cudaSuccess))
+            return SBL_ERR_CUDA;
+        if (stats->keep && round_up(K / 8, 16) > K / 8 &&
+            cudaMemsetAsync(stats->keep, 0, static_cast<size_t>(O) * round_up(K / 8, 16), stream) != cudaSuccess)
+            return SBL_ERR_CUDA;  // row padding of the bitmap reads 0
+    }
 
     const int gblocks = static_cast<int>((count + kGammaBlock - 1) / kGammaBlock);
     gamma_kernel<<<gblocks, 256, 0, stream>>>(W, count, ws, out->gamma);
@@ -445,11 +487,6 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         pa.out.nm_bitmap = out->nm_bitmap;
         pa.out.nm_bitmap_stride =
             static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP));
-        if (cudaMemsetAsync(pa.out.nm_values, 0x55, static_cast<size_t>(O) * pa.out.nm_values_stride,
-                            stream) != cudaSuccess ||
-            cudaMemsetAsync(pa.out.nm_bitmap, 0, static_cast<size_t>(O) * pa.out.nm_bitmap_stride, stream) !=
-                cudaSuccess)
-            return SBL_ERR_CUDA;
     }
     if (formats & SBL_FMT_SP24) {
         pa.out.sp24_values = out->sp24_values;
@@ -457,7 +494,16 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         pa.out.sp24_meta = out->sp24_meta;
         pa.out.sp24_meta_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_SP24, SBL_BUF_SP24_META));
     }
-    if (formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM | SBL_FMT_SP24)) {
+    const bool want_stats = stats && (stats->keep || stats->flips || stats->near_zero || stats->block_threshold);
+    if (want_stats) {
+        pa.stats.prev_keep = stats->prev_keep;
+        pa.stats.keep = stats->keep;
+        pa.stats.keep_stride = static_cast<int64_t>(round_up(K / 8, 16));
+        pa.stats.flips = stats->flips;
+        pa.stats.near_zero = stats->near_zero;
+        pa.stats.threshold = stats->block_threshold;
+    }
+    if ((formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM | SBL_FMT_SP24)) || want_stats) {
         // programmatic dependent launch behind gamma_kernel (see pack_kernel);
         // a thread covers 16 weights
         const int64_t per_cta = 256 * 16 / desc->m;  // groups per CTA
@@ -473,10 +519,8 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const bool sp = (formats & SBL_FMT_SP24) != 0;
-        const cudaError_t e = (desc->m == 8) ? (sp ? cudaLaunchKernelEx(&cfg, pack_kernel<8, true>, pa)
-                                                   : cudaLaunchKernelEx(&cfg, pack_kernel<8, false>, pa))
-                                             : (sp ? cudaLaunchKernelEx(&cfg, pack_kernel<4, true>, pa)
-                                                   : cudaLaunchKernelEx(&cfg, pack_kernel<4, false>, pa));
+        const cudaError_t e = desc->m == 8 ? launch_pack<8>(cfg, pa, sp, want_stats)
+                                           : launch_pack<4>(cfg, pa, sp, want_stats);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         if ((st = launch_status()) != SBL_OK) return st;
     }
@@ -486,6 +530,22 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
         if ((st = launch_status()) != SBL_OK) return st;
     }
     return SBL_OK;
+}
+
+extern "C" {
+
+sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, uint32_t formats,
+                                  const sbl_packed *out, void *workspace, size_t workspace_bytes,
+                                  void *stream_p)
+{
+    return quantize_mask_pack_impl(desc, W, formats, out, nullptr, workspace, workspace_bytes, stream_p);
+}
+
+sbl_status sbl_quantize_mask_pack_stats(const sbl_layer_desc *desc, const float *W, uint32_t formats,
+                                        const sbl_packed *out, const sbl_mask_stats *stats, void *workspace,
+                                        size_t workspace_bytes, void *stream_p)
+{
+    return quantize_mask_pack_impl(desc, W, formats, out, stats, workspace, workspace_bytes, stream_p);
 }
 
 sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq, float *d, void *stream_p)

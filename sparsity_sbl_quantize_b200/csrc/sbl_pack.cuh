@@ -53,6 +53,17 @@ struct PackOut {
     int64_t sp24_meta_stride;
 };
 
+// By-product statistics of the re-mask step (all optional; the counters are
+// zeroed by the host before the launch).
+struct PackStats {
+    const uint8_t *prev_keep;        // keep bitmap of the previous step (bit k%8 of byte k/8)
+    uint8_t *keep;                   // this step's keep bitmap, same layout
+    int64_t keep_stride;             // bytes per bitmap row
+    unsigned long long *flips;       // positions whose keep bit changed
+    unsigned long long *near_zero;   // weights with fl32(|w| / gamma) < 0.5
+    float *threshold;                // [rows, cols / M] largest dropped |w| per group
+};
+
 struct PackArgs {
     const float *W;
     int32_t rows, cols, n;
@@ -60,7 +71,19 @@ struct PackArgs {
     uint64_t inv_cols;     // ceil(2^64 / cols): row = umul64hi(e, inv_cols) exactly for e < 2^28
     const float *gamma;    // written by gamma_kernel
     PackOut out;
+    PackStats stats;
 };
+
+// fl32(|w| / gamma) < 0.5 exactly when |w| < gamma * (0.5 - 2^-26) (the
+// quotients that round to a float below 0.5; the midpoint 0.5 - 2^-26 rounds
+// to the even 0.5), and that product is exact in fp64: |w| is below it
+// exactly when it is below the first fp32 at or above it.  Every weight
+// counts when gamma == 0.
+__device__ __forceinline__ uint32_t near_zero_bound_bits(float gamma)
+{
+    if (!(gamma > 0.0f)) return 0x7f800000u;  // +inf: every finite |w| is below
+    return __float_as_uint(__double2float_ru(static_cast<double>(gamma) * (0.5 - 0x1p-26)));
+}
 
 // gamma: one CTA per tree node of kGammaBlock weights.  Warp w owns the 1024
 // consecutive weights [node*8192 + 1024w, +1024) as eight 128-weight chunks;
@@ -292,6 +315,94 @@ __device__ __forceinline__ void store_group(const PackArgs &a, int32_t row, int3
     }
 }
 
+// The re-mask statistics of one thread's 16 weights, in two parts: the
+// small per-thread results are computed from the weights first (so the
+// weights' registers are freed by the format stores), then stored and the
+// counts reduced over the warp, then the CTA, and added to the counters with
+// one atomic each (every thread of the CTA takes part in that second part).
+template <int M>
+struct ThreadStats {
+    uint32_t keep16, flips, nz;
+    uint32_t drop_max[16 / M];  // largest dropped |w| (as bits) per group
+};
+
+template <int M>
+__device__ __forceinline__ ThreadStats<M> stats_of(const PackArgs &a, const uint32_t (&bits)[16 / M][M],
+                                                   const uint32_t (&keep)[16 / M], uint32_t prev16)
+{
+    constexpr int kBatch = 16 / M;
+    ThreadStats<M> r;
+    r.keep16 = 0;
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) r.keep16 |= keep[b] << (b * M);
+    r.flips = a.stats.prev_keep ? static_cast<uint32_t>(__popc((r.keep16 ^ prev16) & 0xffffu)) : 0u;
+    r.nz = 0;
+    if (a.stats.near_zero) {
+        const uint32_t bound = near_zero_bound_bits(*a.gamma);
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+            for (int i = 0; i < M; ++i) r.nz += ((bits[b][i] & 0x7fffffffu) < bound) ? 1u : 0u;
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+        uint32_t dm = 0u;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const uint32_t key = bits[b][i] & 0x7fffffffu;
+            if (!((keep[b] >> i) & 1u) && key > dm) dm = key;
+        }
+        r.drop_max[b] = dm;
+    }
+    return r;
+}
+
+template <int M>
+__device__ __forceinline__ void stats_finish(const PackArgs &a, bool active, int64_t e0, const ThreadStats<M> &r)
+{
+    uint32_t flips = 0, nz = 0;
+    if (active) {
+        const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
+        const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);
+        if (a.stats.keep)
+            *reinterpret_cast<uint16_t *>(a.stats.keep + static_cast<int64_t>(row) * a.stats.keep_stride + col0 / 8) =
+                static_cast<uint16_t>(r.keep16);
+        if (a.stats.threshold) {
+            float *t = a.stats.threshold + static_cast<int64_t>(row) * (a.cols / M) + col0 / M;
+            if constexpr (M == 8) {
+                *reinterpret_cast<uint2 *>(t) = make_uint2(r.drop_max[0], r.drop_max[1]);
+            } else {
+                *reinterpret_cast<uint4 *>(t) = make_uint4(r.drop_max[0], r.drop_max[1], r.drop_max[2], r.drop_max[3]);
+            }
+        }
+        flips = r.flips;
+        nz = r.nz;
+    }
+    if (!a.stats.flips && !a.stats.near_zero) return;  // uniform over the grid
+    __shared__ uint32_t red[2][8];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        flips += __shfl_xor_sync(0xffffffffu, flips, off);
+        nz += __shfl_xor_sync(0xffffffffu, nz, off);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[0][warp] = flips;
+        red[1][warp] = nz;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long f = 0, z = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            f += red[0][w];
+            z += red[1][w];
+        }
+        if (a.stats.flips && f) atomicAdd(a.stats.flips, f);
+        if (a.stats.near_zero && z) atomicAdd(a.stats.near_zero, z);
+    }
+}
+
 // SP24 form of four-group q of a thread's 16 weights: the group's kept
 // positions (at most two) completed with its smallest positions not kept,
 // i0 < i1; values W_eff[i0], W_eff[i1] go to value bytes 2q, 2q+1 and the
@@ -315,34 +426,12 @@ __device__ __forceinline__ void sp24_group(uint32_t wbytes, uint32_t keep4, int 
 // gamma_kernel (which does not write W); gamma is read after.
 // SP24: also write the 2:4 sparse-MMA operand (a separate instantiation, so
 // the other formats' kernel carries none of its registers).
+// Ternarise and store every requested format of one thread's 16 weights.
 template <int M, bool SP24>
-__global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
+__device__ __forceinline__ void pack_formats(const PackArgs &a, int64_t e0, const uint32_t (&bits)[16 / M][M],
+                                             const uint32_t (&keep)[16 / M])
 {
-    constexpr int kBatch = 16 / M;  // groups per thread
-    const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 16;
-    const bool active = e0 < a.count;  // count % 16 == 0: the 16 weights are all in or all out
-    uint32_t bits[kBatch][M];
-    uint32_t keep[kBatch];
-    if (active) {
-        float4 f[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) f[j] = __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j);
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            uint32_t key[M];
-#pragma unroll
-            for (int i = 0; i < M; ++i) {
-                const int e = b * M + i;
-                const float4 &v = f[e >> 2];
-                const float x = (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
-                bits[b][i] = __float_as_uint(x);
-                key[i] = bits[b][i] & 0x7fffffffu;  // |W| ordered as integers; -0 ties +0
-            }
-            keep[b] = keep_mask<M>(key, a.n);
-        }
-    }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (!active) return;
+    constexpr int kBatch = 16 / M;
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
     const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
     const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);  // 16 | K: same row
@@ -374,6 +463,57 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
         }
     }
 }
+
+// STATS: also the re-mask statistics of PackStats (flip count, near-zero
+// count, per-group threshold, keep bitmap).
+template <int M, bool SP24, bool STATS>
+__global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
+{
+    constexpr int kBatch = 16 / M;  // groups per thread
+    const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 16;
+    const bool active = e0 < a.count;  // count % 16 == 0: the 16 weights are all in or all out
+    uint32_t bits[kBatch][M];
+    uint32_t keep[kBatch];
+    uint32_t prev16 = 0;        // previous step's keep bits of these 16 weights
+    if constexpr (STATS) {
+        // the previous bitmap was written before gamma_kernel started (which
+        // is not launched early), so it may be read before the wait
+        if (active && a.stats.prev_keep) {
+            const int32_t prow = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
+            const int32_t pcol = static_cast<int32_t>(e0 - static_cast<int64_t>(prow) * a.cols);
+            prev16 = *reinterpret_cast<const uint16_t *>(a.stats.prev_keep + static_cast<int64_t>(prow) * a.stats.keep_stride +
+                                                         pcol / 8);
+        }
+    }
+    if (active) {
+        float4 f[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) f[j] = __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j);
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            uint32_t key[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                const int e = b * M + i;
+                const float4 &v = f[e >> 2];
+                const float x = (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
+                bits[b][i] = __float_as_uint(x);
+                key[i] = bits[b][i] & 0x7fffffffu;  // |W| ordered as integers; -0 ties +0
+            }
+            keep[b] = keep_mask<M>(key, a.n);
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if constexpr (STATS) {
+        // every thread takes part in the statistics' CTA-wide reduction
+        ThreadStats<M> st{};
+        if (active) st = stats_of<M>(a, bits, keep, prev16);
+        stats_finish<M>(a, active, e0, st);
+    }
+    if (!active) return;
+    pack_formats<M, SP24>(a, e0, bits, keep);
+}
+
 
 // W_eff^T as bf16 from the int8 W_eff: in [rows, cols] int8 -> out [cols,
 // rows] bf16 bits, through 64 x 64 shared-memory tiles.  rows, cols % 16 == 0.

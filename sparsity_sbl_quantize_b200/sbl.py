@@ -45,6 +45,11 @@ class sbl_packed(ctypes.Structure):
                 ("sp24_values", ctypes.c_void_p), ("sp24_meta", ctypes.c_void_p)]
 
 
+class sbl_mask_stats(ctypes.Structure):
+    _fields_ = [("prev_keep", ctypes.c_void_p), ("keep", ctypes.c_void_p), ("flips", ctypes.c_void_p),
+                ("near_zero", ctypes.c_void_p), ("block_threshold", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _D = ctypes.POINTER(sbl_layer_desc)
 _W = ctypes.POINTER(sbl_packed)
@@ -59,6 +64,8 @@ _lib.sbl_workspace_bytes.restype = _sz
 _lib.sbl_workspace_bytes.argtypes = [_D, _i32, ctypes.c_int]
 _lib.sbl_quantize_mask_pack.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack.argtypes = [_D, _P, _u32, _W, _P, _sz, _P]
+_lib.sbl_quantize_mask_pack_stats.restype = ctypes.c_int
+_lib.sbl_quantize_mask_pack_stats.argtypes = [_D, _P, _u32, _W, ctypes.POINTER(sbl_mask_stats), _P, _sz, _P]
 _lib.sbl_quantize_mask_pack_noalloc.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack_noalloc.argtypes = [_D, _P, _u32, _W, _P]
 _lib.sbl_quantize_act.restype = ctypes.c_int
@@ -73,7 +80,7 @@ _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
-            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
+            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
             "sbl_forward_format", "sbl_backward_dual_ste", "sbl_device_error"]
 
 
@@ -145,6 +152,26 @@ def sbl_quantize_mask_pack(d: sbl_layer_desc, W: torch.Tensor, formats: int, out
     _check(_lib.sbl_quantize_mask_pack(ctypes.byref(d), _ptr(W), formats, ctypes.byref(cp),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream()), "sbl_quantize_mask_pack")
+
+
+def sbl_quantize_mask_pack_stats(d: sbl_layer_desc, W: torch.Tensor, formats: int, p: Packed,
+                                 workspace: torch.Tensor, prev_keep: Optional[torch.Tensor] = None,
+                                 keep: Optional[torch.Tensor] = None, flips: Optional[torch.Tensor] = None,
+                                 near_zero: Optional[torch.Tensor] = None,
+                                 block_threshold: Optional[torch.Tensor] = None):
+    """sbl_quantize_mask_pack plus re-mask statistics; flips / near_zero are
+    one-element int64 device tensors (read as uint64)."""
+    st = sbl_mask_stats(*[(t.data_ptr() if t is not None else None)
+                          for t in (prev_keep, keep, flips, near_zero, block_threshold)])
+    cp = p.c()
+    _check(_lib.sbl_quantize_mask_pack_stats(ctypes.byref(d), _ptr(W), formats, ctypes.byref(cp), ctypes.byref(st),
+                                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()),
+           "sbl_quantize_mask_pack_stats")
+
+
+def keep_bitmap_bytes(d: sbl_layer_desc) -> int:
+    """Bytes per row of the keep bitmap of sbl_mask_stats (the NM bitmap layout)."""
+    return sbl_packed_row_bytes(d, SBL_FMT_NM, SBL_BUF_NM_BITMAP)
 
 
 def sbl_quantize_mask_pack_noalloc(d: sbl_layer_desc, W: torch.Tensor, formats: int, out: Packed) -> None:

@@ -167,3 +167,22 @@ def test_forward_format_recommendation(sbl):
     assert F(sbl.desc(2048, 11008, 3, 4), 16384) == sbl.SBL_FMT_I8
     assert F(sbl.desc(20, 256, 2, 4), 64) == 0                       # invalid descriptor
     assert F(sbl.desc(128, 256, 2, 4), -1) == 0
+
+
+def test_mask_stats_validation(sbl):
+    """Statistics arguments are checked before any device access: a flip
+    count needs the previous bitmap; counters must be 8-byte and arrays
+    16-byte aligned."""
+    good = 0x10000
+    P = ctypes.c_void_p
+    d = sbl.desc(128, 256, 6, 8)
+    w = sbl.sbl_packed(None, None, None, good, None, good)
+    no_prev = sbl.sbl_mask_stats(None, good, good, None, None)
+    assert _raw(sbl, "sbl_quantize_mask_pack_stats", ctypes.byref(d), P(good), sbl.SBL_FMT_I8, ctypes.byref(w),
+                ctypes.byref(no_prev), P(good), 1 << 20, None) == 1
+    odd_counter = sbl.sbl_mask_stats(good, None, good + 4, None, None)
+    assert _raw(sbl, "sbl_quantize_mask_pack_stats", ctypes.byref(d), P(good), sbl.SBL_FMT_I8, ctypes.byref(w),
+                ctypes.byref(odd_counter), P(good), 1 << 20, None) == 3
+    odd_thr = sbl.sbl_mask_stats(None, None, None, None, good + 4)
+    assert _raw(sbl, "sbl_quantize_mask_pack_stats", ctypes.byref(d), P(good), sbl.SBL_FMT_I8, ctypes.byref(w),
+                ctypes.byref(odd_thr), P(good), 1 << 20, None) == 3

@@ -95,6 +95,71 @@ def test_pack_rounding_boundaries():
     check_pack(w, 8, 8)
 
 
+# -------------------------------------------------------- re-mask statistics
+
+def bitmap_of(mask):
+    """Oracle mask (one byte per position) -> keep bitmap rows (bit k%8 of
+    byte k/8, rows padded to 16 bytes)."""
+    o, k = mask.shape
+    rb = oracle.nm_bitmap_row_bytes(k)
+    out = np.zeros((o, rb), dtype=np.uint8)
+    out[:, : k // 8] = np.packbits(mask.astype(np.uint8).reshape(o, k // 8, 8)[..., ::-1], axis=-1)[..., 0]
+    return out
+
+
+@pytest.mark.parametrize("O,K,n,m", [(128, 256, 6, 8), (48, 80, 2, 4), (96, 160, 7, 8), (64, 128, 8, 8),
+                                     (528, 1040, 5, 8), (32, 64, 1, 4), (1008, 1040, 2, 8)])
+def test_pack_stats_bit_exact(O, K, n, m):
+    """Keep bitmap, flip count against the mask of slightly perturbed
+    weights, near-zero count and per-group thresholds: exactly the oracle's,
+    with and without the SP24 instantiation."""
+    sbl = sbl_mod()
+    w_prev = wl.master_weights(O, K, seed=O + K)
+    w = w_prev + np.float32(0.003) * wl.master_weights(O, K, seed=O + K + 1)
+    ref_prev = oracle.Layer(w_prev, n, m)
+    ref = oracle.Layer(w, n, m)
+    dsc = sbl.desc(O, K, n, m)
+    rb = sbl.keep_bitmap_bytes(dsc)
+    prev = to_dev(bitmap_of(ref_prev.mask))
+    fmts = sbl.SBL_FMT_I8 | (sbl.SBL_FMT_SP24 if n <= 2 else 0)
+    for formats in (fmts, 0):
+        p = sbl.alloc_packed(dsc, formats)
+        ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+        keep = torch.full((O, rb), 0xAB, dtype=torch.uint8, device="cuda")
+        flips = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+        nz = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+        thr = torch.empty((O, K // m), dtype=torch.float32, device="cuda")
+        sbl.sbl_quantize_mask_pack_stats(dsc, to_dev(w), formats, p, ws, prev_keep=prev, keep=keep, flips=flips,
+                                         near_zero=nz, block_threshold=thr)
+        np.testing.assert_array_equal(keep.cpu().numpy(), bitmap_of(ref.mask))
+        assert int(flips.item()) == oracle.mask_flips(ref_prev.mask, ref.mask)
+        assert int(nz.item()) == oracle.near_zero(w, ref.gamma)
+        np.testing.assert_array_equal(thr.cpu().numpy().view(np.uint32),
+                                      oracle.block_threshold(w, ref.mask, m).view(np.uint32))
+        if formats & sbl.SBL_FMT_I8:
+            np.testing.assert_array_equal(p.i8.cpu().numpy(), ref.weff)
+        assert float(p.gamma[0].item()) == ref.gamma
+
+
+def test_pack_stats_near_zero_boundary_and_zero_gamma():
+    """Weights at and next to 0.5 gamma (gamma = 1 exactly): exactly 0.5 is
+    not near zero, the float below is; an all-zero matrix counts every
+    weight."""
+    sbl = sbl_mod()
+    base = np.array([0.5, -0.5, 1.5, -1.5, 2.5, -2.5] + [0.75] * 8 + [0.5, 0.5], dtype=np.float32)
+    dn = np.nextafter(np.float32(0.5), np.float32(0))
+    w = np.tile(base, (16, 4)).reshape(16, 64)
+    w[1, 0], w[2, 0] = dn, -dn
+    for mat in (w, np.zeros((16, 64), dtype=np.float32)):
+        ref = oracle.Layer(mat, 6, 8)
+        dsc = sbl.desc(16, 64, 6, 8)
+        p = sbl.alloc_packed(dsc, sbl.SBL_FMT_I8)
+        ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+        nz = torch.zeros((1,), dtype=torch.int64, device="cuda")
+        sbl.sbl_quantize_mask_pack_stats(dsc, to_dev(mat), sbl.SBL_FMT_I8, p, ws, near_zero=nz)
+        assert int(nz.item()) == oracle.near_zero(mat, ref.gamma)
+
+
 # -------------------------------------------------------------- activations
 
 @pytest.mark.parametrize("T,K", [(64, 256), (300, 1040), (1, 16), (7, 8960), (33, 11008), (5, 32768)])
