@@ -48,6 +48,9 @@ def _load():
         lib.sbl_oracle_sp24_meta_row_bytes.argtypes = [i64]
         lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
         lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
+        lib.sbl_oracle_gamma_survivors.restype = f32
+        lib.sbl_oracle_gamma_survivors.argtypes = [p, p, i64, i64]
+        lib.sbl_oracle_nm_mask_quantized.argtypes = [p, i64, i64, i32, i32, p]
         lib.sbl_oracle_mask_flips.restype = i64
         lib.sbl_oracle_mask_flips.argtypes = [p, p, i64]
         lib.sbl_oracle_near_zero.restype = i64
@@ -197,6 +200,21 @@ def pack_sp24(weff, mask):
     return vals, meta
 
 
+def gamma_survivors(w, mask) -> np.float32:
+    w = _f32(w)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    d_out, d_in = w.shape
+    return np.float32(_load().sbl_oracle_gamma_survivors(_ptr(w), _ptr(mask), d_out, d_in))
+
+
+def nm_mask_quantized(wq, n: int, m: int) -> np.ndarray:
+    wq = _i8(wq)
+    d_out, d_in = wq.shape
+    mask = np.empty((d_out, d_in), dtype=np.uint8)
+    _load().sbl_oracle_nm_mask_quantized(_ptr(wq), d_out, d_in, n, m, _ptr(mask))
+    return mask
+
+
 def mask_flips(mask_prev, mask) -> int:
     a = np.ascontiguousarray(mask_prev, dtype=np.uint8)
     b = np.ascontiguousarray(mask, dtype=np.uint8)
@@ -303,12 +321,26 @@ class Layer:
     """The whole forward of one Sparse-BitLinear layer, step by step, as the
     oracle computes it (a convenience bundle for tests and the bench)."""
 
-    def __init__(self, w, n: int, m: int):
+    def __init__(self, w, n: int, m: int, mask_source: str = "master", order: str = "quant_then_mask"):
+        """mask_source "master" ranks |W| (the method) or "quantized" ranks
+        |W_q|; order "quant_then_mask" takes gamma over all weights (the
+        method) or "mask_then_quant" over the survivors ([P1] "Composition
+        Order" ablations).  w may be bf16 bits (uint16), read as fp32 exactly."""
+        w = np.asarray(w)
+        if w.dtype == np.uint16:
+            w = (w.astype(np.uint32) << 16).view(np.float32)
         self.w = _f32(w)
         self.n, self.m = n, m
-        self.gamma = gamma(self.w)
-        self.wq = ternarize(self.w, self.gamma)
-        self.mask = nm_mask(self.w, n, m)
+        if mask_source == "quantized" and order == "mask_then_quant":
+            raise ValueError("a mask from W_q needs gamma, which mask-then-quant takes from the mask")
+        if order == "mask_then_quant":
+            self.mask = nm_mask(self.w, n, m)
+            self.gamma = gamma_survivors(self.w, self.mask)
+            self.wq = ternarize(self.w, self.gamma)
+        else:
+            self.gamma = gamma(self.w)
+            self.wq = ternarize(self.w, self.gamma)
+            self.mask = nm_mask(self.w, n, m) if mask_source == "master" else nm_mask_quantized(self.wq, n, m)
         self.weff = apply_mask(self.wq, self.mask)
 
     def forward(self, x_bf16_bits):

@@ -123,6 +123,54 @@ void sbl_oracle_apply_mask(const int8_t *wq, const uint8_t *mask, int64_t count,
         weff[i] = (int8_t)(mask[i] ? wq[i] : 0);
 }
 
+/* ------------------------------------------------- ablation variants -- */
+
+/* Pairwise tree of R1 over the flat row-major array with |w| at kept
+ * positions and +0.0 at dropped ones. */
+static double abs_sum_tree_masked(const float *w, const uint8_t *mask, int64_t lo, int64_t n)
+{
+    if (n <= 0) return 0.0;
+    if (n == 1) return mask[lo] ? fabs((double)w[lo]) : 0.0;
+    int64_t h = 1;
+    while (h * 2 < n) h *= 2;
+    double left = abs_sum_tree_masked(w, mask, lo, h);
+    double right = abs_sum_tree_masked(w, mask, lo + h, n - h);
+    return left + right;
+}
+
+/* Mask-then-quant ([P1] "Composition Order": W_eff = Q_t(W * M), gamma from
+ * only the Top-N active weights): gamma = mean |W| over the kept positions,
+ * the sum over the same tree as gamma (zeros at dropped positions) divided
+ * by the number of kept positions. */
+float sbl_oracle_gamma_survivors(const float *w, const uint8_t *mask, int64_t d_out, int64_t d_in)
+{
+    int64_t count = d_out * d_in, kept = 0;
+    for (int64_t i = 0; i < count; ++i) kept += mask[i] ? 1 : 0;
+    if (kept == 0) return 0.0f;
+    double s = abs_sum_tree_masked(w, mask, 0, count);
+    return (float)(s / (double)kept);
+}
+
+/* Mask from the quantized weights ([P1] "Composition Order", "Where the mask
+ * is computed"): the same top-n rule ranking |W_q| in {0, 1} instead of |W|;
+ * ties (nearly all) go to the lower index. */
+void sbl_oracle_nm_mask_quantized(const int8_t *wq, int64_t d_out, int64_t d_in, int n, int m, uint8_t *mask)
+{
+    for (int64_t o = 0; o < d_out; ++o)
+        for (int64_t g = 0; g < d_in / m; ++g) {
+            const int8_t *grp = wq + o * d_in + g * m;
+            for (int i = 0; i < m; ++i) {
+                int ki = grp[i] != 0;
+                int rank = 0;
+                for (int j = 0; j < m; ++j) {
+                    int kj = grp[j] != 0;
+                    if (kj > ki || (kj == ki && j < i)) rank++;
+                }
+                mask[o * d_in + g * m + i] = (uint8_t)(rank < n ? 1 : 0);
+            }
+        }
+}
+
 /* -------------------------------------------------------------- packing -- */
 
 /* 2-bit code of a ternary value: {-1, 0, +1} -> {0, 1, 2} ([P5] "Inference

@@ -14,9 +14,11 @@ import test_oracle_pins as pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "sbl_oracle.c")
 
 MUTANTS = {
-    "tie_rule_higher_index": ("(kj == ki && j < i)", "(kj == ki && j > i)"),
+    "tie_rule_higher_index": ("float kj = fabsf(grp[j]);\n                    if (kj > ki || (kj == ki && j < i)) rank++;",
+                              "float kj = fabsf(grp[j]);\n                    if (kj > ki || (kj == ki && j > i)) rank++;"),
     "round_half_away": ("float q = nearbyintf(r);", "float q = roundf(r);"),
-    "sum_split_at_half": ("while (h * 2 < n) h *= 2;", "h = n / 2;"),
+    "sum_split_at_half": ("while (h * 2 < n) h *= 2;\n    double left = abs_sum_tree(w, lo, h);",
+                          "h = n / 2;\n    double left = abs_sum_tree(w, lo, h);"),
     "gamma_over_dout_only": ("return (float)(s / (double)count);", "return (float)(s / (double)d_in);"),
     "act_divide_form": ("float s = bf16_to_f32(row[k]) * r;", "float s = bf16_to_f32(row[k]) / a * 127.0f;"),
     "act_scale_dropped": ("d[t] = a / 127.0f;", "d[t] = a;"),
@@ -26,7 +28,8 @@ MUTANTS = {
     "dx_gamma_dropped": ("dx[t * d_in + k] = (double)gamma * s;", "dx[t * d_in + k] = s;"),
     "mask_not_applied": ("weff[i] = (int8_t)(mask[i] ? wq[i] : 0);", "weff[i] = wq[i];"),
     "sign_extension_codes": ("return (uint8_t)(v + 1);", "return (uint8_t)(v & 3);"),
-    "keep_rank_off_by_one": ("(rank < n ? 1 : 0)", "(rank < n - 1 ? 1 : 0)"),
+    "keep_rank_off_by_one": ("float kj = fabsf(grp[j]);\n                    if (kj > ki || (kj == ki && j < i)) rank++;\n                }\n                mask[o * d_in + g * m + i] = (uint8_t)(rank < n ? 1 : 0);",
+                             "float kj = fabsf(grp[j]);\n                    if (kj > ki || (kj == ki && j < i)) rank++;\n                }\n                mask[o * d_in + g * m + i] = (uint8_t)(rank < n - 1 ? 1 : 0);"),
     "sp24_nibble_fields_swapped": ("unsigned nib = (unsigned)idx[0] | ((unsigned)idx[1] << 2);",
                                    "unsigned nib = (unsigned)idx[1] | ((unsigned)idx[0] << 2);"),
     "sp24_high_nibble_first": ("(nib << (4 * (g % 2)))", "(nib << (4 * (1 - g % 2)))"),
@@ -35,6 +38,9 @@ MUTANTS = {
     "near_zero_inclusive": ("if (r < 0.5f) c++;", "if (r <= 0.5f) c++;"),
     "threshold_from_kept": ("if (mask[k]) continue;\n                float a = fabsf(w[k]);",
                             "if (!mask[k]) continue;\n                float a = fabsf(w[k]);"),
+    "survivor_gamma_over_all": ("return (float)(s / (double)kept);", "return (float)(s / (double)count);"),
+    "quantized_mask_ties_high": ("int kj = grp[j] != 0;\n                    if (kj > ki || (kj == ki && j < i)) rank++;",
+                                 "int kj = grp[j] != 0;\n                    if (kj > ki || (kj == ki && j > i)) rank++;"),
     "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
                            "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
 }
@@ -56,6 +62,8 @@ PIN_CALLS = [
     (pins.test_sp24_hand_example, ()),
     (pins.test_sp24_roundtrip, (2, 4)),
     (pins.test_sp24_roundtrip, (1, 4)),
+    (pins.test_gamma_survivors_hand_row_and_exact_mean, ()),
+    (pins.test_mask_from_quantized_hand_and_brute_force, ()),
     (pins.test_mask_flips_matches_numpy_and_invariants, ()),
     (pins.test_near_zero_matches_numpy_and_gaussian_closed_form, ()),
     (pins.test_block_threshold_brute_force_and_hand_row, ()),

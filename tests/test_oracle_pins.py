@@ -309,6 +309,63 @@ def test_sp24_rejects_masks_that_are_not_2of4():
         oracle.pack_sp24(layer.weff, layer.mask)
 
 
+# ------------------------------------------------------- ablation variants
+
+def test_gamma_survivors_hand_row_and_exact_mean():
+    """Mask-then-quant ("Composition Order": gamma from only the Top-N active
+    weights): the golden 1x8 row keeps 0.9, 0.7, 0.5, 0.3, 0.2, 0.1 at 6:8, so
+    gamma = 2.7 / 6 (not / 8); on random layers gamma is within one fp32 ulp
+    of the exact rational mean of the kept |W|, equals the plain gamma at
+    n = m, and exceeds it otherwise (the survivors are the largest)."""
+    row = np.array([[0.9, -0.1, 0.5, -0.7, 0.05, 0.3, -0.2, 0.0]], dtype=np.float32)
+    mask = oracle.nm_mask(row, 6, 8)
+    kept = [Fraction(float(abs(v))) for v, k in zip(row[0], mask[0]) if k]
+    assert oracle.gamma_survivors(row, mask) == np.float32(float(sum(kept) / 6))
+    for (n, m) in [(6, 8), (2, 4), (3, 8)]:
+        w = wl.master_weights(48, 96, seed=n + m)
+        mask = oracle.nm_mask(w, n, m)
+        g = oracle.gamma_survivors(w, mask)
+        exact = sum(Fraction(float(abs(v))) for v in w[mask == 1]) / int(mask.sum())
+        assert abs(Fraction(float(g)) - exact) <= Fraction(float(np.spacing(g)))
+        assert g > oracle.gamma(w)
+    w = wl.master_weights(16, 64, seed=9)
+    assert oracle.gamma_survivors(w, oracle.nm_mask(w, 8, 8)) == oracle.gamma(w)
+
+
+def test_mask_from_quantized_hand_and_brute_force():
+    """Mask from |W_q| ("Where the mask is computed"): W_q = [1,0,1,-1,0,1,-1,0]
+    at 6:8 keeps the five nonzeros and then the lowest-index zero (position
+    1); in general the top-n of a stable descending order of |W_q|."""
+    wq = np.array([[1, 0, 1, -1, 0, 1, -1, 0]], dtype=np.int8)
+    np.testing.assert_array_equal(oracle.nm_mask_quantized(wq, 6, 8)[0], [1, 1, 1, 1, 0, 1, 1, 0])
+    rng = np.random.default_rng(4)
+    for n, m in [(6, 8), (2, 4), (3, 8), (1, 4)]:
+        q = rng.integers(-1, 2, size=(16, 64)).astype(np.int8)
+        got = oracle.nm_mask_quantized(q, n, m)
+        g = (q != 0).astype(np.int8).reshape(16, 64 // m, m)
+        order = np.argsort(-g, axis=-1, kind="stable")
+        expect = np.zeros_like(g)
+        np.put_along_axis(expect, order[..., :n], 1, axis=-1)
+        np.testing.assert_array_equal(got, expect.reshape(16, 64))
+
+
+def test_layer_variants_invariants():
+    """Layer options: mask-then-quant keeps exactly the master mask and zeroes
+    every dropped position; the quantized-weight mask keeps every nonzero
+    W_q it can (a group with at most n nonzeros keeps all of them)."""
+    w = wl.master_weights(32, 64, seed=12)
+    base = oracle.Layer(w, 6, 8)
+    mtq = oracle.Layer(w, 6, 8, order="mask_then_quant")
+    np.testing.assert_array_equal(mtq.mask, base.mask)
+    assert not mtq.weff[mtq.mask == 0].any()
+    qm = oracle.Layer(w, 6, 8, mask_source="quantized")
+    nz = (qm.wq != 0).reshape(32, 8, 8).sum(-1)
+    kept_nz = ((qm.wq != 0) & (qm.mask == 1)).reshape(32, 8, 8).sum(-1)
+    np.testing.assert_array_equal(kept_nz, np.minimum(nz, 6))
+    with pytest.raises(ValueError):
+        oracle.Layer(w, 6, 8, mask_source="quantized", order="mask_then_quant")
+
+
 # ----------------------------------------------------------- mask statistics
 
 def test_mask_flips_matches_numpy_and_invariants():
