@@ -185,6 +185,38 @@ sbl_status sbl_quantize_mask_pack_stats(const sbl_layer_desc *desc, const float 
                                         const sbl_mask_stats *stats, void *workspace,
                                         size_t workspace_bytes, void *stream);
 
+/* Variants of the weight side, the ablation arms of the Sparse-BitNet
+ * summary ("Composition Order", "Where the mask is computed"; the method
+ * itself is all zeros):
+ *  master_dtype  SBL_MASTER_FP32: W is fp32 [O, K]; SBL_MASTER_BF16: W is
+ *                bf16 bits [O, K] (the pages' master precision), every step
+ *                applied to its exact fp32 value;
+ *  mask_source   SBL_MASK_FROM_MASTER ranks |W|; SBL_MASK_FROM_QUANTIZED
+ *                ranks |W_q| in {0, 1} (ties, i.e. nearly all, to the
+ *                lower index);
+ *  order         SBL_QUANT_THEN_MASK: gamma over all O K weights;
+ *                SBL_MASK_THEN_QUANT: W_eff = Q_t(W * M), gamma = the mean
+ *                |W| over the kept weights only (same fp64 tree with zeros at
+ *                dropped positions, divided by O K n / m).
+ * SBL_MASK_FROM_QUANTIZED with SBL_MASK_THEN_QUANT is circular (the mask
+ * needs gamma, gamma needs the mask): SBL_ERR_UNSUPPORTED. */
+typedef enum { SBL_MASTER_FP32 = 0, SBL_MASTER_BF16 = 1 } sbl_master_dtype;
+typedef enum { SBL_MASK_FROM_MASTER = 0, SBL_MASK_FROM_QUANTIZED = 1 } sbl_mask_source;
+typedef enum { SBL_QUANT_THEN_MASK = 0, SBL_MASK_THEN_QUANT = 1 } sbl_compose_order;
+typedef struct {
+    int32_t master_dtype; /* sbl_master_dtype  */
+    int32_t mask_source;  /* sbl_mask_source   */
+    int32_t order;        /* sbl_compose_order */
+} sbl_pack_variant;
+
+/* sbl_quantize_mask_pack_stats with a variant (NULL = the method: fp32
+ * master weights, mask from |W|, quant-then-mask).  W points to fp32 or bf16
+ * data as the variant says. */
+sbl_status sbl_quantize_mask_pack_ex(const sbl_layer_desc *desc, const void *W,
+                                     const sbl_pack_variant *variant, uint32_t formats,
+                                     const sbl_packed *out, const sbl_mask_stats *stats,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
 /* Same result as sbl_quantize_mask_pack, but the caller passes no workspace
  * and the library allocates nothing.  The paper has no counterpart; this
  * entry point exists for callers that cannot obtain device memory at the
@@ -268,6 +300,18 @@ sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY,
                                  const sbl_packed *w, void *dX, int32_t dx_is_fp32,
                                  float *dW, void *workspace, size_t workspace_bytes,
                                  void *stream);
+
+/* sbl_backward_dual_ste with the mask-gated dW of the pages' ablation
+ * ("Gradient flow through masked weights": gradients blocked at pruned
+ * weights): dW[o, k] = 0 where bit k%8 of byte k/8 of row o of dw_keep is 0
+ * (the keep bitmap of sbl_mask_stats or the SBL_FMT_NM bitmap, rows of
+ * round_up(K/8, 16) bytes); dw_keep == NULL gives the method's ungated dW.
+ * dX is never gated (identity through the mask either way). */
+sbl_status sbl_backward_dual_ste_ex(const sbl_layer_desc *desc, const uint16_t *dY,
+                                    const int8_t *Xq, const float *d, int32_t T,
+                                    const sbl_packed *w, void *dX, int32_t dx_is_fp32,
+                                    float *dW, const uint8_t *dw_keep, void *workspace,
+                                    size_t workspace_bytes, void *stream);
 
 /* Device error word of the current device: 0 when every kernel's bounded
  * waits completed; otherwise a bit per kernel family that gave up a wait.

@@ -315,13 +315,29 @@ namespace {
 constexpr int kDecGroupsSmallT = 1;
 constexpr int kDecGroupsLargeT = 1;
 
+// opt: the kPack* bits of the kernel to run.
 template <int M>
-cudaError_t launch_pack(const cudaLaunchConfig_t &cfg, const PackArgs &pa, bool sp24, bool stats)
+cudaError_t launch_pack(const cudaLaunchConfig_t &cfg, const PackArgs &pa, int opt)
 {
-    if (stats) return sp24 ? cudaLaunchKernelEx(&cfg, pack_kernel<M, true, true>, pa)
-                           : cudaLaunchKernelEx(&cfg, pack_kernel<M, false, true>, pa);
-    return sp24 ? cudaLaunchKernelEx(&cfg, pack_kernel<M, true, false>, pa)
-                : cudaLaunchKernelEx(&cfg, pack_kernel<M, false, false>, pa);
+    switch (opt) {
+    case 0: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 0>, pa);
+    case 1: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 1>, pa);
+    case 2: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 2>, pa);
+    case 3: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 3>, pa);
+    case 4: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 4>, pa);
+    case 5: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 5>, pa);
+    case 6: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 6>, pa);
+    case 7: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 7>, pa);
+    case 8: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 8>, pa);
+    case 9: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 9>, pa);
+    case 10: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 10>, pa);
+    case 11: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 11>, pa);
+    case 12: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 12>, pa);
+    case 13: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 13>, pa);
+    case 14: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 14>, pa);
+    case 15: return cudaLaunchKernelEx(&cfg, pack_kernel<M, 15>, pa);
+    }
+    return cudaErrorInvalidValue;
 }
 
 // cpw: chunks per warp per round, 1, 2, 4 or 8 (at most 4 with two row
@@ -395,11 +411,20 @@ size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op
 }  // extern "C"
 
 // sbl_quantize_mask_pack with optional re-mask statistics (stats may be null).
-static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const float *W, uint32_t formats,
-                                          const sbl_packed *out, const sbl_mask_stats *stats, void *workspace,
+static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void *W, uint32_t formats,
+                                          const sbl_packed *out, const sbl_mask_stats *stats,
+                                          const sbl_pack_variant *variant, void *workspace,
                                           size_t workspace_bytes, void *stream_p)
 {
     sbl_status st = check_desc(desc);
+    const sbl_pack_variant def = {SBL_MASTER_FP32, SBL_MASK_FROM_MASTER, SBL_QUANT_THEN_MASK};
+    const sbl_pack_variant v = variant ? *variant : def;
+    if ((v.master_dtype != SBL_MASTER_FP32 && v.master_dtype != SBL_MASTER_BF16) ||
+        (v.mask_source != SBL_MASK_FROM_MASTER && v.mask_source != SBL_MASK_FROM_QUANTIZED) ||
+        (v.order != SBL_QUANT_THEN_MASK && v.order != SBL_MASK_THEN_QUANT))
+        return SBL_ERR_INVALID_ARG;
+    if (v.mask_source == SBL_MASK_FROM_QUANTIZED && v.order == SBL_MASK_THEN_QUANT) return SBL_ERR_UNSUPPORTED;
+    const bool bf16 = v.master_dtype == SBL_MASTER_BF16;
     if (st != SBL_OK) return st;
     if (!W || !out || !out->gamma) return SBL_ERR_INVALID_ARG;
     const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T | SBL_FMT_SP24;
@@ -464,7 +489,20 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const floa
     }
 
     const int gblocks = static_cast<int>((count + kGammaBlock - 1) / kGammaBlock);
-    gamma_kernel<<<gblocks, 256, 0, stream>>>(W, count, ws, out->gamma);
+    const bool surv = v.order == SBL_MASK_THEN_QUANT;
+    const int64_t divisor = surv ? count / desc->m * desc->n : count;
+    const int gm = surv ? desc->m : 0;
+    if (bf16) {
+        const uint16_t *Wb = static_cast<const uint16_t *>(W);
+        if (gm == 0) gamma_kernel<uint16_t, 0><<<gblocks, 256, 0, stream>>>(Wb, count, ws, out->gamma, desc->n, divisor);
+        else if (gm == 4) gamma_kernel<uint16_t, 4><<<gblocks, 256, 0, stream>>>(Wb, count, ws, out->gamma, desc->n, divisor);
+        else gamma_kernel<uint16_t, 8><<<gblocks, 256, 0, stream>>>(Wb, count, ws, out->gamma, desc->n, divisor);
+    } else {
+        const float *Wf = static_cast<const float *>(W);
+        if (gm == 0) gamma_kernel<float, 0><<<gblocks, 256, 0, stream>>>(Wf, count, ws, out->gamma, desc->n, divisor);
+        else if (gm == 4) gamma_kernel<float, 4><<<gblocks, 256, 0, stream>>>(Wf, count, ws, out->gamma, desc->n, divisor);
+        else gamma_kernel<float, 8><<<gblocks, 256, 0, stream>>>(Wf, count, ws, out->gamma, desc->n, divisor);
+    }
     if ((st = launch_status()) != SBL_OK) return st;
 
     PackArgs pa;
@@ -519,8 +557,9 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const floa
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const bool sp = (formats & SBL_FMT_SP24) != 0;
-        const cudaError_t e = desc->m == 8 ? launch_pack<8>(cfg, pa, sp, want_stats)
-                                           : launch_pack<4>(cfg, pa, sp, want_stats);
+        const int opt = (sp ? kPackSp24 : 0) | (want_stats ? kPackStats : 0) |
+                        (v.mask_source == SBL_MASK_FROM_QUANTIZED ? kPackMaskQ : 0) | (bf16 ? kPackBf16 : 0);
+        const cudaError_t e = desc->m == 8 ? launch_pack<8>(cfg, pa, opt) : launch_pack<4>(cfg, pa, opt);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         if ((st = launch_status()) != SBL_OK) return st;
     }
@@ -538,14 +577,21 @@ sbl_status sbl_quantize_mask_pack(const sbl_layer_desc *desc, const float *W, ui
                                   const sbl_packed *out, void *workspace, size_t workspace_bytes,
                                   void *stream_p)
 {
-    return quantize_mask_pack_impl(desc, W, formats, out, nullptr, workspace, workspace_bytes, stream_p);
+    return quantize_mask_pack_impl(desc, W, formats, out, nullptr, nullptr, workspace, workspace_bytes, stream_p);
 }
 
 sbl_status sbl_quantize_mask_pack_stats(const sbl_layer_desc *desc, const float *W, uint32_t formats,
                                         const sbl_packed *out, const sbl_mask_stats *stats, void *workspace,
                                         size_t workspace_bytes, void *stream_p)
 {
-    return quantize_mask_pack_impl(desc, W, formats, out, stats, workspace, workspace_bytes, stream_p);
+    return quantize_mask_pack_impl(desc, W, formats, out, stats, nullptr, workspace, workspace_bytes, stream_p);
+}
+
+sbl_status sbl_quantize_mask_pack_ex(const sbl_layer_desc *desc, const void *W, const sbl_pack_variant *variant,
+                                     uint32_t formats, const sbl_packed *out, const sbl_mask_stats *stats,
+                                     void *workspace, size_t workspace_bytes, void *stream_p)
+{
+    return quantize_mask_pack_impl(desc, W, formats, out, stats, variant, workspace, workspace_bytes, stream_p);
 }
 
 sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq, float *d, void *stream_p)
@@ -681,19 +727,21 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
     return (desc->in_features >= 1024 && outputs >= 8192LL * 1024) ? SBL_FMT_SP24 : SBL_FMT_I8;
 }
 
-sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq,
-                                 const float *d, int32_t T, const sbl_packed *w, void *dX,
-                                 int32_t dx_is_fp32, float *dW, void *workspace, size_t workspace_bytes,
-                                 void *stream_p)
+}  // extern "C"
+
+static sbl_status backward_impl(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq, const float *d,
+                                int32_t T, const sbl_packed *w, void *dX, int32_t dx_is_fp32, float *dW,
+                                const uint8_t *dw_keep, void *workspace, size_t workspace_bytes, void *stream_p)
 {
     sbl_status st = check_desc(desc);
     if (st != SBL_OK) return st;
     if (T < 0) return SBL_ERR_SHAPE;
     if (!dY || !w || (!dX && !dW)) return SBL_ERR_INVALID_ARG;
+    if (dw_keep && !dW) return SBL_ERR_INVALID_ARG;
     if (dX && (!w->bf16t || !w->gamma)) return SBL_ERR_INVALID_ARG;
     if (dW && (!Xq || !d)) return SBL_ERR_INVALID_ARG;
     if (!aligned16(dY) || (dX && (!aligned16(dX) || !aligned16(w->bf16t) || !aligned16(w->gamma))) ||
-        (dW && (!aligned16(dW) || !aligned16(Xq) || !aligned16(d))))
+        (dW && (!aligned16(dW) || !aligned16(Xq) || !aligned16(d))) || (dw_keep && !aligned16(dw_keep)))
         return SBL_ERR_ALIGNMENT;
     if (dW && (!workspace || workspace_bytes < sbl_workspace_bytes(desc, T, SBL_OP_BACKWARD)))
         return SBL_ERR_WORKSPACE;
@@ -738,10 +786,30 @@ sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY,
         a.out = dW;
         a.ldo = K;
         a.out_fp32 = 1;
+        a.col_keep = dw_keep;
+        a.keep_stride = round_up(K / 8, 16);
         st = launch_gemm<kKindF16>(di, a_t, tp * 2, b_t, tp * 2, O, K, static_cast<int32_t>(tp), a, stream);
         if (st != SBL_OK) return st;
     }
     return SBL_OK;
+}
+
+extern "C" {
+
+sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq,
+                                 const float *d, int32_t T, const sbl_packed *w, void *dX,
+                                 int32_t dx_is_fp32, float *dW, void *workspace, size_t workspace_bytes,
+                                 void *stream_p)
+{
+    return backward_impl(desc, dY, Xq, d, T, w, dX, dx_is_fp32, dW, nullptr, workspace, workspace_bytes, stream_p);
+}
+
+sbl_status sbl_backward_dual_ste_ex(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq,
+                                    const float *d, int32_t T, const sbl_packed *w, void *dX,
+                                    int32_t dx_is_fp32, float *dW, const uint8_t *dw_keep, void *workspace,
+                                    size_t workspace_bytes, void *stream_p)
+{
+    return backward_impl(desc, dY, Xq, d, T, w, dX, dx_is_fp32, dW, dw_keep, workspace, workspace_bytes, stream_p);
 }
 
 }  // extern "C"

@@ -63,6 +63,8 @@ struct GemmArgs {
     int32_t *acc_out;       // optional raw accumulators [M, ldo] (int32 / fp32 bits)
     const float *gamma;     // device scalar (nullptr: 1)
     const float *row_scale; // per-row d_t (nullptr: none)
+    const uint8_t *col_keep;// fp32 output only: keep bitmap [M, keep_stride] (bit n%8 of byte n/8);
+    int64_t keep_stride;    // columns whose bit is 0 are written as 0 (nullptr: none)
     uint32_t *err;
 };
 
@@ -356,11 +358,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint32_t w[32];
                     if (args.out_fp32) {
                         const uint32_t *v = part ? v1 : v0;
+                        // mask-gated output: the 32 keep bits of these columns
+                        const uint32_t keep_bits =
+                            (args.col_keep && row_ok)
+                                ? *reinterpret_cast<const uint32_t *>(args.col_keep + static_cast<int64_t>(m) * args.keep_stride +
+                                                                      col / 8)
+                                : 0xffffffffu;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[i]))
                                                               : __uint_as_float(v[i]);
-                            w[i] = __float_as_uint(__fmul_rn(a, scale));
+                            w[i] = ((keep_bits >> i) & 1u) ? __float_as_uint(__fmul_rn(a, scale)) : 0u;
                         }
                     } else {
 #pragma unroll

@@ -7,6 +7,8 @@
 //     writing the packed formats in one pass over W.
 #pragma once
 
+#include <type_traits>
+
 #include "sbl_device.cuh"
 
 namespace sbl {
@@ -65,7 +67,7 @@ struct PackStats {
 };
 
 struct PackArgs {
-    const float *W;
+    const void *W;         // fp32 or bf16 master weights
     int32_t rows, cols, n;
     int64_t count;         // rows * cols (a multiple of 16)
     uint64_t inv_cols;     // ceil(2^64 / cols): row = umul64hi(e, inv_cols) exactly for e < 2^28
@@ -85,6 +87,23 @@ __device__ __forceinline__ uint32_t near_zero_bound_bits(float gamma)
     return __float_as_uint(__double2float_ru(static_cast<double>(gamma) * (0.5 - 0x1p-26)));
 }
 
+template <int M>
+__device__ __forceinline__ uint32_t keep_mask(const uint32_t (&key)[M], int n);
+
+// Master weights are fp32 or bf16 (uint16_t bits); a bf16 weight is the fp32
+// with the same upper 16 bits, so every step below sees exact fp32 values.
+template <typename WT>
+__device__ __forceinline__ float4 load4(const WT *W, int64_t e)
+{
+    if constexpr (sizeof(WT) == 4) {
+        return __ldg(reinterpret_cast<const float4 *>(W + e));
+    } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(W + e));
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    }
+}
+
 // gamma: one CTA per tree node of kGammaBlock weights.  Warp w owns the 1024
 // consecutive weights [node*8192 + 1024w, +1024) as eight 128-weight chunks;
 // for chunk q lane l loads the float4 at 128q + 4l (coalesced), sums its four
@@ -92,8 +111,13 @@ __device__ __forceinline__ uint32_t near_zero_bound_bits(float gamma)
 // chunk sums, the eight warp sums and finally (in the last CTA to finish) the
 // node partials are combined over the same pairwise tree.  ws->counter must
 // be zero at launch.
-__global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W, int64_t count,
-                                                    GammaWorkspace *ws, float *gamma_out)
+// SURV_M = 0: gamma over all weights; SURV_M = m (4 or 8): mask-then-quant,
+// the sum over the kept |w| only (the group's keep mask from |w| as in
+// pack_kernel; zeros at dropped positions keep the same tree) divided by
+// `divisor` (the number of kept weights).
+template <typename WT, int SURV_M>
+__global__ void __launch_bounds__(256) gamma_kernel(const WT *__restrict__ W, int64_t count,
+                                                    GammaWorkspace *ws, float *gamma_out, int n, int64_t divisor)
 {
     __shared__ double warp_sums[8];
     __shared__ int is_last;
@@ -105,7 +129,37 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
 #pragma unroll
     for (int q = 0; q < 8; ++q) {  // count % 4 == 0: a float4 is all in or all out
         const int64_t e = wbase + 128 * q + 4 * lane;
-        f[q] = (e < count) ? __ldg(reinterpret_cast<const float4 *>(W + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        f[q] = (e < count) ? load4(W, e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if constexpr (SURV_M != 0) {
+        // zero the dropped weights: a group of 4 is one lane's float4, a
+        // group of 8 the float4s of lanes 2i and 2i + 1
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint32_t own[4] = {__float_as_uint(f[q].x) & 0x7fffffffu, __float_as_uint(f[q].y) & 0x7fffffffu,
+                               __float_as_uint(f[q].z) & 0x7fffffffu, __float_as_uint(f[q].w) & 0x7fffffffu};
+            uint32_t keep4;
+            if constexpr (SURV_M == 4) {
+                keep4 = keep_mask<4>(own, n);
+            } else {
+                uint32_t other[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) other[i] = __shfl_xor_sync(0xffffffffu, own[i], 1);
+                const bool odd = lane & 1;
+                uint32_t key[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    key[i] = odd ? other[i] : own[i];
+                    key[4 + i] = odd ? own[i] : other[i];
+                }
+                const uint32_t k8 = keep_mask<8>(key, n);
+                keep4 = odd ? (k8 >> 4) : (k8 & 0xfu);
+            }
+            if (!(keep4 & 1u)) f[q].x = 0.f;
+            if (!(keep4 & 2u)) f[q].y = 0.f;
+            if (!(keep4 & 4u)) f[q].z = 0.f;
+            if (!(keep4 & 8u)) f[q].w = 0.f;
+        }
     }
     double c[8];
 #pragma unroll
@@ -164,7 +218,7 @@ __global__ void __launch_bounds__(256) gamma_kernel(const float *__restrict__ W,
         for (int w = 1; w < kChunks; w *= 2)
 #pragma unroll
             for (int i = 0; i < kChunks; i += 2 * w) cs[i] = cs[i] + cs[i + w];
-        const double mean = __ddiv_rn(cs[0], static_cast<double>(count));
+        const double mean = divisor > 0 ? __ddiv_rn(cs[0], static_cast<double>(divisor)) : 0.0;
         *gamma_out = __double2float_rn(mean);
     }
 }
@@ -466,9 +520,17 @@ __device__ __forceinline__ void pack_formats(const PackArgs &a, int64_t e0, cons
 
 // STATS: also the re-mask statistics of PackStats (flip count, near-zero
 // count, per-group threshold, keep bitmap).
-template <int M, bool SP24, bool STATS>
+// Compile-time options of pack_kernel (a bit mask, so each combination is
+// its own kernel and the common one carries nothing of the others).
+enum : int { kPackSp24 = 1, kPackStats = 2, kPackMaskQ = 4, kPackBf16 = 8 };
+
+template <int M, int OPT>
 __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
 {
+    constexpr bool SP24 = (OPT & kPackSp24) != 0;
+    constexpr bool STATS = (OPT & kPackStats) != 0;
+    constexpr bool MASKQ = (OPT & kPackMaskQ) != 0;
+    using WT = typename std::conditional<(OPT & kPackBf16) != 0, uint16_t, float>::type;
     constexpr int kBatch = 16 / M;  // groups per thread
     const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 16;
     const bool active = e0 < a.count;  // count % 16 == 0: the 16 weights are all in or all out
@@ -488,7 +550,7 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
     if (active) {
         float4 f[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) f[j] = __ldg(reinterpret_cast<const float4 *>(a.W + e0) + j);
+        for (int j = 0; j < 4; ++j) f[j] = load4(static_cast<const WT *>(a.W), e0 + 4 * j);
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
             uint32_t key[M];
@@ -500,10 +562,22 @@ __global__ void __launch_bounds__(256) pack_kernel(PackArgs a)
                 bits[b][i] = __float_as_uint(x);
                 key[i] = bits[b][i] & 0x7fffffffu;  // |W| ordered as integers; -0 ties +0
             }
-            keep[b] = keep_mask<M>(key, a.n);
+            keep[b] = MASKQ ? 0u : keep_mask<M>(key, a.n);
         }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (MASKQ && active) {
+        // ablation: the mask ranks |W_q| in {0, 1} (ties to the lower index),
+        // so it needs gamma first
+        const uint32_t thr = __float_as_uint(ternary_threshold(*a.gamma));
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            uint32_t key01[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) key01[i] = ((bits[b][i] & 0x7fffffffu) >= thr) ? 1u : 0u;
+            keep[b] = keep_mask<M>(key01, a.n);
+        }
+    }
     if constexpr (STATS) {
         // every thread takes part in the statistics' CTA-wide reduction
         ThreadStats<M> st{};

@@ -45,6 +45,15 @@ class sbl_packed(ctypes.Structure):
                 ("sp24_values", ctypes.c_void_p), ("sp24_meta", ctypes.c_void_p)]
 
 
+class sbl_pack_variant(ctypes.Structure):
+    _fields_ = [("master_dtype", ctypes.c_int32), ("mask_source", ctypes.c_int32), ("order", ctypes.c_int32)]
+
+
+SBL_MASTER_FP32, SBL_MASTER_BF16 = 0, 1
+SBL_MASK_FROM_MASTER, SBL_MASK_FROM_QUANTIZED = 0, 1
+SBL_QUANT_THEN_MASK, SBL_MASK_THEN_QUANT = 0, 1
+
+
 class sbl_mask_stats(ctypes.Structure):
     _fields_ = [("prev_keep", ctypes.c_void_p), ("keep", ctypes.c_void_p), ("flips", ctypes.c_void_p),
                 ("near_zero", ctypes.c_void_p), ("block_threshold", ctypes.c_void_p)]
@@ -66,6 +75,11 @@ _lib.sbl_quantize_mask_pack.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack.argtypes = [_D, _P, _u32, _W, _P, _sz, _P]
 _lib.sbl_quantize_mask_pack_stats.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack_stats.argtypes = [_D, _P, _u32, _W, ctypes.POINTER(sbl_mask_stats), _P, _sz, _P]
+_lib.sbl_quantize_mask_pack_ex.restype = ctypes.c_int
+_lib.sbl_quantize_mask_pack_ex.argtypes = [_D, _P, ctypes.POINTER(sbl_pack_variant), _u32, _W,
+                                           ctypes.POINTER(sbl_mask_stats), _P, _sz, _P]
+_lib.sbl_backward_dual_ste_ex.restype = ctypes.c_int
+_lib.sbl_backward_dual_ste_ex.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _P, _sz, _P]
 _lib.sbl_quantize_mask_pack_noalloc.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack_noalloc.argtypes = [_D, _P, _u32, _W, _P]
 _lib.sbl_quantize_act.restype = ctypes.c_int
@@ -81,7 +95,8 @@ _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
-            "sbl_forward_format", "sbl_backward_dual_ste", "sbl_device_error"]
+            "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
+            "sbl_quantize_mask_pack_ex", "sbl_device_error"]
 
 
 class SblError(RuntimeError):
@@ -169,6 +184,22 @@ def sbl_quantize_mask_pack_stats(d: sbl_layer_desc, W: torch.Tensor, formats: in
            "sbl_quantize_mask_pack_stats")
 
 
+def sbl_quantize_mask_pack_ex(d: sbl_layer_desc, W: torch.Tensor, formats: int, p: Packed, workspace: torch.Tensor,
+                              mask_source: int = SBL_MASK_FROM_MASTER, order: int = SBL_QUANT_THEN_MASK,
+                              prev_keep: Optional[torch.Tensor] = None, keep: Optional[torch.Tensor] = None,
+                              flips: Optional[torch.Tensor] = None, near_zero: Optional[torch.Tensor] = None,
+                              block_threshold: Optional[torch.Tensor] = None):
+    """Packing with a weight-side variant; W is float32 or bfloat16."""
+    dtype = SBL_MASTER_BF16 if W.dtype == torch.bfloat16 else SBL_MASTER_FP32
+    v = sbl_pack_variant(dtype, mask_source, order)
+    st = sbl_mask_stats(*[(t.data_ptr() if t is not None else None)
+                          for t in (prev_keep, keep, flips, near_zero, block_threshold)])
+    cp = p.c()
+    _check(_lib.sbl_quantize_mask_pack_ex(ctypes.byref(d), _ptr(W), ctypes.byref(v), formats, ctypes.byref(cp),
+                                          ctypes.byref(st), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _stream()), "sbl_quantize_mask_pack_ex")
+
+
 def keep_bitmap_bytes(d: sbl_layer_desc) -> int:
     """Bytes per row of the keep bitmap of sbl_mask_stats (the NM bitmap layout)."""
     return sbl_packed_row_bytes(d, SBL_FMT_NM, SBL_BUF_NM_BITMAP)
@@ -203,6 +234,17 @@ def sbl_backward_dual_ste(dsc: sbl_layer_desc, dY: torch.Tensor, Xq: Optional[to
     _check(_lib.sbl_backward_dual_ste(ctypes.byref(dsc), _ptr(dY), _ptr(Xq), _ptr(d), T,
                                       ctypes.byref(cp), _ptr(dX), 1 if dx_is_fp32 else 0, _ptr(dW),
                                       _ptr(workspace), nbytes, _stream()), "sbl_backward_dual_ste")
+
+
+def sbl_backward_dual_ste_ex(d: sbl_layer_desc, dY: torch.Tensor, Xq: torch.Tensor, dvec: torch.Tensor, T: int,
+                             p: Packed, dX: Optional[torch.Tensor], dx_fp32: bool, dW: Optional[torch.Tensor],
+                             dw_keep: Optional[torch.Tensor], workspace: Optional[torch.Tensor]):
+    """The backward with dW gated by a keep bitmap (the pages' mask-gated ablation)."""
+    cp = p.c()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.sbl_backward_dual_ste_ex(ctypes.byref(d), _ptr(dY), _ptr(Xq), _ptr(dvec), T, ctypes.byref(cp),
+                                         _ptr(dX), 1 if dx_fp32 else 0, _ptr(dW), _ptr(dw_keep), _ptr(workspace),
+                                         ws_bytes, _stream()), "sbl_backward_dual_ste_ex")
 
 
 def sbl_device_error(clear: bool = False) -> int:

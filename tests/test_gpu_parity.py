@@ -373,6 +373,93 @@ def test_backward_training_workload_sampled():
         assert normwise(dw.cpu().numpy()[io, ik], dw_s) <= FWD_TOL
 
 
+# -------------------------------------------------- ablation variants (f3)
+
+VARIANTS = [("bf16", "master", "quant_then_mask"), ("fp32", "quantized", "quant_then_mask"),
+            ("fp32", "master", "mask_then_quant"), ("bf16", "master", "mask_then_quant"),
+            ("bf16", "quantized", "quant_then_mask")]
+
+
+@pytest.mark.parametrize("dtype,mask_source,order", VARIANTS)
+@pytest.mark.parametrize("O,K,n,m", [(128, 256, 6, 8), (48, 80, 2, 4), (528, 1040, 3, 8), (64, 128, 1, 8),
+                                     (1008, 1040, 2, 4)])
+def test_pack_variants_bit_exact(dtype, mask_source, order, O, K, n, m):
+    """The weight-side ablation arms (bf16 master weights, mask from |W_q|,
+    gamma over the survivors): gamma and every packed format bit for bit
+    against the oracle run with the same variant, plus the statistics."""
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=O + K + n)
+    if dtype == "bf16":
+        wbits = (w.view(np.uint32) >> 16).astype(np.uint16)  # truncated to bf16 (any bf16 value will do)
+        w_dev = torch.from_numpy(wbits.view(np.int16)).view(torch.bfloat16).to("cuda")
+        ref = oracle.Layer(wbits, n, m, mask_source=mask_source, order=order)
+    else:
+        w_dev = to_dev(w)
+        ref = oracle.Layer(w, n, m, mask_source=mask_source, order=order)
+    dsc = sbl.desc(O, K, n, m)
+    fmts = sbl.SBL_FMT_I8 | sbl.SBL_FMT_PK2 | sbl.SBL_FMT_NM | (sbl.SBL_FMT_SP24 if n <= 2 else 0)
+    p = sbl.alloc_packed(dsc, fmts)
+    ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+    keep = torch.empty((O, sbl.keep_bitmap_bytes(dsc)), dtype=torch.uint8, device="cuda")
+    nz = torch.zeros((1,), dtype=torch.int64, device="cuda")
+    thr = torch.empty((O, K // m), dtype=torch.float32, device="cuda")
+    src = {"master": sbl.SBL_MASK_FROM_MASTER, "quantized": sbl.SBL_MASK_FROM_QUANTIZED}[mask_source]
+    odr = {"quant_then_mask": sbl.SBL_QUANT_THEN_MASK, "mask_then_quant": sbl.SBL_MASK_THEN_QUANT}[order]
+    sbl.sbl_quantize_mask_pack_ex(dsc, w_dev, fmts, p, ws, mask_source=src, order=odr, keep=keep, near_zero=nz,
+                                  block_threshold=thr)
+    torch.cuda.synchronize()
+    assert float(p.gamma[0].item()) == ref.gamma
+    np.testing.assert_array_equal(p.i8.cpu().numpy(), ref.weff)
+    np.testing.assert_array_equal(p.pk2.cpu().numpy(), oracle.pack_pk2(ref.weff))
+    vals, bm = oracle.pack_nm(ref.weff, ref.mask, n, m)
+    np.testing.assert_array_equal(p.nm_bitmap.cpu().numpy(), bm)
+    np.testing.assert_array_equal(p.nm_values.cpu().numpy(), vals)
+    np.testing.assert_array_equal(keep.cpu().numpy(), bitmap_of(ref.mask))
+    if n <= 2:
+        sv, sm = oracle.pack_sp24(ref.weff, ref.mask)
+        np.testing.assert_array_equal(p.sp24_values.cpu().numpy(), sv)
+        np.testing.assert_array_equal(p.sp24_meta.cpu().numpy(), sm)
+    assert int(nz.item()) == oracle.near_zero(ref.w, ref.gamma)
+    np.testing.assert_array_equal(thr.cpu().numpy().view(np.uint32),
+                                  oracle.block_threshold(ref.w, ref.mask, m).view(np.uint32))
+
+
+def test_pack_variant_circular_combination_is_unsupported():
+    sbl = sbl_mod()
+    dsc = sbl.desc(32, 64, 6, 8)
+    p = sbl.alloc_packed(dsc, sbl.SBL_FMT_I8)
+    ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+    with pytest.raises(sbl.SblError):
+        sbl.sbl_quantize_mask_pack_ex(dsc, to_dev(wl.master_weights(32, 64, seed=1)), sbl.SBL_FMT_I8, p, ws,
+                                      mask_source=sbl.SBL_MASK_FROM_QUANTIZED, order=sbl.SBL_MASK_THEN_QUANT)
+
+
+@pytest.mark.parametrize("O,K,T,n,m", [(128, 256, 64, 6, 8), (528, 1040, 300, 2, 4), (96, 80, 33, 5, 8)])
+def test_backward_mask_gated_dw(O, K, T, n, m):
+    """The mask-gated dW ablation: dW = (dY^T Xtilde) * M, exactly zero at
+    the pruned positions and within the float tolerance elsewhere; dX as
+    ungated."""
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=O + T)
+    x = wl.activations(T, K, seed=O + T)
+    dy = wl.output_grad(T, O, seed=O + T)
+    layer = GpuLayer(w, n, m, 4 | 8)
+    ref = oracle.Layer(w, n, m)
+    q, d = quantize_act(x)
+    keep = to_dev(bitmap_of(ref.mask))
+    dx = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    dw = torch.empty((O, K), dtype=torch.float32, device="cuda")
+    ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(layer.desc, T, sbl.SBL_OP_BACKWARD))
+    sbl.sbl_backward_dual_ste_ex(layer.desc, bf16_dev(dy), q, d, T, layer.packed, dx, True, dw, keep, ws)
+    torch.cuda.synchronize()
+    qr, dr = oracle.quantize_act(x)
+    dxr, dwr = oracle.backward(dy, ref.weff, ref.gamma, qr, dr)
+    dwg = dw.cpu().numpy()
+    assert not dwg[ref.mask == 0].any()
+    assert normwise(dwg, dwr * ref.mask) <= FWD_TOL
+    assert normwise(dx.cpu().numpy(), dxr) <= FWD_TOL
+
+
 def test_device_error_word_clear():
     sbl = sbl_mod()
     assert sbl.sbl_device_error(clear=True) == 0
