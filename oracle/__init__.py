@@ -48,6 +48,7 @@ def _load():
         lib.sbl_oracle_sp24_meta_row_bytes.argtypes = [i64]
         lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
         lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
+        lib.sbl_oracle_epilogue.argtypes = [p, i64, i64, i32, p, p, p]
         lib.sbl_oracle_gamma_survivors.restype = f32
         lib.sbl_oracle_gamma_survivors.argtypes = [p, p, i64, i64]
         lib.sbl_oracle_nm_mask_quantized.argtypes = [p, i64, i64, i32, i32, p]
@@ -267,6 +268,19 @@ def dequant(acc, g, d):
     yb = np.empty((t, o), dtype=np.uint16)
     _load().sbl_oracle_dequant(_ptr(acc), t, o, float(np.float32(g)), _ptr(d), _ptr(y), _ptr(yb))
     return y, yb
+
+
+def epilogue(y, relu2: bool = False, residual_bf16_bits=None):
+    """Squared-ReLU and residual epilogue on the fp32 output y -> (fp32,
+    bf16 bit patterns)."""
+    y = _f32(y)
+    t, o = y.shape
+    out = np.empty((t, o), dtype=np.float32)
+    ob = np.empty((t, o), dtype=np.uint16)
+    res = None if residual_bf16_bits is None else _u16(residual_bf16_bits)
+    _load().sbl_oracle_epilogue(_ptr(y), t, o, 1 if relu2 else 0, _ptr(res) if res is not None else None,
+                                _ptr(out), _ptr(ob))
+    return out, ob
 
 
 def backward(dy_bf16_bits, weff, g, q, d, want_dx=True, want_dw=True):

@@ -418,6 +418,25 @@ void sbl_oracle_dequant(const int32_t *acc, int64_t tokens, int64_t d_out,
     }
 }
 
+/* Output epilogue after the layer ("Squared ReLU Activation in the
+ * Feed-Forward Network" of the BitNet b1.58 2B4T summary: ReLU^2(x) =
+ * max(0, x)^2, applied to the projection's output; and a residual add):
+ *   v = y                      (the fp32 output of sbl_oracle_dequant)
+ *   v = v > 0 ? fl32(v * v) : 0   when relu2
+ *   v = fl32(v + r)            when a residual r (bf16 [T, O]) is given
+ * written as fp32 and as bf16 (round to nearest even). */
+void sbl_oracle_epilogue(const float *y, int64_t tokens, int64_t d_out, int relu2, const uint16_t *res,
+                         float *out, uint16_t *out_bf16)
+{
+    for (int64_t i = 0; i < tokens * d_out; ++i) {
+        float v = y[i];
+        if (relu2) v = v > 0.0f ? v * v : 0.0f;
+        if (res) v = v + bf16_to_f32(res[i]);
+        if (out) out[i] = v;
+        if (out_bf16) out_bf16[i] = f32_to_bf16(v);
+    }
+}
+
 /* ------------------------------------------------------------ backward -- */
 
 /* [P1] "The Dual Straight-Through Estimator" (dL/dW ~= dL/dW_eff) and the

@@ -41,6 +41,9 @@ MUTANTS = {
     "survivor_gamma_over_all": ("return (float)(s / (double)kept);", "return (float)(s / (double)count);"),
     "quantized_mask_ties_high": ("int kj = grp[j] != 0;\n                    if (kj > ki || (kj == ki && j < i)) rank++;",
                                  "int kj = grp[j] != 0;\n                    if (kj > ki || (kj == ki && j > i)) rank++;"),
+    "relu_not_squared": ("if (relu2) v = v > 0.0f ? v * v : 0.0f;", "if (relu2) v = v > 0.0f ? v : 0.0f;"),
+    "residual_before_activation": ("if (relu2) v = v > 0.0f ? v * v : 0.0f;\n        if (res) v = v + bf16_to_f32(res[i]);",
+                                   "if (res) v = v + bf16_to_f32(res[i]);\n        if (relu2) v = v > 0.0f ? v * v : 0.0f;"),
     "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
                            "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
 }
@@ -62,6 +65,7 @@ PIN_CALLS = [
     (pins.test_sp24_hand_example, ()),
     (pins.test_sp24_roundtrip, (2, 4)),
     (pins.test_sp24_roundtrip, (1, 4)),
+    (pins.test_epilogue_hand_values, ()),
     (pins.test_gamma_survivors_hand_row_and_exact_mean, ()),
     (pins.test_mask_from_quantized_hand_and_brute_force, ()),
     (pins.test_mask_flips_matches_numpy_and_invariants, ()),

@@ -309,6 +309,36 @@ def test_sp24_rejects_masks_that_are_not_2of4():
         oracle.pack_sp24(layer.weff, layer.mask)
 
 
+# --------------------------------------------------------------- epilogue
+
+def test_epilogue_hand_values():
+    """ReLU^2 ("Squared ReLU Activation": max(0, x)^2) then the residual:
+    [-2, -0, 0.5, 3] -> [0, 0, 0.25, 9]; + 1 -> [1, 1, 1.25, 10] (exact),
+    bf16 of 1.25 = 0x3FA0."""
+    y = np.array([[-2.0, -0.0, 0.5, 3.0]], dtype=np.float32)
+    out, _ = oracle.epilogue(y, relu2=True)
+    np.testing.assert_array_equal(out, [[0.0, 0.0, 0.25, 9.0]])
+    assert not np.signbit(out).any()
+    one = np.full((1, 4), 0x3F80, dtype=np.uint16)
+    out, ob = oracle.epilogue(y, relu2=True, residual_bf16_bits=one)
+    np.testing.assert_array_equal(out, [[1.0, 1.0, 1.25, 10.0]])
+    assert ob[0, 2] == 0x3FA0
+    out, _ = oracle.epilogue(y, residual_bf16_bits=one)
+    np.testing.assert_array_equal(out, [[-1.0, 1.0, 1.5, 4.0]])
+
+
+def test_epilogue_matches_numpy_float32_and_torch_bf16():
+    rng = np.random.default_rng(8)
+    y = (rng.standard_normal((64, 96)) * 40).astype(np.float32)
+    r = torch.from_numpy(rng.standard_normal((64, 96)).astype(np.float32)).to(torch.bfloat16)
+    rb = r.view(torch.int16).numpy().view(np.uint16)
+    out, ob = oracle.epilogue(y, relu2=True, residual_bf16_bits=rb)
+    sq = np.where(y > 0, y * y, np.float32(0)).astype(np.float32)
+    expect = (sq + r.to(torch.float32).numpy()).astype(np.float32)
+    np.testing.assert_array_equal(out, expect)
+    np.testing.assert_array_equal(ob, torch.from_numpy(expect).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
 # ------------------------------------------------------- ablation variants
 
 def test_gamma_survivors_hand_row_and_exact_mean():
