@@ -273,6 +273,26 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
                        int32_t T, const sbl_packed *w, sbl_format fmt,
                        void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);
 
+/* Output epilogue fused into the forward (all members optional):
+ *  relu2     non-zero: v = max(v, 0)^2 on the fp32 output (Squared ReLU of the
+ *            BitNet b1.58 2B4T summary, "Squared ReLU Activation in the
+ *            Feed-Forward Network"), v = v > 0 ? fl32(v * v) : +0;
+ *  residual  bf16 bits [T, O] (16-byte aligned): v = fl32(v + residual),
+ *            applied after relu2;
+ * then the bf16 (RNE) or fp32 store as in sbl_forward.  acc_out, when given,
+ * still receives the raw int32 accumulators. */
+typedef struct {
+    int32_t relu2;
+    const uint16_t *residual;
+} sbl_epilogue;
+
+/* sbl_forward with an output epilogue (NULL: exactly sbl_forward).  Every
+ * forward format supports it. */
+sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const float *d,
+                          int32_t T, const sbl_packed *w, sbl_format fmt, void *Y,
+                          int32_t y_is_fp32, int32_t *acc_out, const sbl_epilogue *epi,
+                          void *stream);
+
 /* The forward operand format the library recommends for a layer and a
  * token count: SBL_FMT_SP24 (2:4 sparse tensor-core MMA on CTA pairs) when
  * the mask allows it (n <= 2) and the GEMM is large enough for the sparse

@@ -70,9 +70,17 @@ static sbl_status current_device(DeviceInfo **out)
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindI8, 256, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindI8, 128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Sp24PairCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(sp24_pair_kernel<224, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(sp24_pair_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<128>::kSmemBytes) != cudaSuccess)
             return SBL_ERR_CUDA;
         if (!g_encode) {
@@ -164,7 +172,7 @@ static int choose_bn(int32_t M, int32_t N, int num_sms)
     return 5 * rounds(128) <= 4 * rounds(256) ? 128 : 256;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool EPI>
 static sbl_status launch_gemm_bn(const DeviceInfo *di, const CUtensorMap &ta, const CUtensorMap &tb,
                                  const CUtensorMap &ty, GemmArgs args, cudaStream_t stream)
 {
@@ -182,7 +190,7 @@ static sbl_status launch_gemm_bn(const DeviceInfo *di, const CUtensorMap &ta, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN>, ta, tb, ty, args) != cudaSuccess) return SBL_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, EPI>, ta, tb, ty, args) != cudaSuccess) return SBL_ERR_CUDA;
     return launch_status();
 }
 
@@ -205,8 +213,13 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     args.K = K;
     args.k_blocks = static_cast<int32_t>((static_cast<int64_t>(K) * eb + kBKBytes - 1) / kBKBytes);
     args.err = di->err;
-    return bn == 128 ? launch_gemm_bn<KIND, 128>(di, ta, tb, ty, args, stream)
-                     : launch_gemm_bn<KIND, 256>(di, ta, tb, ty, args, stream);
+    if constexpr (KIND == kKindI8) {
+        if (args.relu2 || args.residual)
+            return bn == 128 ? launch_gemm_bn<KIND, 128, true>(di, ta, tb, ty, args, stream)
+                             : launch_gemm_bn<KIND, 256, true>(di, ta, tb, ty, args, stream);
+    }
+    return bn == 128 ? launch_gemm_bn<KIND, 128, false>(di, ta, tb, ty, args, stream)
+                     : launch_gemm_bn<KIND, 256, false>(di, ta, tb, ty, args, stream);
 }
 
 // 3-D view of the SP24 metadata [O, row_bytes] for the sparse GEMM: dims
@@ -260,7 +273,7 @@ static int choose_pair_bn(int32_t O, int32_t T, int num_sms)
 template <int BN>
 static sbl_status launch_sp24_pair(const DeviceInfo *di, int32_t O, int32_t K, int32_t T, const int8_t *Xq,
                                    const float *d, const sbl_packed *w, void *Y, bool y_fp32, int32_t *acc_out,
-                                   cudaStream_t stream)
+                                   const sbl_epilogue *epi, cudaStream_t stream)
 {
     const int64_t vstride = round_up(K / 2, 16), mstride = round_up(K / 8, 16);
     CUtensorMap ta, tb, te, ty;
@@ -282,6 +295,11 @@ static sbl_status launch_sp24_pair(const DeviceInfo *di, int32_t O, int32_t K, i
     a.gamma = w->gamma;
     a.d = d;
     a.err = di->err;
+    const bool with_epi = epi && (epi->relu2 || epi->residual);
+    if (with_epi) {
+        a.relu2 = epi->relu2 ? 1 : 0;
+        a.residual = epi->residual;
+    }
     const int tiles = a.tiles_m * a.tiles_n;
     const int pairs = tiles < di->num_sms / 2 ? tiles : di->num_sms / 2;
     cudaLaunchConfig_t cfg;
@@ -299,7 +317,9 @@ static sbl_status launch_sp24_pair(const DeviceInfo *di, int32_t O, int32_t K, i
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, sp24_pair_kernel<BN>, ta, tb, te, ty, a) != cudaSuccess) return SBL_ERR_CUDA;
+    const cudaError_t e = with_epi ? cudaLaunchKernelEx(&cfg, sp24_pair_kernel<BN, true>, ta, tb, te, ty, a)
+                                   : cudaLaunchKernelEx(&cfg, sp24_pair_kernel<BN, false>, ta, tb, te, ty, a);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
     return launch_status();
 }
 
@@ -638,9 +658,11 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq,
     return launch_status();
 }
 
-sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
-                       const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32,
-                       int32_t *acc_out, void *stream_p)
+}  // extern "C"
+
+static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
+                               const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32,
+                               int32_t *acc_out, const sbl_epilogue *epi, void *stream_p)
 {
     sbl_status st = check_desc(desc);
     if (st != SBL_OK) return st;
@@ -648,7 +670,7 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
     if (T == 0) return SBL_OK;
     if (!Xq || !d || !w || !Y || !w->gamma) return SBL_ERR_INVALID_ARG;
     if (!aligned16(Xq) || !aligned16(d) || !aligned16(Y) || !aligned16(w->gamma) ||
-        (acc_out && !aligned16(acc_out)))
+        (acc_out && !aligned16(acc_out)) || (epi && epi->residual && !aligned16(epi->residual)))
         return SBL_ERR_ALIGNMENT;
     DeviceInfo *di = nullptr;
     if ((st = current_device(&di)) != SBL_OK) return st;
@@ -666,6 +688,10 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         a.acc_out = acc_out;
         a.gamma = w->gamma;
         a.row_scale = d;
+        if (epi) {
+            a.relu2 = epi->relu2 ? 1 : 0;
+            a.residual = epi->residual;
+        }
         return launch_gemm<kKindI8>(di, Xq, K, w->i8, K, T, O, K, a, stream);
     }
     if (fmt == SBL_FMT_SP24) {
@@ -673,8 +699,8 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
         if (!aligned16(w->sp24_values) || !aligned16(w->sp24_meta)) return SBL_ERR_ALIGNMENT;
         return choose_pair_bn(O, T, di->num_sms) == 224
-                   ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream)
-                   : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, stream);
+                   ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, epi, stream)
+                   : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, epi, stream);
     }
     if (fmt == SBL_FMT_PK2) {
         if (!w->pk2) return SBL_ERR_INVALID_ARG;
@@ -690,6 +716,10 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         a.out = Y;
         a.out_fp32 = y_is_fp32 ? 1 : 0;
         a.acc_out = acc_out;
+        if (epi) {
+            a.relu2 = epi->relu2 ? 1 : 0;
+            a.residual = epi->residual;
+        }
         a.T = T;
         a.K = K;
         a.O = O;
@@ -717,6 +747,22 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
         return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
     }
     return SBL_ERR_UNSUPPORTED;
+}
+
+extern "C" {
+
+sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
+                       const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32,
+                       int32_t *acc_out, void *stream_p)
+{
+    return forward_impl(desc, Xq, d, T, w, fmt, Y, y_is_fp32, acc_out, nullptr, stream_p);
+}
+
+sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
+                          const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32, int32_t *acc_out,
+                          const sbl_epilogue *epi, void *stream_p)
+{
+    return forward_impl(desc, Xq, d, T, w, fmt, Y, y_is_fp32, acc_out, epi, stream_p);
 }
 
 sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)

@@ -48,6 +48,8 @@ struct DecodeArgs {
     void *out;            // [T, O] bf16 bits or fp32
     int32_t out_fp32;
     int32_t *acc_out;     // optional [T, O] int32
+    int32_t relu2;        // output epilogue: v = max(v, 0)^2 ...
+    const uint16_t *residual;  // ... then v = v + residual[t, o] (bf16 [T, O]; nullptr: none)
     int32_t T, K, O;
     int32_t chunks;       // ceil(K / 256)
 };
@@ -274,7 +276,9 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
                  static_cast<uint32_t>(csum[w0 + w][t_out]);
         const int32_t acc_v = static_cast<int32_t>(s);
         const int64_t off = static_cast<int64_t>(t_out) * args.O + row0 + r_out;
-        const float y = __fmul_rn(__int2float_rn(acc_v), scale);
+        float y = __fmul_rn(__int2float_rn(acc_v), scale);
+        if (args.relu2) y = y > 0.0f ? __fmul_rn(y, y) : 0.0f;
+        if (args.residual) y = __fadd_rn(y, __uint_as_float(static_cast<uint32_t>(args.residual[off]) << 16));
         if (args.out_fp32) static_cast<float *>(args.out)[off] = y;
         else {
             const __nv_bfloat16 hb = __float2bfloat16_rn(y);

@@ -65,8 +65,19 @@ struct GemmArgs {
     const float *row_scale; // per-row d_t (nullptr: none)
     const uint8_t *col_keep;// fp32 output only: keep bitmap [M, keep_stride] (bit n%8 of byte n/8);
     int64_t keep_stride;    // columns whose bit is 0 are written as 0 (nullptr: none)
+    int32_t relu2;          // output epilogue: v = max(v, 0)^2 ...
+    const uint16_t *residual;  // ... then v = v + residual[m, n] (bf16 [M, ldo]; nullptr: none)
     uint32_t *err;
 };
+
+// The optional output epilogue of the forward (Squared ReLU, then a bf16
+// residual), in fp32 with round-to-nearest operations.
+__device__ __forceinline__ float epilogue_op(float v, int32_t relu2, uint32_t res_bits16, bool has_res)
+{
+    if (relu2) v = v > 0.0f ? __fmul_rn(v, v) : 0.0f;
+    if (has_res) v = __fadd_rn(v, __uint_as_float(res_bits16 << 16));
+    return v;
+}
 
 template <int KIND, int BN>
 __device__ __forceinline__ constexpr uint32_t gemm_idesc()
@@ -93,7 +104,9 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
     tn = r / gm;
 }
 
-template <int KIND, int BN>
+// EPI: the instantiation that applies the output epilogue (relu2 /
+// residual); the others compile without it.
+template <int KIND, int BN, bool EPI = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs args)
@@ -268,7 +281,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (args.row_scale) scale = row_ok ? __fmul_rn(g, d_m) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
-            if (!args.out_fp32) {
+            if (!args.out_fp32 && !EPI) {
                 // bf16: drain this warp's share of the accumulator, converting
                 // each 64-column chunk to 32 packed words, hand TMEM back, and
                 // only then store -- the MMAs of the tile after next need not
@@ -356,6 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int col = args.out_fp32 ? n0 + 32 * part : n0;
                     if (col >= args.N) break;  // warp-uniform
                     uint32_t w[32];
+                    const bool has_res = EPI && args.residual != nullptr && row_ok;
                     if (args.out_fp32) {
                         const uint32_t *v = part ? v1 : v0;
                         // mask-gated output: the 32 keep bits of these columns
@@ -368,7 +382,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int i = 0; i < 32; ++i) {
                             const float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[i]))
                                                               : __uint_as_float(v[i]);
-                            w[i] = ((keep_bits >> i) & 1u) ? __float_as_uint(__fmul_rn(a, scale)) : 0u;
+                            float y = __fmul_rn(a, scale);
+                            if constexpr (EPI) {
+                                // the residual of columns col + 8q .. + 7, one 16-byte load per 8
+                                const int q = i >> 3;
+                                const uint4 r4 = (has_res && col + 8 * q < args.N)
+                                                     ? *reinterpret_cast<const uint4 *>(args.residual + static_cast<int64_t>(m) * args.ldo + col + 8 * q)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                                const int e = i & 7;
+                                const uint32_t word = e < 2 ? r4.x : e < 4 ? r4.y : e < 6 ? r4.z : r4.w;
+                                y = epilogue_op(y, args.relu2, (word >> (16 * (e & 1))) & 0xffffu, has_res);
+                            }
+                            w[i] = ((keep_bits >> i) & 1u) ? __float_as_uint(y) : 0u;
                         }
                     } else {
 #pragma unroll
@@ -379,7 +404,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                                : __uint_as_float(v[k]);
                             const float a1 = (KIND == kKindI8) ? __int2float_rn(static_cast<int32_t>(v[k + 1]))
                                                                : __uint_as_float(v[k + 1]);
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(a0, scale), __fmul_rn(a1, scale));
+                            float y0 = __fmul_rn(a0, scale), y1 = __fmul_rn(a1, scale);
+                            if constexpr (EPI) {
+                                // word i of the residual row holds columns col + 2i, col + 2i + 1
+                                const int q = i >> 2;
+                                const uint4 r4 = (has_res && col + 8 * q < args.N)
+                                                     ? *reinterpret_cast<const uint4 *>(args.residual + static_cast<int64_t>(m) * args.ldo + col + 8 * q)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                                const int e = i & 3;
+                                const uint32_t word = e == 0 ? r4.x : e == 1 ? r4.y : e == 2 ? r4.z : r4.w;
+                                y0 = epilogue_op(y0, args.relu2, word & 0xffffu, has_res);
+                                y1 = epilogue_op(y1, args.relu2, word >> 16, has_res);
+                            }
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
                             w[i] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
                     }

@@ -44,6 +44,8 @@ struct Sp24Args {
     int32_t *acc_out;          // optional [T, O] int32
     const float *gamma;
     const float *d;            // [T]
+    int32_t relu2;             // output epilogue: v = max(v, 0)^2 ...
+    const uint16_t *residual;  // ... then v = v + residual[t, o] (bf16 [T, O]; nullptr: none)
     uint32_t *err;
 };
 
@@ -100,7 +102,8 @@ __device__ __forceinline__ void tmem_cp_128x256b_pair(uint32_t taddr, uint32_t s
     asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
-template <int BN>
+// EPI: the instantiation with the output epilogue (relu2 / residual).
+template <int BN, bool EPI = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     sp24_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                    static_cast<uint32_t>(acc * BN);
             constexpr int kChunks = BN / 32;
             constexpr int kMine = (kChunks + 1) / 2;  // chunks c = half, half + 2, ... (warp half 0 has the extra)
-            if (!args.out_fp32) {
+            if (!args.out_fp32 && !EPI) {
                 // bf16: drain every chunk of this warp, converting it to 16
                 // packed words of the transposed block (lanes 2i and 2i+1 swap
                 // one value so each holds a word of two weight rows: the even
@@ -343,7 +346,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 continue;
             }
-            // fp32: chunk by chunk, the accumulator handed back after the last load
+            // fp32, or any output with the epilogue: chunk by chunk, the
+            // accumulator handed back after the last load
 #pragma unroll 1
             for (int c = half; c < kChunks; c += 2) {
                 const int t0 = tn * BN + 32 * c;
@@ -364,14 +368,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (t0 + j < args.T)
                             args.acc_out[static_cast<int64_t>(t0 + j) * args.O + o] = static_cast<int32_t>(v[j]);
                 }
-                if (lane == 0) bulk_wait_group_read<0>();
+                if (lane == 0) bulk_wait_group_read<0>();  // every earlier store has read its staging
                 __syncwarp();
+                const bool has_res = EPI && args.residual != nullptr && o < args.O;
+                const bool odd = lane & 1;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float s = __shfl_sync(0xffffffffu, sc, j);
-                    const float y = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[j])), s);
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(buf + static_cast<uint32_t>(j * 128 + lane * 4)), "f"(y)
-                                 : "memory");
+                for (int j = 0; j < 32; j += 2) {
+                    float y[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float s = __shfl_sync(0xffffffffu, sc, j + h);
+                        y[h] = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[j + h])), s);
+                        if constexpr (EPI) {
+                            // the lanes of a warp read consecutive weight rows of one token
+                            const uint32_t rb = (has_res && t0 + j + h < args.T)
+                                                    ? args.residual[static_cast<int64_t>(t0 + j + h) * args.O + o]
+                                                    : 0u;
+                            y[h] = epilogue_op(y[h], args.relu2, rb, has_res);
+                        }
+                    }
+                    if (args.out_fp32) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            asm volatile("st.shared.f32 [%0], %1;" ::"r"(buf + static_cast<uint32_t>((j + h) * 128 + lane * 4)),
+                                         "f"(y[h])
+                                         : "memory");
+                    } else {
+                        // lanes 2i and 2i+1 swap one value: the even lane writes
+                        // token j of weight rows 2i, 2i+1, the odd lane token j+1
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? y[0] : y[1], 1);
+                        const __nv_bfloat162 b2 =
+                            odd ? __floats2bfloat162_rn(other, y[1]) : __floats2bfloat162_rn(y[0], other);
+                        const uint32_t addr = buf + static_cast<uint32_t>((j + (odd ? 1 : 0)) * 64 + (lane & ~1) * 2);
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(*reinterpret_cast<const uint32_t *>(&b2))
+                                     : "memory");
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();

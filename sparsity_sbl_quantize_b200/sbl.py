@@ -54,6 +54,10 @@ SBL_MASK_FROM_MASTER, SBL_MASK_FROM_QUANTIZED = 0, 1
 SBL_QUANT_THEN_MASK, SBL_MASK_THEN_QUANT = 0, 1
 
 
+class sbl_epilogue(ctypes.Structure):
+    _fields_ = [("relu2", ctypes.c_int32), ("residual", ctypes.c_void_p)]
+
+
 class sbl_mask_stats(ctypes.Structure):
     _fields_ = [("prev_keep", ctypes.c_void_p), ("keep", ctypes.c_void_p), ("flips", ctypes.c_void_p),
                 ("near_zero", ctypes.c_void_p), ("block_threshold", ctypes.c_void_p)]
@@ -88,6 +92,8 @@ _lib.sbl_forward.restype = ctypes.c_int
 _lib.sbl_forward.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, _P]
 _lib.sbl_backward_dual_ste.restype = ctypes.c_int
 _lib.sbl_backward_dual_ste.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _sz, _P]
+_lib.sbl_forward_ex.restype = ctypes.c_int
+_lib.sbl_forward_ex.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, ctypes.POINTER(sbl_epilogue), _P]
 _lib.sbl_forward_format.restype = ctypes.c_int
 _lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
@@ -95,7 +101,7 @@ _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
-            "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
+            "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
             "sbl_quantize_mask_pack_ex", "sbl_device_error"]
 
 
@@ -223,6 +229,17 @@ def sbl_forward(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, 
     cp = w.c()
     _check(_lib.sbl_forward(ctypes.byref(dsc), _ptr(Xq), _ptr(d), T, ctypes.byref(cp), fmt, _ptr(Y),
                             1 if y_is_fp32 else 0, _ptr(acc_out), _stream()), "sbl_forward")
+
+
+def sbl_forward_ex(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, w: Packed, fmt: int,
+                   Y: torch.Tensor, relu2: bool = False, residual: Optional[torch.Tensor] = None,
+                   acc_out: Optional[torch.Tensor] = None) -> None:
+    """sbl_forward with the Squared-ReLU / residual output epilogue."""
+    cp = w.c()
+    epi = sbl_epilogue(1 if relu2 else 0, residual.data_ptr() if residual is not None else None)
+    y_fp32 = 1 if Y.dtype == torch.float32 else 0
+    _check(_lib.sbl_forward_ex(ctypes.byref(dsc), _ptr(Xq), _ptr(d), T, ctypes.byref(cp), fmt, _ptr(Y), y_fp32,
+                               _ptr(acc_out), ctypes.byref(epi), _stream()), "sbl_forward_ex")
 
 
 def sbl_backward_dual_ste(dsc: sbl_layer_desc, dY: torch.Tensor, Xq: Optional[torch.Tensor],

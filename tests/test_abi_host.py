@@ -186,3 +186,13 @@ def test_mask_stats_validation(sbl):
     odd_thr = sbl.sbl_mask_stats(None, None, None, None, good + 4)
     assert _raw(sbl, "sbl_quantize_mask_pack_stats", ctypes.byref(d), P(good), sbl.SBL_FMT_I8, ctypes.byref(w),
                 ctypes.byref(odd_thr), P(good), 1 << 20, None) == 3
+
+
+def test_forward_epilogue_validation(sbl):
+    good = 0x10000
+    P = ctypes.c_void_p
+    d = sbl.desc(128, 256, 6, 8)
+    w = sbl.sbl_packed(None, None, None, good, None, good)
+    epi = sbl.sbl_epilogue(1, good + 2)  # misaligned residual
+    assert _raw(sbl, "sbl_forward_ex", ctypes.byref(d), P(good), P(good), 64, ctypes.byref(w), sbl.SBL_FMT_I8,
+                P(good), 0, None, ctypes.byref(epi), None) == 3

@@ -262,6 +262,35 @@ def test_forward_sp24_matches_dense_path_full_size(O, K, T):
     np.testing.assert_array_equal(accs.cpu().numpy()[it, io], oracle.acc_samples(qr, ref.weff, it, io))
 
 
+@pytest.mark.parametrize("fmt_name,O,K,T,n,m", [("I8", 528, 1040, 300, 6, 8), ("I8", 256, 128, 64, 2, 4),
+                                                ("SP24", 528, 1040, 300, 2, 4), ("SP24", 4864, 896, 96, 2, 4),
+                                                ("PK2", 384, 640, 9, 2, 4), ("PK2", 2560, 6912, 1, 2, 4)])
+@pytest.mark.parametrize("relu2,residual", [(True, False), (False, True), (True, True)])
+@pytest.mark.parametrize("fp32", [False, True])
+def test_forward_epilogue_bit_exact(fmt_name, O, K, T, n, m, relu2, residual, fp32):
+    """Squared ReLU and the residual add fused into every forward kernel:
+    bit for bit the oracle's dequantisation followed by its epilogue."""
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=O + T)
+    x = wl.activations(T, K, seed=O + T)
+    fmt = {"I8": sbl.SBL_FMT_I8, "PK2": sbl.SBL_FMT_PK2, "SP24": sbl.SBL_FMT_SP24}[fmt_name]
+    layer = GpuLayer(w, n, m, fmt)
+    ref = oracle.Layer(w, n, m)
+    q, d = quantize_act(x)
+    qr, dr, accr, yr, _ = ref.forward(x)
+    res_bits = (wl.activations(T, O, seed=O + T + 1)) if residual else None
+    out, outb = oracle.epilogue(yr, relu2=relu2, residual_bf16_bits=res_bits)
+    y = torch.empty((T, O), dtype=torch.float32 if fp32 else torch.bfloat16, device="cuda")
+    acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+    sbl.sbl_forward_ex(layer.desc, q, d, T, layer.packed, fmt, y, relu2=relu2,
+                       residual=bf16_dev(res_bits) if residual else None, acc_out=acc)
+    np.testing.assert_array_equal(acc.cpu().numpy(), accr)
+    if fp32:
+        np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), out.view(np.uint32))
+    else:
+        np.testing.assert_array_equal(bits_of(y), outb)
+
+
 def test_forward_zero_tokens_is_noop():
     sbl = sbl_mod()
     layer = GpuLayer(wl.master_weights(32, 64, seed=1), 6, 8, 4)
