@@ -49,6 +49,7 @@ def _load():
         lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
         lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
         lib.sbl_oracle_epilogue.argtypes = [p, i64, i64, i32, p, p, p]
+        lib.sbl_oracle_rmsnorm_quantize_act.argtypes = [p, i64, i64, p, f32, p, p]
         lib.sbl_oracle_gamma_survivors.restype = f32
         lib.sbl_oracle_gamma_survivors.argtypes = [p, p, i64, i64]
         lib.sbl_oracle_nm_mask_quantized.argtypes = [p, i64, i64, i32, i32, p]
@@ -268,6 +269,18 @@ def dequant(acc, g, d):
     yb = np.empty((t, o), dtype=np.uint16)
     _load().sbl_oracle_dequant(_ptr(acc), t, o, float(np.float32(g)), _ptr(d), _ptr(y), _ptr(yb))
     return y, yb
+
+
+def rmsnorm_quantize_act(x_bf16_bits, g_bf16_bits=None, eps: float = 1e-5):
+    """RMSNorm fused with the activation quantiser -> (q int8 [T, K], d fp32 [T])."""
+    x = _u16(x_bf16_bits)
+    t, k = x.shape
+    g = None if g_bf16_bits is None else _u16(g_bf16_bits)
+    q = np.empty((t, k), dtype=np.int8)
+    d = np.empty((t,), dtype=np.float32)
+    _load().sbl_oracle_rmsnorm_quantize_act(_ptr(x), t, k, _ptr(g) if g is not None else None, float(eps),
+                                            _ptr(q), _ptr(d))
+    return q, d
 
 
 def epilogue(y, relu2: bool = False, residual_bf16_bits=None):

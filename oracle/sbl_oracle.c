@@ -418,6 +418,61 @@ void sbl_oracle_dequant(const int32_t *acc, int64_t tokens, int64_t d_out,
     }
 }
 
+/* Pairwise tree (R1's shape) over the squares of a row of bf16 values, fp64:
+ * each square of a bf16 value is exact in fp64. */
+static double square_sum_tree(const uint16_t *x, int64_t lo, int64_t n)
+{
+    if (n <= 0) return 0.0;
+    if (n == 1) {
+        double v = (double)bf16_to_f32(x[lo]);
+        return v * v;
+    }
+    int64_t h = 1;
+    while (h * 2 < n) h *= 2;
+    double left = square_sum_tree(x, lo, h);
+    double right = square_sum_tree(x, lo + h, n - h);
+    return left + right;
+}
+
+/* The norm before the activation quantiser ([P1] forward step 1:
+ * x~ = Q_a(Norm(x)), Norm being RMSNorm) fused with it:
+ *   r   = fl32(1 / sqrt(S / K + eps)) in fp64, S = the pairwise tree of
+ *         x_k^2 over the row in flat order;
+ *   u_k = fl32(fl32(x_k * r) * g_k)   (g: bf16 gains, 1 when absent);
+ * then the quantiser of sbl_oracle_quantize_act on the fp32 u (a = max|u|,
+ * q = clamp(rint(fl32(u * fl32(127 / a)))), d = fl32(a / 127); a == 0 gives
+ * q = 0, d = 0). */
+void sbl_oracle_rmsnorm_quantize_act(const uint16_t *x, int64_t tokens, int64_t d_in, const uint16_t *g,
+                                     float eps, int8_t *q, float *d)
+{
+    for (int64_t t = 0; t < tokens; ++t) {
+        const uint16_t *row = x + t * d_in;
+        double s = square_sum_tree(row, 0, d_in);
+        float r = (float)(1.0 / sqrt(s / (double)d_in + (double)eps));
+        float a = 0.0f;
+        for (int64_t k = 0; k < d_in; ++k) {
+            float u = bf16_to_f32(row[k]) * r;
+            if (g) u = u * bf16_to_f32(g[k]);
+            if (fabsf(u) > a) a = fabsf(u);
+        }
+        if (a == 0.0f) {
+            for (int64_t k = 0; k < d_in; ++k) q[t * d_in + k] = 0;
+            d[t] = 0.0f;
+            continue;
+        }
+        float rq = 127.0f / a;
+        for (int64_t k = 0; k < d_in; ++k) {
+            float u = bf16_to_f32(row[k]) * r;
+            if (g) u = u * bf16_to_f32(g[k]);
+            float v = nearbyintf(u * rq);
+            if (v > 127.0f) v = 127.0f;
+            if (v < -128.0f) v = -128.0f;
+            q[t * d_in + k] = (int8_t)v;
+        }
+        d[t] = a / 127.0f;
+    }
+}
+
 /* Output epilogue after the layer ("Squared ReLU Activation in the
  * Feed-Forward Network" of the BitNet b1.58 2B4T summary: ReLU^2(x) =
  * max(0, x)^2, applied to the projection's output; and a residual add):

@@ -21,7 +21,8 @@ MUTANTS = {
                           "h = n / 2;\n    double left = abs_sum_tree(w, lo, h);"),
     "gamma_over_dout_only": ("return (float)(s / (double)count);", "return (float)(s / (double)d_in);"),
     "act_divide_form": ("float s = bf16_to_f32(row[k]) * r;", "float s = bf16_to_f32(row[k]) / a * 127.0f;"),
-    "act_scale_dropped": ("d[t] = a / 127.0f;", "d[t] = a;"),
+    "act_scale_dropped": ("float v = nearbyintf(s);\n            if (v > 127.0f) v = 127.0f;\n            if (v < -128.0f) v = -128.0f;\n            q[t * d_in + k] = (int8_t)v;\n        }\n        d[t] = a / 127.0f;",
+                          "float v = nearbyintf(s);\n            if (v > 127.0f) v = 127.0f;\n            if (v < -128.0f) v = -128.0f;\n            q[t * d_in + k] = (int8_t)v;\n        }\n        d[t] = a;"),
     "dequant_token_scale_dropped": ("float c = gamma * d[t];", "float c = gamma;"),
     "dw_token_scale_dropped": ("(double)bf16_to_f32(dy[t * d_out + o]) * (double)d[t] *\n                         (double)q[t * d_in + k];",
                                "(double)bf16_to_f32(dy[t * d_out + o]) *\n                         (double)q[t * d_in + k];"),
@@ -44,6 +45,12 @@ MUTANTS = {
     "relu_not_squared": ("if (relu2) v = v > 0.0f ? v * v : 0.0f;", "if (relu2) v = v > 0.0f ? v : 0.0f;"),
     "residual_before_activation": ("if (relu2) v = v > 0.0f ? v * v : 0.0f;\n        if (res) v = v + bf16_to_f32(res[i]);",
                                    "if (res) v = v + bf16_to_f32(res[i]);\n        if (relu2) v = v > 0.0f ? v * v : 0.0f;"),
+    "rmsnorm_eps_dropped": ("float r = (float)(1.0 / sqrt(s / (double)d_in + (double)eps));",
+                            "float r = (float)(1.0 / sqrt(s / (double)d_in));"),
+    "rmsnorm_mean_over_k_minus_1": ("float r = (float)(1.0 / sqrt(s / (double)d_in + (double)eps));",
+                                    "float r = (float)(1.0 / sqrt(s / (double)(d_in - 1) + (double)eps));"),
+    "rmsnorm_gain_ignored": ("            float u = bf16_to_f32(row[k]) * r;\n            if (g) u = u * bf16_to_f32(g[k]);\n            float v = nearbyintf(u * rq);",
+                             "            float u = bf16_to_f32(row[k]) * r;\n            float v = nearbyintf(u * rq);"),
     "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
                            "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
 }
@@ -66,6 +73,7 @@ PIN_CALLS = [
     (pins.test_sp24_roundtrip, (2, 4)),
     (pins.test_sp24_roundtrip, (1, 4)),
     (pins.test_epilogue_hand_values, ()),
+    (pins.test_rmsnorm_quant_matches_numpy_definition, ()),
     (pins.test_gamma_survivors_hand_row_and_exact_mean, ()),
     (pins.test_mask_from_quantized_hand_and_brute_force, ()),
     (pins.test_mask_flips_matches_numpy_and_invariants, ()),

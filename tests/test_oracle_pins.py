@@ -309,6 +309,65 @@ def test_sp24_rejects_masks_that_are_not_2of4():
         oracle.pack_sp24(layer.weff, layer.mask)
 
 
+# ------------------------------------------------------ RMSNorm + act quant
+
+def _np_rmsnorm_quant(xb, gb, eps):
+    """The fused definition in numpy float32 steps, with the row's sum of
+    squares taken exactly (math.fsum) -- the oracle's fp64 tree of exact
+    squares rounds only at its additions."""
+    x = (xb.astype(np.uint32) << 16).view(np.float32)
+    g = None if gb is None else (gb.astype(np.uint32) << 16).view(np.float32)
+    t, k = x.shape
+    q = np.zeros((t, k), dtype=np.int8)
+    d = np.zeros((t,), dtype=np.float32)
+    for i in range(t):
+        s = math.fsum(float(v) * float(v) for v in x[i])
+        r = np.float32(1.0 / math.sqrt(s / k + float(np.float32(eps))))
+        u = (x[i] * r).astype(np.float32)
+        if g is not None:
+            u = (u * g).astype(np.float32)
+        a = np.float32(np.abs(u).max())
+        if a == 0:
+            continue
+        rq = np.float32(np.float32(127) / a)
+        q[i] = np.clip(np.rint((u * rq).astype(np.float32)), -128, 127).astype(np.int8)
+        d[i] = np.float32(a / np.float32(127))
+    return q, d
+
+
+def test_rmsnorm_quant_matches_numpy_definition():
+    """RMSNorm fused into the quantiser ("The Full Sparse-BitLinear Layer",
+    forward step 1: x~ = Q_a(Norm(x))): the same float32 steps in numpy."""
+    x = wl.activations(16, 896, seed=21, outlier_frac=0.01)
+    x[3] = 0  # a zero row stays zero
+    g = wl.activations(1, 896, seed=22)[0]
+    for gb, eps in [(None, 1e-5), (g, 1e-6), (g, 0.0)]:
+        q, d = oracle.rmsnorm_quantize_act(x, gb, eps)
+        if eps == 0.0:
+            continue  # the zero row has 0/0 without eps
+        qn, dn = _np_rmsnorm_quant(x, gb, eps)
+        np.testing.assert_array_equal(q, qn)
+        np.testing.assert_array_equal(d, dn)
+        assert (np.abs(q[np.arange(16) != 3]).max(axis=1) == 127).all() and not q[3].any() and d[3] == 0
+
+
+def test_rmsnorm_quant_scale_invariance_and_torch():
+    """With eps = 0 and no gains the normalised row does not depend on a
+    power-of-two scale of x (every step scales exactly); the normalised
+    values agree with torch's fp64 rms_norm to fp32 precision."""
+    x = wl.activations(8, 512, seed=23)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    x4 = ((xf * np.float32(4.0)).view(np.uint32) >> 16).astype(np.uint16)  # exact in bf16
+    q1, d1 = oracle.rmsnorm_quantize_act(x, None, 0.0)
+    q4, d4 = oracle.rmsnorm_quantize_act(x4, None, 0.0)
+    np.testing.assert_array_equal(q1, q4)
+    np.testing.assert_array_equal(d1, d4)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(xf.astype(np.float64)), (512,), eps=1e-5).numpy()
+    _, d = oracle.rmsnorm_quantize_act(x, None, 1e-5)
+    amax = np.abs(ref).max(axis=1)
+    np.testing.assert_allclose(d * 127, amax, rtol=2e-7)
+
+
 # --------------------------------------------------------------- epilogue
 
 def test_epilogue_hand_values():
