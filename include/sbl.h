@@ -253,6 +253,17 @@ sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const floa
 sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K,
                             int8_t *Xq, float *d, void *stream);
 
+/* RMSNorm fused with the activation quantiser (forward step 1 of the
+ * Sparse-BitNet summary, x~ = Q_a(Norm(x)), Norm read as RMSNorm): per
+ * token, S = the sum of x_k^2 in fp64 over the pairwise tree of the row
+ * (flat order, as for gamma), r = fl32(1 / sqrt(S / K + eps)) computed in
+ * fp64, u_k = fl32(fl32(x_k * r) * g_k) with g the bf16 gains [K] (NULL: 1),
+ * then exactly the quantiser of sbl_quantize_act applied to the fp32 u (no
+ * bf16 rounding in between).  eps: finite, >= 0 (a zero row needs eps > 0).
+ * Shapes, outputs and errors as sbl_quantize_act.  One launch. */
+sbl_status sbl_quantize_act_rmsnorm(const uint16_t *X, int32_t T, int32_t K, const uint16_t *g,
+                                    float eps, int8_t *Xq, float *d, void *stream);
+
 /* Step 5 of the forward: acc[t,o] = sum_k W_eff[o,k] * Xq[t,k] (int32), and
  *   Y[t,o] = fl32(fl32(acc) * fl32(gamma * d[t]))  (bf16 by RNE, or fp32).
  * fmt selects the weight operand: SBL_FMT_I8 runs the tcgen05 int8 tensor

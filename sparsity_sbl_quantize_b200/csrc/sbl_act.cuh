@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
     constexpr int kRowsPerCta = RT >= 256 ? 1 : 256 / RT;
     constexpr int kWarpsPerRow = RT / 32 > 0 ? RT / 32 : 1;
     __shared__ float red[kRowsPerCta][kWarpsPerRow];
+    __shared__ float rsh[kRowsPerCta];
     const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + sub;
     // programmatic dependent launch: X may come from the previous kernel
@@ -88,6 +89,139 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
             }
             reinterpret_cast<uint2 *>(Xq + row * K)[ci] = out;
         }
+    }
+    if (lt == 0) d[row] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
+}
+
+// RMSNorm fused with the quantiser (the norm before Q_a in forward step 1 of
+// the Sparse-BitNet summary): per row, S = sum of x_k^2 in fp64 over the
+// pairwise tree of the row in flat order, r = fl32(1 / sqrt(S / K + eps)),
+// u_k = fl32(fl32(x_k * r) * g_k) (g: bf16 gains, none = 1), then the
+// absmax int8 quantisation of u.  The tree follows the thread layout: thread
+// lt holds chunks ci = lt + c * RT (8 elements each, an aligned 8-leaf
+// subtree); for a fixed slot c the chunks of consecutive lanes are adjacent,
+// so lane butterflies, then a pairwise combination of the row's warps (RT a
+// power of two >= 32), then a pairwise tree over the 8 slots give exactly
+// the row's tree (the tail beyond K is +0.0, which leaves every sum exact).
+template <int RT>
+__global__ void __launch_bounds__(RT > 256 ? RT : 256)
+    act_norm_quant_kernel(const uint16_t *__restrict__ X, int32_t T, int32_t K, const uint16_t *__restrict__ g,
+                          float eps, int8_t *__restrict__ Xq, float *__restrict__ d)
+{
+    static_assert(RT >= 32 && (RT & (RT - 1)) == 0, "rows are whole warps, a power of two");
+    constexpr int kRowsPerCta = RT >= 256 ? 1 : 256 / RT;
+    constexpr int kWarpsPerRow = RT / 32;
+    __shared__ double slots[kRowsPerCta][kWarpsPerRow][kActMaxChunks];
+    __shared__ float red[kRowsPerCta][kWarpsPerRow];
+    __shared__ float rsh[kRowsPerCta];
+    const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
+    const int wr = lt >> 5, lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + sub;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const bool active = row < T;
+    const int chunks = K / 8;
+
+    uint4 v[kActMaxChunks];
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const int ci = lt + c * RT;
+        v[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (active && ci < chunks) v[c] = __ldg(reinterpret_cast<const uint4 *>(X + row * K) + ci);
+    }
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        double sq[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const double lo = static_cast<double>(bf16_lo(w[i])), hi = static_cast<double>(bf16_hi(w[i]));
+            sq[2 * i] = lo * lo;  // exact: a bf16 square has at most 16 significant bits
+            sq[2 * i + 1] = hi * hi;
+        }
+        double cs = ((sq[0] + sq[1]) + (sq[2] + sq[3])) + ((sq[4] + sq[5]) + (sq[6] + sq[7]));
+        // adjacent lanes first: every lane ends with the warp's subtree (a + b == b + a exactly)
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) cs = cs + __shfl_xor_sync(0xffffffffu, cs, off);
+        if (lane == 0) slots[sub][wr][c] = cs;
+    }
+    __syncthreads();
+    if (wr == 0) {
+        // the row's first warp: per slot, the warps' subtrees pairwise in warp
+        // order (lanes >= kWarpsPerRow hold zeros in groups of their own); lane
+        // c keeps slot c; then the 8 slots pairwise over lanes 0..7
+        double mine = 0.0;
+#pragma unroll
+        for (int c = 0; c < kActMaxChunks; ++c) {
+            double x = lane < kWarpsPerRow ? slots[sub][lane][c] : 0.0;
+#pragma unroll
+            for (int off = 1; off < kWarpsPerRow; off <<= 1) x = x + __shfl_xor_sync(0xffffffffu, x, off);
+            x = __shfl_sync(0xffffffffu, x, 0);
+            if (lane == c) mine = x;
+        }
+#pragma unroll
+        for (int off = 1; off < kActMaxChunks; off <<= 1) mine = mine + __shfl_xor_sync(0xffffffffu, mine, off);
+        if (lane == 0) {
+            const double S = mine;
+            rsh[sub] = __double2float_rn(__ddiv_rn(
+                1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps)))));
+        }
+    }
+    __syncthreads();
+    const float r = rsh[sub];
+
+    // u = fl32(fl32(x * r) * g): absmax over the row, then quantise
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const int ci = lt + c * RT;
+        if (!(active && ci < chunks)) continue;
+        const uint4 gv = g ? __ldg(reinterpret_cast<const uint4 *>(g) + ci) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float u0 = __fmul_rn(bf16_lo(w[i]), r), u1 = __fmul_rn(bf16_hi(w[i]), r);
+            if (g) {
+                u0 = __fmul_rn(u0, bf16_lo(gw[i]));
+                u1 = __fmul_rn(u1, bf16_hi(gw[i]));
+            }
+            amax = fmaxf(amax, fmaxf(fabsf(u0), fabsf(u1)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) red[sub][wr] = amax;
+    __syncthreads();
+    amax = red[sub][0];
+#pragma unroll
+    for (int w = 1; w < kWarpsPerRow; ++w) amax = fmaxf(amax, red[sub][w]);
+    if (!active) return;
+    const bool zero = !(amax > 0.0f);
+    const float rq = zero ? 0.0f : __fdiv_rn(127.0f, amax);
+#pragma unroll
+    for (int c = 0; c < kActMaxChunks; ++c) {
+        const int ci = lt + c * RT;
+        if (ci >= chunks) continue;
+        uint2 out = make_uint2(0u, 0u);
+        if (!zero) {
+            const uint4 gv = g ? __ldg(reinterpret_cast<const uint4 *>(g) + ci) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            float u[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                u[2 * i] = __fmul_rn(bf16_lo(w[i]), r);
+                u[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), r);
+                if (g) {
+                    u[2 * i] = __fmul_rn(u[2 * i], bf16_lo(gw[i]));
+                    u[2 * i + 1] = __fmul_rn(u[2 * i + 1], bf16_hi(gw[i]));
+                }
+            }
+            out.x = quant4(u[0], u[1], u[2], u[3], rq);
+            out.y = quant4(u[4], u[5], u[6], u[7], rq);
+        }
+        reinterpret_cast<uint2 *>(Xq + row * K)[ci] = out;
     }
     if (lt == 0) d[row] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
 }

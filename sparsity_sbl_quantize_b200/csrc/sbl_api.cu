@@ -658,6 +658,52 @@ sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq,
     return launch_status();
 }
 
+sbl_status sbl_quantize_act_rmsnorm(const uint16_t *X, int32_t T, int32_t K, const uint16_t *g, float eps, int8_t *Xq,
+                                    float *d, void *stream_p)
+{
+    if (T < 0 || K < 16 || K % 16 != 0 || K > kMaxDim) return SBL_ERR_SHAPE;
+    if (T == 0) return SBL_OK;
+    if (!X || !Xq || !d) return SBL_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return SBL_ERR_INVALID_ARG;  // finite, non-negative
+    if (!aligned16(X) || !aligned16(Xq) || !aligned16(d) || (g && !aligned16(g))) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    const int chunks = K / 8;
+    int rt = 32;
+    while (rt * kActMaxChunks < chunks) rt *= 2;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaSuccess;
+    switch (rt) {
+#define SBL_ACT_CASE(R)                                                        \
+    case R: {                                                                 \
+        constexpr int rows = R >= 256 ? 1 : 256 / R;                          \
+        cfg.gridDim = dim3(static_cast<unsigned>((T + rows - 1) / rows));     \
+        cfg.blockDim = dim3(R > 256 ? R : 256);                               \
+        e = cudaLaunchKernelEx(&cfg, act_norm_quant_kernel<R>, X, T, K, g, eps, Xq, d); \
+        break;                                                                \
+    }
+        SBL_ACT_CASE(32)
+        SBL_ACT_CASE(64)
+        SBL_ACT_CASE(128)
+        SBL_ACT_CASE(256)
+        SBL_ACT_CASE(512)
+        SBL_ACT_CASE(1024)
+#undef SBL_ACT_CASE
+    default: return SBL_ERR_SHAPE;
+    }
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+    return launch_status();
+}
+
 }  // extern "C"
 
 static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,

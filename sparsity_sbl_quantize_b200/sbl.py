@@ -88,6 +88,8 @@ _lib.sbl_quantize_mask_pack_noalloc.restype = ctypes.c_int
 _lib.sbl_quantize_mask_pack_noalloc.argtypes = [_D, _P, _u32, _W, _P]
 _lib.sbl_quantize_act.restype = ctypes.c_int
 _lib.sbl_quantize_act.argtypes = [_P, _i32, _i32, _P, _P, _P]
+_lib.sbl_quantize_act_rmsnorm.restype = ctypes.c_int
+_lib.sbl_quantize_act_rmsnorm.argtypes = [_P, _i32, _i32, _P, ctypes.c_float, _P, _P, _P]
 _lib.sbl_forward.restype = ctypes.c_int
 _lib.sbl_forward.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, _P]
 _lib.sbl_backward_dual_ste.restype = ctypes.c_int
@@ -100,7 +102,7 @@ _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
-            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_forward",
+            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward",
             "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
             "sbl_quantize_mask_pack_ex", "sbl_device_error"]
 
@@ -222,6 +224,12 @@ def sbl_quantize_mask_pack_noalloc(d: sbl_layer_desc, W: torch.Tensor, formats: 
 
 def sbl_quantize_act(X: torch.Tensor, T: int, K: int, Xq: torch.Tensor, d: torch.Tensor) -> None:
     _check(_lib.sbl_quantize_act(_ptr(X), T, K, _ptr(Xq), _ptr(d), _stream()), "sbl_quantize_act")
+
+
+def sbl_quantize_act_rmsnorm(X: torch.Tensor, T: int, K: int, g: Optional[torch.Tensor], eps: float,
+                             Xq: torch.Tensor, d: torch.Tensor) -> None:
+    _check(_lib.sbl_quantize_act_rmsnorm(_ptr(X), T, K, _ptr(g), float(eps), _ptr(Xq), _ptr(d), _stream()),
+           "sbl_quantize_act_rmsnorm")
 
 
 def sbl_forward(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, w: Packed, fmt: int,

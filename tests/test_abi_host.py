@@ -103,6 +103,18 @@ def test_validation_happens_before_any_device_access(sbl):
     assert _raw(sbl, "sbl_quantize_act", None, 4, 256, P(good), P(good), None) == 1
     assert _raw(sbl, "sbl_quantize_act", P(good + 4), 4, 256, P(good), P(good), None) == 3
     assert _raw(sbl, "sbl_quantize_act", P(good), 0, 256, P(good), P(good), None) == 0  # T == 0: no-op
+    F = ctypes.c_float
+    rms = "sbl_quantize_act_rmsnorm"
+    assert _raw(sbl, rms, P(good), 4, 250, None, F(1e-5), P(good), P(good), None) == 2
+    assert _raw(sbl, rms, P(good), 4, 2 * 65536, None, F(1e-5), P(good), P(good), None) == 2
+    assert _raw(sbl, rms, None, 4, 256, None, F(1e-5), P(good), P(good), None) == 1
+    assert _raw(sbl, rms, P(good), 4, 256, None, F(-1.0), P(good), P(good), None) == 1
+    assert _raw(sbl, rms, P(good), 4, 256, None, F(float("nan")), P(good), P(good), None) == 1
+    assert _raw(sbl, rms, P(good), 4, 256, None, F(float("inf")), P(good), P(good), None) == 1
+    assert _raw(sbl, rms, P(good), 4, 256, P(good + 2), F(1e-5), P(good), P(good), None) == 3
+    assert _raw(sbl, rms, P(good), 0, 256, None, F(1e-5), P(good), P(good), None) == 0
+    assert _raw(sbl, rms, P(good), 4, 256, None, F(1e-5), P(good), P(good), None) == 7  # no sm_100 device here
+    assert _raw(sbl, rms, P(good), 4, 256, P(good), F(0.0), P(good), P(good), None) == 7
     d = sbl.desc(128, 256, 6, 8)
     w = sbl.sbl_packed(None, None, None, good, good, good)
     st = _raw(sbl, "sbl_forward", ctypes.byref(d), P(good), P(good), 64, ctypes.byref(w),

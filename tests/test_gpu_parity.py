@@ -172,6 +172,47 @@ def test_act_quant_bit_exact(T, K):
     np.testing.assert_array_equal(d.cpu().numpy()[:T], dr)
 
 
+def _gains(K, seed):
+    rng = np.random.default_rng(seed)
+    return wl.f32_to_bf16_bits(rng.normal(1.0, 0.25, size=K).astype(np.float32))
+
+
+def rmsnorm_quantize_act(x_bits, g_bits, eps):
+    sbl = sbl_mod()
+    t, k = x_bits.shape
+    q = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    d = torch.empty((max(t, 1),), dtype=torch.float32, device="cuda")
+    g = None if g_bits is None else bf16_dev(g_bits)
+    sbl.sbl_quantize_act_rmsnorm(bf16_dev(x_bits), t, k, g, eps, q, d)
+    return q, d
+
+
+# every thread-row width (32 .. 1024 threads), 1 .. 8 chunks per thread, ragged
+# K within a slot, multi-row CTAs with an inactive tail row
+@pytest.mark.parametrize("T,K", [(64, 256), (300, 1040), (1, 16), (7, 8960), (33, 11008), (5, 32768),
+                                 (3, 65536), (9, 40960), (130, 2048), (5, 4112)])
+@pytest.mark.parametrize("gains", [False, True])
+def test_rmsnorm_act_quant_bit_exact(T, K, gains):
+    x = wl.activations(T, K, seed=3 * T + K, outlier_frac=0.01)
+    x[0] = 0  # an all-zero token: S = 0, r = 1/sqrt(eps), q = 0, d = 0
+    if T > 2:
+        x[2] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(x[2]) * np.float32(1e-30))  # tiny magnitudes
+    g = _gains(K, K) if gains else None
+    for eps in (1e-5, 1e-6):
+        q, d = rmsnorm_quantize_act(x, g, eps)
+        qr, dr = oracle.rmsnorm_quantize_act(x, g, eps)
+        np.testing.assert_array_equal(q.cpu().numpy(), qr)
+        np.testing.assert_array_equal(d.cpu().numpy()[:T], dr)
+
+
+def test_rmsnorm_act_quant_eps_zero_nonzero_rows():
+    x = wl.activations(40, 896, seed=11)
+    q, d = rmsnorm_quantize_act(x, None, 0.0)
+    qr, dr = oracle.rmsnorm_quantize_act(x, None, 0.0)
+    np.testing.assert_array_equal(q.cpu().numpy(), qr)
+    np.testing.assert_array_equal(d.cpu().numpy()[:40], dr)
+
+
 # ------------------------------------------------------------------- forward
 
 def run_forward_full_check(O, K, T, n, m, seed, fmt_name="I8", outliers=0.0):
