@@ -38,14 +38,19 @@ METRIC = "Sparse-BitLinear int8 TOPS (prefill/train) & decode GB/s, % of B200 ro
 L2_FLUSH_BYTES = 512 << 20
 LONG_STEP_MS = 1.0  # steps longer than this run at the power-capped (sustained) clock
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
-# the device code of the roofline kernels (the GEMMs and the decode GEMV)
-KERNEL_SOURCES = ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh", "sbl_decode.cuh")
+# the device code of each family of roofline kernels (the GEMMs, the decode GEMV)
+KERNEL_SOURCES = {"gemm": ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh"),
+                  "decode": ("sbl_device.cuh", "sbl_act.cuh", "sbl_decode.cuh")}
+
+
+def kernel_family(workload: str) -> str:
+    return "decode" if wl.WORKLOADS[workload].mode == "decode" else "gemm"
 
 
 UNIT_BYTES = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1024, "MB": 1 << 20, "GB": 1 << 30}
 
 
-def record_traffic(csv_path: str, workload: str, kernel_regex: str, command: str) -> dict:
+def record_traffic(csv_paths, workload: str, kernel_regex: str, command: str) -> dict:
     """Parse an ncu --csv metric list (dram__bytes_read.sum and
     dram__bytes_write.sum per launch) and store the mean read+write bytes per
     launch of the kernels matching kernel_regex for `workload`, tagged with
@@ -54,18 +59,19 @@ def record_traffic(csv_path: str, workload: str, kernel_regex: str, command: str
     import re
     pat = re.compile(kernel_regex)
     per_launch = {}
-    with open(csv_path) as f:
-        lines = [ln for ln in f if ln.startswith('"')]
-    for row in csv.DictReader(lines):
-        if not pat.search(row["Kernel Name"]) or not row["Metric Name"].startswith("dram__bytes_"):
-            continue
-        val = float(row["Metric Value"].replace(",", "")) * UNIT_BYTES[row["Metric Unit"]]
-        per_launch[row["ID"]] = per_launch.get(row["ID"], 0.0) + val
+    for fi, csv_path in enumerate(csv_paths):
+        with open(csv_path) as f:
+            lines = [ln for ln in f if ln.startswith('"')]
+        for row in csv.DictReader(lines):
+            if not pat.search(row["Kernel Name"]) or not row["Metric Name"].startswith("dram__bytes_"):
+                continue
+            val = float(row["Metric Value"].replace(",", "")) * UNIT_BYTES[row["Metric Unit"]]
+            per_launch[(fi, row["ID"])] = per_launch.get((fi, row["ID"]), 0.0) + val
     if not per_launch:
-        raise SystemExit(f"no launches of {kernel_regex} with DRAM metrics in {csv_path}")
+        raise SystemExit(f"no launches of {kernel_regex} with DRAM metrics in {csv_paths}")
     rec = {"kernel_regex": kernel_regex, "launches": len(per_launch),
            "bytes_per_launch": round(sum(per_launch.values()) / len(per_launch)),
-           "kernel_source_sha256": kernel_source_hash(), "command": command}
+           "kernel_source_sha256": kernel_source_hash(kernel_family(workload)), "command": command}
     data = {}
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
@@ -77,12 +83,12 @@ def record_traffic(csv_path: str, workload: str, kernel_regex: str, command: str
     return rec
 
 
-def kernel_source_hash() -> str:
-    """SHA-256 over the CUDA sources of the timed kernels: a stored DRAM
-    traffic figure is reported only while these are unchanged."""
+def kernel_source_hash(family: str) -> str:
+    """SHA-256 over the CUDA sources of a family of timed kernels: a stored
+    DRAM traffic figure is reported only while these are unchanged."""
     import hashlib
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[family]:
         with open(os.path.join(ROOT, "sparsity_sbl_quantize_b200", "csrc", name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
@@ -97,7 +103,7 @@ def stored_traffic(workload: str):
             rec = json.load(f).get(workload)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("kernel_source_sha256") != kernel_source_hash():
+    if not rec or rec.get("kernel_source_sha256") != kernel_source_hash(kernel_family(workload)):
         return None
     return rec.get("bytes_per_launch")
 
@@ -110,7 +116,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen05b_mlp", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+    ap.add_argument("--record-traffic", metavar="NCU_CSV", nargs="+",
                     help="store the mean DRAM bytes per roofline-kernel launch from an ncu --csv metric list "
                          "(dram__bytes_read.sum, dram__bytes_write.sum) for --workload, then exit")
     ap.add_argument("--traffic-command", default="", help="the ncu command that produced NCU_CSV (recorded)")
@@ -180,15 +186,28 @@ class ClockSampler:
         self.uuid = uuid
 
     def start(self):
+        """Start sampling every 50 ms and wait (up to 5 s) for the first row,
+        so that the timed region that follows is covered from its start."""
         try:
-            cmd = ["nvidia-smi", "--query-gpu=uuid," + self.FIELDS, "--format=csv,noheader,nounits",
+            cmd = ["nvidia-smi", "--query-gpu=timestamp,uuid," + self.FIELDS, "--format=csv,noheader,nounits",
                    "-lms", "50"]
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        deadline = time.time() + 5.0
+        while time.time() < deadline and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
 
-    def stop(self):
+    def mark(self):
+        """Host wall-clock time of the start or the end of the timed region."""
+        return time.time()
+
+    def stop(self, *windows):
+        """Stop sampling; summarise the rows taken inside the (t0, t1) host
+        wall-clock windows of the timed regions, or all rows when none fall
+        inside."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -197,21 +216,27 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
+        import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
+            if len(parts) < 9 or (self.uuid and self.uuid not in parts[1]):
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[4:8]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[5:9]))
             except ValueError:
                 continue
-        if not rows:
+        inside = [r for r in rows if any(t0 <= r[0] <= t1 for t0, t1 in windows)]
+        window = "timed region"
+        if not inside:
+            inside, window = rows, "around the timed region (shorter than the 50 ms sampling period)"
+        if not inside:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for *_, r in inside for i in range(4) if r[i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
 
 
 # -------------------------------------------------------------- our impl
@@ -481,6 +506,7 @@ def run_ours(args, wk):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    t_wall0 = clocks.mark()
     # timed region 1: whole steps (the value)
     times = []
     s0 = torch.cuda.Event(enable_timing=True)
@@ -502,7 +528,7 @@ def run_ours(args, wk):
         gemm_ms += sum(a.elapsed_time(b) for a, b, _ in r.kernel_events)
         gemm_ops += sum(o for _, _, o in r.kernel_events)
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    clk = clocks.stop((t_wall0, clocks.mark()))
     if world > 1:
         dist.barrier()
     total_ms = max_over_ranks(sum(times), dist, world, device)
@@ -603,7 +629,8 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 128 << 20)
     clocks = ClockSampler(str(getattr(props, "uuid", "")) or None)
-    clk = None
+    clocks.start()
+    windows = []
     results = {}
     n, m = wk.patterns[0]
     for T in wk.tokens:
@@ -632,15 +659,16 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.stream(s):
                 for lin, dsc, copies, x, q, d, y, _ in layers:  # warm outside capture
-                    sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
+                    sbl.sbl_linear_forward(dsc, x, T, copies[0], sbl.SBL_FMT_PK2, q, d, y)
                     sbl.sbl_forward(dsc, q, d, T, copies[0], sbl.SBL_FMT_PK2, y)
                 torch.cuda.synchronize()
                 with torch.cuda.graph(g, stream=s):
                     for lin, dsc, copies, x, q, d, y, _ in layers:
                         for p in copies:
-                            if mode == "step":
-                                sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
-                            sbl.sbl_forward(dsc, q, d, T, p, sbl.SBL_FMT_PK2, y)
+                            if mode == "step":  # the layer from its bf16 input: Q_a + GEMV
+                                sbl.sbl_linear_forward(dsc, x, T, p, sbl.SBL_FMT_PK2, q, d, y)
+                            else:  # the GEMV alone from the int8 activations
+                                sbl.sbl_forward(dsc, q, d, T, p, sbl.SBL_FMT_PK2, y)
             graphs[mode] = g
         res = {}
         for mode, g in graphs.items():
@@ -648,23 +676,25 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
                 g.replay()
             torch.cuda.synchronize()
             barrier(dist, world)
-            if T == wk.tokens[-1] and mode == "gemv":
-                clocks.start()
+            t_wall0 = clocks.mark()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             for _ in range(args.steps):
                 g.replay()
             e1.record()
             torch.cuda.synchronize()
-            if T == wk.tokens[-1] and mode == "gemv":
-                clk = clocks.stop()
+            windows.append((t_wall0, clocks.mark()))
             ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / args.steps
-            launches = sum(len(c) * (2 if mode == "step" else 1) for _, _, c, *_ in layers)
-            # algorithmic bytes: packed weights + the layer's input (int8 Xq for the
-            # GEMV alone, bf16 X for the step) + bf16 Y + the token scales
-            alg_bytes = sum(len(c) * (bw + T * lin.d_in * (1 if mode == "gemv" else 2) + T * lin.d_out * 2 + 4 * T)
+            # launches: the fused decode kernel is one launch per linear when
+            # T K <= 8192, else the activation kernel and the decode kernel
+            launches = sum(len(c) * (1 if mode == "gemv" or T * lin.d_in <= 8192 else 2)
+                           for lin, _, c, *_ in layers)
+            # algorithmic bytes: the packed weights, bf16 Y and, for the GEMV
+            # alone, int8 Xq + d read; for the step, bf16 X read and Xq + d written
+            alg_bytes = sum(len(c) * (bw + T * lin.d_out * 2 + (T * lin.d_in + 4 * T if mode == "gemv"
+                                                                else 3 * T * lin.d_in + 8 * T))
                             for lin, _, c, _, _, _, _, bw in layers)
-            res[mode] = {"ms_per_graph": ms, "launches": launches,
+            res[mode] = {"ms_per_graph": ms, "launches": launches, "bytes_per_graph": alg_bytes,
                          "gbs": whole_job_rate(alg_bytes, world, ms) / 1e9}
         # end to end through the public API: every step copies the tokens'
         # activations in from pinned host memory and the outputs back
@@ -679,8 +709,7 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
         for _ in range(e_steps):
             for (lin, dsc, copies, x, q, d, y, _), h_in, h_out in zip(layers, hx, hy):
                 x.copy_(h_in, non_blocking=True)
-                sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
-                sbl.sbl_forward(dsc, q, d, T, copies[0], sbl.SBL_FMT_PK2, y)
+                sbl.sbl_linear_forward(dsc, x, T, copies[0], sbl.SBL_FMT_PK2, q, d, y)
                 h_out.copy_(y, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
@@ -691,8 +720,13 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
                       "d2h_bytes_per_step": sum(h.numel() * 2 for h in hy)}
         results[T] = res
     Tm = wk.tokens[-1]
+    clk = clocks.stop(*windows)
     value = statistics.mean(results[T]["step"]["gbs"] for T in wk.tokens)
-    gemv = results[Tm]["gemv"]["gbs"]
+    # the roofline kernel is the decode GEMV (the 'gemv' graphs launch it
+    # alone): its algorithmic bytes over its time, all token counts together
+    gemv_bytes = sum(results[T]["gemv"]["bytes_per_graph"] for T in wk.tokens)
+    gemv_ms = sum(results[T]["gemv"]["ms_per_graph"] for T in wk.tokens)
+    gemv = gemv_bytes * world / (gemv_ms * 1e-3) / 1e9
     e2e = statistics.mean(results[T]["e2e"]["gbs"] for T in wk.tokens)
     err = sbl.sbl_device_error()
     cpu = None
@@ -704,14 +738,18 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "2-bit ternary x int8 -> int32",
         "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32 packed once to 2:4 PK2, X~N(0,1) bf16)",
         "config": {"workload": wk.name, "tokens": wk.tokens,
-                   "step": "per token count: act quant + GEMV of each linear, over rotating weight copies",
+                   "step": "per token count: sbl_linear_forward of each linear (act quant fused into the "
+                           "decode GEMV, one launch, when T K <= 8192; else the activation kernel and the "
+                           "GEMV), over rotating weight copies; 'gemv' is the GEMV alone from int8 activations",
                    "per_token_count": {str(T): results[T] for T in wk.tokens},
                    "l2": "inputs larger than L2: rotating weight copies > 4x L2 inside one CUDA graph",
                    "parallelism": f"independent replicas x{world}"},
-        "roofline": {"kernel": "decode_kernel (PK2 stream, mma.sync u8 x s8)", "bound": "hbm", "achieved": round(gemv, 1),
+        "roofline": {"kernel": "decode_kernel (PK2 stream, mma.sync u8 x s8), both linears, T = 1, 4, 16",
+                     "bound": "hbm", "achieved": round(gemv, 1),
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gemv / pk["hbm_gbs"], 4),
                      "traffic": stored_traffic(wk.name),
-                     "traffic_note": "mean DRAM read+write bytes per decode launch (ncu capture in "
+                     "traffic_note": "mean DRAM read+write bytes per decode launch over both linears and "
+                                     "T = 1, 4, 16, each launch after an L2 flush (ncu captures in "
                                      "profiles/roofline_traffic.json; null when absent or stale)"},
         "e2e": {"value": round(e2e, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": results[Tm]["e2e"]["h2d_bytes_per_step"],
@@ -813,7 +851,9 @@ def main():
     args = parse()
     wk = wl.WORKLOADS[args.workload]
     if args.record_traffic:
-        regex = r"decode_kernel" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
+        # the roofline kernels: the decode GEMV (last template flag 0: not the
+        # fused variant), or the int8 dense and 2:4 sparse forward GEMMs
+        regex = r"decode_kernel<\d+, \d+, \d+, 0>" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
         print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command)))
         return
     if args.impl == "reference":

@@ -304,6 +304,19 @@ sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const fl
                           int32_t y_is_fp32, int32_t *acc_out, const sbl_epilogue *epi,
                           void *stream);
 
+/* A layer's forward from its bf16 input: Xq, d = Q_a(X) exactly as
+ * sbl_quantize_act, then Y exactly as sbl_forward_ex (forward steps 1-5 of
+ * the Sparse-BitNet summary, "The Full Sparse-BitLinear Layer").  X: bf16
+ * [T, K]; Xq int8 [T, K] and d fp32 [T] are outputs (the backward reuses
+ * them); Y and epi as sbl_forward_ex (no accumulator output).  For
+ * SBL_FMT_PK2 with T <= 16, K % 64 == 0 and T K <= 8192 this is ONE launch
+ * (every CTA of the decode kernel quantises the small X in its prologue);
+ * otherwise the activation kernel and the forward kernel, two launches.
+ * Shapes, formats and errors as the two calls. */
+sbl_status sbl_linear_forward(const sbl_layer_desc *desc, const uint16_t *X, int32_t T, const sbl_packed *w,
+                              sbl_format fmt, int8_t *Xq, float *d, void *Y, int32_t y_is_fp32,
+                              const sbl_epilogue *epi, void *stream);
+
 /* The forward operand format the library recommends for a layer and a
  * token count: SBL_FMT_SP24 (2:4 sparse tensor-core MMA on CTA pairs) when
  * the mask allows it (n <= 2) and the GEMM is large enough for the sparse

@@ -44,7 +44,6 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
     constexpr int kRowsPerCta = RT >= 256 ? 1 : 256 / RT;
     constexpr int kWarpsPerRow = RT / 32 > 0 ? RT / 32 : 1;
     __shared__ float red[kRowsPerCta][kWarpsPerRow];
-    __shared__ float rsh[kRowsPerCta];
     const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + sub;
     // programmatic dependent launch: X may come from the previous kernel
@@ -93,16 +92,42 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
     if (lt == 0) d[row] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
 }
 
+// u = fl32(fl32(x * r) * g) of one 8-element chunk (g: bf16 gains or none)
+__device__ __forceinline__ void norm_chunk(const uint4 &v, const uint16_t *__restrict__ g, int ci, int chunks,
+                                           float r, float (&u)[8])
+{
+    const uint4 gv = (g && ci < chunks) ? __ldg(reinterpret_cast<const uint4 *>(g) + ci) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        u[2 * i] = __fmul_rn(bf16_lo(w[i]), r);
+        u[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), r);
+        if (g) {
+            u[2 * i] = __fmul_rn(u[2 * i], bf16_lo(gw[i]));
+            u[2 * i + 1] = __fmul_rn(u[2 * i + 1], bf16_hi(gw[i]));
+        }
+    }
+}
+
 // RMSNorm fused with the quantiser (the norm before Q_a in forward step 1 of
 // the Sparse-BitNet summary): per row, S = sum of x_k^2 in fp64 over the
 // pairwise tree of the row in flat order, r = fl32(1 / sqrt(S / K + eps)),
 // u_k = fl32(fl32(x_k * r) * g_k) (g: bf16 gains, none = 1), then the
-// absmax int8 quantisation of u.  The tree follows the thread layout: thread
-// lt holds chunks ci = lt + c * RT (8 elements each, an aligned 8-leaf
-// subtree); for a fixed slot c the chunks of consecutive lanes are adjacent,
-// so lane butterflies, then a pairwise combination of the row's warps (RT a
-// power of two >= 32), then a pairwise tree over the 8 slots give exactly
-// the row's tree (the tail beyond K is +0.0, which leaves every sum exact).
+// absmax int8 quantisation of u.
+//
+// That tree equals the tree of the row padded with +0.0 to 64 RT elements (a
+// sum with +0.0 is exact), so it is assembled from aligned subtrees of the
+// layout of the plain quantiser: thread lt of a row holds the 8-element
+// chunks lt + c RT (slot c < 8; coalesced loads).  Slot c of warp w is the
+// aligned 256-element block of chunks c RT + 32 w .. + 31, and slot c of the
+// row the aligned block c RT .. (c + 1) RT - 1.  Each chunk is an 8-leaf tree;
+// a reduce-scatter over lanes (xor 1, 2, 4: adjacent lanes first, each lane
+// keeping half, then a quarter, then one of its slot sums) and two
+// butterflies (xor 8, 16) leave in lane L the warp's sum of slot
+// 4 (L & 1) + 2 (L >> 1 & 1) + (L >> 2 & 1); the row's first warp then adds
+// the warps of each slot pairwise and the slots pairwise.  Every addition
+// joins two adjacent aligned subtrees (a + b == b + a exactly).
 template <int RT>
 __global__ void __launch_bounds__(RT > 256 ? RT : 256)
     act_norm_quant_kernel(const uint16_t *__restrict__ X, int32_t T, int32_t K, const uint16_t *__restrict__ g,
@@ -110,9 +135,10 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
 {
     static_assert(RT >= 32 && (RT & (RT - 1)) == 0, "rows are whole warps, a power of two");
     constexpr int kRowsPerCta = RT >= 256 ? 1 : 256 / RT;
-    constexpr int kWarpsPerRow = RT / 32;
-    __shared__ double slots[kRowsPerCta][kWarpsPerRow][kActMaxChunks];
-    __shared__ float red[kRowsPerCta][kWarpsPerRow];
+    constexpr int W = RT / 32;                        // warps per row
+    constexpr int H = (8 * W + 31) / 32;              // (slot, warp) sums per lane of the combining warp
+    __shared__ double wsum[kRowsPerCta][8 * W];       // [slot][warp]
+    __shared__ float wmax[kRowsPerCta][W];
     __shared__ float rsh[kRowsPerCta];
     const int sub = threadIdx.x / RT, lt = threadIdx.x % RT;
     const int wr = lt >> 5, lane = threadIdx.x & 31;
@@ -129,6 +155,7 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
         v[c] = make_uint4(0u, 0u, 0u, 0u);
         if (active && ci < chunks) v[c] = __ldg(reinterpret_cast<const uint4 *>(X + row * K) + ci);
     }
+    double cs[kActMaxChunks];
 #pragma unroll
     for (int c = 0; c < kActMaxChunks; ++c) {
         const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
@@ -139,63 +166,73 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
             sq[2 * i] = lo * lo;  // exact: a bf16 square has at most 16 significant bits
             sq[2 * i + 1] = hi * hi;
         }
-        double cs = ((sq[0] + sq[1]) + (sq[2] + sq[3])) + ((sq[4] + sq[5]) + (sq[6] + sq[7]));
-        // adjacent lanes first: every lane ends with the warp's subtree (a + b == b + a exactly)
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) cs = cs + __shfl_xor_sync(0xffffffffu, cs, off);
-        if (lane == 0) slots[sub][wr][c] = cs;
+        cs[c] = ((sq[0] + sq[1]) + (sq[2] + sq[3])) + ((sq[4] + sq[5]) + (sq[6] + sq[7]));
     }
+    // reduce-scatter over the lanes: keep slots 4 b0 .. 4 b0 + 3, then two of
+    // them, then one
+    const bool b0 = lane & 1, b1 = (lane >> 1) & 1, b2 = (lane >> 2) & 1;
+    double r1[4], r2[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double keep = b0 ? cs[4 + i] : cs[i], give = b0 ? cs[i] : cs[4 + i];
+        r1[i] = keep + __shfl_xor_sync(0xffffffffu, give, 1);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const double keep = b1 ? r1[2 + i] : r1[i], give = b1 ? r1[i] : r1[2 + i];
+        r2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+    }
+    double r3;
+    {
+        const double keep = b2 ? r2[1] : r2[0], give = b2 ? r2[0] : r2[1];
+        r3 = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+    }
+    r3 = r3 + __shfl_xor_sync(0xffffffffu, r3, 8);
+    r3 = r3 + __shfl_xor_sync(0xffffffffu, r3, 16);
+    if (lane < 8) wsum[sub][(4 * b0 + 2 * b1 + b2) * W + wr] = r3;
     __syncthreads();
     if (wr == 0) {
-        // the row's first warp: per slot, the warps' subtrees pairwise in warp
-        // order (lanes >= kWarpsPerRow hold zeros in groups of their own); lane
-        // c keeps slot c; then the 8 slots pairwise over lanes 0..7
-        double mine = 0.0;
+        // value i = h 32 + lane is (slot i / W, warp i % W): warps pairwise
+        // within each slot (xor < W), slots pairwise across the lane groups
+        // (xor W .. 16; lanes past 8 W hold +0.0), then the H blocks pairwise
+        double x[H];
 #pragma unroll
-        for (int c = 0; c < kActMaxChunks; ++c) {
-            double x = lane < kWarpsPerRow ? slots[sub][lane][c] : 0.0;
-#pragma unroll
-            for (int off = 1; off < kWarpsPerRow; off <<= 1) x = x + __shfl_xor_sync(0xffffffffu, x, off);
-            x = __shfl_sync(0xffffffffu, x, 0);
-            if (lane == c) mine = x;
+        for (int h = 0; h < H; ++h) {
+            const int i = h * 32 + lane;
+            x[h] = i < 8 * W ? wsum[sub][i] : 0.0;
         }
 #pragma unroll
-        for (int off = 1; off < kActMaxChunks; off <<= 1) mine = mine + __shfl_xor_sync(0xffffffffu, mine, off);
-        if (lane == 0) {
-            const double S = mine;
+        for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+            for (int h = 0; h < H; ++h) x[h] = x[h] + __shfl_xor_sync(0xffffffffu, x[h], off);
+#pragma unroll
+        for (int step = 1; step < H; step *= 2)
+#pragma unroll
+            for (int h = 0; h < H; h += 2 * step) x[h] = x[h] + x[h + step];
+        if (lane == 0)
             rsh[sub] = __double2float_rn(__ddiv_rn(
-                1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps)))));
-        }
+                1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(x[0], static_cast<double>(K)), static_cast<double>(eps)))));
     }
     __syncthreads();
     const float r = rsh[sub];
 
-    // u = fl32(fl32(x * r) * g): absmax over the row, then quantise
+    // u = fl32(fl32(x * r) * g), computed from the held x in both passes:
+    // max|u| over the row, then the quantised stores
     float amax = 0.0f;
 #pragma unroll
     for (int c = 0; c < kActMaxChunks; ++c) {
-        const int ci = lt + c * RT;
-        if (!(active && ci < chunks)) continue;
-        const uint4 gv = g ? __ldg(reinterpret_cast<const uint4 *>(g) + ci) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        float u[8];
+        norm_chunk(v[c], g, lt + c * RT, chunks, r, u);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float u0 = __fmul_rn(bf16_lo(w[i]), r), u1 = __fmul_rn(bf16_hi(w[i]), r);
-            if (g) {
-                u0 = __fmul_rn(u0, bf16_lo(gw[i]));
-                u1 = __fmul_rn(u1, bf16_hi(gw[i]));
-            }
-            amax = fmaxf(amax, fmaxf(fabsf(u0), fabsf(u1)));
-        }
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(u[i]));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) red[sub][wr] = amax;
+    if (lane == 0) wmax[sub][wr] = amax;
     __syncthreads();
-    amax = red[sub][0];
+    amax = wmax[sub][0];
 #pragma unroll
-    for (int w = 1; w < kWarpsPerRow; ++w) amax = fmaxf(amax, red[sub][w]);
+    for (int w = 1; w < W; ++w) amax = fmaxf(amax, wmax[sub][w]);
     if (!active) return;
     const bool zero = !(amax > 0.0f);
     const float rq = zero ? 0.0f : __fdiv_rn(127.0f, amax);
@@ -205,19 +242,8 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256)
         if (ci >= chunks) continue;
         uint2 out = make_uint2(0u, 0u);
         if (!zero) {
-            const uint4 gv = g ? __ldg(reinterpret_cast<const uint4 *>(g) + ci) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
             float u[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                u[2 * i] = __fmul_rn(bf16_lo(w[i]), r);
-                u[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), r);
-                if (g) {
-                    u[2 * i] = __fmul_rn(u[2 * i], bf16_lo(gw[i]));
-                    u[2 * i + 1] = __fmul_rn(u[2 * i + 1], bf16_hi(gw[i]));
-                }
-            }
+            norm_chunk(v[c], g, ci, chunks, r, u);
             out.x = quant4(u[0], u[1], u[2], u[3], rq);
             out.y = quant4(u[4], u[5], u[6], u[7], rq);
         }

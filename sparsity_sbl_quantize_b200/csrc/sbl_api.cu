@@ -375,6 +375,17 @@ cudaError_t launch_decode_nt(const cudaLaunchConfig_t &cfg, const DecodeArgs &a,
     }
 }
 
+template <int NT>
+cudaError_t launch_decode_fused(const cudaLaunchConfig_t &cfg, const DecodeArgs &a, int cpw)
+{
+    switch (cpw) {
+    case 1: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 1, 1, true>, a);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 2, 1, true>, a);
+    case 4: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, 1, true>, a);
+    default: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 8, 1, true>, a);
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -669,42 +680,77 @@ sbl_status sbl_quantize_act_rmsnorm(const uint16_t *X, int32_t T, int32_t K, con
     DeviceInfo *di = nullptr;
     sbl_status st = current_device(&di);
     if (st != SBL_OK) return st;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    // RT threads per row (the layout of the plain quantiser: 16-byte chunks
+    // lt + c RT, c < 8), 256 / RT rows per CTA when RT < 256
     const int chunks = K / 8;
     int rt = 32;
     while (rt * kActMaxChunks < chunks) rt *= 2;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.stream = stream;
+    cfg.stream = static_cast<cudaStream_t>(stream_p);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaSuccess;
+    cudaError_t e = cudaErrorInvalidValue;
     switch (rt) {
-#define SBL_ACT_CASE(R)                                                        \
-    case R: {                                                                 \
-        constexpr int rows = R >= 256 ? 1 : 256 / R;                          \
-        cfg.gridDim = dim3(static_cast<unsigned>((T + rows - 1) / rows));     \
-        cfg.blockDim = dim3(R > 256 ? R : 256);                               \
-        e = cudaLaunchKernelEx(&cfg, act_norm_quant_kernel<R>, X, T, K, g, eps, Xq, d); \
-        break;                                                                \
+#define SBL_NORM_CASE(R)                                                                   \
+    case R: {                                                                             \
+        constexpr int rows = R >= 256 ? 1 : 256 / R;                                      \
+        cfg.gridDim = dim3(static_cast<unsigned>((T + rows - 1) / rows));                 \
+        cfg.blockDim = dim3(R > 256 ? R : 256);                                           \
+        e = cudaLaunchKernelEx(&cfg, act_norm_quant_kernel<R>, X, T, K, g, eps, Xq, d);   \
+        break;                                                                            \
     }
-        SBL_ACT_CASE(32)
-        SBL_ACT_CASE(64)
-        SBL_ACT_CASE(128)
-        SBL_ACT_CASE(256)
-        SBL_ACT_CASE(512)
-        SBL_ACT_CASE(1024)
-#undef SBL_ACT_CASE
-    default: return SBL_ERR_SHAPE;
+        SBL_NORM_CASE(32)
+        SBL_NORM_CASE(64)
+        SBL_NORM_CASE(128)
+        SBL_NORM_CASE(256)
+        SBL_NORM_CASE(512)
+        SBL_NORM_CASE(1024)
+#undef SBL_NORM_CASE
     }
-    if (e != cudaSuccess) return SBL_ERR_CUDA;
-    return launch_status();
+    return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
 }
 
 }  // extern "C"
+
+// One decode launch: a CTA per 16 output rows; fused: the bf16 activations
+// are quantised in the kernel's prologue into T (K + 16) bytes of shared
+// memory (at most 8.4 KB: T K <= 8192).
+static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream)
+{
+    a.chunks = (a.K + kDecChunk - 1) / kDecChunk;
+    // chunks per warp per round: the whole row in one round up to
+    // K = 16384 (more rounds above)
+    const int need = (a.chunks + 7) / 8;
+    const int cpw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
+    const int rg = fuse ? 1 : a.T <= 8 ? kDecGroupsSmallT : kDecGroupsLargeT;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>((a.O + kDecRows * rg - 1) / (kDecRows * rg)));
+    cfg.blockDim = dim3(static_cast<unsigned>(256 * rg));
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    // programmatic dependent launch: the kernel loads its (read-only)
+    // packed weights before waiting on the previous kernel's outputs
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (fuse) {
+        a.xs_stride = a.K + kDecXsPad;
+        cfg.dynamicSmemBytes = static_cast<size_t>(a.T) * a.xs_stride;
+        e = a.T <= 8 ? launch_decode_fused<1>(cfg, a, cpw) : launch_decode_fused<2>(cfg, a, cpw);
+    } else {
+        e = a.T <= 8 ? (rg == 1 ? launch_decode_nt<1, 1>(cfg, a, cpw) : launch_decode_nt<1, 2>(cfg, a, cpw))
+                     : (rg == 1 ? launch_decode_nt<2, 1>(cfg, a, cpw) : launch_decode_nt<2, 2>(cfg, a, cpw));
+    }
+    return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
+}
 
 static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
                                const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32,
@@ -769,28 +815,7 @@ static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, con
         a.T = T;
         a.K = K;
         a.O = O;
-        a.chunks = (K + kDecChunk - 1) / kDecChunk;
-        // chunks per warp per round: the whole row in one round up to
-        // K = 16384 (more rounds above)
-        const int need = (a.chunks + 7) / 8;
-        const int cpw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
-        const int rg = T <= 8 ? kDecGroupsSmallT : kDecGroupsLargeT;
-        cudaLaunchConfig_t cfg;
-        memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(static_cast<unsigned>((O + kDecRows * rg - 1) / (kDecRows * rg)));
-        cfg.blockDim = dim3(static_cast<unsigned>(256 * rg));
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        // programmatic dependent launch: the kernel loads its (read-only)
-        // packed weights before waiting on the previous kernel's outputs
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t e = T <= 8 ? (rg == 1 ? launch_decode_nt<1, 1>(cfg, a, cpw) : launch_decode_nt<1, 2>(cfg, a, cpw))
-                                     : (rg == 1 ? launch_decode_nt<2, 1>(cfg, a, cpw) : launch_decode_nt<2, 2>(cfg, a, cpw));
-        return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
+        return launch_decode(a, false, stream);
     }
     return SBL_ERR_UNSUPPORTED;
 }
@@ -809,6 +834,49 @@ sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const fl
                           const sbl_epilogue *epi, void *stream_p)
 {
     return forward_impl(desc, Xq, d, T, w, fmt, Y, y_is_fp32, acc_out, epi, stream_p);
+}
+
+sbl_status sbl_linear_forward(const sbl_layer_desc *desc, const uint16_t *X, int32_t T, const sbl_packed *w,
+                              sbl_format fmt, int8_t *Xq, float *d, void *Y, int32_t y_is_fp32,
+                              const sbl_epilogue *epi, void *stream_p)
+{
+    sbl_status st = check_desc(desc);
+    if (st != SBL_OK) return st;
+    if (T < 0) return SBL_ERR_SHAPE;
+    if (T == 0) return SBL_OK;
+    if (!X || !Xq || !d || !w || !Y || !w->gamma) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xq) || !aligned16(d) || !aligned16(Y) || !aligned16(w->gamma) ||
+        (epi && epi->residual && !aligned16(epi->residual)))
+        return SBL_ERR_ALIGNMENT;
+    const int32_t O = desc->out_features, K = desc->in_features;
+    if (fmt == SBL_FMT_PK2 && T <= kDecMaxTokens && K % kDecKUnit == 0 &&
+        static_cast<int64_t>(T) * K <= kDecFuseMaxElems) {
+        if (!w->pk2) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(w->pk2)) return SBL_ERR_ALIGNMENT;
+        DeviceInfo *di = nullptr;
+        if ((st = current_device(&di)) != SBL_OK) return st;
+        DecodeArgs a;
+        memset(&a, 0, sizeof(a));
+        a.pk2 = w->pk2;
+        a.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_PK2, SBL_BUF_MAIN));
+        a.gamma = w->gamma;
+        a.out = Y;
+        a.out_fp32 = y_is_fp32 ? 1 : 0;
+        if (epi) {
+            a.relu2 = epi->relu2 ? 1 : 0;
+            a.residual = epi->residual;
+        }
+        a.T = T;
+        a.K = K;
+        a.O = O;
+        a.x = X;
+        a.xq_out = Xq;
+        a.d_out = d;
+        return launch_decode(a, true, static_cast<cudaStream_t>(stream_p));
+    }
+    // otherwise the activation kernel, then the layer's forward kernel
+    if ((st = sbl_quantize_act(X, T, K, Xq, d, stream_p)) != SBL_OK) return st;
+    return forward_impl(desc, Xq, d, T, w, fmt, Y, y_is_fp32, nullptr, epi, stream_p);
 }
 
 sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)

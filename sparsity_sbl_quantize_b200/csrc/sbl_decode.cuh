@@ -25,10 +25,18 @@
 // so that kernel's weights stream during this one's arithmetic.  The warps'
 // int32 partials meet in shared memory (exact) and one thread per (token,
 // row) dequantises y = fl32(fl32(acc) * fl32(gamma * d_t)).
+//
+// Fused variant (FUSE): the input is the bf16 activation X itself (small:
+// T K <= 8192).  After the wait every CTA loads X in one pass into registers,
+// quantises it per token (absmax int8, the quantiser of the activation
+// kernel) into shared memory, and CTA 0 also stores Xq and d; the MMA loop
+// then reads the activations from shared memory.  One launch per layer
+// instead of two.
 #pragma once
 
 #include <cuda_bf16.h>
 
+#include "sbl_act.cuh"
 #include "sbl_device.cuh"
 
 namespace sbl {
@@ -52,7 +60,18 @@ struct DecodeArgs {
     const uint16_t *residual;  // ... then v = v + residual[t, o] (bf16 [T, O]; nullptr: none)
     int32_t T, K, O;
     int32_t chunks;       // ceil(K / 256)
+    // fused variant only
+    const uint16_t *x;    // bf16 activations [T, K]
+    int8_t *xq_out;       // Q_a(x) [T, K], stored by CTA 0 (nullptr: not stored)
+    float *d_out;         // d_t [T], stored by CTA 0 (nullptr: not stored)
+    int32_t xs_stride;    // bytes per token row of the shared int8 copy (K + 16)
 };
+
+// dynamic shared memory of the fused variant: the int8 activations [T][K + 16]
+constexpr int kDecXsPad = 16;
+// 16-byte groups of X per thread of the fused prologue (T K <= 8 x 4 x 256)
+constexpr int kDecFuseVec = 4;
+constexpr int kDecFuseMaxElems = 8 * kDecFuseVec * 256;
 
 // Programmatic dependent launch: let the next kernel on the stream start
 // launching, and wait for the previous kernel's results.
@@ -97,6 +116,85 @@ __device__ __forceinline__ float ld_global_f32(const float *p)
     return v;
 }
 
+__device__ __forceinline__ uint4 ld_shared16(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t absmax8_bits(const uint4 &v)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    return __float_as_uint(m);  // |x| >= 0: the bit patterns order as the values
+}
+
+// Per-token absmax quantisation of the bf16 rows X[T][K] into the CTA's
+// shared copy xs (row stride xs_stride), by all threads of the CTA in one
+// pass: thread i holds the 16-byte groups i, i + 256, ... (at most
+// kDecFuseVec, T K <= 8 kDecFuseVec blockDim) in registers; per-token maxima
+// meet in shared memory; CTA 0 also stores Xq and d.  The same arithmetic as
+// the activation kernel: a = max|x|, r = fl32(127 / a),
+// q = sat8(rint(fl32(x r))), d = fl32(a / 127); a == 0 gives q = 0, d = 0.
+// s_amax was zeroed, and a barrier passed, before the grid-dependency wait.
+__device__ __forceinline__ void decode_quantize_x(const DecodeArgs &a, uint32_t xs, uint32_t *s_amax)
+{
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const int k8 = a.K >> 3, n = a.T * k8;
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(a.x);
+    uint4 v[kDecFuseVec];
+#pragma unroll
+    for (int u = 0; u < kDecFuseVec; ++u) {
+        const int i = tid + u * nth;
+        v[u] = i < n ? ld_global16(x4 + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    int tcur = -1;
+    uint32_t mcur = 0u;
+#pragma unroll
+    for (int u = 0; u < kDecFuseVec; ++u) {
+        const int i = tid + u * nth;
+        if (i >= n) break;
+        const int t = i / k8;
+        const uint32_t m = absmax8_bits(v[u]);
+        if (t != tcur) {
+            if (tcur >= 0) atomicMax(&s_amax[tcur], mcur);
+            tcur = t;
+            mcur = m;
+        } else {
+            mcur = max(mcur, m);
+        }
+    }
+    if (tcur >= 0) atomicMax(&s_amax[tcur], mcur);
+    __syncthreads();
+    const bool store = blockIdx.x == 0 && a.xq_out != nullptr;
+#pragma unroll
+    for (int u = 0; u < kDecFuseVec; ++u) {
+        const int i = tid + u * nth;
+        if (i >= n) break;
+        const int t = i / k8, kk = i - t * k8;
+        const float amax = __uint_as_float(s_amax[t]);
+        uint2 q = make_uint2(0u, 0u);
+        if (amax > 0.0f) {
+            const float r = __fdiv_rn(127.0f, amax);
+            q.x = quant4(bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y), r);
+            q.y = quant4(bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w), r);
+        }
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(xs + t * a.xs_stride + 8 * kk), "r"(q.x), "r"(q.y)
+                     : "memory");
+        if (store) reinterpret_cast<uint2 *>(a.xq_out + static_cast<int64_t>(t) * a.K)[kk] = q;
+    }
+    if (blockIdx.x == 0 && a.d_out && tid < a.T) {
+        const float amax = __uint_as_float(s_amax[tid]);
+        a.d_out[tid] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    }
+    __syncthreads();
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s)
 {
     uint32_t r;
@@ -131,9 +229,15 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 // NT: n8 token blocks (T <= 8 or T <= 16); CPW: chunks per warp per round;
 // RG: groups of 16 rows per CTA, each worked by 8 warps that split the K
 // chunks of its rows (the groups read the same activations: L1 hits).
-template <int NT, int CPW, int RG>
+template <int NT, int CPW, int RG, bool FUSE = false>
 __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
 {
+    extern __shared__ __align__(16) uint8_t dec_xs[];
+    __shared__ uint32_t s_amax[FUSE ? kDecMaxTokens : 1];
+    if constexpr (FUSE) {
+        if (threadIdx.x < kDecMaxTokens) s_amax[threadIdx.x] = 0u;
+        __syncthreads();
+    }
     constexpr int kWarps = 8;                          // warps per row group
     constexpr int NA = CPW < 4 ? CPW : 4;              // independent MMA chains
     constexpr int G = NT == 1 ? (CPW < 4 ? CPW : 4) : 1;  // chunks loaded together
@@ -180,7 +284,16 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
         }
         if (round0 == 0) {
             pdl_wait_prior();  // activations, scales and gamma
-            if (has_out) scale = __fmul_rn(ld_global_f32(args.gamma), ld_global_f32(args.d + t_out));
+            if constexpr (FUSE) {
+                decode_quantize_x(args, smem_addr(dec_xs), s_amax);
+                if (has_out) {
+                    const float amax = __uint_as_float(s_amax[t_out]);
+                    const float d_t = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+                    scale = __fmul_rn(ld_global_f32(args.gamma), d_t);
+                }
+            } else {
+                if (has_out) scale = __fmul_rn(ld_global_f32(args.gamma), ld_global_f32(args.d + t_out));
+            }
         }
 
         // 2. groups of G chunks: the lane's 64 activations of each chunk and
@@ -198,10 +311,18 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
                 for (int b = 0; b < NT; ++b) {
                     const int t = 8 * b + g;
                     const bool ok = c < args.chunks && pos < args.K && t < args.T;
-                    const int8_t *src = args.xq + static_cast<int64_t>(ok ? t : 0) * args.K + (ok ? pos : 0);
+                    if constexpr (FUSE) {
+                        const uint32_t src = smem_addr(dec_xs) + (ok ? t * args.xs_stride + pos : 0);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        xr[j][b][q] = ok ? ld_global16(src + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
+                        for (int q = 0; q < 4; ++q)
+                            xr[j][b][q] = ok ? ld_shared16(src + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
+                    } else {
+                        const int8_t *src =
+                            args.xq + static_cast<int64_t>(ok ? t : 0) * args.K + (ok ? pos : 0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            xr[j][b][q] = ok ? ld_global16(src + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
             }
 #pragma unroll

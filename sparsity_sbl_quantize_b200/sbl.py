@@ -96,13 +96,16 @@ _lib.sbl_backward_dual_ste.restype = ctypes.c_int
 _lib.sbl_backward_dual_ste.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _sz, _P]
 _lib.sbl_forward_ex.restype = ctypes.c_int
 _lib.sbl_forward_ex.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, ctypes.POINTER(sbl_epilogue), _P]
+_lib.sbl_linear_forward.restype = ctypes.c_int
+_lib.sbl_linear_forward.argtypes = [_D, _P, _i32, _W, ctypes.c_int, _P, _P, _P, _i32,
+                                    ctypes.POINTER(sbl_epilogue), _P]
 _lib.sbl_forward_format.restype = ctypes.c_int
 _lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
-            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward",
+            "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward", "sbl_linear_forward",
             "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
             "sbl_quantize_mask_pack_ex", "sbl_device_error"]
 
@@ -248,6 +251,17 @@ def sbl_forward_ex(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: in
     y_fp32 = 1 if Y.dtype == torch.float32 else 0
     _check(_lib.sbl_forward_ex(ctypes.byref(dsc), _ptr(Xq), _ptr(d), T, ctypes.byref(cp), fmt, _ptr(Y), y_fp32,
                                _ptr(acc_out), ctypes.byref(epi), _stream()), "sbl_forward_ex")
+
+
+def sbl_linear_forward(dsc: sbl_layer_desc, X: torch.Tensor, T: int, w: Packed, fmt: int, Xq: torch.Tensor,
+                       d: torch.Tensor, Y: torch.Tensor, relu2: bool = False,
+                       residual: Optional[torch.Tensor] = None) -> None:
+    """Q_a(X) -> Xq, d, then the forward into Y (one launch for the PK2 decode)."""
+    cp = w.c()
+    epi = sbl_epilogue(1 if relu2 else 0, residual.data_ptr() if residual is not None else None)
+    y_fp32 = 1 if Y.dtype == torch.float32 else 0
+    _check(_lib.sbl_linear_forward(ctypes.byref(dsc), _ptr(X), T, ctypes.byref(cp), fmt, _ptr(Xq), _ptr(d),
+                                   _ptr(Y), y_fp32, ctypes.byref(epi), _stream()), "sbl_linear_forward")
 
 
 def sbl_backward_dual_ste(dsc: sbl_layer_desc, dY: torch.Tensor, Xq: Optional[torch.Tensor],

@@ -103,6 +103,25 @@ def test_validation_happens_before_any_device_access(sbl):
     assert _raw(sbl, "sbl_quantize_act", None, 4, 256, P(good), P(good), None) == 1
     assert _raw(sbl, "sbl_quantize_act", P(good + 4), 4, 256, P(good), P(good), None) == 3
     assert _raw(sbl, "sbl_quantize_act", P(good), 0, 256, P(good), P(good), None) == 0  # T == 0: no-op
+    # linear forward: descriptor, null, alignment, then device
+    lf = "sbl_linear_forward"
+    dd = sbl.desc(128, 256, 6, 8)
+    pw = sbl.sbl_packed(None, None, None, good, good, good)
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good), -1, ctypes.byref(pw), sbl.SBL_FMT_PK2, P(good), P(good),
+                P(good), 0, None, None) == 2
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good), 0, ctypes.byref(pw), sbl.SBL_FMT_PK2, P(good), P(good),
+                P(good), 0, None, None) == 0
+    assert _raw(sbl, lf, ctypes.byref(dd), None, 4, ctypes.byref(pw), sbl.SBL_FMT_PK2, P(good), P(good),
+                P(good), 0, None, None) == 1
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good), 4, ctypes.byref(pw), sbl.SBL_FMT_PK2, None, P(good),
+                P(good), 0, None, None) == 1
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good + 8), 4, ctypes.byref(pw), sbl.SBL_FMT_PK2, P(good),
+                P(good), P(good), 0, None, None) == 3
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good), 4, ctypes.byref(pw), sbl.SBL_FMT_PK2, P(good), P(good),
+                P(good), 0, None, None) == 1  # no PK2 buffer: invalid before the device lookup
+    pk = sbl.sbl_packed(good, None, None, None, None, good)
+    assert _raw(sbl, lf, ctypes.byref(dd), P(good), 4, ctypes.byref(pk), sbl.SBL_FMT_PK2, P(good), P(good),
+                P(good), 0, None, None) == 7  # valid: no sm_100 device here
     F = ctypes.c_float
     rms = "sbl_quantize_act_rmsnorm"
     assert _raw(sbl, rms, P(good), 4, 250, None, F(1e-5), P(good), P(good), None) == 2

@@ -332,6 +332,64 @@ def test_forward_epilogue_bit_exact(fmt_name, O, K, T, n, m, relu2, residual, fp
         np.testing.assert_array_equal(bits_of(y), outb)
 
 
+# sbl_linear_forward: Q_a(X) then the forward, one fused launch for the PK2
+# decode (T K <= 8192), else the activation and forward kernels
+@pytest.mark.parametrize("fmt_name,O,K,T,n,m", [
+    ("PK2", 6912, 2560, 1, 2, 4),    # fused, one token
+    ("PK2", 2560, 6912, 1, 2, 4),    # fused, 4 chunks per warp
+    ("PK2", 48, 2048, 4, 2, 4),      # fused at the size limit (T K = 8192), tokens spread over threads
+    ("PK2", 32, 512, 16, 2, 4),      # fused, two n8 token blocks
+    ("PK2", 64, 2560, 4, 2, 4),      # just past the limit: two launches
+    ("PK2", 16, 192, 8, 6, 8),       # fused, K not a multiple of 256
+    ("PK2", 48, 11008, 7, 2, 4),     # too large to fuse: two launches
+    ("PK2", 32, 16448, 16, 2, 4),    # too large to fuse: two launches
+    ("I8", 528, 1040, 300, 6, 8),    # GEMM path
+    ("SP24", 528, 1040, 300, 2, 4),  # sparse GEMM path
+])
+def test_linear_forward_bit_exact(fmt_name, O, K, T, n, m):
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=O + K)
+    x = wl.activations(T, K, seed=O + T, outlier_frac=0.01)
+    x[0] = 0  # a zero token: q = 0, d = 0, y = 0
+    fmt = {"I8": sbl.SBL_FMT_I8, "PK2": sbl.SBL_FMT_PK2, "SP24": sbl.SBL_FMT_SP24}[fmt_name]
+    layer = GpuLayer(w, n, m, fmt)
+    ref = oracle.Layer(w, n, m)
+    qr, dr, _, yr, ybr = ref.forward(x)
+    xd = bf16_dev(x)
+    q = torch.full((T, K), 99, dtype=torch.int8, device="cuda")
+    d = torch.full((T,), -1.0, dtype=torch.float32, device="cuda")
+    for fp32 in (False, True):
+        y = torch.empty((T, O), dtype=torch.float32 if fp32 else torch.bfloat16, device="cuda")
+        sbl.sbl_linear_forward(layer.desc, xd, T, layer.packed, fmt, q, d, y)
+        np.testing.assert_array_equal(q.cpu().numpy(), qr)
+        np.testing.assert_array_equal(d.cpu().numpy(), dr)
+        if fp32:
+            np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), yr.view(np.uint32))
+        else:
+            np.testing.assert_array_equal(bits_of(y), ybr)
+    assert sbl.sbl_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("O,K,T", [(96, 1536, 5), (2560, 6912, 16)])  # fused; two launches
+def test_linear_forward_fused_decode_epilogue(O, K, T):
+    """The fused decode with Squared ReLU and the residual: the oracle's
+    quantiser, dequantisation and epilogue, bit for bit."""
+    sbl = sbl_mod()
+    w = wl.master_weights(O, K, seed=K)
+    x = wl.activations(T, K, seed=T)
+    layer = GpuLayer(w, 2, 4, sbl.SBL_FMT_PK2)
+    ref = oracle.Layer(w, 2, 4)
+    _, _, _, yr, _ = ref.forward(x)
+    res_bits = wl.activations(T, O, seed=T + 1)
+    _, outb = oracle.epilogue(yr, relu2=True, residual_bf16_bits=res_bits)
+    q = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    d = torch.empty((T,), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, O), dtype=torch.bfloat16, device="cuda")
+    sbl.sbl_linear_forward(layer.desc, bf16_dev(x), T, layer.packed, sbl.SBL_FMT_PK2, q, d, y, relu2=True,
+                           residual=bf16_dev(res_bits))
+    np.testing.assert_array_equal(bits_of(y), outb)
+
+
 def test_forward_zero_tokens_is_noop():
     sbl = sbl_mod()
     layer = GpuLayer(wl.master_weights(32, 64, seed=1), 6, 8, 4)
