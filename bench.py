@@ -40,7 +40,7 @@ LONG_STEP_MS = 1.0  # steps longer than this run at the power-capped (sustained)
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
 # the device code of each family of roofline kernels (the GEMMs, the decode GEMV)
 KERNEL_SOURCES = {"gemm": ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh"),
-                  "decode": ("sbl_device.cuh", "sbl_act.cuh", "sbl_decode.cuh")}
+                  "decode": ("sbl_device.cuh", "sbl_decode.cuh")}
 
 
 def kernel_family(workload: str) -> str:
@@ -686,8 +686,8 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
             windows.append((t_wall0, clocks.mark()))
             ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / args.steps
             # launches: the fused decode kernel is one launch per linear when
-            # T K <= 8192, else the activation kernel and the decode kernel
-            launches = sum(len(c) * (1 if mode == "gemv" or T * lin.d_in <= 8192 else 2)
+            # T K <= 4096, else the activation kernel and the decode kernel
+            launches = sum(len(c) * (1 if mode == "gemv" or T * lin.d_in <= 4096 else 2)
                            for lin, _, c, *_ in layers)
             # algorithmic bytes: the packed weights, bf16 Y and, for the GEMV
             # alone, int8 Xq + d read; for the step, bf16 X read and Xq + d written
@@ -739,7 +739,7 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
         "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32 packed once to 2:4 PK2, X~N(0,1) bf16)",
         "config": {"workload": wk.name, "tokens": wk.tokens,
                    "step": "per token count: sbl_linear_forward of each linear (act quant fused into the "
-                           "decode GEMV, one launch, when T K <= 8192; else the activation kernel and the "
+                           "decode GEMV, one launch, when T K <= 4096; else the activation kernel and the "
                            "GEMV), over rotating weight copies; 'gemv' is the GEMV alone from int8 activations",
                    "per_token_count": {str(T): results[T] for T in wk.tokens},
                    "l2": "inputs larger than L2: rotating weight copies > 4x L2 inside one CUDA graph",

@@ -309,7 +309,7 @@ sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const fl
  * the Sparse-BitNet summary, "The Full Sparse-BitLinear Layer").  X: bf16
  * [T, K]; Xq int8 [T, K] and d fp32 [T] are outputs (the backward reuses
  * them); Y and epi as sbl_forward_ex (no accumulator output).  For
- * SBL_FMT_PK2 with T <= 16, K % 64 == 0 and T K <= 8192 this is ONE launch
+ * SBL_FMT_PK2 with T <= 16, K % 64 == 0 and T K <= 4096 this is ONE launch
  * (every CTA of the decode kernel quantises the small X in its prologue);
  * otherwise the activation kernel and the forward kernel, two launches.
  * Shapes, formats and errors as the two calls. */

@@ -129,7 +129,7 @@ __device__ __forceinline__ void norm_chunk(const uint4 &v, const uint16_t *__res
 // the warps of each slot pairwise and the slots pairwise.  Every addition
 // joins two adjacent aligned subtrees (a + b == b + a exactly).
 template <int RT>
-__global__ void __launch_bounds__(RT > 256 ? RT : 256)
+__global__ void __launch_bounds__(RT > 256 ? RT : 256, RT > 256 ? 1 : 3)
     act_norm_quant_kernel(const uint16_t *__restrict__ X, int32_t T, int32_t K, const uint16_t *__restrict__ g,
                           float eps, int8_t *__restrict__ Xq, float *__restrict__ d)
 {

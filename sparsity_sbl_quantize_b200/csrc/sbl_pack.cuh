@@ -166,13 +166,34 @@ __global__ void __launch_bounds__(256) gamma_kernel(const WT *__restrict__ W, in
     for (int q = 0; q < 8; ++q)
         c[q] = (fabs(static_cast<double>(f[q].x)) + fabs(static_cast<double>(f[q].y))) +
                (fabs(static_cast<double>(f[q].z)) + fabs(static_cast<double>(f[q].w)));
-    // butterfly: after the step with offset `off`, every lane holds the tree
-    // over its aligned group of 2*off lanes (a + b == b + a exactly)
+    // chunk q's tree over the lanes (adjacent lanes first; a + b == b + a
+    // exactly) as a reduce-scatter: at xor 1, 2, 4 each lane keeps half, a
+    // quarter, then one of the chunks; xor 8 and 16 finish it.  Lane L then
+    // holds chunk 4 (L & 1) + 2 (L >> 1 & 1) + (L >> 2 & 1), so the chunks'
+    // pairwise tree ((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)) is the
+    // butterfly xor 4, 2, 1 over lanes 0..7.
+    const bool b0 = lane & 1, b1 = (lane >> 1) & 1, b2 = (lane >> 2) & 1;
+    double r1[4], r2[2];
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1)
+    for (int i = 0; i < 4; ++i) {
+        const double keep = b0 ? c[4 + i] : c[i], give = b0 ? c[i] : c[4 + i];
+        r1[i] = keep + __shfl_xor_sync(0xffffffffu, give, 1);
+    }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) c[q] = c[q] + __shfl_xor_sync(0xffffffffu, c[q], off);
-    const double t = ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
+    for (int i = 0; i < 2; ++i) {
+        const double keep = b1 ? r1[2 + i] : r1[i], give = b1 ? r1[i] : r1[2 + i];
+        r2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+    }
+    double t;
+    {
+        const double keep = b2 ? r2[1] : r2[0], give = b2 ? r2[0] : r2[1];
+        t = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+    }
+    t = t + __shfl_xor_sync(0xffffffffu, t, 8);
+    t = t + __shfl_xor_sync(0xffffffffu, t, 16);
+    t = t + __shfl_xor_sync(0xffffffffu, t, 4);
+    t = t + __shfl_xor_sync(0xffffffffu, t, 2);
+    t = t + __shfl_xor_sync(0xffffffffu, t, 1);
     if (lane == 0) warp_sums[warp] = t;
     __syncthreads();
     if (threadIdx.x == 0) {

@@ -68,6 +68,26 @@ def test_pack_gamma_multi_block_tree():
     check_pack(wl.master_weights(1008, 1040, seed=21), 6, 8)
 
 
+def test_pack_gamma_summation_order():
+    """An input on which the order of the fp64 sum decides gamma's fp32
+    rounding: |W| sums to 2^30 + 64 (the mean lands on an fp32 midpoint) plus
+    8192 x 2^-35 in the second tree node.  Summed pairwise (as the R1 tree
+    does) the tiny values survive and gamma rounds up; added one by one to the
+    large partial they are lost and the tie rounds to even (down)."""
+    w = np.zeros((64, 256), dtype=np.float32)
+    w[0, 0], w[0, 1] = 2.0 ** 30, -64.0
+    w.reshape(-1)[8192:] = 2.0 ** -35
+    w.reshape(-1)[8192::3] *= -1.0
+    seq = 0.0
+    for v in np.abs(w.astype(np.float64)).reshape(-1):
+        seq += v
+    gamma_seq = np.float32(seq / w.size)
+    ref = oracle.Layer(w, 6, 8)
+    assert ref.gamma != gamma_seq  # the input discriminates the two orders
+    assert ref.gamma == np.float32((2.0 ** 30 + 64 + 2.0 ** -22) / w.size)
+    check_pack(w, 6, 8)
+
+
 @pytest.mark.parametrize("n,m", [(6, 8), (2, 4), (2, 8), (1, 4), (3, 4), (7, 8), (5, 8), (3, 8), (1, 8), (4, 8)])
 def test_pack_ties_zero_and_signed_zero(n, m):
     """Tie-heavy weights (few distinct magnitudes), all-zero and all -0.0 rows:
@@ -333,14 +353,15 @@ def test_forward_epilogue_bit_exact(fmt_name, O, K, T, n, m, relu2, residual, fp
 
 
 # sbl_linear_forward: Q_a(X) then the forward, one fused launch for the PK2
-# decode (T K <= 8192), else the activation and forward kernels
+# decode (T K <= 4096), else the activation and forward kernels
 @pytest.mark.parametrize("fmt_name,O,K,T,n,m", [
     ("PK2", 6912, 2560, 1, 2, 4),    # fused, one token
-    ("PK2", 2560, 6912, 1, 2, 4),    # fused, 4 chunks per warp
-    ("PK2", 48, 2048, 4, 2, 4),      # fused at the size limit (T K = 8192), tokens spread over threads
-    ("PK2", 32, 512, 16, 2, 4),      # fused, two n8 token blocks
-    ("PK2", 64, 2560, 4, 2, 4),      # just past the limit: two launches
+    ("PK2", 96, 4096, 1, 2, 4),      # fused at the size limit, 2 chunks per warp
+    ("PK2", 48, 1024, 4, 2, 4),      # fused at the limit, tokens spread over threads
+    ("PK2", 32, 256, 16, 2, 4),      # fused, two n8 token blocks
     ("PK2", 16, 192, 8, 6, 8),       # fused, K not a multiple of 256
+    ("PK2", 2560, 6912, 1, 2, 4),    # past the limit: two launches
+    ("PK2", 64, 2560, 4, 2, 4),      # past the limit: two launches
     ("PK2", 48, 11008, 7, 2, 4),     # too large to fuse: two launches
     ("PK2", 32, 16448, 16, 2, 4),    # too large to fuse: two launches
     ("I8", 528, 1040, 300, 6, 8),    # GEMM path
@@ -370,7 +391,7 @@ def test_linear_forward_bit_exact(fmt_name, O, K, T, n, m):
     assert sbl.sbl_device_error(clear=True) == 0
 
 
-@pytest.mark.parametrize("O,K,T", [(96, 1536, 5), (2560, 6912, 16)])  # fused; two launches
+@pytest.mark.parametrize("O,K,T", [(96, 768, 5), (2560, 6912, 16)])  # fused; two launches
 def test_linear_forward_fused_decode_epilogue(O, K, T):
     """The fused decode with Squared ReLU and the residual: the oracle's
     quantiser, dequantisation and epilogue, bit for bit."""
