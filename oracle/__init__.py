@@ -48,6 +48,12 @@ def _load():
         lib.sbl_oracle_sp24_meta_row_bytes.argtypes = [i64]
         lib.sbl_oracle_pack_sp24.restype = ctypes.c_int
         lib.sbl_oracle_pack_sp24.argtypes = [p, p, i64, i64, p, p]
+        lib.sbl_oracle_t24_lo_row_bytes.restype = i64
+        lib.sbl_oracle_t24_lo_row_bytes.argtypes = [i64]
+        lib.sbl_oracle_t24_hi_row_bytes.restype = i64
+        lib.sbl_oracle_t24_hi_row_bytes.argtypes = [i64]
+        lib.sbl_oracle_pack_t24.restype = ctypes.c_int
+        lib.sbl_oracle_pack_t24.argtypes = [p, i64, i64, p, p]
         lib.sbl_oracle_epilogue.argtypes = [p, i64, i64, i32, p, p, p]
         lib.sbl_oracle_rmsnorm_quantize_act.argtypes = [p, i64, i64, p, f32, p, p]
         lib.sbl_oracle_gamma_survivors.restype = f32
@@ -200,6 +206,27 @@ def pack_sp24(weff, mask):
     if _load().sbl_oracle_pack_sp24(_ptr(weff), _ptr(mask), d_out, d_in, _ptr(vals), _ptr(meta)) != 0:
         raise ValueError("mask keeps more than two positions in a group of four")
     return vals, meta
+
+
+def t24_lo_row_bytes(d_in: int) -> int:
+    return int(_load().sbl_oracle_t24_lo_row_bytes(d_in))
+
+
+def t24_hi_row_bytes(d_in: int) -> int:
+    return int(_load().sbl_oracle_t24_hi_row_bytes(d_in))
+
+
+def pack_t24(weff):
+    """6-bit group codes of W_eff: low plane uint8 [O, lo_row_bytes] and high
+    plane uint8 [O, hi_row_bytes]; raises ValueError when a group of four
+    holds more than two nonzeros."""
+    weff = _i8(weff)
+    d_out, d_in = weff.shape
+    lo = np.empty((d_out, t24_lo_row_bytes(d_in)), dtype=np.uint8)
+    hi = np.empty((d_out, t24_hi_row_bytes(d_in)), dtype=np.uint8)
+    if _load().sbl_oracle_pack_t24(_ptr(weff), d_out, d_in, _ptr(lo), _ptr(hi)) != 0:
+        raise ValueError("a group of four holds more than two nonzeros")
+    return lo, hi
 
 
 def gamma_survivors(w, mask) -> np.float32:

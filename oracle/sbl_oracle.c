@@ -281,6 +281,53 @@ int sbl_oracle_pack_sp24(const int8_t *weff, const uint8_t *mask, int64_t d_out,
     return 0;
 }
 
+int64_t sbl_oracle_t24_lo_row_bytes(int64_t d_in) { return round_up(d_in / 8, 16); }
+
+int64_t sbl_oracle_t24_hi_row_bytes(int64_t d_in) { return round_up(d_in / 16, 16); }
+
+/* T24: W_eff of a layer whose groups of four hold at most two nonzeros (2:4,
+ * 1:4, 2:8, 1:8 masks) in 6 bits per group -- a denser form of the 2-bit
+ * packing of [P5] "Inference Implementation: GPU" (no page gives a layout:
+ * reading R24).  Group g (positions 4g .. 4g+3) with nonzero positions
+ * p < q and sign bits s = 1 for -1, 0 for +1:
+ *   no nonzero   code 0
+ *   one (p)      code 1 + 2p + s_p                        (1 .. 8)
+ *   two (p, q)   code 9 + 4k + 2 s_p + s_q, k the index of (p, q) in
+ *                (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)       (9 .. 32)
+ * Low plane: code & 15 at bits 4 (g % 2) of byte g / 2 of the row; high
+ * plane: code >> 4 at bits 2 (g % 4) of byte g / 4.  Padding bytes 0.
+ * Returns -1 when a group has more than two nonzeros. */
+int sbl_oracle_pack_t24(const int8_t *weff, int64_t d_out, int64_t d_in, uint8_t *lo, uint8_t *hi)
+{
+    static const int pair_index[4][4] = {{-1, 0, 1, 2}, {-1, -1, 3, 4}, {-1, -1, -1, 5}, {-1, -1, -1, -1}};
+    int64_t lb = sbl_oracle_t24_lo_row_bytes(d_in), hb = sbl_oracle_t24_hi_row_bytes(d_in);
+    for (int64_t o = 0; o < d_out; ++o) {
+        uint8_t *lrow = lo + o * lb, *hrow = hi + o * hb;
+        for (int64_t b = 0; b < lb; ++b) lrow[b] = 0;
+        for (int64_t b = 0; b < hb; ++b) hrow[b] = 0;
+        for (int64_t g = 0; g < d_in / 4; ++g) {
+            const int8_t *w = weff + o * d_in + 4 * g;
+            int pos[4], count = 0;
+            for (int i = 0; i < 4; ++i)
+                if (w[i] != 0) pos[count++] = i;
+            unsigned code;
+            if (count == 0) {
+                code = 0;
+            } else if (count == 1) {
+                code = 1u + 2u * (unsigned)pos[0] + (w[pos[0]] < 0 ? 1u : 0u);
+            } else if (count == 2) {
+                code = 9u + 4u * (unsigned)pair_index[pos[0]][pos[1]] + (w[pos[0]] < 0 ? 2u : 0u) +
+                       (w[pos[1]] < 0 ? 1u : 0u);
+            } else {
+                return -1;
+            }
+            lrow[g / 2] = (uint8_t)(lrow[g / 2] | ((code & 15u) << (4 * (g % 2))));
+            hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 4))));
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------ mask statistics -- */
 
 /* Mask flip count between consecutive steps ([P1] "Dynamic Mask

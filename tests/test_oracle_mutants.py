@@ -53,6 +53,14 @@ MUTANTS = {
                              "            float u = bf16_to_f32(row[k]) * r;\n            float v = nearbyintf(u * rq);"),
     "sp24_fill_from_top": ("for (int i = 0; i < 4 && count < 2; ++i) {\n                if (mask[o * d_in + 4 * g + i]) continue;",
                            "for (int i = 3; i >= 0 && count < 2; --i) {\n                if (mask[o * d_in + 4 * g + i]) continue;"),
+    "t24_signs_swapped": ("(w[pos[0]] < 0 ? 2u : 0u) +\n                       (w[pos[1]] < 0 ? 1u : 0u);",
+                          "(w[pos[0]] < 0 ? 1u : 0u) +\n                       (w[pos[1]] < 0 ? 2u : 0u);"),
+    "t24_pair_table_order": ("{{-1, 0, 1, 2}, {-1, -1, 3, 4}, {-1, -1, -1, 5}",
+                             "{{-1, 0, 1, 3}, {-1, -1, 2, 4}, {-1, -1, -1, 5}"),
+    "t24_single_offset": ("code = 1u + 2u * (unsigned)pos[0] + (w[pos[0]] < 0 ? 1u : 0u);",
+                          "code = 2u * (unsigned)pos[0] + (w[pos[0]] < 0 ? 1u : 0u);"),
+    "t24_high_plane_stride": ("hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 4))));",
+                              "hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 2))));"),
 }
 
 PIN_CALLS = [
@@ -72,6 +80,9 @@ PIN_CALLS = [
     (pins.test_sp24_hand_example, ()),
     (pins.test_sp24_roundtrip, (2, 4)),
     (pins.test_sp24_roundtrip, (1, 4)),
+    (pins.test_t24_hand_row, ()),
+    (pins.test_t24_all_groups, ()),
+    (pins.test_t24_roundtrip, (2, 4)),
     (pins.test_epilogue_hand_values, ()),
     (pins.test_rmsnorm_quant_matches_numpy_definition, ()),
     (pins.test_gamma_survivors_hand_row_and_exact_mean, ()),

@@ -309,6 +309,89 @@ def test_sp24_rejects_masks_that_are_not_2of4():
         oracle.pack_sp24(layer.weff, layer.mask)
 
 
+# ------------------------------------------------------------------- T24
+
+T24_PAIRS = [(0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3)]
+
+
+def _t24_group_of_code(c):
+    """The group of four ternary weights a 6-bit T24 code stands for, read
+    off the code's definition (not from the oracle)."""
+    g = [0, 0, 0, 0]
+    if c == 0:
+        return g
+    if c <= 8:
+        p, neg = divmod(c - 1, 2)
+        g[p] = -1 if neg else 1
+        return g
+    k, rest = divmod(c - 9, 4)
+    p, q = T24_PAIRS[k]
+    g[p] = -1 if rest & 2 else 1
+    g[q] = -1 if rest & 1 else 1
+    return g
+
+
+def _t24_decode(lo, hi, d_in):
+    d_out = lo.shape[0]
+    w = np.zeros((d_out, d_in), dtype=np.int8)
+    for o in range(d_out):
+        for g in range(d_in // 4):
+            c = ((int(lo[o, g // 2]) >> (4 * (g % 2))) & 15) | (((int(hi[o, g // 4]) >> (2 * (g % 4))) & 3) << 4)
+            assert c <= 32, "codes above 32 are never written"
+            w[o, 4 * g:4 * g + 4] = _t24_group_of_code(c)
+    return w
+
+
+def test_t24_hand_row():
+    """Groups (0,0,0,0) (0,0,-1,0) (1,0,0,-1) (0,-1,1,0) have codes 0, 1 + 2*2
+    + 1 = 6, 9 + 4*2 + 0 + 1 = 18 ((0,3) is pair 2), 9 + 4*3 + 2 + 0 = 23
+    ((1,2) is pair 3): low plane bytes 0x60 0x72, high plane byte
+    0 | 0 << 2 | 1 << 4 | 1 << 6 = 0x50; padding zero."""
+    w = np.array([[0, 0, 0, 0, 0, 0, -1, 0, 1, 0, 0, -1, 0, -1, 1, 0]], dtype=np.int8)
+    lo, hi = oracle.pack_t24(w)
+    assert lo.shape == (1, 16) and hi.shape == (1, 16)
+    assert list(lo[0, :2]) == [0x60, 0x72] and not lo[0, 2:].any()
+    assert hi[0, 0] == 0x50 and not hi[0, 1:].any()
+
+
+def test_t24_all_groups():
+    """Every one of the 81 sign patterns of a group: the 33 with at most two
+    nonzeros get 33 distinct codes in 0..32 that decode back to the group;
+    the 48 others are refused."""
+    seen = set()
+    for digits in itertools.product([-1, 0, 1], repeat=4):
+        w = np.zeros((1, 16), dtype=np.int8)
+        w[0, 4:8] = digits  # group 1: low nibble 1 of byte 0, high bits 2..3
+        if sum(1 for v in digits if v) > 2:
+            with pytest.raises(ValueError):
+                oracle.pack_t24(w)
+            continue
+        lo, hi = oracle.pack_t24(w)
+        c = (int(lo[0, 0]) >> 4) | (((int(hi[0, 0]) >> 2) & 3) << 4)
+        assert c <= 32 and c not in seen
+        seen.add(c)
+        assert _t24_group_of_code(c) == list(digits)
+        assert lo[0, 0] & 15 == 0 and hi[0, 0] & 0xF3 == 0  # the zero groups stay zero
+    assert seen == set(range(33))
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (2, 8), (1, 8)])
+def test_t24_roundtrip(n, m):
+    """Layers with 2:4-compatible masks: an independent decoder of the two
+    planes gives W_eff back; padding bytes are zero."""
+    w = wl.master_weights(48, 272, seed=n * 10 + m)
+    layer = oracle.Layer(w, n, m)
+    lo, hi = oracle.pack_t24(layer.weff)
+    np.testing.assert_array_equal(_t24_decode(lo, hi, 272), layer.weff)
+    assert not lo[:, 272 // 8:].any() and not hi[:, 272 // 16:].any()
+
+
+def test_t24_rejects_masks_that_are_not_2of4():
+    w = wl.master_weights(16, 64, seed=5)
+    with pytest.raises(ValueError):
+        oracle.pack_t24(oracle.Layer(w, 6, 8).weff)
+
+
 # ------------------------------------------------------ RMSNorm + act quant
 
 def _np_rmsnorm_quant(xb, gb, eps):
