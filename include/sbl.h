@@ -69,20 +69,31 @@ typedef enum {
  *        bytes 2g, 2g+1 ([O, row_bytes(SP24 main)] int8, row_bytes =
  *        K/2 rounded up to 16).  Metadata: nibble i0 | (i1 << 2) at bits
  *        4*(g%2) of byte g/2 ([O, row_bytes(SP24 meta)] uint8, K/8 rounded
- *        up to 16).  Padding bytes are 0.  */
+ *        up to 16).  Padding bytes are 0.
+ *  T24   W_eff in 6 bits per group of four, for the same masks as SP24 (a
+ *        denser form of the 2-bit packing of the BitNet b1.58 2B4T summary,
+ *        "Inference Implementation: GPU"): group g with nonzero positions
+ *        p < q and sign bits s (1 for -1) has code 0 (none), 1 + 2p + s_p
+ *        (one), or 9 + 4k + 2 s_p + s_q (two; k = index of (p, q) in
+ *        (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)).  Low plane: code & 15 at bits
+ *        4*(g%2) of byte g/2 ([O, row_bytes(T24 main)], K/8 rounded up to
+ *        16); high plane: code >> 4 at bits 2*(g%4) of byte g/4 ([O,
+ *        row_bytes(T24 high)], K/16 rounded up to 16).  Padding bytes 0. */
 typedef enum {
     SBL_FMT_PK2 = 1,
     SBL_FMT_NM = 2,
     SBL_FMT_I8 = 4,
     SBL_FMT_BF16T = 8,
-    SBL_FMT_SP24 = 16
+    SBL_FMT_SP24 = 16,
+    SBL_FMT_T24 = 32
 } sbl_format;
 
 /* Which buffer of a format sbl_packed_row_bytes() describes. */
 typedef enum {
     SBL_BUF_MAIN = 0,       /* PK2 / I8 / BF16T data, NM / SP24 values */
     SBL_BUF_NM_BITMAP = 1,  /* NM keep bitmap                          */
-    SBL_BUF_SP24_META = 2   /* SP24 position metadata                  */
+    SBL_BUF_SP24_META = 2,  /* SP24 position metadata                  */
+    SBL_BUF_T24_HI = 3      /* T24 high plane (SBL_BUF_MAIN: low plane) */
 } sbl_buffer;
 
 /* Operations that take a workspace. */
@@ -114,6 +125,8 @@ typedef struct {
     float *gamma;       /* device scalar                                */
     int8_t *sp24_values; /* SBL_FMT_SP24 values                         */
     uint8_t *sp24_meta;  /* SBL_FMT_SP24 position metadata              */
+    uint8_t *t24_lo;     /* SBL_FMT_T24 low plane                       */
+    uint8_t *t24_hi;     /* SBL_FMT_T24 high plane                      */
 } sbl_packed;
 
 /* Human-readable text for a status code (static storage). */
@@ -268,7 +281,8 @@ sbl_status sbl_quantize_act_rmsnorm(const uint16_t *X, int32_t T, int32_t K, con
  *   Y[t,o] = fl32(fl32(acc) * fl32(gamma * d[t]))  (bf16 by RNE, or fp32).
  * fmt selects the weight operand: SBL_FMT_I8 runs the tcgen05 int8 tensor
  * core GEMM (any T); SBL_FMT_PK2 runs the decode kernel that streams the
- * 2-bit codes (T <= 16, K a multiple of 64).  Y: [T, O] bf16 bits
+ * 2-bit codes (T <= 16, K a multiple of 64); SBL_FMT_T24 the same kernel
+ * streaming the 6-bit group codes (same limits; n <= 2, m = 4 or 8).  Y: [T, O] bf16 bits
  * (y_is_fp32 = 0) or fp32.  acc_out: optional [T, O] int32 copy of the
  * accumulators (NULL to skip).  One launch.
  * The SBL_FMT_PK2 kernel is launched with programmatic dependent launch: it

@@ -386,6 +386,17 @@ cudaError_t launch_decode_fused(const cudaLaunchConfig_t &cfg, const DecodeArgs 
     }
 }
 
+template <int NT>
+cudaError_t launch_decode_t24(const cudaLaunchConfig_t &cfg, const DecodeArgs &a, int cpw)
+{
+    switch (cpw) {
+    case 1: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 1, 1, false, true>, a);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 2, 1, false, true>, a);
+    case 4: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, 1, false, true>, a);
+    default: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 8, 1, false, true>, a);
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -421,6 +432,10 @@ size_t sbl_packed_row_bytes(const sbl_layer_desc *desc, sbl_format fmt, sbl_buff
     case SBL_FMT_SP24:
         if (which == SBL_BUF_MAIN) return static_cast<size_t>(round_up(K / 2, 16));
         if (which == SBL_BUF_SP24_META) return static_cast<size_t>(round_up(K / 8, 16));
+        return 0;
+    case SBL_FMT_T24:
+        if (which == SBL_BUF_MAIN) return static_cast<size_t>(round_up(K / 8, 16));
+        if (which == SBL_BUF_T24_HI) return static_cast<size_t>(round_up(K / 16, 16));
         return 0;
     }
     return 0;
@@ -458,12 +473,17 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
     const bool bf16 = v.master_dtype == SBL_MASTER_BF16;
     if (st != SBL_OK) return st;
     if (!W || !out || !out->gamma) return SBL_ERR_INVALID_ARG;
-    const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T | SBL_FMT_SP24;
+    const uint32_t known = SBL_FMT_PK2 | SBL_FMT_NM | SBL_FMT_I8 | SBL_FMT_BF16T | SBL_FMT_SP24 | SBL_FMT_T24;
     if (formats & ~known) return SBL_ERR_INVALID_ARG;
     if (formats & SBL_FMT_SP24) {
         if (!out->sp24_values || !out->sp24_meta) return SBL_ERR_INVALID_ARG;
         if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
         if (!aligned16(out->sp24_values) || !aligned16(out->sp24_meta)) return SBL_ERR_ALIGNMENT;
+    }
+    if (formats & SBL_FMT_T24) {
+        if (!out->t24_lo || !out->t24_hi) return SBL_ERR_INVALID_ARG;
+        if (!sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
+        if (!aligned16(out->t24_lo) || !aligned16(out->t24_hi)) return SBL_ERR_ALIGNMENT;
     }
     if ((formats & SBL_FMT_PK2) && !out->pk2) return SBL_ERR_INVALID_ARG;
     if ((formats & SBL_FMT_NM) && (!out->nm_values || !out->nm_bitmap)) return SBL_ERR_INVALID_ARG;
@@ -557,6 +577,12 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
         pa.out.nm_bitmap_stride =
             static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_NM, SBL_BUF_NM_BITMAP));
     }
+    if (formats & SBL_FMT_T24) {
+        pa.out.t24_lo = out->t24_lo;
+        pa.out.t24_lo_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_MAIN));
+        pa.out.t24_hi = out->t24_hi;
+        pa.out.t24_hi_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_T24_HI));
+    }
     if (formats & SBL_FMT_SP24) {
         pa.out.sp24_values = out->sp24_values;
         pa.out.sp24_values_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_SP24, SBL_BUF_MAIN));
@@ -572,7 +598,7 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
         pa.stats.near_zero = stats->near_zero;
         pa.stats.threshold = stats->block_threshold;
     }
-    if ((formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM | SBL_FMT_SP24)) || want_stats) {
+    if ((formats & (SBL_FMT_PK2 | SBL_FMT_I8 | SBL_FMT_NM | SBL_FMT_SP24 | SBL_FMT_T24)) || want_stats) {
         // programmatic dependent launch behind gamma_kernel (see pack_kernel);
         // a thread covers 16 weights
         const int64_t per_cta = 256 * 16 / desc->m;  // groups per CTA
@@ -587,7 +613,7 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const bool sp = (formats & SBL_FMT_SP24) != 0;
+        const bool sp = (formats & (SBL_FMT_SP24 | SBL_FMT_T24)) != 0;  // the 2:4 formats' instantiation
         const int opt = (sp ? kPackSp24 : 0) | (want_stats ? kPackStats : 0) |
                         (v.mask_source == SBL_MASK_FROM_QUANTIZED ? kPackMaskQ : 0) | (bf16 ? kPackBf16 : 0);
         const cudaError_t e = desc->m == 8 ? launch_pack<8>(cfg, pa, opt) : launch_pack<4>(cfg, pa, opt);
@@ -727,7 +753,7 @@ static_assert(kLinearFuseMaxElems <= kDecFuseMaxElems, "the fused prologue holds
 // One decode launch: a CTA per 16 output rows; fused: the bf16 activations
 // are quantised in the kernel's prologue into T (K + 16) bytes of shared
 // memory (at most 8.4 KB: T K <= 8192).
-static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream)
+static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream, bool t24 = false)
 {
     a.chunks = (a.K + kDecChunk - 1) / kDecChunk;
     // chunks per warp per round: the whole row in one round up to
@@ -749,7 +775,9 @@ static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (fuse) {
+    if (t24) {
+        e = a.T <= 8 ? launch_decode_t24<1>(cfg, a, cpw) : launch_decode_t24<2>(cfg, a, cpw);
+    } else if (fuse) {
         a.xs_stride = a.K + kDecXsPad;
         cfg.dynamicSmemBytes = static_cast<size_t>(a.T) * a.xs_stride;
         e = a.T <= 8 ? launch_decode_fused<1>(cfg, a, cpw) : launch_decode_fused<2>(cfg, a, cpw);
@@ -801,6 +829,32 @@ static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, con
         return choose_pair_bn(O, T, di->num_sms) == 224
                    ? launch_sp24_pair<224>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, epi, stream)
                    : launch_sp24_pair<128>(di, O, K, T, Xq, d, w, Y, y_is_fp32 != 0, acc_out, epi, stream);
+    }
+    if (fmt == SBL_FMT_T24) {
+        if (!w->t24_lo || !w->t24_hi) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(w->t24_lo) || !aligned16(w->t24_hi)) return SBL_ERR_ALIGNMENT;
+        if (T > kDecMaxTokens || K % kDecKUnit != 0 || !sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
+        DecodeArgs a;
+        memset(&a, 0, sizeof(a));
+        a.pk2 = w->t24_lo;  // valid row base for the (unused) PK2 pointers
+        a.t24_lo = w->t24_lo;
+        a.t24_lo_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_MAIN));
+        a.t24_hi = w->t24_hi;
+        a.t24_hi_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_T24_HI));
+        a.xq = Xq;
+        a.d = d;
+        a.gamma = w->gamma;
+        a.out = Y;
+        a.out_fp32 = y_is_fp32 ? 1 : 0;
+        a.acc_out = acc_out;
+        if (epi) {
+            a.relu2 = epi->relu2 ? 1 : 0;
+            a.residual = epi->residual;
+        }
+        a.T = T;
+        a.K = K;
+        a.O = O;
+        return launch_decode(a, false, stream, true);
     }
     if (fmt == SBL_FMT_PK2) {
         if (!w->pk2) return SBL_ERR_INVALID_ARG;

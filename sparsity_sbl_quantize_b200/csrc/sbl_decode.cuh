@@ -60,6 +60,11 @@ struct DecodeArgs {
     const uint16_t *residual;  // ... then v = v + residual[t, o] (bf16 [T, O]; nullptr: none)
     int32_t T, K, O;
     int32_t chunks;       // ceil(K / 256)
+    // T24 variant only: the 6-bit group codes' planes
+    const uint8_t *t24_lo;
+    int64_t t24_lo_stride;
+    const uint8_t *t24_hi;
+    int64_t t24_hi_stride;
     // fused variant only
     const uint16_t *x;    // bf16 activations [T, K]
     int8_t *xq_out;       // Q_a(x) [T, K], stored by CTA 0 (nullptr: not stored)
@@ -93,6 +98,17 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p)
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
+    return v;
+}
+
+// A lane's T24 weights of one row and chunk: 8 low-plane bytes and 4
+// high-plane bytes (read once, no L1 allocation) as (lo, lo, hi, 0).
+__device__ __forceinline__ uint4 ld_stream_t24(const void *lo, const void *hi)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(lo));
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v.z) : "l"(hi));
+    v.w = 0u;
     return v;
 }
 
@@ -195,6 +211,48 @@ __device__ __forceinline__ void decode_quantize_x(const DecodeArgs &a, uint32_t 
     __syncthreads();
 }
 
+// T24 decoding: the PK2 byte (2-bit codes w + 1 of four weights) of a 6-bit
+// group code (0: none; 1 + 2p + s_p: one; 9 + 4k + 2 s_p + s_q: two at pair
+// k of (0,1) (0,2) (0,3) (1,2) (1,3) (2,3); s = 1 for -1).  Codes above 32
+// are never written; they decode as zeros.
+__device__ __forceinline__ uint32_t t24_pk2_byte(uint32_t c)
+{
+    uint32_t b = 0x55u;  // four zero weights
+    if (c >= 1u && c <= 8u) {
+        const uint32_t p = (c - 1u) >> 1, neg = (c - 1u) & 1u;
+        b = (b & ~(3u << (2 * p))) | ((neg ? 0u : 2u) << (2 * p));
+    } else if (c >= 9u && c <= 32u) {
+        const uint32_t k = (c - 9u) >> 2, r = (c - 9u) & 3u;
+        const uint32_t pq = (0x323121302010ull >> (8 * k)) & 0xffu;  // q << 4 | p
+        const uint32_t p = pq & 15u, q = pq >> 4;
+        b = (b & ~(3u << (2 * p)) & ~(3u << (2 * q))) | (((r & 2u) ? 0u : 2u) << (2 * p)) |
+            (((r & 1u) ? 0u : 2u) << (2 * q));
+    }
+    return b;
+}
+
+// Two PK2 bytes of a pair of groups from its 12-bit index: the low-plane byte
+// (two nibbles) | the pair's 4 high-plane bits << 8.
+__device__ __forceinline__ uint32_t t24_pair_pk2(uint32_t idx)
+{
+    const uint32_t lo = idx & 0xffu, hi = idx >> 8;
+    return t24_pk2_byte((lo & 15u) | ((hi & 3u) << 4)) | (t24_pk2_byte((lo >> 4) | ((hi >> 2) << 4)) << 8);
+}
+
+// The four PK2 words of a lane's 64 weights of one row from its 8 low-plane
+// bytes (v.x, v.y) and 32 high-plane bits (v.z): word j is pairs 2j and
+// 2j + 1 through the shared table.
+__device__ __forceinline__ void t24_decode(const uint4 &v, const uint16_t *lut, uint32_t (&w)[4])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = j < 2 ? v.x : v.y;
+        const uint32_t i0 = ((lo >> (16 * (j & 1))) & 0xffu) | (((v.z >> (8 * j)) & 15u) << 8);
+        const uint32_t i1 = ((lo >> (16 * (j & 1) + 8)) & 0xffu) | (((v.z >> (8 * j + 4)) & 15u) << 8);
+        w[j] = static_cast<uint32_t>(lut[i0]) | (static_cast<uint32_t>(lut[i1]) << 16);
+    }
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s)
 {
     uint32_t r;
@@ -229,13 +287,20 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 // NT: n8 token blocks (T <= 8 or T <= 16); CPW: chunks per warp per round;
 // RG: groups of 16 rows per CTA, each worked by 8 warps that split the K
 // chunks of its rows (the groups read the same activations: L1 hits).
-template <int NT, int CPW, int RG, bool FUSE = false>
+// T24: the weights come as 6-bit group codes (two planes), expanded to PK2
+// words through a 4096-entry shared table built before the wait.
+template <int NT, int CPW, int RG, bool FUSE = false, bool T24 = false>
 __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
 {
     extern __shared__ __align__(16) uint8_t dec_xs[];
     __shared__ uint32_t s_amax[FUSE ? kDecMaxTokens : 1];
+    __shared__ uint16_t t24_lut[T24 ? 4096 : 1];
     if constexpr (FUSE) {
         if (threadIdx.x < kDecMaxTokens) s_amax[threadIdx.x] = 0u;
+        __syncthreads();
+    }
+    if constexpr (T24) {
+        for (int i = threadIdx.x; i < 4096; i += blockDim.x) t24_lut[i] = static_cast<uint16_t>(t24_pair_pk2(i));
         __syncthreads();
     }
     constexpr int kWarps = 8;                          // warps per row group
@@ -252,6 +317,11 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
     // 64-byte chunk (weights pos = 256 c + 64 tg .. pos + 63, bytes pos / 4 ..)
     const uint8_t *wA = args.pk2 + static_cast<int64_t>(okA ? row0 + g : 0) * args.pk2_stride;
     const uint8_t *wB = args.pk2 + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.pk2_stride;
+    // T24: the same rows of the two planes (8 + 4 bytes per lane and chunk)
+    const uint8_t *lA = T24 ? args.t24_lo + static_cast<int64_t>(okA ? row0 + g : 0) * args.t24_lo_stride : nullptr;
+    const uint8_t *lB = T24 ? args.t24_lo + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.t24_lo_stride : nullptr;
+    const uint8_t *hA = T24 ? args.t24_hi + static_cast<int64_t>(okA ? row0 + g : 0) * args.t24_hi_stride : nullptr;
+    const uint8_t *hB = T24 ? args.t24_hi + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.t24_hi_stride : nullptr;
     // output (t, r) of the row group belongs to thread 16 t + r of the group
     // (the group of thread i is i / 256, the same as its warp's)
     const int t_out = (threadIdx.x & 255) >> 4, r_out = threadIdx.x & 15;
@@ -279,8 +349,13 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
             const int c = round0 + wig + kWarps * i;
             const int pos = c * kDecChunk + 64 * tg;
             const bool ok = c < args.chunks && pos < args.K;
-            wa[i] = (ok && okA) ? ld_stream16(wA + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
-            wb[i] = (ok && okB) ? ld_stream16(wB + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (T24) {
+                wa[i] = (ok && okA) ? ld_stream_t24(lA + pos / 8, hA + pos / 16) : make_uint4(0u, 0u, 0u, 0u);
+                wb[i] = (ok && okB) ? ld_stream_t24(lB + pos / 8, hB + pos / 16) : make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                wa[i] = (ok && okA) ? ld_stream16(wA + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
+                wb[i] = (ok && okB) ? ld_stream16(wB + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
+            }
         }
         if (round0 == 0) {
             pdl_wait_prior();  // activations, scales and gamma
@@ -343,12 +418,20 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
                         xt[b][q] = transpose4x4(v);
                     }
                 }
+                uint32_t pa[4], pb[4];  // the lane's PK2 words of rows g and g + 8
+                if constexpr (T24) {
+                    t24_decode(wa[i], t24_lut, pa);
+                    t24_decode(wb[i], t24_lut, pb);
+                } else {
+                    pa[0] = wa[i].x, pa[1] = wa[i].y, pa[2] = wa[i].z, pa[3] = wa[i].w;
+                    pb[0] = wb[i].x, pb[1] = wb[i].y, pb[2] = wb[i].z, pb[3] = wb[i].w;
+                }
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     // step s takes word s/2 of the lane's 16 bytes and the
                     // code shifts ja (K slots 0..15) and ja + 1 (K slots 16..31)
                     const int wi = s >> 1, ja = 2 * (s & 1);
-                    const uint32_t ra = word_of(wa[i], wi), rb = word_of(wb[i], wi);
+                    const uint32_t ra = pa[wi], rb = pb[wi];
                     const uint32_t a0 = (ra >> (2 * ja)) & 0x03030303u;
                     const uint32_t a1 = (rb >> (2 * ja)) & 0x03030303u;
                     const uint32_t a2 = (ra >> (2 * ja + 2)) & 0x03030303u;

@@ -53,6 +53,10 @@ struct PackOut {
     int64_t sp24_values_stride;
     uint8_t *sp24_meta;
     int64_t sp24_meta_stride;
+    uint8_t *t24_lo;
+    int64_t t24_lo_stride;
+    uint8_t *t24_hi;
+    int64_t t24_hi_stride;
 };
 
 // By-product statistics of the re-mask step (all optional; the counters are
@@ -494,13 +498,34 @@ __device__ __forceinline__ void sp24_group(uint32_t wbytes, uint32_t keep4, int 
     meta |= (i0 | (i1 << 2)) << (4 * q);
 }
 
+// T24 code of one group of four W_eff bytes (int8 -1 / 0 / +1): 0 (no
+// nonzero), 1 + 2p + s_p (one at p), 9 + 4k + 2 s_p + s_q (two, p < q, k the
+// index of (p, q) in (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)); s = 1 for -1.
+__device__ __forceinline__ uint32_t t24_code(uint32_t wbytes)
+{
+    uint32_t nz = 0u, neg = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t b = (wbytes >> (8 * i)) & 0xffu;
+        nz |= (b != 0u ? 1u : 0u) << i;
+        neg |= (b >> 7) << i;
+    }
+    if (nz == 0u) return 0u;
+    const uint32_t p = static_cast<uint32_t>(__ffs(nz) - 1);
+    if (__popc(nz) == 1) return 1u + 2u * p + ((neg >> p) & 1u);
+    const uint32_t q = static_cast<uint32_t>(31 - __clz(nz));
+    const uint32_t k = p * (7u - p) / 2u + (q - p - 1u);
+    return 9u + 4u * k + 2u * ((neg >> p) & 1u) + ((neg >> q) & 1u);
+}
+
 // Mask + ternarise + pack: thread t of CTA c owns the 16 consecutive weights
 // (two groups of 8 or four of 4) starting at (256 c + t) * 16.  Launched with
 // programmatic dependent launch right behind gamma_kernel: W is loaded and the
 // N:M keep masks (which need only |W|) are computed before waiting for
 // gamma_kernel (which does not write W); gamma is read after.
-// SP24: also write the 2:4 sparse-MMA operand (a separate instantiation, so
-// the other formats' kernel carries none of its registers).
+// SP24: also write the 2:4 formats that were asked for, the sparse-MMA
+// operand and the 6-bit T24 codes (a separate instantiation, so the other
+// formats' kernel carries none of their registers).
 // Ternarise and store every requested format of one thread's 16 weights.
 template <int M, bool SP24>
 __device__ __forceinline__ void pack_formats(const PackArgs &a, int64_t e0, const uint32_t (&bits)[16 / M][M],
@@ -510,22 +535,45 @@ __device__ __forceinline__ void pack_formats(const PackArgs &a, int64_t e0, cons
     const uint32_t thr_bits = __float_as_uint(ternary_threshold(*a.gamma));
     const int32_t row = static_cast<int32_t>(__umul64hi(static_cast<uint64_t>(e0), a.inv_cols));
     const int32_t col0 = static_cast<int32_t>(e0 - static_cast<int64_t>(row) * a.cols);  // 16 | K: same row
-    uint32_t sp_vals[2] = {0u, 0u}, sp_meta = 0u;
+    uint32_t sp_vals[2] = {0u, 0u}, sp_meta = 0u, t_lo = 0u, t_hi = 0u;
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
         uint32_t w0, w1;
         ternarise_group<M>(bits[b], keep[b], thr_bits, w0, w1);
         store_group<M>(a, row, col0 / M + b, w0, w1, keep[b]);
         if constexpr (SP24) {
+            // the thread's four groups of four, j = 0..3
+            const int j0 = M == 4 ? b : 2 * b;
             if constexpr (M == 4) {
                 sp24_group(w0, keep[b], b, sp_vals, sp_meta);
             } else {
                 sp24_group(w0, keep[b], 2 * b, sp_vals, sp_meta);
                 sp24_group(w1, keep[b] >> 4, 2 * b + 1, sp_vals, sp_meta);
             }
+            const uint32_t c0 = t24_code(w0);
+            t_lo |= (c0 & 15u) << (4 * j0);
+            t_hi |= (c0 >> 4) << (2 * j0);
+            if constexpr (M == 8) {
+                const uint32_t c1 = t24_code(w1);
+                t_lo |= (c1 & 15u) << (4 * (j0 + 1));
+                t_hi |= (c1 >> 4) << (2 * (j0 + 1));
+            }
         }
     }
     if constexpr (SP24) {
+        if (a.out.t24_lo) {
+            // 2 low-plane bytes and 1 high-plane byte per thread
+            uint8_t *lrow = a.out.t24_lo + static_cast<int64_t>(row) * a.out.t24_lo_stride;
+            uint8_t *hrow = a.out.t24_hi + static_cast<int64_t>(row) * a.out.t24_hi_stride;
+            *reinterpret_cast<uint16_t *>(lrow + col0 / 8) = static_cast<uint16_t>(t_lo);
+            hrow[col0 / 16] = static_cast<uint8_t>(t_hi);
+            if (col0 + 16 == a.cols) {
+                for (int64_t b = a.cols / 8; b < a.out.t24_lo_stride; ++b) lrow[b] = 0;
+                for (int64_t b = a.cols / 16; b < a.out.t24_hi_stride; ++b) hrow[b] = 0;
+            }
+        }
+    }
+    if (SP24 && a.out.sp24_values) {
         // 8 value bytes and 16 metadata bits per thread; the thread that ends
         // a row also zeroes the row padding
         uint8_t *vrow = reinterpret_cast<uint8_t *>(a.out.sp24_values) + static_cast<int64_t>(row) * a.out.sp24_values_stride;

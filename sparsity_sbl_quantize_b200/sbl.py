@@ -24,8 +24,8 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 SBL_OK = 0
-SBL_FMT_PK2, SBL_FMT_NM, SBL_FMT_I8, SBL_FMT_BF16T, SBL_FMT_SP24 = 1, 2, 4, 8, 16
-SBL_BUF_MAIN, SBL_BUF_NM_BITMAP, SBL_BUF_SP24_META = 0, 1, 2
+SBL_FMT_PK2, SBL_FMT_NM, SBL_FMT_I8, SBL_FMT_BF16T, SBL_FMT_SP24, SBL_FMT_T24 = 1, 2, 4, 8, 16, 32
+SBL_BUF_MAIN, SBL_BUF_NM_BITMAP, SBL_BUF_SP24_META, SBL_BUF_T24_HI = 0, 1, 2, 3
 SBL_OP_QUANTIZE_MASK_PACK, SBL_OP_BACKWARD = 0, 1
 
 STATUS_NAMES = {0: "SBL_OK", 1: "SBL_ERR_INVALID_ARG", 2: "SBL_ERR_SHAPE", 3: "SBL_ERR_ALIGNMENT",
@@ -42,7 +42,8 @@ class sbl_packed(ctypes.Structure):
     _fields_ = [("pk2", ctypes.c_void_p), ("nm_values", ctypes.c_void_p),
                 ("nm_bitmap", ctypes.c_void_p), ("i8", ctypes.c_void_p),
                 ("bf16t", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
-                ("sp24_values", ctypes.c_void_p), ("sp24_meta", ctypes.c_void_p)]
+                ("sp24_values", ctypes.c_void_p), ("sp24_meta", ctypes.c_void_p),
+                ("t24_lo", ctypes.c_void_p), ("t24_hi", ctypes.c_void_p)]
 
 
 class sbl_pack_variant(ctypes.Structure):
@@ -147,11 +148,13 @@ class Packed:
     bf16t: Optional[torch.Tensor] = None
     sp24_values: Optional[torch.Tensor] = None
     sp24_meta: Optional[torch.Tensor] = None
+    t24_lo: Optional[torch.Tensor] = None
+    t24_hi: Optional[torch.Tensor] = None
 
     def c(self) -> sbl_packed:
         return sbl_packed(*[(t.data_ptr() if t is not None else None)
                             for t in (self.pk2, self.nm_values, self.nm_bitmap, self.i8, self.bf16t,
-                                      self.gamma, self.sp24_values, self.sp24_meta)])
+                                      self.gamma, self.sp24_values, self.sp24_meta, self.t24_lo, self.t24_hi)])
 
 
 # ------------------------------------------------------------------ C calls
@@ -316,6 +319,10 @@ def alloc_packed(d: sbl_layer_desc, formats: int, device="cuda") -> Packed:
         p.sp24_values = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_SP24)), dtype=torch.int8, device=device)
         p.sp24_meta = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_SP24, SBL_BUF_SP24_META)),
                                   dtype=torch.uint8, device=device)
+    if formats & SBL_FMT_T24:
+        p.t24_lo = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_T24)), dtype=torch.uint8, device=device)
+        p.t24_hi = torch.empty((O, sbl_packed_row_bytes(d, SBL_FMT_T24, SBL_BUF_T24_HI)),
+                               dtype=torch.uint8, device=device)
     return p
 
 

@@ -64,6 +64,9 @@ class GpuLayer:
         if p.sp24_values is not None:
             out["sp24_values"] = p.sp24_values.cpu().numpy()
             out["sp24_meta"] = p.sp24_meta.cpu().numpy()
+        if p.t24_lo is not None:
+            out["t24_lo"] = p.t24_lo.cpu().numpy()
+            out["t24_hi"] = p.t24_hi.cpu().numpy()
         return out
 
 

@@ -54,6 +54,8 @@ def test_row_bytes_match_oracle_formats(sbl, O, K, n, m):
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_BF16T) == 2 * O
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_SP24) == oracle.sp24_value_row_bytes(K)
     assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_SP24, sbl.SBL_BUF_SP24_META) == oracle.sp24_meta_row_bytes(K)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_T24) == oracle.t24_lo_row_bytes(K)
+    assert sbl.sbl_packed_row_bytes(d, sbl.SBL_FMT_T24, sbl.SBL_BUF_T24_HI) == oracle.t24_hi_row_bytes(K)
 
 
 @pytest.mark.parametrize("O,K,n,m", [(0, 256, 6, 8), (128, 250, 6, 8), (128, 256, 9, 8),
@@ -184,6 +186,28 @@ def test_sp24_validation(sbl):
     skew = sbl.sbl_packed(None, None, None, None, None, good, good + 8, good)
     assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_SP24,
                 ctypes.byref(skew), ws, 1 << 20, None) == 3
+
+
+def test_t24_validation(sbl):
+    """The 6-bit group code exists for the same masks as SP24 (n <= 2): other
+    n:m are unsupported in the pack; missing or misaligned planes are
+    rejected first; the decode takes at most 16 tokens."""
+    good = 0x10000
+    P = ctypes.c_void_p
+    ws = P(good)
+    d68 = sbl.desc(128, 256, 6, 8)
+    d24 = sbl.desc(128, 256, 2, 4)
+    w = sbl.sbl_packed(None, None, None, None, None, good, None, None, good, good)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d68), P(good), sbl.SBL_FMT_T24,
+                ctypes.byref(w), ws, 1 << 20, None) == 4
+    nohi = sbl.sbl_packed(None, None, None, None, None, good, None, None, good, None)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_T24,
+                ctypes.byref(nohi), ws, 1 << 20, None) == 1
+    skew = sbl.sbl_packed(None, None, None, None, None, good, None, None, good + 8, good)
+    assert _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d24), P(good), sbl.SBL_FMT_T24,
+                ctypes.byref(skew), ws, 1 << 20, None) == 3
+    assert _raw(sbl, "sbl_forward", ctypes.byref(d24), P(good), P(good), 17, ctypes.byref(w),
+                sbl.SBL_FMT_T24, P(good), 0, None, None) in (4, 7)
 
 
 def test_forward_format_recommendation(sbl):

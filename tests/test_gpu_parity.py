@@ -26,11 +26,12 @@ FWD_TOL = 1e-3  # only used where bit-exactness is not expected (backward)
 
 
 SP24 = 16
+T24 = 32
 
 
 def check_pack(w, n, m, formats=ALL_FORMATS):
     if n <= 2 and formats == ALL_FORMATS:
-        formats |= SP24  # the sparse MMA operand exists for 2:4-compatible masks
+        formats |= SP24 | T24  # the 2:4 formats exist for 2:4-compatible masks
     layer = GpuLayer(w, n, m, formats)
     got = layer.host()
     ref = oracle.Layer(w, n, m)
@@ -50,6 +51,10 @@ def check_pack(w, n, m, formats=ALL_FORMATS):
         vals, meta = oracle.pack_sp24(ref.weff, ref.mask)
         np.testing.assert_array_equal(got["sp24_values"], vals)
         np.testing.assert_array_equal(got["sp24_meta"], meta)
+    if "t24_lo" in got:
+        lo, hi = oracle.pack_t24(ref.weff)
+        np.testing.assert_array_equal(got["t24_lo"], lo)
+        np.testing.assert_array_equal(got["t24_hi"], hi)
     return layer, ref
 
 
@@ -244,9 +249,9 @@ def run_forward_full_check(O, K, T, n, m, seed, fmt_name="I8", outliers=0.0):
     q, d = quantize_act(x)
     qr, dr, accr, yr, ybr = ref.forward(x)
     np.testing.assert_array_equal(q.cpu().numpy(), qr)
-    fmt = {"I8": sbl.SBL_FMT_I8, "PK2": sbl.SBL_FMT_PK2, "SP24": sbl.SBL_FMT_SP24}[fmt_name]
-    if fmt_name == "SP24":
-        layer = GpuLayer(w, n, m, sbl.SBL_FMT_SP24)
+    fmt = {"I8": sbl.SBL_FMT_I8, "PK2": sbl.SBL_FMT_PK2, "SP24": sbl.SBL_FMT_SP24, "T24": sbl.SBL_FMT_T24}[fmt_name]
+    if fmt_name in ("SP24", "T24"):
+        layer = GpuLayer(w, n, m, fmt)
     yb, acc = forward(layer, q, d, fmt)
     np.testing.assert_array_equal(acc.cpu().numpy(), accr)
     np.testing.assert_array_equal(bits_of(yb), ybr)
@@ -281,6 +286,32 @@ def test_forward_single_layer_workload_outliers():
                                    (48, 2560, 12)])   # a CTA of two 16-row groups, one past O
 def test_forward_decode_pk2_bit_exact(O, K, T):
     run_forward_full_check(O, K, T, 2, 4, seed=O + K + T, fmt_name="PK2")
+
+
+# T24: the decode kernel from the 6-bit group codes (2:4-compatible masks)
+@pytest.mark.parametrize("O,K,T,n,m", [(48, 11008, 7, 2, 4), (32, 16448, 16, 2, 4), (16, 192, 8, 2, 4),
+                                       (6912, 2560, 1, 2, 4), (2560, 6912, 16, 2, 4), (96, 1024, 3, 1, 4),
+                                       (64, 2048, 12, 2, 8), (32, 512, 1, 1, 8)])
+def test_forward_decode_t24_bit_exact(O, K, T, n, m):
+    run_forward_full_check(O, K, T, n, m, seed=O + K + T + n, fmt_name="T24")
+
+
+def test_forward_t24_epilogue_and_packed_planes():
+    """Squared ReLU and the residual on the T24 decode; the planes the pack
+    wrote next to SP24 equal the oracle's."""
+    sbl = sbl_mod()
+    O, K, T = 64, 2560, 5
+    w = wl.master_weights(O, K, seed=9)
+    x = wl.activations(T, K, seed=9)
+    layer, ref = check_pack(w, 2, 4)
+    _, _, _, yr, _ = ref.forward(x)
+    res_bits = wl.activations(T, O, seed=10)
+    _, outb = oracle.epilogue(yr, relu2=True, residual_bf16_bits=res_bits)
+    q, d = quantize_act(x)
+    y = torch.empty((T, O), dtype=torch.bfloat16, device="cuda")
+    sbl.sbl_forward_ex(layer.desc, q, d, T, layer.packed, sbl.SBL_FMT_T24, y, relu2=True,
+                       residual=bf16_dev(res_bits))
+    np.testing.assert_array_equal(bits_of(y), outb)
 
 
 def test_forward_decode_pk2_six_of_eight():
