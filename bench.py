@@ -851,9 +851,10 @@ def main():
     args = parse()
     wk = wl.WORKLOADS[args.workload]
     if args.record_traffic:
-        # the roofline kernels: the decode GEMV (last template flag 0: not the
-        # fused variant), or the int8 dense and 2:4 sparse forward GEMMs
-        regex = r"decode_kernel<\d+, \d+, \d+, 0>" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
+        # the roofline kernels: the decode GEMV from PK2 codes (the last two
+        # template flags 0: not the fused, not the T24 variant), or the int8
+        # dense and 2:4 sparse forward GEMMs
+        regex = r"decode_kernel<\d+, \d+, \d+, 0, 0>" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
         print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command)))
         return
     if args.impl == "reference":

@@ -776,6 +776,7 @@ static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream, b
     cfg.numAttrs = 1;
     cudaError_t e;
     if (t24) {
+        cfg.dynamicSmemBytes = 4096 * sizeof(uint16_t);  // the pair table
         e = a.T <= 8 ? launch_decode_t24<1>(cfg, a, cpw) : launch_decode_t24<2>(cfg, a, cpw);
     } else if (fuse) {
         a.xs_stride = a.K + kDecXsPad;
@@ -836,11 +837,10 @@ static sbl_status forward_impl(const sbl_layer_desc *desc, const int8_t *Xq, con
         if (T > kDecMaxTokens || K % kDecKUnit != 0 || !sp24_fits(desc)) return SBL_ERR_UNSUPPORTED;
         DecodeArgs a;
         memset(&a, 0, sizeof(a));
-        a.pk2 = w->t24_lo;  // valid row base for the (unused) PK2 pointers
-        a.t24_lo = w->t24_lo;
-        a.t24_lo_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_MAIN));
+        a.pk2 = w->t24_lo;  // the low plane takes the place of the PK2 codes
+        a.pk2_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_MAIN));
         a.t24_hi = w->t24_hi;
-        a.t24_hi_stride = static_cast<int64_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_T24_HI));
+        a.t24_hi_stride = static_cast<int32_t>(sbl_packed_row_bytes(desc, SBL_FMT_T24, SBL_BUF_T24_HI));
         a.xq = Xq;
         a.d = d;
         a.gamma = w->gamma;

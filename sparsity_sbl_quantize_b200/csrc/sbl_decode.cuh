@@ -48,7 +48,7 @@ constexpr int kDecChunk = 256;      // weights of one row in a warp's K chunk
 constexpr int kDecPartStride = 20;  // padded token row of the partial sums
 
 struct DecodeArgs {
-    const uint8_t *pk2;
+    const uint8_t *pk2;   // PK2 codes (T24 variant: the low plane of the group codes)
     int64_t pk2_stride;   // bytes per packed row
     const int8_t *xq;     // [T, K]
     const float *d;       // [T]
@@ -60,16 +60,17 @@ struct DecodeArgs {
     const uint16_t *residual;  // ... then v = v + residual[t, o] (bf16 [T, O]; nullptr: none)
     int32_t T, K, O;
     int32_t chunks;       // ceil(K / 256)
-    // T24 variant only: the 6-bit group codes' planes
-    const uint8_t *t24_lo;
-    int64_t t24_lo_stride;
-    const uint8_t *t24_hi;
-    int64_t t24_hi_stride;
     // fused variant only
-    const uint16_t *x;    // bf16 activations [T, K]
+    union {
+        const uint16_t *x;       // bf16 activations [T, K]
+        const uint8_t *t24_hi;   // T24 variant: the high plane (pk2 holds the low plane)
+    };
     int8_t *xq_out;       // Q_a(x) [T, K], stored by CTA 0 (nullptr: not stored)
     float *d_out;         // d_t [T], stored by CTA 0 (nullptr: not stored)
-    int32_t xs_stride;    // bytes per token row of the shared int8 copy (K + 16)
+    union {
+        int32_t xs_stride;      // bytes per token row of the shared int8 copy (K + 16)
+        int32_t t24_hi_stride;  // T24 variant: bytes per row of the high plane
+    };
 };
 
 // dynamic shared memory of the fused variant: the int8 activations [T][K + 16]
@@ -288,13 +289,15 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 // RG: groups of 16 rows per CTA, each worked by 8 warps that split the K
 // chunks of its rows (the groups read the same activations: L1 hits).
 // T24: the weights come as 6-bit group codes (two planes), expanded to PK2
-// words through a 4096-entry shared table built before the wait.
+// words through a 4096-entry table in dynamic shared memory (8 KiB) built
+// before the wait.
 template <int NT, int CPW, int RG, bool FUSE = false, bool T24 = false>
 __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
 {
     extern __shared__ __align__(16) uint8_t dec_xs[];
     __shared__ uint32_t s_amax[FUSE ? kDecMaxTokens : 1];
-    __shared__ uint16_t t24_lut[T24 ? 4096 : 1];
+    static_assert(!(T24 && FUSE), "T24 and the fused prologue share the dynamic shared memory");
+    uint16_t *t24_lut = reinterpret_cast<uint16_t *>(dec_xs);  // T24: 4096 entries of dynamic shared memory
     if constexpr (FUSE) {
         if (threadIdx.x < kDecMaxTokens) s_amax[threadIdx.x] = 0u;
         __syncthreads();
@@ -317,11 +320,6 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
     // 64-byte chunk (weights pos = 256 c + 64 tg .. pos + 63, bytes pos / 4 ..)
     const uint8_t *wA = args.pk2 + static_cast<int64_t>(okA ? row0 + g : 0) * args.pk2_stride;
     const uint8_t *wB = args.pk2 + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.pk2_stride;
-    // T24: the same rows of the two planes (8 + 4 bytes per lane and chunk)
-    const uint8_t *lA = T24 ? args.t24_lo + static_cast<int64_t>(okA ? row0 + g : 0) * args.t24_lo_stride : nullptr;
-    const uint8_t *lB = T24 ? args.t24_lo + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.t24_lo_stride : nullptr;
-    const uint8_t *hA = T24 ? args.t24_hi + static_cast<int64_t>(okA ? row0 + g : 0) * args.t24_hi_stride : nullptr;
-    const uint8_t *hB = T24 ? args.t24_hi + static_cast<int64_t>(okB ? row0 + g + 8 : 0) * args.t24_hi_stride : nullptr;
     // output (t, r) of the row group belongs to thread 16 t + r of the group
     // (the group of thread i is i / 256, the same as its warp's)
     const int t_out = (threadIdx.x & 255) >> 4, r_out = threadIdx.x & 15;
@@ -350,8 +348,12 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
             const int pos = c * kDecChunk + 64 * tg;
             const bool ok = c < args.chunks && pos < args.K;
             if constexpr (T24) {
-                wa[i] = (ok && okA) ? ld_stream_t24(lA + pos / 8, hA + pos / 16) : make_uint4(0u, 0u, 0u, 0u);
-                wb[i] = (ok && okB) ? ld_stream_t24(lB + pos / 8, hB + pos / 16) : make_uint4(0u, 0u, 0u, 0u);
+                // the same rows of the two planes (8 + 4 bytes per lane and chunk)
+                const int64_t ra = okA ? row0 + g : 0, rb = okB ? row0 + g + 8 : 0;
+                wa[i] = (ok && okA) ? ld_stream_t24(wA + pos / 8, args.t24_hi + ra * args.t24_hi_stride + pos / 16)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+                wb[i] = (ok && okB) ? ld_stream_t24(wB + pos / 8, args.t24_hi + rb * args.t24_hi_stride + pos / 16)
+                                    : make_uint4(0u, 0u, 0u, 0u);
             } else {
                 wa[i] = (ok && okA) ? ld_stream16(wA + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
                 wb[i] = (ok && okB) ? ld_stream16(wB + pos / 4) : make_uint4(0u, 0u, 0u, 0u);
@@ -418,20 +420,20 @@ __global__ void __launch_bounds__(256 * RG) decode_kernel(DecodeArgs args)
                         xt[b][q] = transpose4x4(v);
                     }
                 }
-                uint32_t pa[4], pb[4];  // the lane's PK2 words of rows g and g + 8
                 if constexpr (T24) {
-                    t24_decode(wa[i], t24_lut, pa);
-                    t24_decode(wb[i], t24_lut, pb);
-                } else {
-                    pa[0] = wa[i].x, pa[1] = wa[i].y, pa[2] = wa[i].z, pa[3] = wa[i].w;
-                    pb[0] = wb[i].x, pb[1] = wb[i].y, pb[2] = wb[i].z, pb[3] = wb[i].w;
+                    // the chunk's codes become its PK2 words, in place
+                    uint32_t t[4];
+                    t24_decode(wa[i], t24_lut, t);
+                    wa[i] = make_uint4(t[0], t[1], t[2], t[3]);
+                    t24_decode(wb[i], t24_lut, t);
+                    wb[i] = make_uint4(t[0], t[1], t[2], t[3]);
                 }
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     // step s takes word s/2 of the lane's 16 bytes and the
                     // code shifts ja (K slots 0..15) and ja + 1 (K slots 16..31)
                     const int wi = s >> 1, ja = 2 * (s & 1);
-                    const uint32_t ra = pa[wi], rb = pb[wi];
+                    const uint32_t ra = word_of(wa[i], wi), rb = word_of(wb[i], wi);
                     const uint32_t a0 = (ra >> (2 * ja)) & 0x03030303u;
                     const uint32_t a1 = (rb >> (2 * ja)) & 0x03030303u;
                     const uint32_t a2 = (ra >> (2 * ja + 2)) & 0x03030303u;
