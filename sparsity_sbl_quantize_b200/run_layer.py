@@ -1,6 +1,6 @@
 """Run one Sparse-BitLinear layer forward on the GPU and time it.
 
-    python -m sparsity_sbl_quantize_b200.run_layer O K T[,T2,...] [--nm 2:4] [--format sp24|i8|pk2]
+    python -m sparsity_sbl_quantize_b200.run_layer O K T[,T2,...] [--nm 2:4] [--format sp24|i8|pk2|t24]
                                                    [--iters 20] [--warmup 3]
 
 Packs a seeded synthetic layer (W ~ N(0, 0.02) fp32, X ~ N(0, 1) bf16, the
@@ -19,7 +19,7 @@ import torch
 from . import sbl
 from . import workloads as wl
 
-FORMATS = {"i8": sbl.SBL_FMT_I8, "pk2": sbl.SBL_FMT_PK2, "sp24": sbl.SBL_FMT_SP24}
+FORMATS = {"i8": sbl.SBL_FMT_I8, "pk2": sbl.SBL_FMT_PK2, "sp24": sbl.SBL_FMT_SP24, "t24": sbl.SBL_FMT_T24}
 
 
 def main() -> None:
