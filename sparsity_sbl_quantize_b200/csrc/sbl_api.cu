@@ -329,11 +329,10 @@ using namespace sbl;
 
 namespace {
 
-// Row groups (16 rows, 8 warps each) per decode CTA, for T <= 8 and T > 8.
-// One group measured fastest for both: two groups halve the activation
-// re-reads from L2 but lose more to fewer, larger CTAs.
-constexpr int kDecGroupsSmallT = 1;
-constexpr int kDecGroupsLargeT = 1;
+// Row groups (16 rows, 8 warps each) per decode CTA: the kernel supports
+// more than one, but one measured fastest for every T (two groups halve the
+// activation re-reads from L2 but lose more to fewer, larger CTAs).
+constexpr int kDecRowGroups = 1;
 
 // opt: the kPack* bits of the kernel to run.
 template <int M>
@@ -360,18 +359,15 @@ cudaError_t launch_pack(const cudaLaunchConfig_t &cfg, const PackArgs &pa, int o
     return cudaErrorInvalidValue;
 }
 
-// cpw: chunks per warp per round, 1, 2, 4 or 8 (at most 4 with two row
-// groups, whose 512 threads get at most 128 registers each).
-template <int NT, int RG>
+// cpw: chunks per warp per round, 1, 2, 4 or 8.
+template <int NT>
 cudaError_t launch_decode_nt(const cudaLaunchConfig_t &cfg, const DecodeArgs &a, int cpw)
 {
     switch (cpw) {
-    case 1: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 1, RG>, a);
-    case 2: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 2, RG>, a);
-    case 4: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, RG>, a);
-    default:
-        if constexpr (RG == 1) return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 8, RG>, a);
-        else return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, RG>, a);
+    case 1: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 1, kDecRowGroups>, a);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 2, kDecRowGroups>, a);
+    case 4: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 4, kDecRowGroups>, a);
+    default: return cudaLaunchKernelEx(&cfg, decode_kernel<NT, 8, kDecRowGroups>, a);
     }
 }
 
@@ -760,7 +756,7 @@ static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream, b
     // K = 16384 (more rounds above)
     const int need = (a.chunks + 7) / 8;
     const int cpw = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
-    const int rg = fuse ? 1 : a.T <= 8 ? kDecGroupsSmallT : kDecGroupsLargeT;
+    const int rg = kDecRowGroups;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>((a.O + kDecRows * rg - 1) / (kDecRows * rg)));
@@ -783,8 +779,7 @@ static sbl_status launch_decode(DecodeArgs &a, bool fuse, cudaStream_t stream, b
         cfg.dynamicSmemBytes = static_cast<size_t>(a.T) * a.xs_stride;
         e = a.T <= 8 ? launch_decode_fused<1>(cfg, a, cpw) : launch_decode_fused<2>(cfg, a, cpw);
     } else {
-        e = a.T <= 8 ? (rg == 1 ? launch_decode_nt<1, 1>(cfg, a, cpw) : launch_decode_nt<1, 2>(cfg, a, cpw))
-                     : (rg == 1 ? launch_decode_nt<2, 1>(cfg, a, cpw) : launch_decode_nt<2, 2>(cfg, a, cpw));
+        e = a.T <= 8 ? launch_decode_nt<1>(cfg, a, cpw) : launch_decode_nt<2>(cfg, a, cpw);
     }
     return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
 }
