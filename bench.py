@@ -150,6 +150,13 @@ def algorithmic_ops(wk, tokens):
     return total
 
 
+def decode_step_bytes(wk, tokens):
+    """Algorithmic bytes of one decode step at T tokens: per linear the 2-bit
+    weights, bf16 X read, int8 Xq and fp32 d written, bf16 Y written."""
+    return sum(lin.d_out * lin.d_in / 4 + 3.0 * tokens * lin.d_in + 8.0 * tokens + 2.0 * tokens * lin.d_out
+               for lin in wk.linears)
+
+
 # ------------------------------------------------------------------ ranks
 
 def max_over_ranks(value: float, dist, world: int, device) -> float:
@@ -770,32 +777,43 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
 
 def cpu_baseline(wk, budget_s=12.0):
     """Time the oracle, as it stands (single thread, plain C), on a bounded
-    sample of the workload: full weight packing and activation quantisation
-    of the first linear, and its GEMM + dequantisation on the first T_s tokens,
-    scaled so the sample takes about `budget_s` seconds."""
+    sample of the workload: the full weight packing of the first linear, and
+    its activation quantisation, GEMM and dequantisation (training: also the
+    fp64 Dual-STE backward, dX and dW) on the first T_s tokens of the step,
+    T_s chosen from a short probe so that the sample takes about `budget_s`
+    seconds.  The packing is charged pro rata, T_s / T of it, since one step
+    packs once for all T tokens."""
     import oracle
     lin = wk.linears[0]
     n, m = wk.patterns[0]
     T = wk.tokens[-1]
+    train = wk.mode == "train"
     w = wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed)
-    x = wl.activations(min(T, 256), lin.d_in, seed=wk.seed)
     t0 = time.perf_counter()
     layer = oracle.Layer(w, n, m)
     t_pack = time.perf_counter() - t0
-    ts = 8
-    t0 = time.perf_counter()
-    layer.forward(x[:ts])
-    t_probe = time.perf_counter() - t0
-    ts = int(max(1, min(x.shape[0], ts * max(1.0, (budget_s - t_pack) / max(t_probe, 1e-6)))))
-    t0 = time.perf_counter()
-    layer.forward(x[:ts])
-    t_fwd = time.perf_counter() - t0
-    ops = 2.0 * ts * lin.d_out * lin.d_in * n / m
-    value = ops / (t_fwd + t_pack * ts / T) / 1e12
+
+    def run(ts):
+        # the first ts rows of the step's inputs (row-major draws: a prefix
+        # of the full-size draw)
+        x = wl.activations(ts, lin.d_in, seed=wk.seed)
+        dy = wl.output_grad(ts, lin.d_out, seed=wk.seed) if train else None
+        t0 = time.perf_counter()
+        q, d, _, _, _ = layer.forward(x)
+        if train:
+            oracle.backward(dy, layer.weff, layer.gamma, q, d)
+        return time.perf_counter() - t0
+
+    probe = 4 if train else 8
+    t_probe = run(probe)
+    ts = int(max(1, min(T, probe * max(1.0, (budget_s - t_pack - t_probe) / max(t_probe, 1e-6)))))
+    t_run = run(ts)
+    per_token = 2.0 * lin.d_out * lin.d_in * n / m + (4.0 * lin.d_out * lin.d_in if train else 0.0)
+    value = per_token * ts / (t_run + t_pack * ts / T) / 1e12
+    what = "act quant + GEMM + dequant + fp64 Dual-STE backward (dX, dW)" if train else "act quant + GEMM + dequant"
     return {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
             "sample": f"{lin.name} {lin.d_in}->{lin.d_out} at {n}:{m}: full pack (charged pro rata "
-                      f"{ts}/{T} tokens) + act quant + GEMM + dequant on {ts} tokens; "
-                      f"pack {t_pack:.2f}s, forward {t_fwd:.2f}s"}
+                      f"{ts}/{T} tokens) + {what} on {ts} tokens; pack {t_pack:.2f}s, rest {t_run:.2f}s"}
 
 
 def cpu_baseline_decode(wk, budget_s=10.0):
@@ -836,10 +854,18 @@ def run_reference(args, wk):
             res.append(r)
     value = statistics.mean(r["value"] for r in res)
     unit = res[-1]["unit"]
+    # one whole step of the workload at the sample's rate
+    if wk.mode == "decode":
+        step_units = sum(decode_step_bytes(wk, T) for T in wk.tokens) / 1e9
+    else:
+        step_units = algorithmic_ops(wk, wk.tokens[-1]) / 1e12
+    dtype = "int8 x ternary -> int64 (plain C)" + ("; backward f64" if wk.mode == "train" else "")
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8 x ternary -> int64 (plain C)", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": round(step_units / value * 1e3, 1),
+        "ms_per_step_basis": "one whole step's algorithmic work at the sampled rate",
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
         "config": {"workload": wk.name}, "impl": "reference",
         "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": res[-1]["sample"]},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

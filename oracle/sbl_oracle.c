@@ -23,7 +23,8 @@
  *       Quantization: Per-Token Absmax to 8-Bit Integers", "Inference
  *       Implementation: GPU (Custom CUDA Kernels)" (2-bit packing).
  *
- * Readings where the pages are silent (each one also listed in the design doc):
+ * Readings where the pages are silent (R1-R24 name them everywhere in this
+ * repository):
  *  R1  sum of |W|: fp64, pairwise tree in flat row-major order, zero-padded
  *      to a power of two (split at the largest power of two below n).
  *  R2  gamma = (float)(S / (double)(d_out*d_in)); no epsilon; gamma == 0

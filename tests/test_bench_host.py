@@ -147,3 +147,40 @@ def test_algorithmic_ops_counts_kept_weights_and_the_backward():
     train = wl.WORKLOADS["qwen3b_train"]
     dense = sum(2.0 * 16384 * lin.d_out * lin.d_in for lin in train.linears)
     assert bench.algorithmic_ops(train, 16384) == pytest.approx(dense * (6 / 8 + 2))
+
+
+def test_reference_arm_line_on_the_host(capsys, monkeypatch):
+    """The oracle arm prints one line in our arm's metric and unit, with the
+    cpu_baseline and e2e objects; rank 0 alone prints under torchrun."""
+    import argparse
+    wk = wl.WORKLOADS["single_256x128"]
+    args = argparse.Namespace(steps=2, warmup=1, ref_step_seconds=0.2)
+    bench.run_reference(args, wk)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TOPS" and line["value"] > 0
+    assert line["metric"] == bench.METRIC and line["config"] == {"workload": "single_256x128"}
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["higher_is_better"] is True
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # one whole step's algorithmic work at the sampled rate
+    assert line["ms_per_step"] == pytest.approx(bench.algorithmic_ops(wk, wk.tokens[-1]) / 1e12 / line["value"] * 1e3,
+                                                rel=1e-3, abs=0.1)
+    monkeypatch.setenv("RANK", "1")
+    bench.run_reference(args, wk)
+    assert capsys.readouterr().out == ""
+
+
+def test_cpu_baseline_training_sample_includes_the_backward(monkeypatch):
+    """For the training workload the sample runs the fp64 Dual-STE backward
+    too, and its operation count includes 4 T O K for it."""
+    import oracle
+    calls = []
+    real = oracle.backward
+    monkeypatch.setattr(oracle, "backward", lambda *a, **k: calls.append(a[0].shape) or real(*a, **k))
+    small = wl.Workload(name="tiny_train", seed=5, tokens=[64], linears=[wl.Linear("up", d_in=64, d_out=32)],
+                        patterns=[(6, 8)], mode="train")
+    cb = bench.cpu_baseline(small, budget_s=0.2)
+    assert calls and calls[-1][1] == 32 and "backward" in cb["sample"]
+    ts = int(cb["sample"].split(" on ")[1].split(" tokens")[0])
+    assert 1 <= ts <= 64
