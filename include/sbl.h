@@ -144,8 +144,9 @@ size_t sbl_packed_row_bytes(const sbl_layer_desc *desc, sbl_format fmt, sbl_buff
  * by SBL_OP_QUANTIZE_MASK_PACK).  0 for an invalid descriptor. */
 size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op);
 
-/* Steps 2-4 of the forward ("compute mask from master weights", "ternary
- * quantization of master weights", "apply mask to quantized weights"):
+/* Steps 2-4 of the forward in "The Full Sparse-BitLinear Layer" (the
+ * mask from the master weights, their ternary quantization, the mask
+ * applied to the ternary weights):
  *   gamma = mean |W| over all O*K master weights (sum in fp64 over a
  *           pairwise tree in flat row-major order, then rounded to fp32);
  *   W_q   = clamp(round_half_even(fl32(W / gamma)), -1, 1)  (0 if gamma==0);
