@@ -332,7 +332,10 @@ def test_forward_sp24_bit_exact(O, K, T, n, m):
 
 @pytest.mark.parametrize("O,K,T", [(896, 4864, 4096),    # MLP down projection (128-token pair tiles)
                                    (4864, 896, 4096),    # MLP gate/up (224-token pair tiles)
-                                   (2048, 1024, 4000)])  # 224-token tiles with a ragged last tile
+                                   (2048, 1024, 4000),   # 224-token tiles with a ragged last tile
+                                   # the 1.5B decoder linears on which the format rule picks the
+                                   # sparse kernel at T = 8192 (down, gate/up, q/o)
+                                   (1536, 8960, 8192), (8960, 1536, 8192), (1536, 1536, 8192)])
 def test_forward_sp24_matches_dense_path_full_size(O, K, T):
     """The sparse and dense tensor-core paths compute the same integers: at
     full workload sizes their accumulators and outputs agree bit for bit, and
