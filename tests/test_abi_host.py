@@ -251,3 +251,36 @@ def test_forward_epilogue_validation(sbl):
     epi = sbl.sbl_epilogue(1, good + 2)  # misaligned residual
     assert _raw(sbl, "sbl_forward_ex", ctypes.byref(d), P(good), P(good), 64, ctypes.byref(w), sbl.SBL_FMT_I8,
                 P(good), 0, None, ctypes.byref(epi), None) == 3
+
+
+def test_binding_refuses_to_load_without_the_library(tmp_path):
+    """No CPU fallback: the binding, placed where no libsbl.so sits, raises on
+    import instead of offering any other implementation."""
+    import importlib.util
+    src = os.path.join(ROOT, "sparsity_sbl_quantize_b200", "sbl.py")
+    dst = tmp_path / "sbl.py"
+    dst.write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("sbl_without_library", dst)
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="libsbl.so is missing"):
+        spec.loader.exec_module(mod)
+
+
+def test_compute_calls_fail_loudly_without_a_device(sbl):
+    """On a host without a CUDA device the compute entry points raise (the
+    binding's stream lookup, or the library's device check); nothing runs
+    elsewhere and the outputs stay untouched."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    d = sbl.desc(32, 64, 6, 8)
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    q = torch.zeros((4, 64), dtype=torch.int8)
+    dv = torch.zeros((4,), dtype=torch.float32)
+    with pytest.raises((sbl.SblError, RuntimeError)):
+        sbl.sbl_quantize_act(x, 4, 64, q, dv)
+    p = sbl.Packed(gamma=torch.zeros(4, dtype=torch.float32), i8=torch.zeros((32, 64), dtype=torch.int8))
+    y = torch.zeros((4, 32), dtype=torch.bfloat16)
+    with pytest.raises((sbl.SblError, RuntimeError)):
+        sbl.sbl_forward(d, q, dv, 4, p, sbl.SBL_FMT_I8, y)
+    assert torch.count_nonzero(y) == 0 and torch.count_nonzero(q) == 0
