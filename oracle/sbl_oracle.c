@@ -452,7 +452,7 @@ static uint16_t f32_to_bf16(float f)
 }
 
 /* [P1] forward step 5: one scalar absorbs the weight scale gamma and the
- * token scale max|x|/127; reading R6. */
+ * token scale max|x|/127; reading R7. */
 void sbl_oracle_dequant(const int32_t *acc, int64_t tokens, int64_t d_out,
                         float gamma, const float *d, float *y, uint16_t *y_bf16)
 {

@@ -59,6 +59,19 @@ MUTANTS = {
                              "{{-1, 0, 1, 3}, {-1, -1, 2, 4}, {-1, -1, -1, 5}"),
     "t24_single_offset": ("code = 1u + 2u * (unsigned)pos[0] + (w[pos[0]] < 0 ? 1u : 0u);",
                           "code = 2u * (unsigned)pos[0] + (w[pos[0]] < 0 ? 1u : 0u);"),
+    "ternarize_clip_dropped": ("if (q > 1.0f) q = 1.0f;\n        if (q < -1.0f) q = -1.0f;\n        wq[i] = (int8_t)q;",
+                               "wq[i] = (int8_t)q;"),
+    "pk2_codes_msb_first": ("int sh = (int)(2 * (k % 4));", "int sh = (int)(2 * (3 - k % 4));"),
+    "pk2_padding_zero": ("for (int64_t b = 0; b < rb; ++b) row[b] = 0x55;", "for (int64_t b = 0; b < rb; ++b) row[b] = 0;"),
+    "nm_bitmap_msb_first": ("brow[k / 8] = (uint8_t)(brow[k / 8] | (1u << (k % 8)));",
+                            "brow[k / 8] = (uint8_t)(brow[k / 8] | (1u << (7 - k % 8)));"),
+    "nm_values_msb_first": ("int sh = (int)(2 * (slot % 4));", "int sh = (int)(2 * (3 - slot % 4));"),
+    "gemm_weights_transposed": ("s += (int64_t)q[t * d_in + k] * (int64_t)weff[o * d_in + k];",
+                                "s += (int64_t)q[t * d_in + k] * (int64_t)weff[k * d_out + o];"),
+    "acc_samples_token_for_row": ("acc += (int64_t)q[t * d_in + k] * (int64_t)weff[o * d_in + k];",
+                                  "acc += (int64_t)q[o * d_in + k] * (int64_t)weff[t * d_in + k];"),
+    "dx_samples_gamma_dropped": ("out[s] = (double)gamma * acc;", "out[s] = acc;"),
+    "bf16_truncates": ("u += 0x7fffu + lsb;", "u += 0u * lsb;"),
     "t24_high_plane_stride": ("hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 4))));",
                               "hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 2))));"),
 }
@@ -90,6 +103,10 @@ PIN_CALLS = [
     (pins.test_mask_flips_matches_numpy_and_invariants, ()),
     (pins.test_near_zero_matches_numpy_and_gaussian_closed_form, ()),
     (pins.test_block_threshold_brute_force_and_hand_row, ()),
+    (pins.test_gemm_acc_matches_numpy_int64, ()),
+    (pins.test_gemm_acc_brute_force_tiny, ()),
+    (pins.test_sampled_variants_agree_with_full, ()),
+    (pins.test_epilogue_matches_numpy_float32_and_torch_bf16, ()),
 ]
 
 
