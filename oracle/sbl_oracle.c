@@ -23,8 +23,8 @@
  *       Quantization: Per-Token Absmax to 8-Bit Integers", "Inference
  *       Implementation: GPU (Custom CUDA Kernels)" (2-bit packing).
  *
- * Readings where the pages are silent (R1-R24 name them everywhere in this
- * repository):
+ * Readings where the pages are silent, garbled or at odds (the same
+ * R-numbers are used throughout this repository):
  *  R1  sum of |W|: fp64, pairwise tree in flat row-major order, zero-padded
  *      to a power of two (split at the largest power of two below n).
  *  R2  gamma = (float)(S / (double)(d_out*d_in)); no epsilon; gamma == 0
@@ -32,13 +32,19 @@
  *  R3  W_q = clamp(rint_half_even(fl32(W / gamma)), -1, 1).
  *  R4  mask: keep rank < n where rank counts strictly larger |W| plus equal
  *      |W| at a lower index (lower index wins ties; -0 ties +0).
- *  R5  activation: a = max|x|; a == 0 -> q = 0, d = 0; otherwise
+ *  R5  the mask ranks the master weights and is applied after ternarisation;
+ *      gamma is taken over all weights, masked ones included.
+ *  R6  activation: a = max|x|; a == 0 -> q = 0, d = 0; otherwise
  *      r = fl32(127 / a), q = clamp(rint_half_even(fl32(x * r)), -128, 127),
  *      d = fl32(a / 127).
- *  R6  output: c_t = fl32(gamma * d_t), y = fl32(fl32(acc) * c_t), bf16 by
+ *  R7  output: c_t = fl32(gamma * d_t), y = fl32(fl32(acc) * c_t), bf16 by
  *      round-to-nearest-even.
- *  R7  Dual-STE backward: identity through mask and quantiser;
- *      dX = gamma * dY * W_eff, dW = dY^T * Xtilde with Xtilde = d_t * q.
+ *  R8  Dual-STE backward: identity through mask and quantiser, no clip
+ *      window: dX = gamma * dY * W_eff.
+ *  R9  dW = dY^T * Xtilde with Xtilde = d_t * q (the forward's operand).
+ * The later readings (R10-R24) cover the packed formats, the statistics,
+ * the ablation arms, the epilogue and the norm; each function below names
+ * the one it follows.
  */
 #include <fenv.h>
 #include <math.h>
@@ -95,8 +101,8 @@ void sbl_oracle_ternarize(const float *w, int64_t count, float gamma, int8_t *wq
 /* ----------------------------------------------------------------- mask -- */
 
 /* [P1] "N:M Mask Generation": per contiguous group of m weights along the
- * input dimension keep the n with the largest |W| of the master weights.
- * Reading R4 for ties. */
+ * input dimension keep the n with the largest |W| of the master weights
+ * (reading R5).  Reading R4 for ties. */
 void sbl_oracle_nm_mask(const float *w, int64_t d_out, int64_t d_in,
                         int n, int m, uint8_t *mask)
 {
@@ -116,7 +122,8 @@ void sbl_oracle_nm_mask(const float *w, int64_t d_out, int64_t d_in,
     }
 }
 
-/* [P1] "Composition Order": W_eff = W_q (elementwise) M. */
+/* [P1] "Composition Order": W_eff = W_q (elementwise) M, the mask applied
+ * after ternarisation (reading R5). */
 void sbl_oracle_apply_mask(const int8_t *wq, const uint8_t *mask, int64_t count,
                            int8_t *weff)
 {
@@ -139,8 +146,9 @@ static double abs_sum_tree_masked(const float *w, const uint8_t *mask, int64_t l
     return left + right;
 }
 
-/* Mask-then-quant ([P1] "Composition Order": W_eff = Q_t(W * M), gamma from
- * only the Top-N active weights): gamma = mean |W| over the kept positions,
+/* Mask-then-quant ([P1] "Composition Order": W_eff = Q_t(W * M), the scale
+ * taken over the surviving weights alone; reading R18): gamma = mean |W|
+ * over the kept positions,
  * the sum over the same tree as gamma (zeros at dropped positions) divided
  * by the number of kept positions. */
 float sbl_oracle_gamma_survivors(const float *w, const uint8_t *mask, int64_t d_out, int64_t d_in)
@@ -153,8 +161,8 @@ float sbl_oracle_gamma_survivors(const float *w, const uint8_t *mask, int64_t d_
 }
 
 /* Mask from the quantized weights ([P1] "Composition Order", "Where the mask
- * is computed"): the same top-n rule ranking |W_q| in {0, 1} instead of |W|;
- * ties (nearly all) go to the lower index. */
+ * is computed"; reading R19): the same top-n rule ranking |W_q| in {0, 1}
+ * instead of |W|; ties (nearly all) go to the lower index. */
 void sbl_oracle_nm_mask_quantized(const int8_t *wq, int64_t d_out, int64_t d_in, int n, int m, uint8_t *mask)
 {
     for (int64_t o = 0; o < d_out; ++o)
@@ -182,8 +190,8 @@ static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 int64_t sbl_oracle_pk2_row_bytes(int64_t d_in) { return round_up(d_in / 4, 16); }
 
-/* PK2: weight k of a row at bits 2*(k%4) of byte k/4; padding bytes hold
- * code 1 in every slot (0x55, i.e. zero weights). */
+/* PK2 (reading R12): weight k of a row at bits 2*(k%4) of byte k/4; padding
+ * bytes hold code 1 in every slot (0x55, i.e. zero weights). */
 void sbl_oracle_pack_pk2(const int8_t *weff, int64_t d_out, int64_t d_in, uint8_t *out)
 {
     int64_t rb = sbl_oracle_pk2_row_bytes(d_in);
@@ -235,8 +243,9 @@ int64_t sbl_oracle_sp24_value_row_bytes(int64_t d_in) { return round_up(d_in / 2
 
 int64_t sbl_oracle_sp24_meta_row_bytes(int64_t d_in) { return round_up(d_in / 8, 16); }
 
-/* SP24: W_eff as the 2:4-compressed operand of the sparse tensor-core MMA
- * (two stored values per group of four positions plus their 2-bit indices).
+/* SP24 (reading R14): W_eff as the 2:4-compressed operand of the sparse
+ * tensor-core MMA (two stored values per group of four positions plus their
+ * 2-bit indices).
  * For group g of a row (positions 4g .. 4g+3) the two positions i0 < i1 are
  * the group's kept positions, completed, when fewer than two are kept, with
  * the smallest positions of the group that are not kept.  Values: int8
@@ -332,9 +341,9 @@ int sbl_oracle_pack_t24(const int8_t *weff, int64_t d_out, int64_t d_in, uint8_t
 /* ------------------------------------------------------ mask statistics -- */
 
 /* Mask flip count between consecutive steps ([P1] "Dynamic Mask
- * Recomputation at Every Training Step": the flip rate r_t measures how
- * many mask positions change from one step to the next; r_t = flips / count
- * is the rate).  Masks are one byte per position (0 or 1). */
+ * Recomputation at Every Training Step", flip rate r_t; reading R15): the
+ * number of positions whose keep bit differs between the two masks, so that
+ * r_t = flips / count.  Masks are one byte per position (0 or 1). */
 int64_t sbl_oracle_mask_flips(const uint8_t *mask_prev, const uint8_t *mask, int64_t count)
 {
     int64_t flips = 0;
@@ -343,8 +352,8 @@ int64_t sbl_oracle_mask_flips(const uint8_t *mask_prev, const uint8_t *mask, int
     return flips;
 }
 
-/* Near-zero mass ([P1] "Polarization analysis": the fraction of weights
- * whose normalized magnitude |W| / gamma falls below 0.5), as a count:
+/* Near-zero mass ([P1] "Polarization analysis": the share of weights with
+ * |W| / gamma under 0.5; reading R16), as a count:
  * #{ fl32(|w| / gamma) < 0.5 }; every weight counts when gamma == 0 (all
  * weights are then 0 and quantise to 0). */
 int64_t sbl_oracle_near_zero(const float *w, int64_t count, float gamma)
@@ -358,8 +367,8 @@ int64_t sbl_oracle_near_zero(const float *w, int64_t count, float gamma)
     return c;
 }
 
-/* Per-block pruning threshold ([P1] "Magnitude stratification": the
- * magnitude of the (N+1)-th largest weight in each block of M): for row o
+/* Per-block pruning threshold ([P1] "Magnitude stratification", threshold
+ * t; reading R17): for row o
  * and group g, the largest |W| among the group's positions the mask drops,
  * which is the (n+1)-th largest |W| of the group; 0 when n == m (nothing is
  * dropped).  Output fp32 [d_out, d_in / m]. */
@@ -391,7 +400,7 @@ static float bf16_to_f32(uint16_t b)
 
 /* [P1] 3.4 activation quantisation equation; [P5] "Activation Quantization:
  * Per-Token Absmax": one scale per token, 127 / max|x|, rounding to the
- * nearest integer; reading R5. */
+ * nearest integer; reading R6. */
 void sbl_oracle_quantize_act(const uint16_t *x, int64_t tokens, int64_t d_in,
                              int8_t *q, float *d)
 {
@@ -489,7 +498,7 @@ static double square_sum_tree(const uint16_t *x, int64_t lo, int64_t n)
  *   u_k = fl32(fl32(x_k * r) * g_k)   (g: bf16 gains, 1 when absent);
  * then the quantiser of sbl_oracle_quantize_act on the fp32 u (a = max|u|,
  * q = clamp(rint(fl32(u * fl32(127 / a)))), d = fl32(a / 127); a == 0 gives
- * q = 0, d = 0). */
+ * q = 0, d = 0).  Reading R23. */
 void sbl_oracle_rmsnorm_quantize_act(const uint16_t *x, int64_t tokens, int64_t d_in, const uint16_t *g,
                                      float eps, int8_t *q, float *d)
 {
@@ -527,7 +536,7 @@ void sbl_oracle_rmsnorm_quantize_act(const uint16_t *x, int64_t tokens, int64_t 
  *   v = y                      (the fp32 output of sbl_oracle_dequant)
  *   v = v > 0 ? fl32(v * v) : 0   when relu2
  *   v = fl32(v + r)            when a residual r (bf16 [T, O]) is given
- * written as fp32 and as bf16 (round to nearest even). */
+ * written as fp32 and as bf16 (round to nearest even).  Reading R22. */
 void sbl_oracle_epilogue(const float *y, int64_t tokens, int64_t d_out, int relu2, const uint16_t *res,
                          float *out, uint16_t *out_bf16)
 {
@@ -544,7 +553,7 @@ void sbl_oracle_epilogue(const float *y, int64_t tokens, int64_t d_out, int relu
 
 /* [P1] "The Dual Straight-Through Estimator" (dL/dW ~= dL/dW_eff) and the
  * backward walk-through (gradient flows through mask and quantiser as
- * identity); reading R7, evaluated in fp64.
+ * identity); readings R8 and R9, evaluated in fp64.
  *   dX[t,k] = gamma * sum_o dY[t,o] * W_eff[o,k]
  *   dW[o,k] = sum_t dY[t,o] * d_t * q[t,k]     (unmasked) */
 void sbl_oracle_backward(const uint16_t *dy, const int8_t *weff, float gamma,
