@@ -284,3 +284,20 @@ def test_compute_calls_fail_loudly_without_a_device(sbl):
     with pytest.raises((sbl.SblError, RuntimeError)):
         sbl.sbl_forward(d, q, dv, 4, p, sbl.SBL_FMT_I8, y)
     assert torch.count_nonzero(y) == 0 and torch.count_nonzero(q) == 0
+
+
+def test_c99_program_against_the_library(sbl, tmp_path):
+    """The header compiles as strict C99 (no CUDA header, no C++), every
+    declared function links against libsbl.so, and a plain C program sees
+    the documented sizes, format rule and argument checks."""
+    import subprocess
+    import torch
+    lib_dir = os.path.dirname(sbl.LIB_PATH)
+    exe = tmp_path / "abi_host_check"
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "abi_host_check.c"),
+                    "-L", lib_dir, "-lsbl", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    if not torch.cuda.is_available():
+        assert "(no device)" in r.stdout
