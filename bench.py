@@ -292,7 +292,7 @@ class Runner:
                 # re-mask statistics of every training step: this step's keep
                 # bitmap against the previous step's, near-zero count, thresholds
                 rb = sbl.keep_bitmap_bytes(dsc0)
-                n0, m0 = wk.patterns[0]
+                _, m0 = wk.patterns[0]
                 L["stats"] = {"prev": torch.zeros((lin.d_out, rb), dtype=torch.uint8, device=device),
                               "keep": torch.zeros((lin.d_out, rb), dtype=torch.uint8, device=device),
                               "flips": torch.zeros((1,), dtype=torch.int64, device=device),
@@ -330,7 +330,7 @@ class Runner:
             st = L["stats"]
             lin = L["lin"]
             count = lin.d_out * lin.d_in
-            dsc, p = L["packed"][self.wk.patterns[0]]
+            _, p = L["packed"][self.wk.patterns[0]]
             g = float(p.gamma[0].item())
             out[lin.name] = {"flip_rate": int(st["flips"].item()) / count,
                              "near_zero_fraction": int(st["near_zero"].item()) / count,

@@ -11,7 +11,6 @@ Parity pins for every function are in ``tests/test_oracle_pins.py``.
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 
