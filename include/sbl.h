@@ -377,6 +377,77 @@ sbl_status sbl_backward_dual_ste_ex(const sbl_layer_desc *desc, const uint16_t *
  * Synchronises the device.  `clear` != 0 resets it to 0 afterwards. */
 sbl_status sbl_device_error(uint32_t *code, int32_t clear);
 
+/* ------------------------------------------------ packed-layer container --
+ * A self-describing byte image of a packed layer, so that packed weights
+ * (for decode: PK2 or T24 and gamma) can be stored and reloaded without
+ * the master weights.  Host code only: these calls never touch a device.
+ * The caller copies the device buffers to host memory before
+ * sbl_container_write, and back to the device after sbl_container_read.
+ *
+ * Layout (integers little-endian):
+ *   bytes  0-3   magic "SBLP"
+ *          4-7   container version (SBL_CONTAINER_VERSION)
+ *          8-23  out_features, in_features, n, m (int32 each)
+ *         24-27  format mask (SBL_FMT_* bits)
+ *         28-31  gamma (fp32 bits)
+ *         32-39  payload bytes (everything after the 64-byte header)
+ *         40-47  64-bit FNV-1a hash of the payload
+ *         48-51  sbl_version() of the writer
+ *         52-63  zero
+ *   payload: for each format present, in the order PK2, NM values, NM
+ *   bitmap, I8, BF16T, SP24 values, SP24 metadata, T24 low plane, T24 high
+ *   plane, the buffer exactly as sbl_quantize_mask_pack writes it (rows x
+ *   sbl_packed_row_bytes; K rows for BF16T), each starting at a multiple of
+ *   64 bytes from the start of the image (zero bytes between; with rows a
+ *   multiple of 16 and row bytes a multiple of 16, every buffer is a
+ *   multiple of 256 bytes, so in practice none are needed).
+ * The hash covers every payload byte, so any change to a stored buffer or
+ * to its fill is detected on reading. */
+#define SBL_CONTAINER_VERSION 1
+#define SBL_CONTAINER_HEADER_BYTES 64
+
+/* Host buffers of a packed layer, one per stored buffer (the layouts of
+ * sbl_packed).  Only the members of the formats in use must be non-null;
+ * they need no alignment. */
+typedef struct {
+    void *pk2;
+    void *nm_values;
+    void *nm_bitmap;
+    void *i8;
+    void *bf16t;
+    void *sp24_values;
+    void *sp24_meta;
+    void *t24_lo;
+    void *t24_hi;
+} sbl_host_buffers;
+
+/* Size of the image for a descriptor and format mask; 0 when the
+ * descriptor or the mask is invalid (unknown bits; SBL_FMT_SP24 or
+ * SBL_FMT_T24 with n > 2). */
+size_t sbl_container_bytes(const sbl_layer_desc *desc, uint32_t formats);
+
+/* Write the image of (desc, formats, gamma, src) into dst[0 .. dst_bytes).
+ * SBL_ERR_INVALID_ARG: null desc/src/dst, a null buffer of a present format,
+ * unknown format bits or a non-finite gamma; SBL_ERR_SHAPE: invalid
+ * descriptor, or dst_bytes below sbl_container_bytes; SBL_ERR_UNSUPPORTED:
+ * SP24 or T24 with n > 2. */
+sbl_status sbl_container_write(const sbl_layer_desc *desc, uint32_t formats, float gamma,
+                               const sbl_host_buffers *src, void *dst, size_t dst_bytes);
+
+/* Check an image and report what it holds.  Any of desc, formats, gamma
+ * may be NULL.  SBL_ERR_INVALID_ARG: null src, shorter than its header or
+ * its payload, wrong magic, a payload size that does not match the
+ * descriptor and formats, or a hash mismatch; SBL_ERR_UNSUPPORTED: a
+ * container version this library does not read; SBL_ERR_SHAPE: an invalid
+ * descriptor. */
+sbl_status sbl_container_info(const void *src, size_t src_bytes, sbl_layer_desc *desc, uint32_t *formats,
+                              float *gamma);
+
+/* Check an image as sbl_container_info does, then copy every stored buffer
+ * into dst (each member of a stored format must be non-null and hold the
+ * buffer's rows x row bytes).  Nothing is written unless the image checks. */
+sbl_status sbl_container_read(const void *src, size_t src_bytes, const sbl_host_buffers *dst);
+
 #ifdef __cplusplus
 }
 #endif

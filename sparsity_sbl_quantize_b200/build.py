@@ -2,9 +2,10 @@
 
     python -m sparsity_sbl_quantize_b200.build [--force] [--verbose]
 
-nvcc cross-compiles for sm_100a without a GPU.  The library is one
-translation unit (csrc/sbl_api.cu includes the kernel headers) linked against
-the static CUDA runtime; the driver entry point for tensor-map encoding is
+nvcc cross-compiles for sm_100a without a GPU.  The library is two
+translation units -- csrc/sbl_api.cu (the ABI; it includes the kernel
+headers) and csrc/sbl_container.cpp (the host-only packed-layer container)
+-- linked against the static CUDA runtime; the driver entry point for tensor-map encoding is
 looked up at run time, so libcuda is not a link dependency.
 """
 from __future__ import annotations
@@ -36,7 +37,7 @@ def _nvcc() -> str:
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  [os.path.join(INCLUDE, "sbl.h")])
+                  glob.glob(os.path.join(CSRC, "*.cpp")) + [os.path.join(INCLUDE, "sbl.h")])
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
@@ -45,7 +46,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
-           os.path.join(CSRC, "sbl_api.cu")]
+           os.path.join(CSRC, "sbl_api.cu"), os.path.join(CSRC, "sbl_container.cpp")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))

@@ -64,6 +64,11 @@ class sbl_mask_stats(ctypes.Structure):
                 ("near_zero", ctypes.c_void_p), ("block_threshold", ctypes.c_void_p)]
 
 
+class sbl_host_buffers(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("pk2", "nm_values", "nm_bitmap", "i8", "bf16t", "sp24_values", "sp24_meta", "t24_lo", "t24_hi")]
+
+
 _P = ctypes.c_void_p
 _D = ctypes.POINTER(sbl_layer_desc)
 _W = ctypes.POINTER(sbl_packed)
@@ -104,11 +109,20 @@ _lib.sbl_forward_format.restype = ctypes.c_int
 _lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
+_lib.sbl_container_bytes.restype = _sz
+_lib.sbl_container_bytes.argtypes = [_D, _u32]
+_lib.sbl_container_write.restype = ctypes.c_int
+_lib.sbl_container_write.argtypes = [_D, _u32, ctypes.c_float, ctypes.POINTER(sbl_host_buffers), _P, _sz]
+_lib.sbl_container_info.restype = ctypes.c_int
+_lib.sbl_container_info.argtypes = [_P, _sz, _D, ctypes.POINTER(_u32), ctypes.POINTER(ctypes.c_float)]
+_lib.sbl_container_read.restype = ctypes.c_int
+_lib.sbl_container_read.argtypes = [_P, _sz, ctypes.POINTER(sbl_host_buffers)]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward", "sbl_linear_forward",
             "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
-            "sbl_quantize_mask_pack_ex", "sbl_device_error"]
+            "sbl_quantize_mask_pack_ex", "sbl_device_error", "sbl_container_bytes", "sbl_container_write",
+            "sbl_container_info", "sbl_container_read"]
 
 
 class SblError(RuntimeError):
@@ -329,3 +343,77 @@ def alloc_packed(d: sbl_layer_desc, formats: int, device="cuda") -> Packed:
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """Workspace as a 256-byte aligned torch buffer (torch's allocator aligns to 512)."""
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------- packed-layer container (host)
+
+_BUFFERS = ("pk2", "nm_values", "nm_bitmap", "i8", "bf16t", "sp24_values", "sp24_meta", "t24_lo", "t24_hi")
+
+
+def _host_buffers(p: Packed) -> sbl_host_buffers:
+    """sbl_host_buffers over the host (CPU, contiguous) tensors of p."""
+    ptrs = []
+    for name in _BUFFERS:
+        t = getattr(p, name)
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name}: the container works on contiguous host tensors")
+        ptrs.append(t.data_ptr() if t is not None else None)
+    return sbl_host_buffers(*ptrs)
+
+
+def sbl_container_bytes(d: sbl_layer_desc, formats: int) -> int:
+    return int(_lib.sbl_container_bytes(ctypes.byref(d), formats))
+
+
+def sbl_container_write(d: sbl_layer_desc, formats: int, gamma: float, src: Packed) -> bytes:
+    """The container image of a packed layer whose buffers are host tensors."""
+    n = sbl_container_bytes(d, formats)  # 0 for an invalid descriptor or mask: the call reports which
+    buf = ctypes.create_string_buffer(max(n, 1))
+    hb = _host_buffers(src)
+    _check(_lib.sbl_container_write(ctypes.byref(d), formats, float(gamma), ctypes.byref(hb), buf, n),
+           "sbl_container_write")
+    return buf.raw
+
+
+def sbl_container_info(image: bytes):
+    """(desc, formats, gamma) of a checked container image."""
+    d = sbl_layer_desc()
+    f = _u32(0)
+    g = ctypes.c_float(0.0)
+    _check(_lib.sbl_container_info(image, len(image), ctypes.byref(d), ctypes.byref(f), ctypes.byref(g)),
+           "sbl_container_info")
+    return d, int(f.value), float(g.value)
+
+
+def sbl_container_read(image: bytes, dst: Packed) -> None:
+    """Copy the stored buffers of a checked image into dst's host tensors."""
+    hb = _host_buffers(dst)
+    _check(_lib.sbl_container_read(image, len(image), ctypes.byref(hb)), "sbl_container_read")
+
+
+def save_packed(path: str, d: sbl_layer_desc, formats: int, p: Packed) -> None:
+    """Store a packed layer (device or host tensors) with its descriptor and
+    gamma; the device buffers are copied to host memory first."""
+    host = Packed(gamma=p.gamma.detach().cpu(),
+                  **{name: (getattr(p, name).detach().cpu().contiguous() if getattr(p, name) is not None else None)
+                     for name in _BUFFERS})
+    image = sbl_container_write(d, formats, float(host.gamma.reshape(-1)[0]), host)
+    with open(path, "wb") as f:
+        f.write(image)
+
+
+def load_packed(path: str, device="cuda"):
+    """Read a stored packed layer: (desc, formats, Packed on `device`)."""
+    with open(path, "rb") as f:
+        image = f.read()
+    d, formats, gamma = sbl_container_info(image)
+    host = alloc_packed(d, formats, device="cpu")
+    sbl_container_read(image, host)
+    host.gamma.zero_()
+    host.gamma[0] = gamma
+    if device == "cpu":
+        return d, formats, host
+    dev = Packed(gamma=host.gamma.to(device),
+                 **{name: (getattr(host, name).to(device) if getattr(host, name) is not None else None)
+                    for name in _BUFFERS})
+    return d, formats, dev

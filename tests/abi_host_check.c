@@ -118,6 +118,36 @@ int main(void)
           SBL_ERR_WORKSPACE);
     CHECK(sbl_device_error(NULL, 0) == SBL_ERR_INVALID_ARG);
 
+    /* the packed-layer container, host memory only */
+    {
+        static uint8_t pk2[16 * 16], i8[16 * 64], image[4096], back_pk2[16 * 16], back_i8[16 * 64];
+        const sbl_layer_desc dc = {16, 64, 2, 4};
+        for (size_t i = 0; i < sizeof(pk2); ++i) pk2[i] = (uint8_t)(i * 7 + 1);
+        for (size_t i = 0; i < sizeof(i8); ++i) i8[i] = (uint8_t)(i % 3);
+        sbl_host_buffers src, dst;
+        memset(&src, 0, sizeof(src));
+        memset(&dst, 0, sizeof(dst));
+        src.pk2 = pk2;
+        src.i8 = i8;
+        dst.pk2 = back_pk2;
+        dst.i8 = back_i8;
+        const uint32_t fm = SBL_FMT_PK2 | SBL_FMT_I8;
+        const size_t nb = sbl_container_bytes(&dc, fm);
+        CHECK(nb == SBL_CONTAINER_HEADER_BYTES + sizeof(pk2) + sizeof(i8));
+        CHECK(sbl_container_write(&dc, fm, 0.25f, &src, image, nb - 1) == SBL_ERR_SHAPE);
+        CHECK(sbl_container_write(&dc, fm, 0.25f, &src, image, sizeof(image)) == SBL_OK);
+        sbl_layer_desc di;
+        uint32_t fi = 0;
+        float gi = 0.0f;
+        CHECK(sbl_container_info(image, nb, &di, &fi, &gi) == SBL_OK);
+        CHECK(di.out_features == 16 && di.in_features == 64 && di.n == 2 && di.m == 4 && fi == fm && gi == 0.25f);
+        CHECK(sbl_container_read(image, nb, &dst) == SBL_OK);
+        CHECK(memcmp(back_pk2, pk2, sizeof(pk2)) == 0 && memcmp(back_i8, i8, sizeof(i8)) == 0);
+        image[nb - 1] ^= 1u;
+        CHECK(sbl_container_info(image, nb, NULL, NULL, NULL) == SBL_ERR_INVALID_ARG);
+        CHECK(sbl_container_info(image, 10, NULL, NULL, NULL) == SBL_ERR_INVALID_ARG);
+    }
+
     if (no_device) {
         /* valid calls: the only thing left is the device, which is absent */
         CHECK(sbl_quantize_act(A, 4, 256, B, B, NULL) == SBL_ERR_DEVICE);
