@@ -20,6 +20,7 @@ bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -223,7 +224,6 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
@@ -480,7 +480,7 @@ def run_ours(args, wk):
     if world > 1:
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", init_method="env://",
-                                timeout=__import__("datetime").timedelta(seconds=120))
+                                timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)
     from sparsity_sbl_quantize_b200 import sbl
     pk = peaks()
