@@ -377,6 +377,18 @@ sbl_status sbl_backward_dual_ste_ex(const sbl_layer_desc *desc, const uint16_t *
  * Synchronises the device.  `clear` != 0 resets it to 0 afterwards. */
 sbl_status sbl_device_error(uint32_t *code, int32_t clear);
 
+/* Bit of the device error word set only by sbl_selftest_wait_expiry. */
+#define SBL_DEVICE_ERROR_SELFTEST 0x80000000u
+
+/* Self-test of failure detection: one launch of one CTA whose single thread
+ * waits on a shared-memory mbarrier that nothing arrives at, through the
+ * bounded wait every kernel of the library uses.  After the wait limit
+ * (1 s) the wait gives up, sets SBL_DEVICE_ERROR_SELFTEST in the device
+ * error word and the kernel returns, leaving the context usable.  Enqueued
+ * on `stream`; read the result with sbl_device_error.  SBL_ERR_DEVICE
+ * without an sm_100 device. */
+sbl_status sbl_selftest_wait_expiry(void *stream);
+
 /* ------------------------------------------------ packed-layer container --
  * A self-describing byte image of a packed layer, so that packed weights
  * (for decode: PK2 or T24 and gamma) can be stored and reloaded without

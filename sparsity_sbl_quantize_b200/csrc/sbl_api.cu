@@ -1042,6 +1042,23 @@ static_assert(SBL_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SBL_NOALLOC_SCRATCH_BYTES];
 static std::mutex g_noalloc_mutex;
 static void *g_noalloc_ptr[kMaxDevices];
+
+// Self-test of the bounded waits: one thread waits, through the same
+// mbar_wait every kernel uses, on a fresh mbarrier that nothing arrives at.
+// After kWaitLimitNs the wait records SBL_DEVICE_ERROR_SELFTEST and the
+// kernel returns.  No copy, MMA or tensor memory is outstanding when it does.
+static_assert((SBL_DEVICE_ERROR_SELFTEST & (kErrGemmProducer | kErrGemmMma | kErrGemmEpilogue | kErrDecode |
+                                            kErrPack)) == 0,
+              "the self-test bit is distinct from every kernel family's bit");
+__global__ void __launch_bounds__(32) wait_expiry_kernel(uint32_t *err)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_addr(&bar);
+    mbar_init(b, 1);
+    fence_barrier_init();
+    mbar_wait(b, 0, err, SBL_DEVICE_ERROR_SELFTEST);
+}
 }  // namespace sbl
 
 extern "C" {
@@ -1067,6 +1084,15 @@ sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const floa
         scratch = g_noalloc_ptr[dev];
     }
     return sbl_quantize_mask_pack(desc, W, formats, out, scratch, SBL_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+sbl_status sbl_selftest_wait_expiry(void *stream)
+{
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    wait_expiry_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(di->err);
+    return launch_status();
 }
 
 sbl_status sbl_device_error(uint32_t *code, int32_t clear)

@@ -109,6 +109,8 @@ _lib.sbl_forward_format.restype = ctypes.c_int
 _lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
 _lib.sbl_device_error.argtypes = [ctypes.POINTER(_u32), _i32]
+_lib.sbl_selftest_wait_expiry.restype = ctypes.c_int
+_lib.sbl_selftest_wait_expiry.argtypes = [_P]
 _lib.sbl_container_bytes.restype = _sz
 _lib.sbl_container_bytes.argtypes = [_D, _u32]
 _lib.sbl_container_write.restype = ctypes.c_int
@@ -121,7 +123,8 @@ _lib.sbl_container_read.argtypes = [_P, _sz, ctypes.POINTER(sbl_host_buffers)]
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward", "sbl_linear_forward",
             "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
-            "sbl_quantize_mask_pack_ex", "sbl_device_error", "sbl_container_bytes", "sbl_container_write",
+            "sbl_quantize_mask_pack_ex", "sbl_device_error", "sbl_selftest_wait_expiry", "sbl_container_bytes",
+            "sbl_container_write",
             "sbl_container_info", "sbl_container_read"]
 
 
@@ -307,6 +310,14 @@ def sbl_device_error(clear: bool = False) -> int:
     code = _u32(0)
     _check(_lib.sbl_device_error(ctypes.byref(code), 1 if clear else 0), "sbl_device_error")
     return int(code.value)
+
+
+SBL_DEVICE_ERROR_SELFTEST = 0x80000000
+
+
+def sbl_selftest_wait_expiry() -> None:
+    """Enqueue the bounded-wait self-test; its bit appears in sbl_device_error."""
+    _check(_lib.sbl_selftest_wait_expiry(_stream()), "sbl_selftest_wait_expiry")
 
 
 # ------------------------------------------------- allocation helpers (torch)

@@ -153,6 +153,7 @@ int main(void)
         CHECK(sbl_quantize_act(A, 4, 256, B, B, NULL) == SBL_ERR_DEVICE);
         CHECK(sbl_forward(&d68, A, B, 4, &w, SBL_FMT_I8, B, 0, NULL, NULL) == SBL_ERR_DEVICE);
         CHECK(sbl_quantize_mask_pack(&d68, (const float *)A, SBL_FMT_I8, &w, B, ws_pack, NULL) == SBL_ERR_DEVICE);
+        CHECK(sbl_selftest_wait_expiry(NULL) == SBL_ERR_DEVICE);
     }
 
     if (failures) {
