@@ -25,6 +25,13 @@
  *    SBL_ERR_DEVICE.
  *  - A device-side wait that exceeds its time limit (it never should) makes
  *    the kernel record a code readable with sbl_device_error() and return.
+ *  - Host calls are thread-safe: the per-device setup of the first call is
+ *    done once under a lock.  Calls may run concurrently (several host
+ *    threads, several streams) as long as they share no output buffer and
+ *    no workspace; sbl_quantize_mask_pack_noalloc shares one scratch per
+ *    device, so its calls must be ordered on one stream.
+ *  - Results are deterministic: the same inputs give bit-identical outputs
+ *    whatever the stream, the concurrency or the launch order.
  */
 #ifndef SBL_H
 #define SBL_H
