@@ -410,9 +410,10 @@ sbl_status sbl_selftest_wait_expiry(void *stream);
  *         24-27  format mask (SBL_FMT_* bits)
  *         28-31  gamma (fp32 bits)
  *         32-39  payload bytes (everything after the 64-byte header)
- *         40-47  64-bit FNV-1a hash of the payload
+ *         40-47  64-bit FNV-1a hash of every byte of the image except
+ *                these eight (header and payload)
  *         48-51  sbl_version() of the writer
- *         52-63  zero
+ *         52-63  zero (a reader refuses anything else)
  *   payload: for each format present, in the order PK2, NM values, NM
  *   bitmap, I8, BF16T, SP24 values, SP24 metadata, T24 low plane, T24 high
  *   plane, the buffer exactly as sbl_quantize_mask_pack writes it (rows x
@@ -420,8 +421,8 @@ sbl_status sbl_selftest_wait_expiry(void *stream);
  *   64 bytes from the start of the image (zero bytes between; with rows a
  *   multiple of 16 and row bytes a multiple of 16, every buffer is a
  *   multiple of 256 bytes, so in practice none are needed).
- * The hash covers every payload byte, so any change to a stored buffer or
- * to its fill is detected on reading. */
+ * The hash covers the header (gamma included) and every payload byte, so
+ * any change to a stored value is detected on reading. */
 #define SBL_CONTAINER_VERSION 1
 #define SBL_CONTAINER_HEADER_BYTES 64
 
@@ -456,7 +457,8 @@ sbl_status sbl_container_write(const sbl_layer_desc *desc, uint32_t formats, flo
 /* Check an image and report what it holds.  Any of desc, formats, gamma
  * may be NULL.  SBL_ERR_INVALID_ARG: null src, shorter than its header or
  * its payload, wrong magic, a payload size that does not match the
- * descriptor and formats, or a hash mismatch; SBL_ERR_UNSUPPORTED: a
+ * descriptor and formats, nonzero reserved bytes, or a hash mismatch;
+ * SBL_ERR_UNSUPPORTED: a
  * container version this library does not read; SBL_ERR_SHAPE: an invalid
  * descriptor. */
 sbl_status sbl_container_info(const void *src, size_t src_bytes, sbl_layer_desc *desc, uint32_t *formats,

@@ -62,15 +62,25 @@ size_t image_bytes(const sbl_layer_desc *d, uint32_t formats)
     return off;
 }
 
-// 64-bit FNV-1a (offset basis 14695981039346656037, prime 1099511628211).
-uint64_t fnv1a64(const uint8_t *p, size_t n)
+// 64-bit FNV-1a (offset basis 14695981039346656037, prime 1099511628211),
+// continued from h over p[0 .. n).
+uint64_t fnv1a64(uint64_t h, const uint8_t *p, size_t n)
 {
-    uint64_t h = 14695981039346656037ull;
     for (size_t i = 0; i < n; ++i) {
         h ^= p[i];
         h *= 1099511628211ull;
     }
     return h;
+}
+
+constexpr uint64_t kFnvBasis = 14695981039346656037ull;
+constexpr size_t kHashAt = 40;  // the 8 hash bytes: the only bytes the hash skips
+
+// The hash of an image of `total` bytes: every byte except bytes 40-47.
+uint64_t image_hash(const uint8_t *img, size_t total)
+{
+    uint64_t h = fnv1a64(kFnvBasis, img, kHashAt);
+    return fnv1a64(h, img + kHashAt + 8, total - kHashAt - 8);
 }
 
 void put32(uint8_t *p, uint32_t v)
@@ -130,8 +140,9 @@ sbl_status parse(const void *src, size_t src_bytes, sbl_layer_desc *desc, uint32
     const uint64_t payload = get64(h + 32);
     const size_t expect = image_bytes(&d, f);
     if (payload != expect - SBL_CONTAINER_HEADER_BYTES || src_bytes < expect) return SBL_ERR_INVALID_ARG;
-    if (fnv1a64(h + SBL_CONTAINER_HEADER_BYTES, static_cast<size_t>(payload)) != get64(h + 40))
-        return SBL_ERR_INVALID_ARG;
+    for (int i = 52; i < SBL_CONTAINER_HEADER_BYTES; ++i)
+        if (h[i] != 0) return SBL_ERR_INVALID_ARG;
+    if (image_hash(h, expect) != get64(h + kHashAt)) return SBL_ERR_INVALID_ARG;
     if (desc) *desc = d;
     if (formats) *formats = f;
     if (gamma) {
@@ -186,8 +197,8 @@ sbl_status sbl_container_write(const sbl_layer_desc *desc, uint32_t formats, flo
     memcpy(&gb, &gamma, 4);
     put32(out + 28, gb);
     put64(out + 32, total - SBL_CONTAINER_HEADER_BYTES);
-    put64(out + 40, fnv1a64(out + SBL_CONTAINER_HEADER_BYTES, total - SBL_CONTAINER_HEADER_BYTES));
     put32(out + 48, as_u32(sbl_version()));
+    put64(out + kHashAt, image_hash(out, total));  // last: it covers every other byte
     return SBL_OK;
 }
 

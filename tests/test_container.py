@@ -73,7 +73,7 @@ def test_round_trip_is_bit_exact(sbl, O, K, n, m):
 def test_layout_matches_its_documentation(sbl):
     """Header fields at their documented offsets, little-endian; buffers in
     the documented order, each at a multiple of 64 bytes, zeros between; the
-    hash is 64-bit FNV-1a of everything after the 64-byte header."""
+    hash is 64-bit FNV-1a of every byte except its own eight."""
     O, K, n, m = 48, 96, 2, 4
     layer, p, fm = oracle_packed(sbl, O, K, n, m)
     d = sbl.desc(O, K, n, m)
@@ -82,7 +82,7 @@ def test_layout_matches_its_documentation(sbl):
     version, o, k, nn, mm, fmt, gbits, payload, h, lib = struct.unpack_from("<IiiiiIIQQi", image, 4)
     assert (version, o, k, nn, mm, fmt) == (1, O, K, n, m, fm)
     assert gbits == int(np.float32(layer.gamma).view(np.uint32))
-    assert payload == len(image) - 64 and h == fnv1a64(image[64:])
+    assert payload == len(image) - 64 and h == fnv1a64(image[:40] + image[48:])
     assert lib == sbl.sbl_version() and image[52:64] == bytes(12)
     off = 64
     for name in ORDER:
@@ -113,6 +113,10 @@ def test_damage_is_refused(sbl):
         bad = bytearray(image)
         bad[pos] ^= 0x01
         assert status(bad) == 1, pos
+    for off in (28, 48, 60):                             # gamma, writer version, reserved
+        bad = bytearray(image)
+        bad[off] ^= 0x01
+        assert status(bad) == 1, off
     bad = bytearray(image)
     bad[0:4] = b"SBLQ"
     assert status(bad) == 1                              # magic
@@ -175,3 +179,42 @@ def test_save_and_load_through_a_file(sbl, tmp_path):
     assert float(p2.gamma[0]) == layer.gamma
     for name in ORDER:
         assert torch.equal(getattr(p, name).view(torch.uint8), getattr(p2, name).view(torch.uint8)), name
+
+
+def test_reader_survives_random_damage(sbl):
+    """Seeded fuzzing of the reader: random byte flips, truncations and
+    header fields (including huge or negative sizes) must each give a status,
+    never a crash or a read outside the image; an intact image still reads."""
+    import random
+    layer, p, fm = oracle_packed(sbl, 32, 64, 2, 4)
+    d = sbl.desc(32, 64, 2, 4)
+    image = sbl.sbl_container_write(d, fm, layer.gamma, p)
+    rnd = random.Random(11)
+    dst = sbl.alloc_packed(d, fm, device="cpu")
+    outcomes = {}
+    for i in range(3000):
+        bad = bytearray(image)
+        kind = i % 4
+        if kind == 0:                                    # flip a few random bytes
+            for _ in range(rnd.randint(1, 4)):
+                bad[rnd.randrange(len(bad))] ^= rnd.randint(1, 255)
+        elif kind == 1:                                  # truncate anywhere
+            bad = bad[:rnd.randrange(len(bad))]
+        elif kind == 2:                                  # rewrite one header field
+            off = rnd.choice([4, 8, 12, 16, 20, 24, 28, 32, 40, 48])
+            width = 8 if off in (32, 40) else 4
+            bad[off:off + width] = rnd.getrandbits(8 * width).to_bytes(width, "little")
+        else:                                            # a plausible but different descriptor
+            struct.pack_into("<iiii", bad, 8, rnd.choice([16, 65536, 1 << 20, -16]),
+                             rnd.choice([16, 64, 65536, -64]), rnd.randint(-1, 9), rnd.choice([4, 8, 0]))
+        try:
+            sbl.sbl_container_info(bytes(bad))
+            sbl.sbl_container_read(bytes(bad), dst)
+            st = 0
+        except sbl.SblError as e:
+            st = e.status
+        outcomes[st] = outcomes.get(st, 0) + 1
+    assert set(outcomes) <= {0, 1, 2, 4}
+    assert outcomes.get(0, 0) <= 1                       # no damaged image is accepted
+    sbl.sbl_container_read(image, dst)
+    assert torch.equal(dst.pk2, p.pk2)
