@@ -300,3 +300,61 @@ def test_c99_program_against_the_library(sbl, tmp_path):
     assert r.returncode == 0, r.stderr
     if not torch.cuda.is_available():
         assert "(no device)" in r.stdout
+
+
+def test_argument_fuzzing_without_a_device(sbl):
+    """Random descriptors, token counts, format bits and pointers (null,
+    misaligned, plausible) through every entry point: each call returns a
+    documented status and none crashes.  Runs only when the library reports
+    that no device is present, so no pointer here can reach a kernel."""
+    import random
+    code = ctypes.c_uint32(0)
+    if _raw(sbl, "sbl_device_error", ctypes.byref(code), 0) != 7:
+        pytest.skip("a device is present: fake pointers must not reach kernels")
+    rnd = random.Random(3)
+    P = ctypes.c_void_p
+    ints = [-(1 << 31), -1, 0, 1, 2, 3, 4, 6, 7, 8, 9, 15, 16, 17, 64, 80, 256, 1040, 65536, 65552, 1 << 20,
+            (1 << 31) - 1]
+
+    def ptr():
+        return rnd.choice([None, P(0x10000), P(0x10008), P(0x20000), P(0x30001)])
+
+    def desc():
+        return sbl.desc(rnd.choice(ints), rnd.choice(ints), rnd.choice(ints), rnd.choice(ints))
+
+    def packed():
+        return sbl.sbl_packed(*[rnd.choice([None, 0x40000, 0x40004]) for _ in range(10)])
+
+    statuses = set()
+    for _ in range(4000):
+        d, w, T, f = desc(), packed(), rnd.choice(ints), rnd.choice([0, 1, 2, 4, 8, 16, 32, 63, 64, 1 << 31])
+        which = rnd.randrange(9)
+        if which == 0:
+            st = _raw(sbl, "sbl_forward", ctypes.byref(d), ptr(), ptr(), T, ctypes.byref(w), f, ptr(),
+                      rnd.randint(0, 1), ptr(), None)
+        elif which == 1:
+            st = _raw(sbl, "sbl_quantize_act", ptr(), T, rnd.choice(ints), ptr(), ptr(), None)
+        elif which == 2:
+            st = _raw(sbl, "sbl_quantize_act_rmsnorm", ptr(), T, rnd.choice(ints), ptr(),
+                      ctypes.c_float(rnd.choice([0.0, 1e-5, -1.0, float("nan")])), ptr(), ptr(), None)
+        elif which == 3:
+            st = _raw(sbl, "sbl_linear_forward", ctypes.byref(d), ptr(), T, ctypes.byref(w), f, ptr(), ptr(),
+                      ptr(), 0, None, None)
+        elif which == 4:
+            st = _raw(sbl, "sbl_backward_dual_ste", ctypes.byref(d), ptr(), ptr(), ptr(), T, ctypes.byref(w),
+                      ptr(), 1, ptr(), ptr(), rnd.choice([0, 256, 1 << 30]), None)
+        elif which == 5:
+            st = _raw(sbl, "sbl_quantize_mask_pack", ctypes.byref(d), ptr(), f, ctypes.byref(w), ptr(),
+                      rnd.choice([0, 256, 1 << 20]), None)
+        elif which == 6:
+            st = _raw(sbl, "sbl_quantize_mask_pack_noalloc", ctypes.byref(d), ptr(), f, ctypes.byref(w), None)
+        elif which == 7:
+            n = _raw(sbl, "sbl_packed_row_bytes", ctypes.byref(d), f, rnd.randrange(5))
+            n2 = _raw(sbl, "sbl_workspace_bytes", ctypes.byref(d), T, rnd.randrange(3))
+            st = 0 if n >= 0 and n2 >= 0 else -1
+        else:
+            fmt = _raw(sbl, "sbl_forward_format", ctypes.byref(d), T)
+            st = 0 if fmt in (0, 4, 16) else -1
+        statuses.add(st)
+    assert statuses <= set(range(8))
+    assert {1, 2, 7} <= statuses  # invalid arguments, bad sizes, and calls that reached the device check
