@@ -72,6 +72,10 @@ MUTANTS = {
                                   "acc += (int64_t)q[o * d_in + k] * (int64_t)weff[t * d_in + k];"),
     "dx_samples_gamma_dropped": ("out[s] = (double)gamma * acc;", "out[s] = acc;"),
     "bf16_truncates": ("u += 0x7fffu + lsb;", "u += 0u * lsb;"),
+    "dx_weights_transposed": ("s += (double)bf16_to_f32(dy[t * d_out + o]) * (double)weff[o * d_in + k];",
+                              "s += (double)bf16_to_f32(dy[t * d_out + o]) * (double)weff[k * d_out + o];"),
+    "dequant_accumulator_transposed": ("float v = (float)acc[t * d_out + o] * c;",
+                                       "float v = (float)acc[o * tokens + t] * c;"),
     "t24_high_plane_stride": ("hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 4))));",
                               "hrow[g / 4] = (uint8_t)(hrow[g / 4] | ((code >> 4) << (2 * (g % 2))));"),
 }
