@@ -218,3 +218,44 @@ def test_reader_survives_random_damage(sbl):
     assert outcomes.get(0, 0) <= 1                       # no damaged image is accepted
     sbl.sbl_container_read(image, dst)
     assert torch.equal(dst.pk2, p.pk2)
+
+
+def test_every_format_subset_round_trips_random_bytes(sbl):
+    """Any valid descriptor and any subset of the formats it allows: random
+    buffer bytes come back unchanged, and the image size is the header plus
+    the buffers."""
+    import random
+    rnd = random.Random(7)
+    bits = [sbl.SBL_FMT_PK2, sbl.SBL_FMT_NM, sbl.SBL_FMT_I8, sbl.SBL_FMT_BF16T, sbl.SBL_FMT_SP24, sbl.SBL_FMT_T24]
+    for trial in range(60):
+        m = rnd.choice([4, 8])
+        n = rnd.randint(1, m)
+        O = 16 * rnd.randint(1, 12)
+        K = 16 * rnd.randint(1, 20)
+        if K % m:
+            continue
+        d = sbl.desc(O, K, n, m)
+        allowed = [b for b in bits if n <= 2 or b not in (sbl.SBL_FMT_SP24, sbl.SBL_FMT_T24)]
+        fm = 0
+        for b in allowed:
+            if rnd.random() < 0.5:
+                fm |= b
+        src = sbl.alloc_packed(d, fm, device="cpu")
+        total = 64
+        for name in ORDER:
+            t = getattr(src, name)
+            if t is not None:
+                t.view(torch.uint8).copy_(torch.randint(0, 256, t.view(torch.uint8).shape, dtype=torch.uint8))
+                total += t.numel() * t.element_size()
+        g = rnd.uniform(-1.0, 1.0)
+        image = sbl.sbl_container_write(d, fm, g, src)
+        assert len(image) == total == sbl.sbl_container_bytes(d, fm)
+        d2, f2, g2 = sbl.sbl_container_info(image)
+        assert (d2.out_features, d2.in_features, d2.n, d2.m, f2) == (O, K, n, m, fm)
+        assert g2 == float(np.float32(g))
+        dst = sbl.alloc_packed(d, fm, device="cpu")
+        sbl.sbl_container_read(image, dst)
+        for name in ORDER:
+            a, b = getattr(src, name), getattr(dst, name)
+            if a is not None:
+                assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), (trial, name)
