@@ -358,9 +358,17 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens);
  * dY: [T, O] bf16 bits; Xq, d: the forward's quantised activations; w must
  * hold SBL_FMT_BF16T and gamma.  dX may be NULL (skips dX), dW may be NULL
  * (skips dW).  Arithmetic: tensor cores with fp32 accumulation; dY and W_eff
- * enter dX as bf16 (exact), dY*d[t] enters dW rounded to fp16 and Xq as fp16
- * (exact).  Requires |dY * d| < 65504.  workspace: at least
- * sbl_workspace_bytes(desc, T, SBL_OP_BACKWARD) bytes, 256-byte aligned. */
+ * enter dX as bf16 (exact).  For dW, one power of two 2^s per call is chosen
+ * from M = max |fl32(dY[t,o] * d[t])| so that M 2^s lies in [2^14, 2^15);
+ * fl32(dY * d[t]) 2^s enters the MMA rounded to fp16 (relative error at most
+ * 2^-11 per product), Xq as fp16 (exact), and the fp32 result is multiplied
+ * by 2^-s (exact).  Any finite dY works, whatever its magnitude: only
+ * products below 2^-29 M (fp16 subnormals) lose precision, and those below
+ * 2^-40 M (or below 2^-126 in fp32) count as zero; s is clamped to
+ * [-126, 126].  Five launches with dW (an absmax reduction over dY, two
+ * transposes, the GEMM; the memset of the prescale word), one for dX.
+ * workspace: at least sbl_workspace_bytes(desc, T, SBL_OP_BACKWARD) bytes,
+ * 256-byte aligned. */
 sbl_status sbl_backward_dual_ste(const sbl_layer_desc *desc, const uint16_t *dY,
                                  const int8_t *Xq, const float *d, int32_t T,
                                  const sbl_packed *w, void *dX, int32_t dx_is_fp32,

@@ -4,9 +4,11 @@
 //     Sparse-BitNet summary, activation quantization equation): one row of X
 //     is read once into registers, reduced to max|x|, then scaled, rounded
 //     half-to-even and stored as int8 with d_t = max|x| / 127;
-//   * the operand preparation of the Dual-STE backward: dY * d_t as fp16
-//     transposed to [O, T], and the int8 activations as fp16 transposed to
-//     [K, T], so both dW operands are K-major for the tensor cores.
+//   * the operand preparation of the Dual-STE backward: dY * d_t * 2^s as
+//     fp16 transposed to [O, T] (2^s a power of two chosen per call from the
+//     largest |dY * d_t|, so that fp16's narrow range holds the products of
+//     gradients of any scale), and the int8 activations as fp16 transposed
+//     to [K, T], so both dW operands are K-major for the tensor cores.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -252,20 +254,91 @@ __global__ void __launch_bounds__(RT > 256 ? RT : 256, RT > 256 ? 1 : 3)
     if (lt == 0) d[row] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
 }
 
+// The dW operand's power-of-two prescale.  grad_absmax_kernel leaves in *m the
+// fp32 bits of M = max over (t, o) of |fl32(dY[t, o] * d_t)| (computed per row
+// as fl32(max_o |dY[t, o]| * |d_t|), the same value since rounding is
+// monotone); *m must be 0 before the launch.  From M, s is chosen so that
+// M * 2^s lies in [2^14, 2^15): the largest product then sits in fp16's top
+// binade with room for rounding (fp16 ends at 65504), and products down to
+// 2^-29 M stay fp16 normals.  M == 0 gives s = 0; s is clamped to [-126, 126]
+// so that 2^s and 2^-s are fp32 normals, which makes both scalings exact.
+__device__ __forceinline__ int grad_prescale_exponent(uint32_t m_bits)
+{
+    if (m_bits == 0u) return 0;
+    const int e = static_cast<int>(m_bits >> 23);  // biased exponent; 0 for fp32 subnormals
+    const int s = 141 - (e > 0 ? e : 1);           // M in [2^(e-127), 2^(e-126)) -> M 2^s in [2^14, 2^15)
+    return s < -126 ? -126 : (s > 126 ? 126 : s);
+}
+
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float(static_cast<uint32_t>(s + 127) << 23); }
+
+// One warp per row of dY [T, O] (bf16 bits, O % 8 == 0): the row's largest
+// |dY| as bf16 bits (|x| of a finite bf16 orders like its bits & 0x7fff),
+// times |d_t|, reduced over the CTA, then one atomicMax on the fp32 bits of
+// the non-negative result.
+__global__ void __launch_bounds__(256, 4) grad_absmax_kernel(const uint16_t *__restrict__ dY,
+                                                          const float *__restrict__ d, int32_t T, int32_t O,
+                                                          uint32_t *__restrict__ m)
+{
+    __shared__ uint32_t red[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunks = O / 8;
+    uint32_t best = 0u;
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp; row < T; row += static_cast<int64_t>(gridDim.x) * 8) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(dY + row * O);
+        uint32_t mx = 0u;  // two 16-bit maxima, one per half
+        int c = lane;
+        auto absmax8 = [](const uint4 &a) {
+            return __vmaxu2(__vmaxu2(a.x & 0x7fff7fffu, a.y & 0x7fff7fffu),
+                            __vmaxu2(a.z & 0x7fff7fffu, a.w & 0x7fff7fffu));
+        };
+        for (; c + 96 < chunks; c += 128) {
+            const uint4 a = __ldg(p + c), b = __ldg(p + c + 32), e = __ldg(p + c + 64), f = __ldg(p + c + 96);
+            mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(absmax8(a), absmax8(b)), __vmaxu2(absmax8(e), absmax8(f))));
+        }
+        for (; c < chunks; c += 32) mx = __vmaxu2(mx, absmax8(__ldg(p + c)));
+        // the sign bit of each half is cleared before every max, so the maxima
+        // compare magnitudes only
+        uint32_t h = max(mx & 0xffffu, mx >> 16);
+        h = __reduce_max_sync(0xffffffffu, h);
+        const float v = __fmul_rn(__uint_as_float(h << 16), fabsf(d[row]));
+        best = max(best, __float_as_uint(v));
+    }
+    if (lane == 0) red[warp] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = red[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) b = max(b, red[w]);
+        if (b) atomicMax(m, b);
+    }
+}
+
 // out[c, r] = fp16(conv(in[r, c])) for r < rows, c < cols; out has row stride
 // ld_out >= rows, and out[c, r] = 0 for rows <= r < ld_out (padding).
-// Mode 0: in is bf16 bits, value = fl32(bf16 * scale[r]) rounded to fp16.
+// Mode 0: in is bf16 bits, value = fl32(fl32(bf16 * scale[r]) * 2^s) rounded
+//         to fp16, with s = grad_prescale_exponent(*pre) (the bits
+//         grad_absmax_kernel left); block (0, 0) stores 2^-s to *inv_pre for
+//         the GEMM epilogue that undoes the prescale.
 // Mode 1: in is int8, value = fp16(in) (exact).
 // 64 x 64 tiles through shared memory; cols % 16 == 0.
 template <int MODE>
 __global__ void __launch_bounds__(256) transpose_to_f16_kernel(const void *__restrict__ in,
                                                                int32_t rows, int32_t cols,
                                                                const float *__restrict__ scale,
+                                                               const uint32_t *__restrict__ pre,
+                                                               float *__restrict__ inv_pre,
                                                                __half *__restrict__ out,
                                                                int64_t ld_out)
 {
     __shared__ float tile[64][65];
     const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+    float factor = 1.0f;
+    if (MODE == 0) {
+        const int s = grad_prescale_exponent(*pre);
+        factor = pow2f(s);
+        if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *inv_pre = pow2f(-s);
+    }
     // load: 64 rows x 64 columns, 16 consecutive columns per thread-quarter
     for (int idx = threadIdx.x; idx < 64 * 4; idx += 256) {
         const int r = idx >> 2, cq = (idx & 3) * 16;
@@ -282,8 +355,8 @@ __global__ void __launch_bounds__(256) transpose_to_f16_kernel(const void *__res
                     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        vals[8 * h + 2 * i] = __fmul_rn(bf16_lo(w[i]), s);
-                        vals[8 * h + 2 * i + 1] = __fmul_rn(bf16_hi(w[i]), s);
+                        vals[8 * h + 2 * i] = __fmul_rn(__fmul_rn(bf16_lo(w[i]), s), factor);
+                        vals[8 * h + 2 * i + 1] = __fmul_rn(__fmul_rn(bf16_hi(w[i]), s), factor);
                     }
                 }
             } else {

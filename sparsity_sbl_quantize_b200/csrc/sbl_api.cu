@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "sbl.h"
@@ -444,8 +445,10 @@ size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op
     if (op == SBL_OP_BACKWARD) {
         if (tokens < 0) return 0;
         const int64_t tp = round_up(tokens > 0 ? tokens : 1, 64);
+        // the two transposed fp16 operands, then 256 bytes for the prescale
+        // (the bits of max |dY d_t| and 2^-s)
         return static_cast<size_t>(round_up(static_cast<int64_t>(desc->out_features) * tp * 2, 256) +
-                                   round_up(static_cast<int64_t>(desc->in_features) * tp * 2, 256));
+                                   round_up(static_cast<int64_t>(desc->in_features) * tp * 2, 256) + 256);
     }
     return 0;
 }
@@ -986,23 +989,35 @@ static sbl_status backward_impl(const sbl_layer_desc *desc, const uint16_t *dY, 
         if (st != SBL_OK) return st;
     }
     if (dW) {
-        // dW[O, K] = sum_t (dY[t, o] * d_t) * q[t, k]: both operands transposed to
-        // [*, T_pad] fp16 so the reduction over tokens is K-major
+        // dW[O, K] = 2^-s sum_t (dY[t, o] d_t 2^s) q[t, k]: both operands
+        // transposed to [*, T_pad] fp16 so the reduction over tokens is
+        // K-major; 2^s puts the largest |dY d_t| in fp16's top binade, so
+        // gradients of any magnitude keep fp16's 11 bits, and the GEMM's
+        // epilogue multiplies by 2^-s (both scalings are exact)
         const int64_t tp = round_up(T, 64);
-        __half *a_t = static_cast<__half *>(workspace);
-        __half *b_t = reinterpret_cast<__half *>(static_cast<uint8_t *>(workspace) +
-                                                 round_up(static_cast<int64_t>(O) * tp * 2, 256));
+        uint8_t *wsb = static_cast<uint8_t *>(workspace);
+        __half *a_t = reinterpret_cast<__half *>(wsb);
+        const int64_t a_bytes = round_up(static_cast<int64_t>(O) * tp * 2, 256);
+        __half *b_t = reinterpret_cast<__half *>(wsb + a_bytes);
+        uint32_t *pre = reinterpret_cast<uint32_t *>(wsb + a_bytes + round_up(static_cast<int64_t>(K) * tp * 2, 256));
+        float *inv_pre = reinterpret_cast<float *>(pre + 1);
+        if (cudaMemsetAsync(pre, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+        const int64_t rows_per_cta = 8;
+        const int64_t mx_grid = std::min<int64_t>((T + rows_per_cta - 1) / rows_per_cta, 8LL * di->num_sms);
+        grad_absmax_kernel<<<static_cast<unsigned>(mx_grid), 256, 0, stream>>>(dY, d, T, O, pre);
+        if ((st = launch_status()) != SBL_OK) return st;
         dim3 ga((O + 63) / 64, static_cast<unsigned>(tp / 64));
-        transpose_to_f16_kernel<0><<<ga, 256, 0, stream>>>(dY, T, O, d, a_t, tp);
+        transpose_to_f16_kernel<0><<<ga, 256, 0, stream>>>(dY, T, O, d, pre, inv_pre, a_t, tp);
         if ((st = launch_status()) != SBL_OK) return st;
         dim3 gb((K + 63) / 64, static_cast<unsigned>(tp / 64));
-        transpose_to_f16_kernel<1><<<gb, 256, 0, stream>>>(Xq, T, K, nullptr, b_t, tp);
+        transpose_to_f16_kernel<1><<<gb, 256, 0, stream>>>(Xq, T, K, nullptr, nullptr, nullptr, b_t, tp);
         if ((st = launch_status()) != SBL_OK) return st;
         GemmArgs a;
         memset(&a, 0, sizeof(a));
         a.out = dW;
         a.ldo = K;
         a.out_fp32 = 1;
+        a.gamma = inv_pre;
         a.col_keep = dw_keep;
         a.keep_stride = round_up(K / 8, 16);
         st = launch_gemm<kKindF16>(di, a_t, tp * 2, b_t, tp * 2, O, K, static_cast<int32_t>(tp), a, stream);

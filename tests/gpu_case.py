@@ -95,3 +95,32 @@ def normwise(gpu: np.ndarray, ref: np.ndarray) -> float:
     ref = np.asarray(ref, dtype=np.float64)
     den = np.abs(ref).max()
     return float(np.abs(np.asarray(gpu, dtype=np.float64) - ref).max() / (den if den > 0 else 1.0))
+
+
+def elementwise_rel(gpu: np.ndarray, ref: np.ndarray, floor: float = 1e-2) -> float:
+    """Largest elementwise relative error over the entries with |ref| >= floor * max|ref|
+    (reported beside the normwise figure; cancellation makes it ill-posed below the floor)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    gpu = np.asarray(gpu, dtype=np.float64)
+    big = np.abs(ref) >= floor * np.abs(ref).max()
+    if not big.any():
+        return 0.0
+    return float((np.abs(gpu[big] - ref[big]) / np.abs(ref[big])).max())
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """One bf16 ulp at |x| (8 significant bits: 2^(E-7) for |x| in [2^E, 2^(E+1)))."""
+    _, e = np.frexp(np.abs(np.asarray(x, dtype=np.float64)))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Exact conversion for values that are already bf16 numbers (checked)."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    assert not (b & 0xFFFF).any(), "not a bf16 value"
+    return (b >> 16).astype(np.uint16)
+
