@@ -263,6 +263,48 @@ sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const floa
                                           uint32_t formats, const sbl_packed *out,
                                           void *stream);
 
+/* ------------------------------------------- column-parallel sharding --
+ * A layer split by rows (out_features) over ranks: every rank holds rows
+ * [first_row, first_row + rows) of W, N:M groups stay inside a row, and only
+ * gamma needs the whole matrix.  gamma's fp64 pairwise tree (flat row-major
+ * order) has as its first level the sums of consecutive 8192-weight blocks;
+ * when every shard starts at a multiple of 8192 weights (first_row * K %
+ * 8192 == 0), each shard's blocks are blocks of the whole matrix, so
+ *   1. sbl_gamma_partials on every rank (its blocks' sums, fp64),
+ *   2. gather them in rank (= row) order (any collective; NCCL all-gather),
+ *   3. sbl_gamma_combine on the gathered sums (the rest of the same tree),
+ *   4. sbl_quantize_mask_pack_shard on every rank with that gamma
+ * give every rank bit for bit the gamma and the packed rows of the unsharded
+ * sbl_quantize_mask_pack.  The pages describe no distributed execution; this
+ * is the library's own split of the same definitions. */
+
+/* Number of first-level sums of a shard: ceil(rows * K / 8192). */
+size_t sbl_gamma_node_count(const sbl_layer_desc *shard);
+
+/* The shard's first-level sums: node_sums[j] = the fp64 tree sum of |W| over
+ * the shard's flat weights [8192 j, min(8192 (j + 1), rows K)).
+ * shard: (rows, K, n, m) as a layer descriptor; W: the shard's fp32 rows
+ * [rows, K]; first_row: the shard's first row in the whole matrix, used only
+ * to check the alignment (SBL_ERR_SHAPE unless first_row * K is a multiple of
+ * 8192); node_sums: sbl_gamma_node_count(shard) doubles (device);
+ * workspace: as for sbl_quantize_mask_pack.  Two launches (a memset, the
+ * gamma kernel) and a device-to-device copy. */
+sbl_status sbl_gamma_partials(const sbl_layer_desc *shard, const float *W, int64_t first_row, double *node_sums,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* gamma = fl32(S / total_weights), S = the pairwise tree over the gathered
+ * first-level sums of the whole matrix (nodes = ceil(total_weights / 8192),
+ * else SBL_ERR_SHAPE; total_weights <= 2^28).  node_sums and gamma: device.
+ * One launch of one CTA. */
+sbl_status sbl_gamma_combine(const double *node_sums, int64_t nodes, int64_t total_weights, float *gamma,
+                             void *stream);
+
+/* sbl_quantize_mask_pack of a shard's rows with the given gamma: out->gamma
+ * is an INPUT here (from sbl_gamma_combine); no workspace.  One launch (plus
+ * the BF16T transpose when asked for). */
+sbl_status sbl_quantize_mask_pack_shard(const sbl_layer_desc *shard, const float *W, uint32_t formats,
+                                        const sbl_packed *out, void *stream);
+
 /* Step 1 of the forward, per-token absmax int8 quantisation (BitNet b1.58
  * 2B4T summary, "Activation Quantization: Per-Token Absmax"; Sparse-BitNet
  * summary, activation quantization equation):
@@ -338,6 +380,62 @@ sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const fl
 sbl_status sbl_linear_forward(const sbl_layer_desc *desc, const uint16_t *X, int32_t T, const sbl_packed *w,
                               sbl_format fmt, int8_t *Xq, float *d, void *Y, int32_t y_is_fp32,
                               const sbl_epilogue *epi, void *stream);
+
+/* One layer of a batched decode forward (sbl_forward_batch).  The layer's
+ * forward steps 4-5 ("The Full Sparse-BitLinear Layer" of the Sparse-BitNet
+ * summary) from its 2-bit PK2 weights, exactly as sbl_forward with
+ * SBL_FMT_PK2:
+ *   Y[t,o] = fl32(fl32(sum_k W_eff[o,k] Xq[t,k]) * fl32(gamma * d[t])).
+ * desc       the layer (in_features a multiple of 64, at most 14336);
+ * pk2, gamma its packed weights (sbl_packed.pk2 and .gamma);
+ * xq, d      its int8 activations [T, K] and token scales [T] (inputs), or,
+ *            when input_is_previous_output is nonzero, unused: the input is
+ *            then the bf16 output Y of the batch's previous layer, quantised
+ *            per token exactly as sbl_quantize_act (that layer must have
+ *            out_features == this layer's in_features and y_is_fp32 == 0);
+ * xq_out, d_out  with input_is_previous_output: where to store that
+ *            quantised input and its scales (optional, NULL to skip);
+ * y          [T, O] bf16 bits (y_is_fp32 == 0) or fp32. */
+typedef struct {
+    sbl_layer_desc desc;
+    const uint8_t *pk2;
+    const float *gamma;
+    const int8_t *xq;
+    const float *d;
+    void *y;
+    int32_t y_is_fp32;
+    int32_t input_is_previous_output;
+    int8_t *xq_out;
+    float *d_out;
+} sbl_batch_layer;
+
+#define SBL_BATCH_MAX_LAYERS 256
+
+/* Workspace bytes of sbl_forward_batch for `count` layers: 0 when no layer
+ * takes its input from the previous one, else 128 per layer. */
+size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count);
+
+/* The decode forward of `count` layers (1 <= count <= SBL_BATCH_MAX_LAYERS)
+ * at T tokens (1 <= T <= 16) in ONE persistent launch: one CTA per SM
+ * streams every layer's packed rows through a shared-memory ring by bulk
+ * copies, ahead of the arithmetic and across layer boundaries, and computes
+ * each layer as sbl_forward does (bit-identical results).  Independent
+ * layers (no input_is_previous_output) run back to back with no
+ * synchronisation between them.  A chained layer waits, inside the kernel,
+ * until every output of the layer before it is written (a completion count
+ * in the workspace; the wait is bounded and records SBL_DEVICE_ERROR bits on
+ * expiry), then quantises that output in-kernel; chained batches are launched
+ * cooperatively (every CTA resident) and do not let the next kernel start
+ * early.  workspace: sbl_forward_batch_workspace_bytes bytes (NULL when 0),
+ * 256-byte aligned; the library zeroes it (one memset) before the launch.
+ * Unchained batches are launched with programmatic dependent launch like
+ * sbl_forward (the weights are read before the wait on the previous kernel).
+ * Errors: SBL_ERR_SHAPE for count, T or a descriptor out of range;
+ * SBL_ERR_UNSUPPORTED for in_features not a multiple of 64 or above 14336;
+ * SBL_ERR_INVALID_ARG for a null pointer a layer needs, a chained first
+ * layer, or a chain whose shapes or output type do not match. */
+sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32_t T, void *workspace,
+                             size_t workspace_bytes, void *stream);
 
 /* The forward operand format the library recommends for a layer and a
  * token count: SBL_FMT_SP24 (2:4 sparse tensor-core MMA on CTA pairs) when

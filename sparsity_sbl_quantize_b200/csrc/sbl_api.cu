@@ -13,6 +13,7 @@
 #include "sbl.h"
 #include "sbl_act.cuh"
 #include "sbl_decode.cuh"
+#include "sbl_gemv.cuh"
 #include "sbl_sp24.cuh"
 #include "sbl_gemm.cuh"
 #include "sbl_pack.cuh"
@@ -82,7 +83,11 @@ static sbl_status current_device(DeviceInfo **out)
             cudaFuncSetAttribute(sp24_pair_kernel<224, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Sp24PairCfg<128>::kSmemBytes) != cudaSuccess)
+                                 Sp24PairCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemv_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGvSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemv_stream_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGvSmemBytes) != cudaSuccess)
             return SBL_ERR_CUDA;
         if (!g_encode) {
             void *fn = nullptr;
@@ -456,10 +461,13 @@ size_t sbl_workspace_bytes(const sbl_layer_desc *desc, int32_t tokens, sbl_op op
 }  // extern "C"
 
 // sbl_quantize_mask_pack with optional re-mask statistics (stats may be null).
+// gamma_given: out->gamma already holds gamma (a column shard's, from
+// sbl_gamma_combine): no workspace, no gamma kernel, and the packing kernel in
+// plain stream order.
 static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void *W, uint32_t formats,
                                           const sbl_packed *out, const sbl_mask_stats *stats,
                                           const sbl_pack_variant *variant, void *workspace,
-                                          size_t workspace_bytes, void *stream_p)
+                                          size_t workspace_bytes, void *stream_p, bool gamma_given = false)
 {
     sbl_status st = check_desc(desc);
     const sbl_pack_variant def = {SBL_MASTER_FP32, SBL_MASK_FROM_MASTER, SBL_QUANT_THEN_MASK};
@@ -504,9 +512,11 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
             (stats->block_threshold && !aligned16(stats->block_threshold)))
             return SBL_ERR_ALIGNMENT;
     }
-    if (!workspace || workspace_bytes < sbl_workspace_bytes(desc, 0, SBL_OP_QUANTIZE_MASK_PACK))
-        return SBL_ERR_WORKSPACE;
-    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    if (!gamma_given) {
+        if (!workspace || workspace_bytes < sbl_workspace_bytes(desc, 0, SBL_OP_QUANTIZE_MASK_PACK))
+            return SBL_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    }
     DeviceInfo *di = nullptr;
     if ((st = current_device(&di)) != SBL_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
@@ -514,7 +524,8 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
     const int32_t O = desc->out_features, K = desc->in_features;
     const int64_t count = static_cast<int64_t>(O) * K;
     GammaWorkspace *ws = static_cast<GammaWorkspace *>(workspace);
-    if (cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+    if (!gamma_given && cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess)
+        return SBL_ERR_CUDA;
     if (formats & SBL_FMT_NM) {
         // presets the packing kernel edits in place (set before gamma_kernel,
         // so the packing kernel follows gamma_kernel directly: a memset in
@@ -542,7 +553,9 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
     const bool surv = v.order == SBL_MASK_THEN_QUANT;
     const int64_t divisor = surv ? count / desc->m * desc->n : count;
     const int gm = surv ? desc->m : 0;
-    if (bf16) {
+    if (gamma_given) {
+        // gamma is in out->gamma already
+    } else if (bf16) {
         const uint16_t *Wb = static_cast<const uint16_t *>(W);
         if (gm == 0) gamma_kernel<uint16_t, 0><<<gblocks, 256, 0, stream>>>(Wb, count, ws, out->gamma, desc->n, divisor);
         else if (gm == 4) gamma_kernel<uint16_t, 4><<<gblocks, 256, 0, stream>>>(Wb, count, ws, out->gamma, desc->n, divisor);
@@ -611,7 +624,7 @@ static sbl_status quantize_mask_pack_impl(const sbl_layer_desc *desc, const void
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = gamma_given ? 0 : 1;
         const bool sp = (formats & (SBL_FMT_SP24 | SBL_FMT_T24)) != 0;  // the 2:4 formats' instantiation
         const int opt = (sp ? kPackSp24 : 0) | (want_stats ? kPackStats : 0) |
                         (v.mask_source == SBL_MASK_FROM_QUANTIZED ? kPackMaskQ : 0) | (bf16 ? kPackBf16 : 0);
@@ -648,6 +661,62 @@ sbl_status sbl_quantize_mask_pack_ex(const sbl_layer_desc *desc, const void *W, 
                                      void *workspace, size_t workspace_bytes, void *stream_p)
 {
     return quantize_mask_pack_impl(desc, W, formats, out, stats, variant, workspace, workspace_bytes, stream_p);
+}
+
+size_t sbl_gamma_node_count(const sbl_layer_desc *shard)
+{
+    if (check_desc(shard) != SBL_OK) return 0;
+    const int64_t count = static_cast<int64_t>(shard->out_features) * shard->in_features;
+    return static_cast<size_t>((count + kGammaBlock - 1) / kGammaBlock);
+}
+
+sbl_status sbl_gamma_partials(const sbl_layer_desc *shard, const float *W, int64_t first_row, double *node_sums,
+                              void *workspace, size_t workspace_bytes, void *stream_p)
+{
+    sbl_status st = check_desc(shard);
+    if (st != SBL_OK) return st;
+    if (!W || !node_sums) return SBL_ERR_INVALID_ARG;
+    const int64_t K = shard->in_features;
+    if (first_row < 0 || first_row > kMaxDim || (first_row * K) % kGammaBlock != 0) return SBL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(node_sums)) return SBL_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < sbl_workspace_bytes(shard, 0, SBL_OP_QUANTIZE_MASK_PACK))
+        return SBL_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    const int64_t count = static_cast<int64_t>(shard->out_features) * K;
+    const int nodes = static_cast<int>((count + kGammaBlock - 1) / kGammaBlock);
+    GammaWorkspace *ws = static_cast<GammaWorkspace *>(workspace);
+    if (cudaMemsetAsync(&ws->counter, 0, sizeof(uint32_t), stream) != cudaSuccess) return SBL_ERR_CUDA;
+    gamma_kernel<float, 0><<<nodes, 256, 0, stream>>>(W, count, ws, nullptr, shard->n, count, nullptr);
+    if ((st = launch_status()) != SBL_OK) return st;
+    if (cudaMemcpyAsync(node_sums, ws->partials, static_cast<size_t>(nodes) * sizeof(double),
+                        cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return SBL_ERR_CUDA;
+    return SBL_OK;
+}
+
+sbl_status sbl_gamma_combine(const double *node_sums, int64_t nodes, int64_t total_weights, float *gamma,
+                             void *stream_p)
+{
+    if (!node_sums || !gamma) return SBL_ERR_INVALID_ARG;
+    if (total_weights < 1 || total_weights > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials ||
+        nodes != (total_weights + kGammaBlock - 1) / kGammaBlock)
+        return SBL_ERR_SHAPE;
+    if (!aligned16(node_sums) || !aligned16(gamma)) return SBL_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    gamma_combine_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream_p)>>>(node_sums, static_cast<int>(nodes),
+                                                                             total_weights, gamma);
+    return launch_status();
+}
+
+sbl_status sbl_quantize_mask_pack_shard(const sbl_layer_desc *shard, const float *W, uint32_t formats,
+                                        const sbl_packed *out, void *stream_p)
+{
+    return quantize_mask_pack_impl(shard, W, formats, out, nullptr, nullptr, nullptr, 0, stream_p, true);
 }
 
 sbl_status sbl_quantize_act(const uint16_t *X, int32_t T, int32_t K, int8_t *Xq, float *d, void *stream_p)
@@ -949,6 +1018,115 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
 
 }  // extern "C"
 
+// ------------------------------------------------------ batched decode --
+static_assert(SBL_BATCH_MAX_LAYERS <= kGvMaxProblems, "the launch parameters hold every layer of a batch");
+static_assert(sizeof(GvArgs) <= 32000, "kernel parameters are limited to 32764 bytes");
+constexpr int32_t kGvMaxK = 4 * kGvStageBytes / 16;  // 16-row items of K / 4 bytes per row fill a stage
+
+static bool batch_has_chain(const sbl_batch_layer *layers, int32_t count)
+{
+    for (int32_t i = 0; i < count; ++i)
+        if (layers[i].input_is_previous_output) return true;
+    return false;
+}
+
+extern "C" {
+
+size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count)
+{
+    if (!layers || count < 1 || count > SBL_BATCH_MAX_LAYERS) return 0;
+    if (!batch_has_chain(layers, count)) return 0;
+    return static_cast<size_t>(round_up(static_cast<int64_t>(count) * kGvSyncWords * 4, 256));
+}
+
+sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32_t T, void *workspace,
+                             size_t workspace_bytes, void *stream_p)
+{
+    if (!layers) return SBL_ERR_INVALID_ARG;
+    if (count < 1 || count > SBL_BATCH_MAX_LAYERS || T < 1 || T > kDecMaxTokens) return SBL_ERR_SHAPE;
+    static GvArgs a;  // 18 KB of launch parameters, filled under the lock below
+    static std::mutex batch_mutex;
+    std::lock_guard<std::mutex> lock(batch_mutex);
+    memset(&a, 0, sizeof(a));
+    int32_t items = 0;
+    bool chain = false;
+    for (int32_t i = 0; i < count; ++i) {
+        const sbl_batch_layer &L = layers[i];
+        sbl_status st = check_desc(&L.desc);
+        if (st != SBL_OK) return st;
+        const int32_t O = L.desc.out_features, K = L.desc.in_features;
+        if (K % kDecKUnit != 0 || K > kGvMaxK) return SBL_ERR_UNSUPPORTED;
+        if (!L.pk2 || !L.gamma || !L.y) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(L.pk2) || !aligned16(L.gamma) || !aligned16(L.y)) return SBL_ERR_ALIGNMENT;
+        const bool ch = L.input_is_previous_output != 0;
+        if (ch) {
+            if (i == 0) return SBL_ERR_INVALID_ARG;
+            const sbl_batch_layer &P = layers[i - 1];
+            if (P.desc.out_features != K || P.y_is_fp32) return SBL_ERR_INVALID_ARG;
+            if ((L.xq_out && !aligned16(L.xq_out)) || (L.d_out && !aligned16(L.d_out))) return SBL_ERR_ALIGNMENT;
+            chain = true;
+        } else {
+            if (!L.xq || !L.d) return SBL_ERR_INVALID_ARG;
+            if (!aligned16(L.xq) || !aligned16(L.d)) return SBL_ERR_ALIGNMENT;
+        }
+        const bool rows16 = 32 * (K / 4) > kGvStageBytes;
+        const int32_t item_rows = rows16 ? 16 : 32;
+        GvProblem &g = a.p[i];
+        g.pk2 = L.pk2;
+        g.gamma = L.gamma;
+        g.xq = ch ? nullptr : L.xq;
+        g.d = ch ? nullptr : L.d;
+        g.y = L.y;
+        g.xq_out = ch ? L.xq_out : nullptr;
+        g.d_out = ch ? L.d_out : nullptr;
+        g.O = O;
+        g.K = K;
+        g.item0 = items;
+        g.flags = (L.y_is_fp32 ? kGvOutFp32 : 0) | (ch ? kGvChained : 0) | (rows16 ? kGvRows16 : 0);
+        if (ch) a.p[i - 1].flags |= kGvPublish;
+        items += (O + item_rows - 1) / item_rows;
+    }
+    const size_t need = sbl_forward_batch_workspace_bytes(layers, count);
+    if (chain) {
+        if (!workspace || workspace_bytes < need) return SBL_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    }
+    DeviceInfo *di = nullptr;
+    sbl_status st = current_device(&di);
+    if (st != SBL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    if (chain && cudaMemsetAsync(workspace, 0, static_cast<size_t>(count) * kGvSyncWords * 4, stream) != cudaSuccess)
+        return SBL_ERR_CUDA;
+    a.count = count;
+    a.T = T;
+    a.items = items;
+    a.early_trigger = chain ? 0 : 1;
+    a.sync = chain ? static_cast<uint32_t *>(workspace) : nullptr;
+    a.err = di->err;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(items < di->num_sms ? items : di->num_sms));
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = kGvSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (chain) {
+        // the CTAs wait on one another: all of them must be resident
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = T <= 8 ? cudaLaunchKernelEx(&cfg, gemv_stream_kernel<1>, a)
+                                 : cudaLaunchKernelEx(&cfg, gemv_stream_kernel<2>, a);
+    return e == cudaSuccess ? launch_status() : SBL_ERR_CUDA;
+}
+
+}  // extern "C"
+
 static sbl_status backward_impl(const sbl_layer_desc *desc, const uint16_t *dY, const int8_t *Xq, const float *d,
                                 int32_t T, const sbl_packed *w, void *dX, int32_t dx_is_fp32, float *dW,
                                 const uint8_t *dw_keep, void *workspace, size_t workspace_bytes, void *stream_p)
@@ -1048,11 +1226,12 @@ sbl_status sbl_backward_dual_ste_ex(const sbl_layer_desc *desc, const uint16_t *
 
 // ------------------------------------------------ no-allocation variant --
 // File-scope scratch for sbl_quantize_mask_pack_noalloc: holds the gamma
-// partial sums, the finishing counter and the ternary threshold.  In host
-// code the symbol is only a handle; its device address comes from
-// cudaGetSymbolAddress, looked up once per device on the first call.
+// partial sums and the finishing counter.  In host code the symbol is only a
+// handle; its device address comes from cudaGetSymbolAddress, looked up once
+// per device on the first call.
 namespace sbl {
-static_assert(SBL_NOALLOC_SCRATCH_BYTES >= sizeof(GammaWorkspace), "scratch too small");
+static_assert(SBL_NOALLOC_SCRATCH_BYTES >= (sizeof(GammaWorkspace) + 255) / 256 * 256,
+              "scratch smaller than the workspace sbl_workspace_bytes asks for");
 static_assert(SBL_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte granularity");
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SBL_NOALLOC_SCRATCH_BYTES];
 static std::mutex g_noalloc_mutex;
@@ -1063,7 +1242,7 @@ static void *g_noalloc_ptr[kMaxDevices];
 // After kWaitLimitNs the wait records SBL_DEVICE_ERROR_SELFTEST and the
 // kernel returns.  No copy, MMA or tensor memory is outstanding when it does.
 static_assert((SBL_DEVICE_ERROR_SELFTEST & (kErrGemmProducer | kErrGemmMma | kErrGemmEpilogue | kErrDecode |
-                                            kErrPack)) == 0,
+                                            kErrPack | kErrGemv)) == 0,
               "the self-test bit is distinct from every kernel family's bit");
 __global__ void __launch_bounds__(32) wait_expiry_kernel(uint32_t *err)
 {
@@ -1086,6 +1265,9 @@ sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const floa
     // the scratch holds kGammaMaxPartials partial sums of kGammaBlock weights
     const int64_t count = static_cast<int64_t>(desc->out_features) * desc->in_features;
     if (count > static_cast<int64_t>(kGammaBlock) * kGammaMaxPartials) return SBL_ERR_SHAPE;
+    // an sm_100 device first (other devices get SBL_ERR_DEVICE, as every call)
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBL_ERR_DEVICE;
     void *scratch = nullptr;
@@ -1093,7 +1275,10 @@ sbl_status sbl_quantize_mask_pack_noalloc(const sbl_layer_desc *desc, const floa
         std::lock_guard<std::mutex> lock(g_noalloc_mutex);
         if (!g_noalloc_ptr[dev]) {
             void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SBL_ERR_CUDA;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+                cudaGetLastError();  // leave no pending error for the thread's next launch check
+                return SBL_ERR_CUDA;
+            }
             g_noalloc_ptr[dev] = p;
         }
         scratch = g_noalloc_ptr[dev];

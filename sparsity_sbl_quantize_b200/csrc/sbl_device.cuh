@@ -17,6 +17,7 @@ enum : uint32_t {
     kErrGemmEpilogue = 1u << 2,
     kErrDecode = 1u << 3,
     kErrPack = 1u << 4,
+    kErrGemv = 1u << 5,
 };
 
 // Every device-side wait gives up after this long and records an error.
@@ -129,6 +130,46 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_group()
 {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// L2 policy for data read exactly once (streamed weights): evict first, so
+// the reused activations and outputs keep their L2 lines.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global into this CTA's shared memory, completing on `bar` as
+// transaction bytes.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                             uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// Wait until *counter >= target (acquire at GPU scope), giving up after
+// kWaitLimitNs with `code` set in *err.
+__device__ __forceinline__ bool wait_counter_geq(const uint32_t *counter, uint32_t target, uint32_t *err,
+                                                 uint32_t code)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= target) return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, code);
+            return false;
+        }
+        __nanosleep(64);
+    }
 }
 
 // Order this thread's generic-proxy shared-memory writes before later

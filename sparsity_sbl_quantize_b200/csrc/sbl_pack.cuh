@@ -108,22 +108,68 @@ __device__ __forceinline__ float4 load4(const WT *W, int64_t e)
     }
 }
 
+// Second level of the gamma tree, over the node partials parts[0 .. nparts)
+// (nparts <= kGammaMaxPartials): chunks of 2048 partials (tree nodes); in each
+// chunk thread t loads [8t, 8t + 8) (all threads, loads in flight together), a
+// butterfly and a shared-memory tree combine the 256 thread sums, and the <= 16
+// chunk sums finish pairwise (zeros past the end).  Called by all 256 threads
+// of a CTA; the result is valid in thread 0.
+__device__ __forceinline__ double gamma_tree_finish(const double *parts, int nparts, double *warp_sums,
+                                                   double *chunk_sums)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = (nparts + 2047) / 2048;
+    for (int c = 0; c < nchunks; ++c) {
+        double v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int j = c * 2048 + threadIdx.x * 8 + i;
+            v[i] = (j < nparts) ? __ldcg(&parts[j]) : 0.0;
+        }
+        double u = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) u = u + __shfl_xor_sync(0xffffffffu, u, off);
+        if (lane == 0) warp_sums[warp] = u;
+        __syncthreads();
+        if (threadIdx.x == 0)
+            chunk_sums[c] = ((warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3])) +
+                            ((warp_sums[4] + warp_sums[5]) + (warp_sums[6] + warp_sums[7]));
+        __syncthreads();
+    }
+    double total = 0.0;
+    if (threadIdx.x == 0) {
+        constexpr int kChunks = kGammaMaxPartials / 2048;
+        double cs[kChunks];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) cs[c] = (c < nchunks) ? chunk_sums[c] : 0.0;
+#pragma unroll
+        for (int w = 1; w < kChunks; w *= 2)
+#pragma unroll
+            for (int i = 0; i < kChunks; i += 2 * w) cs[i] = cs[i] + cs[i + w];
+        total = cs[0];
+    }
+    return total;
+}
+
 // gamma: one CTA per tree node of kGammaBlock weights.  Warp w owns the 1024
 // consecutive weights [node*8192 + 1024w, +1024) as eight 128-weight chunks;
 // for chunk q lane l loads the float4 at 128q + 4l (coalesced), sums its four
 // leaves, and a butterfly over the lanes completes the chunk's tree; the eight
 // chunk sums, the eight warp sums and finally (in the last CTA to finish) the
 // node partials are combined over the same pairwise tree.  ws->counter must
-// be zero at launch.
+// be zero at launch.  gamma_out and sum_out (the fp64 sum itself) are
+// optional; with neither, the node partials in ws are the result.
 // SURV_M = 0: gamma over all weights; SURV_M = m (4 or 8): mask-then-quant,
 // the sum over the kept |w| only (the group's keep mask from |w| as in
 // pack_kernel; zeros at dropped positions keep the same tree) divided by
 // `divisor` (the number of kept weights).
 template <typename WT, int SURV_M>
 __global__ void __launch_bounds__(256) gamma_kernel(const WT *__restrict__ W, int64_t count,
-                                                    GammaWorkspace *ws, float *gamma_out, int n, int64_t divisor)
+                                                    GammaWorkspace *ws, float *gamma_out, int n, int64_t divisor,
+                                                    double *sum_out = nullptr)
 {
     __shared__ double warp_sums[8];
+    __shared__ double chunk_sums[kGammaMaxPartials / 2048];
     __shared__ int is_last;
     // the pack kernel may launch now: it only streams W before waiting for us
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -210,40 +256,29 @@ __global__ void __launch_bounds__(256) gamma_kernel(const WT *__restrict__ W, in
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    // Second level, over the same tree: chunks of 2048 partials (tree nodes);
-    // in each chunk thread t loads [8t, 8t + 8) (all threads, loads in flight
-    // together), a shared-memory tree combines the 256 thread sums, and the
-    // <= 16 chunk sums finish pairwise (zeros past the end).
-    const int nparts = static_cast<int>(gridDim.x);
-    __shared__ double chunk_sums[kGammaMaxPartials / 2048];
-    const int nchunks = (nparts + 2047) / 2048;
-    for (int c = 0; c < nchunks; ++c) {
-        double v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int j = c * 2048 + threadIdx.x * 8 + i;
-            v[i] = (j < nparts) ? __ldcg(&ws->partials[j]) : 0.0;
-        }
-        double u = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) u = u + __shfl_xor_sync(0xffffffffu, u, off);
-        if (lane == 0) warp_sums[warp] = u;
-        __syncthreads();
-        if (threadIdx.x == 0)
-            chunk_sums[c] = ((warp_sums[0] + warp_sums[1]) + (warp_sums[2] + warp_sums[3])) +
-                            ((warp_sums[4] + warp_sums[5]) + (warp_sums[6] + warp_sums[7]));
-        __syncthreads();
-    }
+    if (!gamma_out && !sum_out) return;  // node partials only (a column shard's first level)
+    const double total = gamma_tree_finish(ws->partials, static_cast<int>(gridDim.x), warp_sums, chunk_sums);
     if (threadIdx.x == 0) {
-        constexpr int kChunks = kGammaMaxPartials / 2048;
-        double cs[kChunks];
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) cs[c] = (c < nchunks) ? chunk_sums[c] : 0.0;
-#pragma unroll
-        for (int w = 1; w < kChunks; w *= 2)
-#pragma unroll
-            for (int i = 0; i < kChunks; i += 2 * w) cs[i] = cs[i] + cs[i + w];
-        const double mean = divisor > 0 ? __ddiv_rn(cs[0], static_cast<double>(divisor)) : 0.0;
+        if (sum_out) *sum_out = total;
+        if (gamma_out) {
+            const double mean = divisor > 0 ? __ddiv_rn(total, static_cast<double>(divisor)) : 0.0;
+            *gamma_out = __double2float_rn(mean);
+        }
+    }
+}
+
+// Combine the first-level node sums of every column shard (gathered in row
+// order) over the same tree: gamma = fl32(tree(nodes) / divisor).  One CTA
+// of 256 threads.
+__global__ void __launch_bounds__(256) gamma_combine_kernel(const double *__restrict__ nodes, int nparts,
+                                                            int64_t divisor, float *gamma_out)
+{
+    __shared__ double warp_sums[8];
+    __shared__ double chunk_sums[kGammaMaxPartials / 2048];
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the node sums may come from the previous kernel
+    const double total = gamma_tree_finish(nodes, nparts, warp_sums, chunk_sums);
+    if (threadIdx.x == 0) {
+        const double mean = divisor > 0 ? __ddiv_rn(total, static_cast<double>(divisor)) : 0.0;
         *gamma_out = __double2float_rn(mean);
     }
 }

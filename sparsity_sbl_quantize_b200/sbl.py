@@ -69,6 +69,15 @@ class sbl_host_buffers(ctypes.Structure):
                 ("pk2", "nm_values", "nm_bitmap", "i8", "bf16t", "sp24_values", "sp24_meta", "t24_lo", "t24_hi")]
 
 
+class sbl_batch_layer(ctypes.Structure):
+    _fields_ = [("desc", sbl_layer_desc), ("pk2", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("xq", ctypes.c_void_p), ("d", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("y_is_fp32", ctypes.c_int32), ("input_is_previous_output", ctypes.c_int32),
+                ("xq_out", ctypes.c_void_p), ("d_out", ctypes.c_void_p)]
+
+
+SBL_BATCH_MAX_LAYERS = 256
+
 _P = ctypes.c_void_p
 _D = ctypes.POINTER(sbl_layer_desc)
 _W = ctypes.POINTER(sbl_packed)
@@ -105,6 +114,18 @@ _lib.sbl_forward_ex.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P
 _lib.sbl_linear_forward.restype = ctypes.c_int
 _lib.sbl_linear_forward.argtypes = [_D, _P, _i32, _W, ctypes.c_int, _P, _P, _P, _i32,
                                     ctypes.POINTER(sbl_epilogue), _P]
+_lib.sbl_forward_batch_workspace_bytes.restype = _sz
+_lib.sbl_forward_batch_workspace_bytes.argtypes = [ctypes.POINTER(sbl_batch_layer), _i32]
+_lib.sbl_forward_batch.restype = ctypes.c_int
+_lib.sbl_forward_batch.argtypes = [ctypes.POINTER(sbl_batch_layer), _i32, _i32, _P, _sz, _P]
+_lib.sbl_gamma_node_count.restype = _sz
+_lib.sbl_gamma_node_count.argtypes = [_D]
+_lib.sbl_gamma_partials.restype = ctypes.c_int
+_lib.sbl_gamma_partials.argtypes = [_D, _P, ctypes.c_int64, _P, _P, _sz, _P]
+_lib.sbl_gamma_combine.restype = ctypes.c_int
+_lib.sbl_gamma_combine.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, _P, _P]
+_lib.sbl_quantize_mask_pack_shard.restype = ctypes.c_int
+_lib.sbl_quantize_mask_pack_shard.argtypes = [_D, _P, _u32, _W, _P]
 _lib.sbl_forward_format.restype = ctypes.c_int
 _lib.sbl_forward_format.argtypes = [_D, _i32]
 _lib.sbl_device_error.restype = ctypes.c_int
@@ -122,7 +143,9 @@ _lib.sbl_container_read.argtypes = [_P, _sz, ctypes.POINTER(sbl_host_buffers)]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward", "sbl_linear_forward",
-            "sbl_forward_ex", "sbl_forward_format", "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
+            "sbl_forward_ex", "sbl_forward_format", "sbl_forward_batch", "sbl_forward_batch_workspace_bytes",
+            "sbl_gamma_node_count", "sbl_gamma_partials", "sbl_gamma_combine", "sbl_quantize_mask_pack_shard",
+            "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
             "sbl_quantize_mask_pack_ex", "sbl_device_error", "sbl_selftest_wait_expiry", "sbl_container_bytes",
             "sbl_container_write",
             "sbl_container_info", "sbl_container_read"]
@@ -321,6 +344,50 @@ def sbl_selftest_wait_expiry() -> None:
 
 
 # ------------------------------------------------- allocation helpers (torch)
+
+def batch_layer(dsc: sbl_layer_desc, w: "Packed", Y: torch.Tensor, Xq: Optional[torch.Tensor] = None,
+                d: Optional[torch.Tensor] = None, y_is_fp32: bool = False, chained: bool = False,
+                xq_out: Optional[torch.Tensor] = None, d_out: Optional[torch.Tensor] = None) -> sbl_batch_layer:
+    """One entry of a batched decode forward (the tensors must outlive the call)."""
+    def addr(t):
+        return t.data_ptr() if t is not None else None
+    return sbl_batch_layer(dsc, w.pk2.data_ptr(), w.gamma.data_ptr(), addr(Xq), addr(d), Y.data_ptr(),
+                           1 if y_is_fp32 else 0, 1 if chained else 0, addr(xq_out), addr(d_out))
+
+
+def batch_array(layers) -> ctypes.Array:
+    return (sbl_batch_layer * len(layers))(*layers)
+
+
+def sbl_forward_batch_workspace_bytes(layers: ctypes.Array, count: int) -> int:
+    return int(_lib.sbl_forward_batch_workspace_bytes(layers, count))
+
+
+def sbl_forward_batch(layers: ctypes.Array, count: int, T: int, workspace: Optional[torch.Tensor] = None) -> None:
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.sbl_forward_batch(layers, count, T, _ptr(workspace), nbytes, _stream()), "sbl_forward_batch")
+
+
+def sbl_gamma_node_count(shard: sbl_layer_desc) -> int:
+    return int(_lib.sbl_gamma_node_count(ctypes.byref(shard)))
+
+
+def sbl_gamma_partials(shard: sbl_layer_desc, W: torch.Tensor, first_row: int, node_sums: torch.Tensor,
+                       workspace: torch.Tensor) -> None:
+    _check(_lib.sbl_gamma_partials(ctypes.byref(shard), _ptr(W), first_row, _ptr(node_sums), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream()), "sbl_gamma_partials")
+
+
+def sbl_gamma_combine(node_sums: torch.Tensor, nodes: int, total_weights: int, gamma: torch.Tensor) -> None:
+    _check(_lib.sbl_gamma_combine(_ptr(node_sums), nodes, total_weights, _ptr(gamma), _stream()),
+           "sbl_gamma_combine")
+
+
+def sbl_quantize_mask_pack_shard(shard: sbl_layer_desc, W: torch.Tensor, formats: int, out: "Packed") -> None:
+    cp = out.c()
+    _check(_lib.sbl_quantize_mask_pack_shard(ctypes.byref(shard), _ptr(W), formats, ctypes.byref(cp), _stream()),
+           "sbl_quantize_mask_pack_shard")
+
 
 def sbl_forward_format(d: sbl_layer_desc, tokens: int) -> int:
     return int(_lib.sbl_forward_format(ctypes.byref(d), tokens))

@@ -358,3 +358,65 @@ def test_argument_fuzzing_without_a_device(sbl):
         statuses.add(st)
     assert statuses <= set(range(8))
     assert {1, 2, 7} <= statuses  # invalid arguments, bad sizes, and calls that reached the device check
+
+
+def test_batch_forward_validation_before_device(sbl):
+    """sbl_forward_batch: count, T, descriptors, K limits, null pointers, chain
+    rules, alignment and the workspace are checked before the device lookup;
+    a valid call on a host without a GPU reports SBL_ERR_DEVICE."""
+    good = 0x10000
+
+    def layer(O=128, K=256, chained=False, y_fp32=0, xq=good, pk2=good):
+        return sbl.sbl_batch_layer(sbl.desc(O, K, 2, 4), pk2, good, xq, good, good, y_fp32, 1 if chained else 0,
+                                   None, None)
+
+    def call(layers, T=4, ws=None, ws_bytes=0, count=None):
+        arr = sbl.batch_array(layers)
+        return _raw(sbl, "sbl_forward_batch", arr, len(layers) if count is None else count, T,
+                    ctypes.c_void_p(ws) if ws else None, ws_bytes, None)
+
+    assert _raw(sbl, "sbl_forward_batch", None, 1, 4, None, 0, None) == 1
+    assert call([layer()], T=0) == 2 and call([layer()], T=17) == 2
+    assert call([layer()], count=0) == 2 and call([layer()], count=257) == 2
+    assert call([layer(K=250)]) == 2                       # invalid descriptor
+    assert call([layer(K=272)]) == 4                       # K not a multiple of 64
+    assert call([layer(K=14400)]) == 4                     # K above the stage limit
+    assert call([layer(pk2=None)]) == 1 and call([layer(xq=None)]) == 1
+    assert call([layer(pk2=good + 8)]) == 3
+    assert call([layer(chained=True)]) == 1                # a chain needs a previous layer
+    assert call([layer(O=256), layer(O=128, K=512, chained=True)]) == 1   # shapes do not chain
+    assert call([layer(O=512, y_fp32=1), layer(K=512, chained=True)]) == 1  # fp32 output cannot chain
+    chain = [layer(O=512), layer(K=512, chained=True, xq=None)]
+    nws = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array(chain), 2)
+    assert nws == 256
+    assert sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer()]), 1) == 0
+    assert call(chain) == 5 and call(chain, ws=good, ws_bytes=nws - 1) == 5
+    assert call(chain, ws=good + 16, ws_bytes=nws) == 3
+    assert call(chain, ws=good, ws_bytes=nws) == 7         # valid: no sm_100 device here
+    assert call([layer(), layer(O=64, K=14336)], T=16) == 7
+
+
+def test_sharding_calls_validate_before_device(sbl):
+    good = 0x10000
+    P = ctypes.c_void_p
+    d = sbl.desc(64, 1040, 6, 8)
+    assert sbl.sbl_gamma_node_count(d) == (64 * 1040 + 8191) // 8192
+    assert sbl.sbl_gamma_node_count(sbl.desc(64, 250, 6, 8)) == 0
+    nb = sbl.sbl_workspace_bytes(d, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK)
+    part = "sbl_gamma_partials"
+    assert _raw(sbl, part, ctypes.byref(d), None, 0, P(good), P(good), nb, None) == 1
+    assert _raw(sbl, part, ctypes.byref(d), P(good), 16, P(good), P(good), nb, None) == 2   # misaligned shard
+    assert _raw(sbl, part, ctypes.byref(d), P(good), -8, P(good), P(good), nb, None) == 2
+    assert _raw(sbl, part, ctypes.byref(d), P(good + 4), 0, P(good), P(good), nb, None) == 3
+    assert _raw(sbl, part, ctypes.byref(d), P(good), 0, P(good), P(good), nb - 1, None) == 5
+    assert _raw(sbl, part, ctypes.byref(d), P(good), 0, P(good), P(good), nb, None) == 7  # no device here
+    comb = "sbl_gamma_combine"
+    assert _raw(sbl, comb, None, 4, 4 * 8192, P(good), None) == 1
+    assert _raw(sbl, comb, P(good), 3, 4 * 8192, P(good), None) == 2
+    assert _raw(sbl, comb, P(good), 1, 0, P(good), None) == 2
+    assert _raw(sbl, comb, P(good), 5, 4 * 8192 + 1, P(good), None) == 7
+    w = sbl.sbl_packed(None, None, None, good, None, good)
+    assert _raw(sbl, "sbl_quantize_mask_pack_shard", ctypes.byref(d), P(good), sbl.SBL_FMT_I8, ctypes.byref(w),
+                None) == 7
+    assert _raw(sbl, "sbl_quantize_mask_pack_shard", ctypes.byref(d), None, sbl.SBL_FMT_I8, ctypes.byref(w),
+                None) == 1

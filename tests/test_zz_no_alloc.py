@@ -66,6 +66,20 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     assert sbl.sbl_device_error() == 0
 
 
+def test_noalloc_matches_the_oracle():
+    """gamma and W_eff from the no-allocation call against the oracle
+    directly (besides the regular entry point), twice in a row."""
+    import oracle
+    sbl = _sbl()
+    w = wl.master_weights(528, 1040, seed=11)
+    ref = oracle.Layer(w, 6, 8)
+    for _ in range(2):
+        _, got = _both(sbl, w, 6, 8)
+        assert np.float32(got.gamma[0].item()) == ref.gamma
+        np.testing.assert_array_equal(got.i8.cpu().numpy(), ref.weff)
+        np.testing.assert_array_equal(got.pk2.cpu().numpy(), oracle.pack_pk2(ref.weff))
+
+
 def test_noalloc_rejects_layers_beyond_its_scratch():
     sbl = _sbl()
     # 2^28 weights is the limit; 16384 x 16400 is over it -> SBL_ERR_SHAPE
