@@ -10,7 +10,10 @@ masked ternary x int8 GEMM with its dequantisation (plus the Dual-STE
 backward for the training workload, or the packed-weight GEMV for decode).
 Inputs are resident in HBM when the timed region starts; the L2 is flushed
 between timed steps (outside the timed events).  The default workload is the
-Qwen2.5-0.5B MLP linears (896->4864 x2, 4864->896) at T=4096, 6:8 and 2:4.
+largest single-GPU one, the Qwen2.5-3B training step (2048->11008, 11008->2048
+at T=16384, 6:8: re-mask, forward, Dual-STE backward); the same JSON line
+carries a `decode` object with the BitNet-2B decode GEMV (GB/s, T = 1, 4, 16),
+the other half of the metric.
 
 Rank 0 prints one JSON line.  Under torchrun every rank runs the same step on
 its own GPU (independent problems, weak scaling, no data-path collective);
@@ -41,7 +44,7 @@ LONG_STEP_MS = 1.0  # steps longer than this run at the power-capped (sustained)
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
 # the device code of each family of roofline kernels (the GEMMs, the decode GEMV)
 KERNEL_SOURCES = {"gemm": ("sbl_device.cuh", "sbl_gemm.cuh", "sbl_sp24.cuh"),
-                  "decode": ("sbl_device.cuh", "sbl_decode.cuh")}
+                  "decode": ("sbl_device.cuh", "sbl_decode.cuh", "sbl_gemv.cuh")}
 
 
 def kernel_family(workload: str) -> str:
@@ -115,8 +118,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen05b_mlp", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="qwen3b_train", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="leave out the decode object that prefill/train lines carry")
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="threads of the oracle timing (default: every core this process may use)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV", nargs="+",
                     help="store the mean DRAM bytes per roofline-kernel launch from an ncu --csv metric list "
                          "(dram__bytes_read.sum, dram__bytes_write.sum) for --workload, then exit")
@@ -158,6 +165,53 @@ def decode_step_bytes(wk, tokens):
                for lin in wk.linears)
 
 
+def workload_config(wk, world: int) -> dict:
+    """What the workload is (shapes, patterns, mode, ranks): the same object in
+    both arms' lines, so that their ratio is on one configuration."""
+    return {"workload": wk.name, "tokens": wk.tokens if wk.mode == "decode" else wk.tokens[-1],
+            "linears": [f"{l.name}:{l.d_in}->{l.d_out}" for l in wk.linears],
+            "patterns": [f"{n}:{m}" for n, m in wk.patterns], "mode": wk.mode,
+            "parallelism": f"independent replicas x{world}"}
+
+
+# Dense int8 tensor-core rate of one B200 SM per clock: 2 x the 8192 bf16
+# flops per clock per SM at which 148 SMs give the dense bf16 figure of
+# 2.25 PFLOP/s (at 1.855 GHz); 148 x 16384 x 1.855 GHz = 4.5 POPS, the dense
+# int8 figure.
+INT8_OPS_PER_CLOCK_PER_SM = 16384
+B200_SMS = 148
+
+
+def clock_scaled_int8_peak(sm_mhz):
+    """The int8 peak at the SM clock sampled during the timed region (TOPS)."""
+    if not sm_mhz:
+        return None
+    return INT8_OPS_PER_CLOCK_PER_SM * B200_SMS * sm_mhz * 1e6 / 1e12
+
+
+def cpu_threads(requested: int = 0) -> int:
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except AttributeError:
+        avail = os.cpu_count() or 1
+    return max(1, min(requested, avail) if requested else avail)
+
+
+def slices(n: int, parts: int):
+    """`parts` contiguous, disjoint, near-equal ranges covering 0 .. n-1."""
+    parts = max(1, min(parts, n))
+    b = [n * i // parts for i in range(parts + 1)]
+    return [(b[i], b[i + 1]) for i in range(parts) if b[i + 1] > b[i]]
+
+
+def run_parallel(pool, jobs):
+    """Run the callables (each calls one unchanged oracle function on its own
+    slice; ctypes releases the GIL for the C call) and wait for all."""
+    if pool is None:
+        return [j() for j in jobs]
+    return [f.result() for f in [pool.submit(j) for j in jobs]]
+
+
 # ------------------------------------------------------------------ ranks
 
 def max_over_ranks(value: float, dist, world: int, device) -> float:
@@ -183,6 +237,61 @@ def barrier(dist, world: int):
 
 # ------------------------------------------------------------------ clocks
 
+class _NvmlPoller:
+    """Samples the SM clock, its maximum, the power draw and the four
+    slowdown reasons of one GPU through NVML every `period` seconds, writing
+    rows in nvidia-smi's CSV form (timestamp, uuid, clocks.sm, clocks.max.sm,
+    power.draw, hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown,
+    sw_power_cap) from a background thread; only reads the GPU's state."""
+
+    def __init__(self, uuid, f, period=0.005):
+        import threading
+        import pynvml as nv
+        nv.nvmlInit()
+        self.nv, self.f, self.period = nv, f, period
+        self.h = None
+        for i in range(nv.nvmlDeviceGetCount()):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            u = nv.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if not uuid or uuid in u:
+                self.h, self.uuid = h, u
+                break
+        if self.h is None:
+            raise RuntimeError("GPU not found through NVML")
+        self.bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                     nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        self.stop_ev = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        smax = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        while not self.stop_ev.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                break
+            stamp = datetime.datetime.now().strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            flags = ", ".join("Active" if r & b else "Not Active" for b in self.bits)
+            self.f.write(f"{stamp}, {self.uuid}, {sm}, {smax}, {pw:.2f}, {flags}\n")
+            self.f.flush()
+            self.stop_ev.wait(self.period)
+
+    def terminate(self):
+        self.stop_ev.set()
+
+    def wait(self, timeout=None):
+        self.thread.join(timeout)
+        return 0
+
+    def kill(self):
+        self.stop_ev.set()
+
+
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -194,16 +303,20 @@ class ClockSampler:
         self.uuid = uuid
 
     def start(self):
-        """Start sampling every 50 ms and wait (up to 5 s) for the first row,
-        so that the timed region that follows is covered from its start."""
+        """Start sampling (every 5 ms through NVML, else every 50 ms through
+        nvidia-smi) and wait (up to 5 s) for the first row, so that the timed
+        region that follows is covered from its start."""
         try:
-            cmd = ["nvidia-smi", "--query-gpu=timestamp,uuid," + self.FIELDS, "--format=csv,noheader,nounits",
-                   "-lms", "50"]
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+            self.proc = _NvmlPoller(self.uuid, self.f)
         except Exception:
-            self.proc = None
-            return
+            try:
+                cmd = ["nvidia-smi", "--query-gpu=timestamp,uuid," + self.FIELDS, "--format=csv,noheader,nounits",
+                       "-lms", "50"]
+                self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+                return
         deadline = time.time() + 5.0
         while time.time() < deadline and os.path.getsize(self.path) == 0:
             time.sleep(0.02)
@@ -237,7 +350,7 @@ class ClockSampler:
         inside = [r for r in rows if any(t0 <= r[0] <= t1 for t0, t1 in windows)]
         window = "timed region"
         if not inside:
-            inside, window = rows, "around the timed region (shorter than the 50 ms sampling period)"
+            inside, window = rows, "around the timed region (shorter than the sampling period)"
         if not inside:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -581,27 +694,33 @@ def run_ours(args, wk):
     err = sbl.sbl_device_error()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wk, budget_s=12.0)
+        cpu = cpu_baselines(wk, 12.0, cpu_threads(args.cpu_threads))
+    sm_mhz = clk.get("sm_mhz") if clk else None
+    clock_peak = clock_scaled_int8_peak(sm_mhz)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (fp32 dequant, bf16 out)",
-        "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32, X~N(0,1) bf16)",
-        "config": {"workload": wk.name, "tokens": r.T,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (fp32 dequant, bf16 out)"
+        + ("; backward bf16/fp16 x -> fp32" if wk.mode == "train" else ""),
+        "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32, X~N(0,1) bf16"
+                + (", dY~N(0,1) bf16)" if wk.mode == "train" else ")"),
+        "config": workload_config(wk, world),
+        "timing": {"l2": "flushed between timed steps (512 MiB write outside the events)",
                    "launch": "one CUDA graph per step; each N:M pass on its own stream, packing and "
-                             "activation quantisation of independent linears forked onto side streams",
-                   "linears": [f"{l.name}:{l.d_in}->{l.d_out}" for l in wk.linears],
-                   "patterns": [f"{n}:{m}" for n, m in wk.patterns], "mode": wk.mode,
-                   "l2": "flushed between timed steps (512 MiB write outside the events)",
-                   "parallelism": f"independent replicas x{world}",
-                   "dense_equivalent_tops": round(value * dense_factor(wk), 3),
-                   "forward_formats": r.formats_used(),
-                   **({"remask_statistics": r.stats_summary()} if wk.mode == "train" else {})},
+                             "activation quantisation of independent linears forked onto side streams"},
+        "details": {"dense_equivalent_tops": round(value * dense_factor(wk), 3),
+                    "forward_formats": r.formats_used(),
+                    **({"remask_statistics": r.stats_summary()} if wk.mode == "train" else {})},
         "roofline": {"kernel": gemm_kernel_names(r, sbl), "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": round(int8_peak, 1), "unit": "TOPS",
                      "frac": round(achieved / int8_peak, 4),
                      "peak_note": f"int8 dense = 2 x {pk['source']} bf16 {peak_kind} {bf16_peak} TFLOP/s "
-                                  f"({'step longer' if long_step else 'step shorter'} than {LONG_STEP_MS} ms)",
+                                  f"({'step longer' if long_step else 'step shorter'} than {LONG_STEP_MS} ms); "
+                                  "the targets are judged on this fraction",
+                     "clock_scaled_peak": round(clock_peak, 1) if clock_peak else None,
+                     "clock_scaled_frac": round(achieved / clock_peak, 4) if clock_peak else None,
+                     "clock_scaled_note": f"{INT8_OPS_PER_CLOCK_PER_SM} int8 ops/clock/SM x {B200_SMS} SMs x the "
+                                          "median SM clock sampled during the timed region",
                      "traffic": stored_traffic(wk.name),
                      "traffic_note": "mean DRAM read+write bytes per GEMM launch of the step (ncu capture in "
                                      "profiles/roofline_traffic.json; null when absent or stale)"},
@@ -615,6 +734,11 @@ def run_ours(args, wk):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    del r, g, g_k, flush
+    torch.cuda.empty_cache()
+    if not args.no_decode and wk.mode != "decode":
+        line["decode"] = measure_decode(args, wl.WORKLOADS["bitnet2b_decode"], sbl, torch, dist, world, rank,
+                                        device, pk)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -629,10 +753,20 @@ def dense_factor(wk):
 
 # ----------------------------------------------------------------- decode
 
-def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
-    """Decode GEMV from pre-packed 2:4 PK2 weights.  R distinct weight copies
-    (> 4x L2 in total) are launched back to back in a CUDA graph, so every
-    launch streams its weights from HBM."""
+def measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
+    """Decode GEMV from pre-packed 2:4 PK2 weights over R distinct weight
+    copies per linear (> 4x L2 in total), so every layer streams its weights
+    from HBM.  Per token count, three ways of running the same layers:
+      batch  the step: sbl_quantize_act of each linear's input, then ONE
+             sbl_forward_batch launch over every copy of both linears (the
+             persistent streaming GEMV); 'batch_gemv' times that launch alone
+             (the roofline kernel);
+      chain  one sbl_forward_batch launch over a chain up_0, down_0, up_1, ...
+             in which every layer quantises the previous layer's bf16 output
+             in the kernel (a dependent multi-layer decode);
+      launch one sbl_forward (PK2 decode kernel) launch per copy, in a CUDA
+             graph (the per-layer launch path, for comparison).
+    Returns the decode measurement as a dict (the keys of a bench line)."""
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 128 << 20)
     clocks = ClockSampler(str(getattr(props, "uuid", "")) or None)
@@ -640,43 +774,73 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
     windows = []
     results = {}
     n, m = wk.patterns[0]
+    wbytes = {}
+    for li, lin in enumerate(wk.linears):
+        dsc = sbl.desc(lin.d_out, lin.d_in, n, m)
+        wbytes[li] = lin.d_out * sbl.sbl_packed_row_bytes(dsc, sbl.SBL_FMT_PK2)
+    R = max(8, int(4 * l2 // min(wbytes.values())) + 1)
+    R = min(R, sbl.SBL_BATCH_MAX_LAYERS // len(wk.linears))
+    copies = {}
+    for li, lin in enumerate(wk.linears):
+        dsc = sbl.desc(lin.d_out, lin.d_in, n, m)
+        w = torch.from_numpy(wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed, layer=li)).to(device)
+        ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
+        copies[li] = (dsc, [])
+        for _ in range(R):
+            p = sbl.alloc_packed(dsc, sbl.SBL_FMT_PK2)
+            sbl.sbl_quantize_mask_pack(dsc, w, sbl.SBL_FMT_PK2, p, ws)
+            copies[li][1].append(p)
+        del w
+    torch.cuda.synchronize()
     for T in wk.tokens:
-        layers = []
+        io = []
         for li, lin in enumerate(wk.linears):
-            dsc = sbl.desc(lin.d_out, lin.d_in, n, m)
-            w = torch.from_numpy(wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed, layer=li)).to(device)
-            bytes_w = lin.d_out * sbl.sbl_packed_row_bytes(dsc, sbl.SBL_FMT_PK2)
-            R = max(8, int(4 * l2 // bytes_w) + 1)
-            ws = sbl.alloc_workspace(sbl.sbl_workspace_bytes(dsc, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK))
-            copies = []
-            for _ in range(R):
-                p = sbl.alloc_packed(dsc, sbl.SBL_FMT_PK2)
-                sbl.sbl_quantize_mask_pack(dsc, w, sbl.SBL_FMT_PK2, p, ws)
-                copies.append(p)
             x = torch.from_numpy(wl.activations(T, lin.d_in, seed=wk.seed, layer=li).view(np.int16)
                                  ).view(torch.bfloat16).to(device)
             q = torch.empty((T, lin.d_in), dtype=torch.int8, device=device)
-            d = torch.empty((T,), dtype=torch.float32, device=device)
-            y = torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=device)
-            layers.append((lin, dsc, copies, x, q, d, y, bytes_w))
-        torch.cuda.synchronize()
+            d = torch.empty((max(T, 4),), dtype=torch.float32, device=device)
+            ys = [torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=device) for _ in range(R)]
+            io.append((lin, x, q, d, ys))
+        entries = [sbl.batch_layer(copies[li][0], copies[li][1][r], io[li][4][r], io[li][2], io[li][3])
+                   for r in range(R) for li in range(len(wk.linears))]
+        batch = sbl.batch_array(entries)
+        # the chain: up_r, down_r, up_r+1, ... each from the previous layer's output
+        chain_entries, chain_y = [], []
+        for r in range(R):
+            for li, (lin, x, q, d, ys) in enumerate(io):
+                first = not chain_entries
+                y = torch.empty((T, lin.d_out), dtype=torch.bfloat16, device=device)
+                chain_y.append(y)
+                chain_entries.append(sbl.batch_layer(copies[li][0], copies[li][1][r], y, q if first else None,
+                                                     d if first else None, chained=not first))
+        chain = sbl.batch_array(chain_entries)
+        chain_ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(chain, len(chain_entries)))
         s = torch.cuda.Stream(device)
+
+        def enqueue(mode):
+            if mode in ("batch", "batch_gemv"):
+                if mode == "batch":
+                    for lin, x, q, d, ys in io:
+                        sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
+                sbl.sbl_forward_batch(batch, len(entries), T)
+            elif mode == "chain":
+                sbl.sbl_forward_batch(chain, len(chain_entries), T, chain_ws)
+            else:
+                for li, (lin, x, q, d, ys) in enumerate(io):
+                    for r, p in enumerate(copies[li][1]):
+                        sbl.sbl_forward(copies[li][0], q, d, T, p, sbl.SBL_FMT_PK2, ys[r])
         graphs = {}
-        for mode in ("gemv", "step"):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(s):
-                for lin, dsc, copies, x, q, d, y, _ in layers:  # warm outside capture
-                    sbl.sbl_linear_forward(dsc, x, T, copies[0], sbl.SBL_FMT_PK2, q, d, y)
-                    sbl.sbl_forward(dsc, q, d, T, copies[0], sbl.SBL_FMT_PK2, y)
-                torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            for lin, x, q, d, ys in io:
+                sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
+            for mode in ("batch", "batch_gemv", "chain", "launch"):
+                enqueue(mode)  # warm outside capture
+            torch.cuda.synchronize()
+            for mode in ("batch", "batch_gemv", "chain", "launch"):
+                g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=s):
-                    for lin, dsc, copies, x, q, d, y, _ in layers:
-                        for p in copies:
-                            if mode == "step":  # the layer from its bf16 input: Q_a + GEMV
-                                sbl.sbl_linear_forward(dsc, x, T, p, sbl.SBL_FMT_PK2, q, d, y)
-                            else:  # the GEMV alone from the int8 activations
-                                sbl.sbl_forward(dsc, q, d, T, p, sbl.SBL_FMT_PK2, y)
-            graphs[mode] = g
+                    enqueue(mode)
+                graphs[mode] = g
         res = {}
         for mode, g in graphs.items():
             for _ in range(max(3, args.warmup)):
@@ -692,81 +856,104 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
             torch.cuda.synchronize()
             windows.append((t_wall0, clocks.mark()))
             ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / args.steps
-            # launches: the fused decode kernel is one launch per linear when
-            # T K <= 4096, else the activation kernel and the decode kernel
-            launches = sum(len(c) * (1 if mode == "gemv" or T * lin.d_in <= 4096 else 2)
-                           for lin, _, c, *_ in layers)
-            # algorithmic bytes: the packed weights, bf16 Y and, for the GEMV
-            # alone, int8 Xq + d read; for the step, bf16 X read and Xq + d written
-            alg_bytes = sum(len(c) * (bw + T * lin.d_out * 2 + (T * lin.d_in + 4 * T if mode == "gemv"
-                                                                else 3 * T * lin.d_in + 8 * T))
-                            for lin, _, c, _, _, _, _, bw in layers)
-            res[mode] = {"ms_per_graph": ms, "launches": launches, "bytes_per_graph": alg_bytes,
-                         "gbs": whole_job_rate(alg_bytes, world, ms) / 1e9}
+            per_layer = [(lin.d_out * lin.d_in / 4, lin) for lin, *_ in io]
+            if mode == "chain":
+                # weights, the bf16 input read (first layer: int8 + scales) and output written
+                alg = sum(wb + 2 * T * lin.d_in + 2 * T * lin.d_out for wb, lin in per_layer) * R
+                launches = 1
+            else:
+                alg = sum(wb + T * lin.d_in + 4 * T + 2 * T * lin.d_out for wb, lin in per_layer) * R
+                launches = len(entries) if mode == "launch" else 1
+                if mode == "batch":
+                    alg += sum(3 * T * lin.d_in + 8 * T for _, lin in per_layer)
+                    launches += len(io)
+            res[mode] = {"ms_per_graph": ms, "launches": launches, "bytes_per_graph": alg,
+                         "gbs": whole_job_rate(alg, world, ms) / 1e9}
         # end to end through the public API: every step copies the tokens'
         # activations in from pinned host memory and the outputs back
-        hx = [torch.empty(x.shape, dtype=torch.bfloat16).pin_memory() for _, _, _, x, *_ in layers]
-        hy = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for *_, y, _ in layers]
-        for h, (_, _, _, x, *_) in zip(hx, layers):
+        hx = [torch.empty(x.shape, dtype=torch.bfloat16).pin_memory() for _, x, *_ in io]
+        hy = [torch.empty(ys[0].shape, dtype=torch.bfloat16).pin_memory() for *_, ys in io]
+        for h, (_, x, *_) in zip(hx, io):
             h.copy_(x)
         e_steps = max(2, min(args.steps, 10))
         barrier(dist, world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(e_steps):
-            for (lin, dsc, copies, x, q, d, y, _), h_in, h_out in zip(layers, hx, hy):
+            for (lin, x, q, d, ys), h_in in zip(io, hx):
                 x.copy_(h_in, non_blocking=True)
-                sbl.sbl_linear_forward(dsc, x, T, copies[0], sbl.SBL_FMT_PK2, q, d, y)
-                h_out.copy_(y, non_blocking=True)
+                sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
+            sbl.sbl_forward_batch(batch, len(entries), T)
+            for (lin, x, q, d, ys), h_out in zip(io, hy):
+                h_out.copy_(ys[0], non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, world, device) / e_steps
-        e_bytes = sum(bw + T * lin.d_in * 2 + T * lin.d_out * 2 + 4 * T for lin, _, _, _, _, _, _, bw in layers)
+        e_bytes = res["batch"]["bytes_per_graph"]
         res["e2e"] = {"ms_per_step": e_ms, "gbs": whole_job_rate(e_bytes, world, e_ms) / 1e9,
                       "h2d_bytes_per_step": sum(h.numel() * 2 for h in hx),
                       "d2h_bytes_per_step": sum(h.numel() * 2 for h in hy)}
+        # self-check: the batched launch equals the per-layer launches bit for bit
+        graphs["launch"].replay()
+        torch.cuda.synchronize()
+        ref = [y.clone() for *_, ys in io for y in ys]
+        graphs["batch"].replay()
+        torch.cuda.synchronize()
+        if not all(torch.equal(a.view(torch.int16), b.view(torch.int16))
+                   for a, b in zip(ref, [y for *_, ys in io for y in ys])):
+            raise SystemExit("decode self-check failed: the batched and per-layer launches differ")
         results[T] = res
+        del graphs
     Tm = wk.tokens[-1]
     clk = clocks.stop(*windows)
-    value = statistics.mean(results[T]["step"]["gbs"] for T in wk.tokens)
-    # the roofline kernel is the decode GEMV (the 'gemv' graphs launch it
-    # alone): its algorithmic bytes over its time, all token counts together
-    gemv_bytes = sum(results[T]["gemv"]["bytes_per_graph"] for T in wk.tokens)
-    gemv_ms = sum(results[T]["gemv"]["ms_per_graph"] for T in wk.tokens)
+    value = statistics.mean(results[T]["batch"]["gbs"] for T in wk.tokens)
+    # the roofline kernel is the streaming GEMV (the 'batch_gemv' graphs launch
+    # it alone): its algorithmic bytes over its time, all token counts together
+    gemv_bytes = sum(results[T]["batch_gemv"]["bytes_per_graph"] for T in wk.tokens)
+    gemv_ms = sum(results[T]["batch_gemv"]["ms_per_graph"] for T in wk.tokens)
     gemv = gemv_bytes * world / (gemv_ms * 1e-3) / 1e9
     e2e = statistics.mean(results[T]["e2e"]["gbs"] for T in wk.tokens)
     err = sbl.sbl_device_error()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_decode(wk)
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(results[Tm]["step"]["ms_per_graph"], 4),
+        cpu = cpu_baselines(wk, 10.0, cpu_threads(args.cpu_threads))
+    out = {
+        "metric": "decode GEMV GB/s (BitNet-2B linears, 2:4, pre-packed 2-bit)", "value": round(value, 1),
+        "unit": "GB/s", "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(results[Tm]["batch"]["ms_per_graph"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "2-bit ternary x int8 -> int32",
         "data": "synthetic (seeded numpy PCG64; W~N(0,0.02) fp32 packed once to 2:4 PK2, X~N(0,1) bf16)",
-        "config": {"workload": wk.name, "tokens": wk.tokens,
-                   "step": "per token count: sbl_linear_forward of each linear (act quant fused into the "
-                           "decode GEMV, one launch, when T K <= 4096; else the activation kernel and the "
-                           "GEMV), over rotating weight copies; 'gemv' is the GEMV alone from int8 activations",
-                   "per_token_count": {str(T): results[T] for T in wk.tokens},
-                   "l2": "inputs larger than L2: rotating weight copies > 4x L2 inside one CUDA graph",
-                   "parallelism": f"independent replicas x{world}"},
-        "roofline": {"kernel": "decode_kernel (PK2 stream, mma.sync u8 x s8), both linears, T = 1, 4, 16",
+        "config": workload_config(wk, world),
+        "timing": {"step": f"per token count: sbl_quantize_act of each linear's input, then one "
+                           f"sbl_forward_batch launch over {R} weight copies of each linear (the persistent "
+                           "streaming GEMV); value = the mean GB/s over T = 1, 4, 16",
+                   "l2": f"inputs larger than L2: {R} rotating weight copies per linear, > 4x L2"},
+        "per_token_count": {str(T): results[T] for T in wk.tokens},
+        "roofline": {"kernel": "gemv_stream_kernel (persistent; PK2 rows bulk-copied into a shared-memory ring; "
+                               "mma.sync u8 x s8), both linears, T = 1, 4, 16",
                      "bound": "hbm", "achieved": round(gemv, 1),
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gemv / pk["hbm_gbs"], 4),
+                     "peak_note": f"{pk['source']} HBM copy bandwidth",
                      "traffic": stored_traffic(wk.name),
-                     "traffic_note": "mean DRAM read+write bytes per decode launch over both linears and "
-                                     "T = 1, 4, 16, each launch after an L2 flush (ncu captures in "
-                                     "profiles/roofline_traffic.json; null when absent or stale)"},
+                     "traffic_note": "DRAM read+write bytes per streaming-GEMV launch scaled to the bench's launch "
+                                     "(ncu capture in profiles/roofline_traffic.json; null when absent or stale)"},
         "e2e": {"value": round(e2e, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": results[Tm]["e2e"]["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": results[Tm]["e2e"]["d2h_bytes_per_step"]},
-        "gpu_launches": sum(results[T]["step"]["launches"] for T in wk.tokens) * args.steps,
+        "gpu_launches": sum(results[T]["batch"]["launches"] for T in wk.tokens) * args.steps,
         "clocks": clk,
         "device_error": err,
     }
     if cpu is not None:
-        line["cpu_baseline"] = cpu
+        out["cpu_baseline"] = cpu
+    return out
+
+
+def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
+    """The decode workload alone, as the bench line."""
+    line = {"metric": METRIC, "n_gpus": world}
+    line.update(measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk))
+    line["metric"] = METRIC
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -775,99 +962,184 @@ def run_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
 
 # ------------------------------------------------------------ CPU baseline
 
-def cpu_baseline(wk, budget_s=12.0):
-    """Time the oracle, as it stands (single thread, plain C), on a bounded
-    sample of the workload: the full weight packing of the first linear, and
-    its activation quantisation, GEMM and dequantisation (training: also the
-    fp64 Dual-STE backward, dX and dW) on the first T_s tokens of the step,
-    T_s chosen from a short probe so that the sample takes about `budget_s`
-    seconds.  The packing is charged pro rata, T_s / T of it, since one step
-    packs once for all T tokens."""
+def _oracle_pack(w, n, m, pool, threads):
+    """The oracle's weight side: gamma over all of W (one fp64 tree), then
+    ternarisation, N:M mask and masking of disjoint row slices in parallel."""
     import oracle
+    from functools import partial
+    g = oracle.gamma(w)
+
+    def job(a, b):
+        ws = w[a:b]
+        return oracle.apply_mask(oracle.ternarize(ws, g), oracle.nm_mask(ws, n, m))
+    parts = run_parallel(pool, [partial(job, a, b) for a, b in slices(w.shape[0], threads)])
+    return g, np.concatenate(parts)
+
+
+def _oracle_forward(x, weff, g, pool, threads):
+    """Act quant, GEMM and dequantisation of disjoint token slices."""
+    import oracle
+    from functools import partial
+
+    def job(a, b):
+        q, d = oracle.quantize_act(x[a:b])
+        oracle.dequant(oracle.gemm_acc(q, weff), g, d)
+        return q, d
+    res = run_parallel(pool, [partial(job, a, b) for a, b in slices(x.shape[0], threads)])
+    return np.concatenate([r[0] for r in res]), np.concatenate([r[1] for r in res])
+
+
+def _oracle_backward(dy, weff, g, q, d, pool, threads):
+    """The fp64 Dual-STE backward: dX over disjoint token slices, dW over
+    disjoint output-row slices."""
+    import oracle
+    from functools import partial
+
+    def dx_job(a, b):
+        oracle.backward(dy[a:b], weff, g, q[a:b], d[a:b], want_dw=False)
+
+    def dw_job(a, b):
+        oracle.backward(np.ascontiguousarray(dy[:, a:b]), weff[a:b], g, q, d, want_dx=False)
+    run_parallel(pool, [partial(dx_job, a, b) for a, b in slices(dy.shape[0], threads)] +
+                 [partial(dw_job, a, b) for a, b in slices(weff.shape[0], threads)])
+
+
+def _pool(threads):
+    from concurrent.futures import ThreadPoolExecutor
+    return ThreadPoolExecutor(max_workers=threads) if threads > 1 else None
+
+
+def cpu_baseline(wk, budget_s=12.0, threads=1):
+    """Time the oracle, as it stands (plain C, each output computed by the
+    same loop), on a bounded sample of the workload, on `threads` host cores:
+    disjoint slices of the outputs go to the threads (ctypes releases the GIL
+    during each C call).  The sample is the full weight packing of the first
+    linear and its activation quantisation, GEMM and dequantisation
+    (training: also the fp64 Dual-STE backward, dX and dW) on the first T_s
+    tokens of the step, T_s chosen from a short probe so that the sample takes
+    about `budget_s` seconds.  The packing is charged pro rata, T_s / T of it,
+    since one step packs once for all T tokens."""
     lin = wk.linears[0]
     n, m = wk.patterns[0]
     T = wk.tokens[-1]
     train = wk.mode == "train"
     w = wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed)
-    t0 = time.perf_counter()
-    layer = oracle.Layer(w, n, m)
-    t_pack = time.perf_counter() - t0
-
-    def run(ts):
-        # the first ts rows of the step's inputs (row-major draws: a prefix
-        # of the full-size draw)
-        x = wl.activations(ts, lin.d_in, seed=wk.seed)
-        dy = wl.output_grad(ts, lin.d_out, seed=wk.seed) if train else None
+    pool = _pool(threads)
+    try:
         t0 = time.perf_counter()
-        q, d, _, _, _ = layer.forward(x)
-        if train:
-            oracle.backward(dy, layer.weff, layer.gamma, q, d)
-        return time.perf_counter() - t0
+        g, weff = _oracle_pack(w, n, m, pool, threads)
+        t_pack = time.perf_counter() - t0
 
-    probe = 4 if train else 8
-    t_probe = run(probe)
-    ts = int(max(1, min(T, probe * max(1.0, (budget_s - t_pack - t_probe) / max(t_probe, 1e-6)))))
-    t_run = run(ts)
+        def run(ts):
+            # the first ts rows of the step's inputs (row-major draws: a
+            # prefix of the full-size draw)
+            x = wl.activations(ts, lin.d_in, seed=wk.seed)
+            dy = wl.output_grad(ts, lin.d_out, seed=wk.seed) if train else None
+            t0 = time.perf_counter()
+            q, d = _oracle_forward(x, weff, g, pool, threads)
+            if train:
+                _oracle_backward(dy, weff, g, q, d, pool, threads)
+            return time.perf_counter() - t0
+
+        probe = max(4 if train else 8, threads)
+        t_probe = run(probe)
+        ts = int(max(1, min(T, probe * max(1.0, (budget_s - t_pack - t_probe) / max(t_probe, 1e-6)))))
+        t_run = run(ts)
+    finally:
+        if pool is not None:
+            pool.shutdown()
     per_token = 2.0 * lin.d_out * lin.d_in * n / m + (4.0 * lin.d_out * lin.d_in if train else 0.0)
-    value = per_token * ts / (t_run + t_pack * ts / T) / 1e12
+    seconds = t_run + t_pack * ts / T
+    value = per_token * ts / seconds / 1e12
     what = "act quant + GEMM + dequant + fp64 Dual-STE backward (dX, dW)" if train else "act quant + GEMM + dequant"
-    return {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
+    return {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle", "sampled_tokens": ts,
+            "seconds": round(seconds, 3), "sampled_ops": per_token * ts,
             "sample": f"{lin.name} {lin.d_in}->{lin.d_out} at {n}:{m}: full pack (charged pro rata "
-                      f"{ts}/{T} tokens) + {what} on {ts} tokens; pack {t_pack:.2f}s, rest {t_run:.2f}s"}
+                      f"{ts}/{T} tokens) + {what} on {ts} tokens, {threads} thread(s) over disjoint output "
+                      f"slices; pack {t_pack:.2f}s, rest {t_run:.2f}s"}
 
 
-def cpu_baseline_decode(wk, budget_s=10.0):
-    """The oracle's GEMV (GEMM + dequantisation from W_eff, T tokens of the
-    first linear) timed on one host core, in the decode metric's unit:
+def cpu_baseline_decode(wk, budget_s=10.0, threads=1):
+    """The oracle's GEMV (act quant, then GEMM + dequantisation from W_eff for
+    disjoint output-row slices on `threads` cores; T tokens of the first
+    linear) repeated for about budget_s, in the decode metric's unit:
     algorithmic bytes (2-bit weights + bf16 X + bf16 Y + scales) per second."""
     import oracle
+    from functools import partial
     lin = wk.linears[0]
     n, m = wk.patterns[0]
     T = wk.tokens[-1]
     layer = oracle.Layer(wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed), n, m)
     x = wl.activations(T, lin.d_in, seed=wk.seed)
+    pool = _pool(threads)
+
+    def job(q, d, a, b):
+        oracle.dequant(oracle.gemm_acc(q, layer.weff[a:b]), layer.gamma, d)
     reps, t = 0, 0.0
-    t0 = time.perf_counter()
-    while t < budget_s and reps < 1000:
-        layer.forward(x)
-        reps += 1
-        t = time.perf_counter() - t0
+    try:
+        t0 = time.perf_counter()
+        while t < budget_s and reps < 100000:
+            q, d = oracle.quantize_act(x)
+            run_parallel(pool, [partial(job, q, d, a, b) for a, b in slices(lin.d_out, threads)])
+            reps += 1
+            t = time.perf_counter() - t0
+    finally:
+        if pool is not None:
+            pool.shutdown()
     alg = lin.d_out * lin.d_in / 4 + T * lin.d_in * 2 + T * lin.d_out * 2 + 4 * T
-    return {"value": alg * reps / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+    return {"value": alg * reps / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": round(t, 3), "sampled_bytes": alg * reps,
             "sample": f"{lin.name} {lin.d_in}->{lin.d_out} at {n}:{m}, T={T}: {reps} GEMVs "
-                      f"(act quant + GEMM + dequant from W_eff) in {t:.1f}s"}
+                      f"(act quant + GEMM + dequant from W_eff, {threads} thread(s) over disjoint output "
+                      f"rows) in {t:.1f}s"}
+
+
+def cpu_baselines(wk, budget_s, threads):
+    """The oracle on every allowed core, with the single-thread figure beside it."""
+    fn = cpu_baseline_decode if wk.mode == "decode" else cpu_baseline
+    multi = fn(wk, budget_s, threads)
+    if threads > 1:
+        one = fn(wk, budget_s / 2, 1)
+        multi["single_thread"] = {k: one[k] for k in ("value", "unit", "cores", "sample")}
+    return multi
 
 
 def run_reference(args, wk):
     """The oracle arm: the plain-C oracle timed on the host cores, in our
-    arm's metric and unit (TOPS, or GB/s for decode).  Under torchrun rank 0
-    alone runs and prints; the other ranks exit without work."""
+    arm's metric and unit (TOPS, or GB/s for decode), on the same workload
+    configuration.  Each step is a bounded sample of the workload (so the run
+    ends within minutes); `value` is the sample's work over its time and
+    `ms_per_step` the time one sample took.  Under torchrun rank 0 alone runs
+    and prints; the other ranks exit without work."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    threads = cpu_threads(args.cpu_threads)
     budget = args.ref_step_seconds or max(2.0, 120.0 / max(1, args.steps + args.warmup))
     res = []
+    fn = cpu_baseline_decode if wk.mode == "decode" else cpu_baseline
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline_decode(wk, budget) if wk.mode == "decode" else cpu_baseline(wk, budget_s=budget)
+        r = fn(wk, budget, threads)
         if i >= args.warmup:
             res.append(r)
-    value = statistics.mean(r["value"] for r in res)
-    unit = res[-1]["unit"]
-    # one whole step of the workload at the sample's rate
+    seconds = sum(r["seconds"] for r in res)
     if wk.mode == "decode":
-        step_units = sum(decode_step_bytes(wk, T) for T in wk.tokens) / 1e9
+        value = sum(r["sampled_bytes"] for r in res) / seconds / 1e9
     else:
-        step_units = algorithmic_ops(wk, wk.tokens[-1]) / 1e12
+        value = sum(r["sampled_ops"] for r in res) / seconds / 1e12
+    unit = res[-1]["unit"]
     dtype = "int8 x ternary -> int64 (plain C)" + ("; backward f64" if wk.mode == "train" else "")
+    cpu = {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": res[-1]["sample"]}
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(step_units / value * 1e3, 1),
-        "ms_per_step_basis": "one whole step's algorithmic work at the sampled rate",
+        "warmup": args.warmup, "ms_per_step": round(seconds / len(res) * 1e3, 1),
+        "ms_per_step_basis": "wall time of one step's bounded sample (the work the value counts)",
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-        "config": {"workload": wk.name}, "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": res[-1]["sample"]},
+        "config": workload_config(wk, world), "impl": "reference",
+        "sampled_tokens": res[-1].get("sampled_tokens", wk.tokens[-1]),
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -877,10 +1149,9 @@ def main():
     args = parse()
     wk = wl.WORKLOADS[args.workload]
     if args.record_traffic:
-        # the roofline kernels: the decode GEMV from PK2 codes (the last two
-        # template flags 0: not the fused, not the T24 variant), or the int8
-        # dense and 2:4 sparse forward GEMMs
-        regex = r"decode_kernel<\d+, \d+, \d+, 0, 0>" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
+        # the roofline kernels: the persistent streaming decode GEMV, or the
+        # int8 dense and 2:4 sparse forward GEMMs
+        regex = r"gemv_stream_kernel" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
         print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command)))
         return
     if args.impl == "reference":
