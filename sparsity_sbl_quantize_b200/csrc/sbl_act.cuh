@@ -22,16 +22,26 @@ constexpr int kActMaxChunks = 8;  // 16-byte chunks (8 bf16) per thread
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Round-half-even of |v| < 2^22 by the fp32 adder: fl(v + 1.5 2^23) has ulp 1
+// and lies in [2^23, 2^24), so its bits are 0x4B400000 + rint(v), and the low
+// byte is rint(v) as an int8 bit pattern when rint(v) is in [-128, 127].  The
+// quantiser's products satisfy |fl32(x fl32(127 / a))| <= 127 (1 + 2^-24) for
+// |x| <= a, so rint lies in [-127, 127] and the clamp to [-128, 127] never
+// binds; one FADD replaces the float-to-int conversion.
+__device__ __forceinline__ uint32_t rne_byte(float v)
+{
+    return __float_as_uint(__fadd_rn(v, 12582912.0f));
+}
+
+// Four int8 codes sat8(rint(fl32(x r))) packed LSB first.
 __device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float r)
 {
-    int q[4] = {__float2int_rn(__fmul_rn(a, r)), __float2int_rn(__fmul_rn(b, r)),
-                __float2int_rn(__fmul_rn(c, r)), __float2int_rn(__fmul_rn(d, r))};
-    uint32_t w = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int v = min(127, max(-128, q[i]));
-        w |= (static_cast<uint32_t>(v) & 0xffu) << (8 * i);
-    }
+    const uint32_t q0 = rne_byte(__fmul_rn(a, r)), q1 = rne_byte(__fmul_rn(b, r));
+    const uint32_t q2 = rne_byte(__fmul_rn(c, r)), q3 = rne_byte(__fmul_rn(d, r));
+    uint32_t lo, hi, w;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(q0), "r"(q1));
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(q2), "r"(q3));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(w) : "r"(lo), "r"(hi));
     return w;
 }
 
