@@ -804,6 +804,7 @@ def measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
         entries = [sbl.batch_layer(copies[li][0], copies[li][1][r], io[li][4][r], io[li][2], io[li][3])
                    for r in range(R) for li in range(len(wk.linears))]
         batch = sbl.batch_array(entries)
+        batch_ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(batch, len(entries), T))
         # the chain: up_r, down_r, up_r+1, ... each from the previous layer's output
         chain_entries, chain_y = [], []
         for r in range(R):
@@ -814,7 +815,7 @@ def measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
                 chain_entries.append(sbl.batch_layer(copies[li][0], copies[li][1][r], y, q if first else None,
                                                      d if first else None, chained=not first))
         chain = sbl.batch_array(chain_entries)
-        chain_ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(chain, len(chain_entries)))
+        chain_ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(chain, len(chain_entries), T))
         s = torch.cuda.Stream(device)
 
         def enqueue(mode):
@@ -822,7 +823,7 @@ def measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
                 if mode == "batch":
                     for lin, x, q, d, ys in io:
                         sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
-                sbl.sbl_forward_batch(batch, len(entries), T)
+                sbl.sbl_forward_batch(batch, len(entries), T, batch_ws)
             elif mode == "chain":
                 sbl.sbl_forward_batch(chain, len(chain_entries), T, chain_ws)
             else:
@@ -883,7 +884,7 @@ def measure_decode(args, wk, sbl, torch, dist, world, rank, device, pk):
             for (lin, x, q, d, ys), h_in in zip(io, hx):
                 x.copy_(h_in, non_blocking=True)
                 sbl.sbl_quantize_act(x, T, lin.d_in, q, d)
-            sbl.sbl_forward_batch(batch, len(entries), T)
+            sbl.sbl_forward_batch(batch, len(entries), T, batch_ws)
             for (lin, x, q, d, ys), h_out in zip(io, hy):
                 h_out.copy_(ys[0], non_blocking=True)
         e1.record()

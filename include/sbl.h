@@ -411,9 +411,13 @@ typedef struct {
 
 #define SBL_BATCH_MAX_LAYERS 256
 
-/* Workspace bytes of sbl_forward_batch for `count` layers: 0 when no layer
- * takes its input from the previous one, else 128 per layer. */
-size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count);
+/* Workspace bytes of sbl_forward_batch for these `count` layers at T tokens:
+ * 128 per layer when some layer takes its input from the previous one, plus,
+ * per distinct unchained input (the same xq pointer and in_features), T K
+ * bytes rounded up to 256 and 256 more (the input as the MMA loop reads it:
+ * every 16-byte group 4 x 4 transposed, and its per-token sums).  0 for
+ * invalid arguments. */
+size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count, int32_t T);
 
 /* The decode forward of `count` layers (1 <= count <= SBL_BATCH_MAX_LAYERS)
  * at T tokens (1 <= T <= 16) in ONE persistent launch: one CTA per SM
@@ -426,10 +430,13 @@ size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t 
  * in the workspace; the wait is bounded and records SBL_DEVICE_ERROR bits on
  * expiry), then quantises that output in-kernel; chained batches are launched
  * cooperatively (every CTA resident) and do not let the next kernel start
- * early.  workspace: sbl_forward_batch_workspace_bytes bytes (NULL when 0),
- * 256-byte aligned; the library zeroes it (one memset) before the launch.
+ * early.  Each distinct unchained input is first rearranged once into the
+ * workspace by a small kernel (its groups transposed, its token sums).
+ * workspace: sbl_forward_batch_workspace_bytes bytes, 256-byte aligned; the
+ * library zeroes the completion words (one memset) before the launch.
  * Unchained batches are launched with programmatic dependent launch like
  * sbl_forward (the weights are read before the wait on the previous kernel).
+ * Two launches (one when every layer after the first is chained).
  * Errors: SBL_ERR_SHAPE for count, T or a descriptor out of range;
  * SBL_ERR_UNSUPPORTED for in_features not a multiple of 64 or above 14336;
  * SBL_ERR_INVALID_ARG for a null pointer a layer needs, a chained first

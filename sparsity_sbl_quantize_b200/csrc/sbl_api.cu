@@ -1020,7 +1020,7 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
 
 // ------------------------------------------------------ batched decode --
 static_assert(SBL_BATCH_MAX_LAYERS <= kGvMaxProblems, "the launch parameters hold every layer of a batch");
-static_assert(sizeof(GvArgs) <= 32000, "kernel parameters are limited to 32764 bytes");
+static_assert(sizeof(GvArgs) <= 32000 && sizeof(GvPrepArgs) <= 32000, "kernel parameters are limited to 32764 bytes");
 constexpr int32_t kGvMaxK = 4 * kGvStageBytes / 16;  // 16-row items of K / 4 bytes per row fill a stage
 
 static bool batch_has_chain(const sbl_batch_layer *layers, int32_t count)
@@ -1030,13 +1030,40 @@ static bool batch_has_chain(const sbl_batch_layer *layers, int32_t count)
     return false;
 }
 
+// Index of the first unchained layer with the same input (activations and
+// width) as layer i, so that each distinct input is prepared once.
+static int32_t batch_input_owner(const sbl_batch_layer *layers, int32_t i)
+{
+    for (int32_t j = 0; j < i; ++j)
+        if (!layers[j].input_is_previous_output && layers[j].xq == layers[i].xq &&
+            layers[j].desc.in_features == layers[i].desc.in_features)
+            return j;
+    return i;
+}
+
+// Workspace layout: [completion words, 128 bytes per layer, when chained]
+// [per distinct unchained input: T K bytes of prepared activations rounded to
+// 256, then 256 bytes of column sums].
+static int64_t batch_workspace_layout(const sbl_batch_layer *layers, int32_t count, int32_t T, int64_t *offsets)
+{
+    int64_t off = batch_has_chain(layers, count) ? round_up(static_cast<int64_t>(count) * kGvSyncWords * 4, 256) : 0;
+    for (int32_t i = 0; i < count; ++i) {
+        if (offsets) offsets[i] = -1;
+        if (layers[i].input_is_previous_output || batch_input_owner(layers, i) != i) continue;
+        if (offsets) offsets[i] = off;
+        off += round_up(static_cast<int64_t>(T) * layers[i].desc.in_features, 256) + 256;
+    }
+    return off;
+}
+
 extern "C" {
 
-size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count)
+size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t count, int32_t T)
 {
-    if (!layers || count < 1 || count > SBL_BATCH_MAX_LAYERS) return 0;
-    if (!batch_has_chain(layers, count)) return 0;
-    return static_cast<size_t>(round_up(static_cast<int64_t>(count) * kGvSyncWords * 4, 256));
+    if (!layers || count < 1 || count > SBL_BATCH_MAX_LAYERS || T < 1 || T > kDecMaxTokens) return 0;
+    for (int32_t i = 0; i < count; ++i)
+        if (check_desc(&layers[i].desc) != SBL_OK) return 0;
+    return static_cast<size_t>(batch_workspace_layout(layers, count, T, nullptr));
 }
 
 sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32_t T, void *workspace,
@@ -1044,10 +1071,14 @@ sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32
 {
     if (!layers) return SBL_ERR_INVALID_ARG;
     if (count < 1 || count > SBL_BATCH_MAX_LAYERS || T < 1 || T > kDecMaxTokens) return SBL_ERR_SHAPE;
-    static GvArgs a;  // 18 KB of launch parameters, filled under the lock below
+    // launch parameters (18 KB and 9 KB), filled under the lock below
+    static GvArgs a;
+    static GvPrepArgs prep;
+    static int64_t offsets[SBL_BATCH_MAX_LAYERS];
     static std::mutex batch_mutex;
     std::lock_guard<std::mutex> lock(batch_mutex);
     memset(&a, 0, sizeof(a));
+    memset(&prep, 0, sizeof(prep));
     int32_t items = 0;
     bool chain = false;
     for (int32_t i = 0; i < count; ++i) {
@@ -1069,12 +1100,12 @@ sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32
             if (!L.xq || !L.d) return SBL_ERR_INVALID_ARG;
             if (!aligned16(L.xq) || !aligned16(L.d)) return SBL_ERR_ALIGNMENT;
         }
-        const bool rows16 = 32 * (K / 4) > kGvStageBytes;
-        const int32_t item_rows = rows16 ? 16 : 32;
+        // as many 16-row tiles per item (4, 2 or 1) as one stage holds
+        const int32_t tiles = 64 * (K / 4) <= kGvStageBytes ? 4 : 32 * (K / 4) <= kGvStageBytes ? 2 : 1;
+        const int32_t item_rows = 16 * tiles;
         GvProblem &g = a.p[i];
         g.pk2 = L.pk2;
         g.gamma = L.gamma;
-        g.xq = ch ? nullptr : L.xq;
         g.d = ch ? nullptr : L.d;
         g.y = L.y;
         g.xq_out = ch ? L.xq_out : nullptr;
@@ -1082,26 +1113,56 @@ sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32
         g.O = O;
         g.K = K;
         g.item0 = items;
-        g.flags = (L.y_is_fp32 ? kGvOutFp32 : 0) | (ch ? kGvChained : 0) | (rows16 ? kGvRows16 : 0);
+        g.flags = (L.y_is_fp32 ? kGvOutFp32 : 0) | (ch ? kGvChained : 0) |
+                  ((tiles == 4 ? 2 : tiles == 2 ? 1 : 0) << kGvTilesShift);
         if (ch) a.p[i - 1].flags |= kGvPublish;
         items += (O + item_rows - 1) / item_rows;
     }
-    const size_t need = sbl_forward_batch_workspace_bytes(layers, count);
-    if (chain) {
-        if (!workspace || workspace_bytes < need) return SBL_ERR_WORKSPACE;
-        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    const int64_t need = batch_workspace_layout(layers, count, T, offsets);
+    if (!workspace || workspace_bytes < static_cast<size_t>(need)) return SBL_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SBL_ERR_ALIGNMENT;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    for (int32_t i = 0; i < count; ++i) {
+        if (layers[i].input_is_previous_output) continue;
+        const int32_t owner = batch_input_owner(layers, i);
+        const int64_t off = offsets[owner];
+        const int32_t K = layers[i].desc.in_features;
+        a.p[i].xt = reinterpret_cast<const int8_t *>(wsb + off);
+        a.p[i].colsum = reinterpret_cast<const int32_t *>(wsb + off + round_up(static_cast<int64_t>(T) * K, 256));
+        if (owner == i) {
+            GvPrepInput &in = prep.in[prep.inputs++];
+            in.xq = layers[i].xq;
+            in.xt = reinterpret_cast<int8_t *>(wsb + off);
+            in.colsum = reinterpret_cast<int32_t *>(wsb + off + round_up(static_cast<int64_t>(T) * K, 256));
+            in.K = K;
+        }
     }
+    prep.T = T;
     DeviceInfo *di = nullptr;
     sbl_status st = current_device(&di);
     if (st != SBL_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
     if (chain && cudaMemsetAsync(workspace, 0, static_cast<size_t>(count) * kGvSyncWords * 4, stream) != cudaSuccess)
         return SBL_ERR_CUDA;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    if (prep.inputs > 0) {
+        cudaLaunchConfig_t pc;
+        memset(&pc, 0, sizeof(pc));
+        pc.gridDim = dim3(static_cast<unsigned>(prep.inputs * T));
+        pc.blockDim = dim3(256);
+        pc.stream = stream;
+        pc.attrs = pdl;
+        pc.numAttrs = chain ? 0 : 1;
+        if (cudaLaunchKernelEx(&pc, gemv_prep_kernel, prep) != cudaSuccess) return SBL_ERR_CUDA;
+        if ((st = launch_status()) != SBL_OK) return st;
+    }
     a.count = count;
     a.T = T;
     a.items = items;
     a.early_trigger = chain ? 0 : 1;
-    a.sync = chain ? static_cast<uint32_t *>(workspace) : nullptr;
+    a.sync = chain ? reinterpret_cast<uint32_t *>(wsb) : nullptr;
     a.err = di->err;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
@@ -1115,8 +1176,7 @@ sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
     } else {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[0] = pdl[0];
     }
     cfg.attrs = attr;
     cfg.numAttrs = 1;

@@ -9,18 +9,24 @@
 // the BitNet b1.58 2B4T summary, "Inference Implementation: GPU").  What
 // differs is how the weights reach the SMs:
 //
-//  * one CTA per SM runs for the whole batch; its work items are 32-row
-//    blocks of the layers (16 rows when K is large), taken round-robin over
-//    the grid in batch order;
+//  * one CTA per SM runs for the whole batch; its work items are blocks of
+//    64, 32 or 16 rows of a layer (as many 16-row tiles as one 56 KB stage
+//    holds at that K), taken round-robin over the grid in batch order;
 //  * a producer warp streams each item's packed rows -- contiguous, since a
 //    PK2 row is exactly K / 4 bytes when K % 64 == 0 -- with ONE bulk copy
 //    (cp.async.bulk, evict-first in L2) into a ring of shared-memory stages,
 //    as far ahead as the ring allows and across layer boundaries: the
 //    weights never depend on the activations, so no launch gap or
 //    dependency stalls the stream;
-//  * eight consumer warps split the item's 256-weight K chunks, each doing
-//    both 16-row tiles per activation fragment, free the stage, and meet in
-//    shared memory (exact int32 partials) where 32 T threads dequantise;
+//  * sixteen consumer warps share an item: each owns one of its tiles and
+//    takes that tile's 128-weight K slices round-robin with the other warps
+//    of the tile (balanced for any K), frees the stage, and the warps meet in
+//    shared memory (exact int32 partials) where the item's T x rows outputs
+//    are summed and dequantised;
+//  * an unchained layer reads its int8 activations in a prepared layout
+//    (every 16-byte group 4 x 4 transposed, written once per launch by a
+//    small kernel together with the per-token sums that remove the +1 code
+//    bias), so the inner loop is loads, masks and MMAs only;
 //  * the 2-bit codes enter the MMA masked in place (one op per four weights)
 //    rather than shifted down: code position j of every byte keeps its
 //    factor 4^j, which a separate accumulator per j carries and an exact
@@ -42,11 +48,12 @@
 namespace sbl {
 
 constexpr int kGvMaxProblems = 256;
-constexpr int kGvWarps = 8;                       // consumer warps
+constexpr int kGvWarps = 16;                      // consumer warps
 constexpr int kGvThreads = 32 * (kGvWarps + 1);   // + the producer warp
-constexpr int kGvStageBytes = 56 * 1024;          // one item: 32 rows x K/4 for K <= 7168
+constexpr int kGvStageBytes = 56 * 1024;          // one item: 16 tiles x K/4 bytes per row
 constexpr int kGvStages = 3;
-constexpr int kGvPartStride = 36;                 // padded row count of a token's partials
+constexpr int kGvSlice = 128;                     // weights of a row in one K slice of a unit
+constexpr int kGvPartStride = 20;                 // padded row count (16 rows) of a token's partials
 constexpr int kGvSyncWords = 32;                  // per layer: [0] items done, [1 + t] max |y_t| bits
 constexpr int kGvSmemBytes = kGvStages * kGvStageBytes + 2 * kGvWarps * kDecMaxTokens * kGvPartStride * 4 +
                              2 * kGvWarps * kDecMaxTokens * 4 + 2 * kGvStages * 8;
@@ -55,13 +62,14 @@ enum : int32_t {
     kGvOutFp32 = 1,   // Y is fp32 (else bf16)
     kGvChained = 2,   // the input is the previous layer's bf16 output
     kGvPublish = 4,   // the next layer is chained on this one: publish max |y| and item counts
-    kGvRows16 = 8,    // items of 16 rows (large K), else 32
+    kGvTilesShift = 8,  // bits 8-10: log2 of the 16-row tiles per item (0, 1 or 2)
 };
 
 struct GvProblem {
     const uint8_t *pk2;  // PK2 codes [O, K / 4]
     const float *gamma;  // device scalar
-    const int8_t *xq;    // [T, K] int8 activations (unchained layers)
+    const int8_t *xt;    // unchained: the int8 activations [T, K], each 16-byte group 4 x 4 transposed
+    const int32_t *colsum;  // unchained: sum_k Xq[t, k] per token [T]
     const float *d;      // [T] token scales (unchained layers)
     void *y;             // [T, O] bf16 bits or fp32
     int8_t *xq_out;      // chained: Q_a of the input, stored by the CTA of item 0 (optional)
@@ -78,7 +86,7 @@ struct GvArgs {
     GvProblem p[kGvMaxProblems];
 };
 
-__device__ __forceinline__ void gv_consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void gv_consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kGvWarps * 32) : "memory"); }
 
 __device__ __forceinline__ uint4 ld_global_cg16(const void *p)
 {
@@ -97,21 +105,15 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
     return v;
 }
 
-// Lane (g, tg)'s 64 activations of token t at positions pos .. pos + 63 as
-// four 16-byte int8 groups.  Unchained: the int8 input.  Chained: the previous
-// layer's bf16 outputs, quantised with r = fl32(127 / a_t) (a_t == 0: zeros).
-__device__ __forceinline__ void gv_load_x(const GvProblem &P, const GvProblem &prev, bool chained, int t, int pos,
-                                          float r, uint4 (&x)[4])
+// Lane (g, tg)'s 32 activations of token t at positions pos .. pos + 31 of a
+// chained layer as two 16-byte int8 groups: the previous layer's bf16
+// outputs, quantised with r = fl32(127 / a_t) (a_t == 0: zeros).
+__device__ __forceinline__ void gv_load_x_chained(const GvProblem &prev, int K, int t, int pos, float r,
+                                                  uint4 (&x)[2])
 {
-    if (!chained) {
-        const int8_t *src = P.xq + static_cast<int64_t>(t) * P.K + pos;
+    const uint16_t *src = static_cast<const uint16_t *>(prev.y) + static_cast<int64_t>(t) * K + pos;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) x[q] = ld_global16(src + 16 * q);
-        return;
-    }
-    const uint16_t *src = static_cast<const uint16_t *>(prev.y) + static_cast<int64_t>(t) * P.K + pos;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
         const uint4 a = ld_global_cg16(src + 16 * q), b = ld_global_cg16(src + 16 * q + 8);
         if (r == 0.0f) {
             x[q] = make_uint4(0u, 0u, 0u, 0u);
@@ -124,12 +126,84 @@ __device__ __forceinline__ void gv_load_x(const GvProblem &P, const GvProblem &p
     }
 }
 
+// One K slice of one tile: four MMAs.  The lane's 8 weight bytes of a row are
+// words 0 and 1, word wi holding positions pos + 16 wi .. + 15 with byte e
+// the four positions pos + 16 wi + 4 e + j at bits 2 j.  Masking code position
+// j in place (one op) leaves byte e = c(pos + 16 wi + 4 e + j) 4^j, which
+// pairs with word j of the transposed activation group wi (byte e =
+// x(pos + 16 wi + 4 e + j)); the 4^j stays in that j's accumulator.
+template <int NT>
+__device__ __forceinline__ void gv_mma_slice(int32_t (&acc)[4][NT][4], uint2 wa, uint2 wb,
+                                             const uint4 (&xt)[NT][2])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t mj = 0x03030303u << (2 * j);
+        const uint32_t a0 = wa.x & mj, a1 = wb.x & mj, a2 = wa.y & mj, a3 = wb.y & mj;
+#pragma unroll
+        for (int b = 0; b < NT; ++b)
+            mma_u8s8(acc[j][b], a0, a1, a2, a3, word_of(xt[b][0], j), word_of(xt[b][1], j));
+    }
+}
+
+__device__ __forceinline__ uint2 ld_shared8(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+// The activations of the unchained layers in the layout the MMA loop reads:
+// one CTA per (distinct input, token) writes the token's row with every
+// 16-byte group 4 x 4 transposed (word j = bytes j, 4 + j, 8 + j, 12 + j) and
+// the row's sum.  Done once per input and launch instead of once per item.
+struct GvPrepInput {
+    const int8_t *xq;  // [T, K]
+    int8_t *xt;        // [T, K]
+    int32_t *colsum;   // [T]
+    int32_t K;
+};
+
+struct GvPrepArgs {
+    int32_t inputs, T;
+    GvPrepInput in[kGvMaxProblems];
+};
+
+__global__ void __launch_bounds__(256) gemv_prep_kernel(const __grid_constant__ GvPrepArgs a)
+{
+    __shared__ int32_t red[8];
+    const GvPrepInput &I = a.in[blockIdx.x / a.T];
+    const int t = blockIdx.x % a.T;
+    pdl_launch_dependents();
+    pdl_wait_prior();  // Xq may come from the previous kernel
+    const uint4 *src = reinterpret_cast<const uint4 *>(I.xq + static_cast<int64_t>(t) * I.K);
+    uint4 *dst = reinterpret_cast<uint4 *>(I.xt + static_cast<int64_t>(t) * I.K);
+    int s = 0;
+    for (int i = threadIdx.x; i < I.K / 16; i += blockDim.x) {
+        const uint4 v = ld_global16(src + i);
+        s = __dp4a(static_cast<int>(v.x), 0x01010101, s);
+        s = __dp4a(static_cast<int>(v.y), 0x01010101, s);
+        s = __dp4a(static_cast<int>(v.z), 0x01010101, s);
+        s = __dp4a(static_cast<int>(v.w), 0x01010101, s);
+        dst[i] = transpose4x4(v);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int total = 0;
+        for (int w = 0; w < 8; ++w) total += red[w];
+        I.colsum[t] = total;
+    }
+}
+
 // NT: n8 token blocks (T <= 8: 1, T <= 16: 2).
 template <int NT>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid_constant__ GvArgs args)
 {
     extern __shared__ __align__(128) uint8_t gv_smem[];
-    int32_t *part = reinterpret_cast<int32_t *>(gv_smem + kGvStages * kGvStageBytes);  // [2][warp][t][row]
+    int32_t *part = reinterpret_cast<int32_t *>(gv_smem + kGvStages * kGvStageBytes);  // [2][warp][t][row of tile]
     int32_t *csum = part + 2 * kGvWarps * kDecMaxTokens * kGvPartStride;                 // [2][warp][t]
     uint64_t *bars = reinterpret_cast<uint64_t *>(csum + 2 * kGvWarps * kDecMaxTokens);
     const uint32_t stage0 = smem_addr(gv_smem);
@@ -166,7 +240,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         for (int item = blockIdx.x; item < args.items; item += gridDim.x) {
             while (p + 1 < args.count && item >= args.p[p + 1].item0) ++p;
             const GvProblem &P = args.p[p];
-            const int item_rows = (P.flags & kGvRows16) ? 16 : 32;
+            const int item_rows = 16 << ((P.flags >> kGvTilesShift) & 7);
             const int r0 = (item - P.item0) * item_rows;
             const int rows = min(item_rows, P.O - r0);
             const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(P.K / 4);
@@ -212,11 +286,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
             if (s_fail[buf]) break;
             ready_p = p;
         }
-        const int item_rows = (P.flags & kGvRows16) ? 16 : 32;
+        const int tl2 = (P.flags >> kGvTilesShift) & 7;  // log2 of the tiles per item (0, 1, 2)
+        const int tiles = 1 << tl2;
+        const int item_rows = 16 * tiles;
         const int r0 = (item - P.item0) * item_rows;
         const int rows = min(item_rows, P.O - r0);
         const int K = P.K, kb = K / 4;
-        const int chunks = (K + kDecChunk - 1) / kDecChunk;
+        const int slices = (K + kGvSlice - 1) / kGvSlice;
+        const int tile = warp & (tiles - 1);           // this warp's tile, fixed for the item
+        const bool tile_in = 16 * tile < rows;         // warp-uniform
+        const int rA = 16 * tile + g, rB = rA + 8;     // the lane's two rows in the item
+        // the tile's warps take its K slices round-robin: slice (warp >> tl2) + i (16 >> tl2)
+        const int sl0 = warp >> tl2, sl_step = kGvWarps >> tl2;
         // this lane's tokens 8 b + g: the quantisation factor of a chained input
         float rq[NT];
 #pragma unroll
@@ -234,80 +315,86 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, args.err, kErrGemv)) && lane == 0)
             s_fail[buf] = 1;
         const uint32_t st = stage0 + static_cast<uint32_t>(stage * kGvStageBytes);
-        const bool tile1 = rows > 16;  // warp-uniform
-        // acc[u][j][b]: tile u, code position j (weights scaled by 4^j), token block b
-        int32_t acc[2][4][NT][4];
+        const uint32_t rowA = st + static_cast<uint32_t>(rA * kb), rowB = st + static_cast<uint32_t>(rB * kb);
+        const bool inA = rA < rows, inB = rB < rows;
+        // acc[j][b]: code position j (weights scaled by 4^j), token block b
+        int32_t acc[4][NT][4];
         uint32_t cs[NT];
 #pragma unroll
         for (int b = 0; b < NT; ++b) {
             cs[b] = 0u;
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[u][j][b][0] = acc[u][j][b][1] = acc[u][j][b][2] = acc[u][j][b][3] = 0;
+            for (int j = 0; j < 4; ++j) acc[j][b][0] = acc[j][b][1] = acc[j][b][2] = acc[j][b][3] = 0;
         }
-        const bool store_xq = chained && P.xq_out && item == P.item0;
-        for (int c = warp; c < chunks; c += kGvWarps) {
-            const int pos = c * kDecChunk + 64 * tg;
-            const bool kin = pos < K;
-            // the lane's 16 bytes of rows g, g + 8, 16 + g, 24 + g (zeros past K or the item)
-            uint4 w[4];
+        if (tile_in) {
+            const uint2 zero_codes = make_uint2(0x55555555u, 0x55555555u);
+            if (!chained) {
+                // the prepared activations: two 16-byte loads per slice and token
+                // block (L1 hits after the first item of a layer), no arithmetic
+                const int8_t *xrow[NT];
+                bool tin[NT];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int row = g + 8 * r;
-                w[r] = (kin && row < rows) ? ld_shared16(st + static_cast<uint32_t>(row * kb + pos / 4))
-                                           : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-            }
-            uint4 xt[NT][4];
-#pragma unroll
-            for (int b = 0; b < NT; ++b) {
-                const int t = 8 * b + g;
-                uint4 x[4];
-                if (kin && t < T) {
-                    gv_load_x(P, prev, chained, t, pos, rq[b], x);
-                    if (store_xq) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(P.xq_out + static_cast<int64_t>(t) * K + pos);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = x[q];
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) x[q] = make_uint4(0u, 0u, 0u, 0u);
+                for (int b = 0; b < NT; ++b) {
+                    const int t = 8 * b + g;
+                    tin[b] = t < T;
+                    xrow[b] = P.xt + static_cast<int64_t>(tin[b] ? t : 0) * K + 32 * tg;
                 }
+                for (int sl = sl0; sl < slices; sl += sl_step) {
+                    const int off = sl * kGvSlice;  // this slice's first weight
+                    const bool kin = off + 32 * tg < K;
+                    const uint32_t bo = static_cast<uint32_t>(off / 4 + 8 * tg);
+                    const uint2 wa = (kin && inA) ? ld_shared8(rowA + bo) : zero_codes;
+                    const uint2 wb = (kin && inB) ? ld_shared8(rowB + bo) : zero_codes;
+                    uint4 xt[NT][2];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    int s = static_cast<int>(cs[b]);
-                    s = __dp4a(static_cast<int>(x[q].x), 0x01010101, s);
-                    s = __dp4a(static_cast<int>(x[q].y), 0x01010101, s);
-                    s = __dp4a(static_cast<int>(x[q].z), 0x01010101, s);
-                    s = __dp4a(static_cast<int>(x[q].w), 0x01010101, s);
-                    cs[b] = static_cast<uint32_t>(s);
-                    xt[b][q] = transpose4x4(x[q]);
-                }
-            }
-            // Weight word wi of a row holds positions 16 wi .. 16 wi + 15, byte
-            // e the four positions 16 wi + 4 e + j at bits 2 j.  Masking code
-            // position j in place (one op) leaves byte e = c(16 wi + 4 e + j) 4^j,
-            // which pairs with word j of the transposed activation group wi
-            // (byte e = x(16 wi + 4 e + j)).  One MMA takes words (0, 1) or
-            // (2, 3) of a row at one j; the 4^j stays in that j's accumulator.
+                    for (int b = 0; b < NT; ++b) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t mj = 0x03030303u << (2 * j);
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        if (u == 1 && !tile1) break;
-                        const uint32_t a0 = word_of(w[2 * u], 2 * h) & mj;
-                        const uint32_t a1 = word_of(w[2 * u + 1], 2 * h) & mj;
-                        const uint32_t a2 = word_of(w[2 * u], 2 * h + 1) & mj;
-                        const uint32_t a3 = word_of(w[2 * u + 1], 2 * h + 1) & mj;
-#pragma unroll
-                        for (int b = 0; b < NT; ++b)
-                            mma_u8s8(acc[u][j][b], a0, a1, a2, a3, word_of(xt[b][2 * h], j),
-                                     word_of(xt[b][2 * h + 1], j));
+                        for (int q = 0; q < 2; ++q)
+                            xt[b][q] = (kin && tin[b]) ? ld_global16(xrow[b] + off + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
                     }
+                    gv_mma_slice<NT>(acc, wa, wb, xt);
+                }
+            } else {
+                // the previous layer's bf16 output, quantised here; the warps of
+                // tile 0 also sum the codes (the +1 bias) and, in the layer's
+                // first item, store the quantised input
+                const bool sums = tile == 0;
+                const bool store_xq = sums && P.xq_out && item == P.item0;
+                for (int sl = sl0; sl < slices; sl += sl_step) {
+                    const int pos = sl * kGvSlice + 32 * tg;
+                    const bool kin = pos < K;
+                    const uint32_t bo = static_cast<uint32_t>(pos / 4);
+                    const uint2 wa = (kin && inA) ? ld_shared8(rowA + bo) : zero_codes;
+                    const uint2 wb = (kin && inB) ? ld_shared8(rowB + bo) : zero_codes;
+                    uint4 xt[NT][2];
+#pragma unroll
+                    for (int b = 0; b < NT; ++b) {
+                        const int t = 8 * b + g;
+                        uint4 x[2];
+                        if (kin && t < T) {
+                            gv_load_x_chained(prev, K, t, pos, rq[b], x);
+                            if (store_xq) {
+                                uint4 *dst = reinterpret_cast<uint4 *>(P.xq_out + static_cast<int64_t>(t) * K + pos);
+                                dst[0] = x[0];
+                                dst[1] = x[1];
+                            }
+                        } else {
+                            x[0] = x[1] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            if (sums) {
+                                int sum = static_cast<int>(cs[b]);
+                                sum = __dp4a(static_cast<int>(x[q].x), 0x01010101, sum);
+                                sum = __dp4a(static_cast<int>(x[q].y), 0x01010101, sum);
+                                sum = __dp4a(static_cast<int>(x[q].z), 0x01010101, sum);
+                                sum = __dp4a(static_cast<int>(x[q].w), 0x01010101, sum);
+                                cs[b] = static_cast<uint32_t>(sum);
+                            }
+                            xt[b][q] = transpose4x4(x[q]);
+                        }
+                    }
+                    gv_mma_slice<NT>(acc, wa, wb, xt);
                 }
             }
         }
@@ -316,25 +403,22 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         if (lane == 0) mbar_arrive(empty_bar(stage));
         if (++stage == kGvStages) stage = 0, phase ^= 1u;
 
-        // partials: part[buf][warp][token][row], column sums csum[buf][warp][token]
+        // partials: part[buf][warp][token][row of the warp's tile]; code sums
+        // (chained layers) csum[buf][warp][token]
         int32_t *pw = part + (buf * kGvWarps + warp) * kDecMaxTokens * kGvPartStride;
 #pragma unroll
         for (int b = 0; b < NT; ++b) {
             const int tA = 8 * b + 2 * tg;
+            // fold the code positions back: acc[j] is a multiple of 4^j
+            // (every product is), so the arithmetic shifts are exact
+            int32_t v[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                // fold the code positions back: acc[j] is a multiple of 4^j
-                // (every product is), so the arithmetic shifts are exact
-                int32_t v[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    v[e] = acc[u][0][b][e] + (acc[u][1][b][e] >> 2) + (acc[u][2][b][e] >> 4) + (acc[u][3][b][e] >> 6);
-                const int rA = 16 * u + g;
-                pw[tA * kGvPartStride + rA] = v[0];
-                pw[(tA + 1) * kGvPartStride + rA] = v[1];
-                pw[tA * kGvPartStride + rA + 8] = v[2];
-                pw[(tA + 1) * kGvPartStride + rA + 8] = v[3];
-            }
+            for (int e = 0; e < 4; ++e)
+                v[e] = acc[0][b][e] + (acc[1][b][e] >> 2) + (acc[2][b][e] >> 4) + (acc[3][b][e] >> 6);
+            pw[tA * kGvPartStride + g] = v[0];
+            pw[(tA + 1) * kGvPartStride + g] = v[1];
+            pw[tA * kGvPartStride + g + 8] = v[2];
+            pw[(tA + 1) * kGvPartStride + g + 8] = v[3];
             uint32_t s = cs[b];
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
@@ -343,26 +427,33 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         gv_consumer_sync();
         if (s_fail[buf]) break;
 
-        // thread (t, r): sum the warps' partials (wrapping int32 arithmetic is
-        // exact when the result fits), dequantise, store
+        // thread (t, r): the tile's warps' partials summed (wrapping int32
+        // arithmetic is exact when the result fits), the code sums removed,
+        // dequantised, stored
         const float gam = ld_global_f32(P.gamma);
         const bool publish = (P.flags & kGvPublish) != 0;
-        for (int o = threadIdx.x; o < T * 32; o += kGvWarps * 32) {
-            const int t = o >> 5, r = o & 31;
-            float d_t;
-            if (chained) {
-                const float a = __uint_as_float(ld_acquire_u32(args.sync + (p - 1) * kGvSyncWords + 1 + t));
-                d_t = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
-            } else {
-                d_t = ld_global_f32(P.d + t);
-            }
+        const int n_out = T * item_rows;
+        for (int o0 = warp * 32; o0 < n_out; o0 += kGvWarps * 32) {  // warp-uniform
+            const int o = o0 + lane;
+            const bool valid = o < n_out;
+            const int t = valid ? o >> (4 + tl2) : 0, r = o - t * item_rows;
+            const int tl = r >> 4, rr = r & 15;
             uint32_t absbits = 0u;
-            if (r < rows) {
-                uint32_t s = 0u;
-#pragma unroll
-                for (int w = 0; w < kGvWarps; ++w)
-                    s += static_cast<uint32_t>(part[((buf * kGvWarps + w) * kDecMaxTokens + t) * kGvPartStride + r]) -
-                         static_cast<uint32_t>(csum[(buf * kGvWarps + w) * kDecMaxTokens + t]);
+            if (valid && r < rows) {
+                float d_t;
+                uint32_t bias = 0u;
+                if (chained) {
+                    const float a = __uint_as_float(ld_acquire_u32(args.sync + (p - 1) * kGvSyncWords + 1 + t));
+                    d_t = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+                    for (int w = 0; w < kGvWarps; w += tiles)  // the warps of tile 0
+                        bias += static_cast<uint32_t>(csum[(buf * kGvWarps + w) * kDecMaxTokens + t]);
+                } else {
+                    d_t = ld_global_f32(P.d + t);
+                    bias = static_cast<uint32_t>(__ldcg(P.colsum + t));
+                }
+                uint32_t s = 0u - bias;
+                for (int w = tl; w < kGvWarps; w += tiles)
+                    s += static_cast<uint32_t>(part[((buf * kGvWarps + w) * kDecMaxTokens + t) * kGvPartStride + rr]);
                 const float y = __fmul_rn(__int2float_rn(static_cast<int32_t>(s)), __fmul_rn(gam, d_t));
                 const int64_t off = static_cast<int64_t>(t) * P.O + r0 + r;
                 if (P.flags & kGvOutFp32) {
@@ -375,9 +466,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
                 }
             }
             if (publish) {
-                // max |y_t| of the bf16 outputs (their fp32 bits order like the values)
-                absbits = __reduce_max_sync(0xffffffffu, absbits);
-                if (lane == 0 && absbits) atomicMax(args.sync + p * kGvSyncWords + 1 + t, absbits << 16);
+                // max |y_t| of the bf16 outputs (their fp32 bits order like the
+                // values): the lanes of one token are the whole warp, or each
+                // half of it when the item has 16 rows
+                uint32_t m = absbits;
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+                if (item_rows >= 32) m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                if (valid && (lane & (item_rows >= 32 ? 31 : 15)) == 0 && m)
+                    atomicMax(args.sync + p * kGvSyncWords + 1 + t, m << 16);
             }
         }
         if (chained && item == P.item0 && P.d_out && threadIdx.x < T) {

@@ -115,7 +115,7 @@ _lib.sbl_linear_forward.restype = ctypes.c_int
 _lib.sbl_linear_forward.argtypes = [_D, _P, _i32, _W, ctypes.c_int, _P, _P, _P, _i32,
                                     ctypes.POINTER(sbl_epilogue), _P]
 _lib.sbl_forward_batch_workspace_bytes.restype = _sz
-_lib.sbl_forward_batch_workspace_bytes.argtypes = [ctypes.POINTER(sbl_batch_layer), _i32]
+_lib.sbl_forward_batch_workspace_bytes.argtypes = [ctypes.POINTER(sbl_batch_layer), _i32, _i32]
 _lib.sbl_forward_batch.restype = ctypes.c_int
 _lib.sbl_forward_batch.argtypes = [ctypes.POINTER(sbl_batch_layer), _i32, _i32, _P, _sz, _P]
 _lib.sbl_gamma_node_count.restype = _sz
@@ -359,8 +359,8 @@ def batch_array(layers) -> ctypes.Array:
     return (sbl_batch_layer * len(layers))(*layers)
 
 
-def sbl_forward_batch_workspace_bytes(layers: ctypes.Array, count: int) -> int:
-    return int(_lib.sbl_forward_batch_workspace_bytes(layers, count))
+def sbl_forward_batch_workspace_bytes(layers: ctypes.Array, count: int, T: int) -> int:
+    return int(_lib.sbl_forward_batch_workspace_bytes(layers, count, T))
 
 
 def sbl_forward_batch(layers: ctypes.Array, count: int, T: int, workspace: Optional[torch.Tensor] = None) -> None:

@@ -387,13 +387,22 @@ def test_batch_forward_validation_before_device(sbl):
     assert call([layer(O=256), layer(O=128, K=512, chained=True)]) == 1   # shapes do not chain
     assert call([layer(O=512, y_fp32=1), layer(K=512, chained=True)]) == 1  # fp32 output cannot chain
     chain = [layer(O=512), layer(K=512, chained=True, xq=None)]
-    nws = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array(chain), 2)
-    assert nws == 256
-    assert sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer()]), 1) == 0
+    nws = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array(chain), 2, 4)
+    # completion words of two layers (256) + the first layer's prepared input (4 x 256 + 256)
+    assert nws == 256 + 1024 + 256
+    one = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer()]), 1, 4)
+    assert one == 1024 + 256
+    # two layers on one input share its prepared copy; a second input gets its own
+    assert sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer(), layer()]), 2, 4) == one
+    assert sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer(), layer(xq=good + 4096)]), 2, 4) == 2 * one
+    assert sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array([layer()]), 1, 0) == 0
     assert call(chain) == 5 and call(chain, ws=good, ws_bytes=nws - 1) == 5
     assert call(chain, ws=good + 16, ws_bytes=nws) == 3
     assert call(chain, ws=good, ws_bytes=nws) == 7         # valid: no sm_100 device here
-    assert call([layer(), layer(O=64, K=14336)], T=16) == 7
+    big = [layer(), layer(O=64, K=14336)]
+    assert call(big, T=16) == 5
+    nb = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array(big), 2, 16)
+    assert call(big, T=16, ws=good, ws_bytes=nb) == 7
 
 
 def test_sharding_calls_validate_before_device(sbl):

@@ -47,8 +47,8 @@ def test_batch_independent_layers_bit_exact(T):
         entries.append(sbl.batch_layer(layer.desc, layer.packed, y, q, d, y_is_fp32=fp32))
         keep.append((layer, ref, x, q, d, y, fp32))
     arr = sbl.batch_array(entries)
-    assert sbl.sbl_forward_batch_workspace_bytes(arr, len(entries)) == 0
-    sbl.sbl_forward_batch(arr, len(entries), T)
+    ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(arr, len(entries), T))
+    sbl.sbl_forward_batch(arr, len(entries), T, ws)
     torch.cuda.synchronize()
     assert sbl.sbl_device_error() == 0
     for layer, ref, x, q, d, y, fp32 in keep:
@@ -83,7 +83,7 @@ def test_batch_chain_matches_oracle_layer_by_layer(T):
         entries.append(e)
         keep.append((ref, y, xq_out, d_out, layer))  # the layer's buffers must outlive the call
     arr = sbl.batch_array(entries)
-    nws = sbl.sbl_forward_batch_workspace_bytes(arr, len(entries))
+    nws = sbl.sbl_forward_batch_workspace_bytes(arr, len(entries), T)
     assert nws >= 128 * len(entries)
     ws = sbl.alloc_workspace(nws)
     for rep in range(2):  # a second call on the same workspace starts from zero again
@@ -116,7 +116,7 @@ def test_batch_chain_then_independent_layer():
     arr = sbl.batch_array([sbl.batch_layer(a.desc, a.packed, ya, qa, da),
                            sbl.batch_layer(b.desc, b.packed, yb, chained=True),
                            sbl.batch_layer(c.desc, c.packed, yc, qc, dc)])
-    ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(arr, 3))
+    ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(arr, 3, T))
     sbl.sbl_forward_batch(arr, 3, T, ws)
     torch.cuda.synchronize()
     _, yab = oracle_forward_bits(ra, xa)
@@ -144,7 +144,9 @@ def test_batch_full_decode_workload_equals_single_launches():
                 sbl.sbl_forward(layers[li].desc, q, d, T, layers[li].packed, sbl.SBL_FMT_PK2, y1)
                 entries.append(sbl.batch_layer(layers[li].desc, layers[li].packed, y, q, d))
                 outs.append((y, y1, q, d))
-        sbl.sbl_forward_batch(sbl.batch_array(entries), len(entries), T)
+        arr = sbl.batch_array(entries)
+        ws = sbl.alloc_workspace(sbl.sbl_forward_batch_workspace_bytes(arr, len(entries), T))
+        sbl.sbl_forward_batch(arr, len(entries), T, ws)
         torch.cuda.synchronize()
         for y, y1, _, _ in outs:
             assert torch.equal(y.view(torch.int16), y1.view(torch.int16))

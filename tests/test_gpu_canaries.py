@@ -133,3 +133,61 @@ def test_guard_bands_fused_decode_one_token():
     qr, dr = oracle.quantize_act(wl.activations(T, K, seed=4))
     np.testing.assert_array_equal(q.cpu().numpy(), qr)
     np.testing.assert_array_equal(dv.cpu().numpy(), dr)
+
+
+def test_guard_bands_batched_decode_and_sharding():
+    """The batched decode (independent layers with ragged row blocks and a
+    chain storing its quantised inputs) and the sharded weight side write
+    only their buffers, workspaces included."""
+    sbl = sbl_mod()
+    g = Guarded()
+    T = 3
+    shapes = [(48, 320), (80, 8960), (272, 1536)]  # items of 4, 1 and 2 tiles, partial last items
+    entries, keep = [], []
+    for i, (O, K) in enumerate(shapes):
+        d = sbl.desc(O, K, 2, 4)
+        p = _packed(sbl, g, d, sbl.SBL_FMT_PK2)
+        ws = g.take((sbl.sbl_workspace_bytes(d, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK),), torch.uint8)
+        sbl.sbl_quantize_mask_pack(d, torch.from_numpy(wl.master_weights(O, K, seed=i)).cuda(), sbl.SBL_FMT_PK2, p, ws)
+        q, dv = g.take((T, K), torch.int8), g.take((T,), torch.float32)
+        sbl.sbl_quantize_act(bf16_dev(wl.activations(T, K, seed=i)), T, K, q, dv)
+        y = g.take((T, O), torch.bfloat16)
+        entries.append(sbl.batch_layer(d, p, y, q, dv))
+        keep.append((p, q, dv, y))
+    # a chained pair 320 -> 64 -> 128 after them (its first layer shares the
+    # first input above)
+    d1 = sbl.desc(64, 320, 6, 8)
+    p1 = _packed(sbl, g, d1, sbl.SBL_FMT_PK2)
+    d2 = sbl.desc(128, 64, 6, 8)
+    p2 = _packed(sbl, g, d2, sbl.SBL_FMT_PK2)
+    for i, (d, p) in enumerate(((d1, p1), (d2, p2))):
+        ws = g.take((sbl.sbl_workspace_bytes(d, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK),), torch.uint8)
+        w = torch.from_numpy(wl.master_weights(d.out_features, d.in_features, seed=10 + i)).cuda()
+        sbl.sbl_quantize_mask_pack(d, w, sbl.SBL_FMT_PK2, p, ws)
+    q1, d1v = keep[0][1], keep[0][2]
+    y1, y2 = g.take((T, 64), torch.bfloat16), g.take((T, 128), torch.bfloat16)
+    xo, do = g.take((T, 64), torch.int8), g.take((T,), torch.float32)
+    entries.append(sbl.batch_layer(d1, p1, y1, q1, d1v))
+    entries.append(sbl.batch_layer(d2, p2, y2, chained=True, xq_out=xo, d_out=do))
+    arr = sbl.batch_array(entries)
+    bws = g.take((sbl.sbl_forward_batch_workspace_bytes(arr, len(entries), T),), torch.uint8)
+    sbl.sbl_forward_batch(arr, len(entries), T, bws)
+
+    # sharded weight side: two shards of a 1104 x 2048 layer
+    O, K = 1104, 2048
+    w = torch.from_numpy(wl.master_weights(O, K, seed=5)).cuda()
+    from sparsity_sbl_quantize_b200 import sharding
+    parts = []
+    for first, rows in sharding.column_shards(O, K, 2):
+        ds = sbl.desc(rows, K, 6, 8)
+        ws = g.take((sbl.sbl_workspace_bytes(ds, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK),), torch.uint8)
+        nodes = g.take((sbl.sbl_gamma_node_count(ds),), torch.float64)
+        sbl.sbl_gamma_partials(ds, w[first:first + rows].contiguous(), first, nodes, ws)
+        parts.append((ds, first, rows, nodes))
+    allnodes = torch.cat([n for *_, n in parts])
+    for ds, first, rows, _ in parts:
+        p = _packed(sbl, g, ds, sbl.SBL_FMT_I8 | sbl.SBL_FMT_PK2)
+        sbl.sbl_gamma_combine(allnodes, allnodes.numel(), O * K, p.gamma)
+        sbl.sbl_quantize_mask_pack_shard(ds, w[first:first + rows].contiguous(), sbl.SBL_FMT_I8 | sbl.SBL_FMT_PK2, p)
+    g.check()
+    assert sbl.sbl_device_error(clear=True) == 0
