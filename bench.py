@@ -54,11 +54,14 @@ def kernel_family(workload: str) -> str:
 UNIT_BYTES = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1024, "MB": 1 << 20, "GB": 1 << 30}
 
 
-def record_traffic(csv_paths, workload: str, kernel_regex: str, command: str) -> dict:
+def record_traffic(csv_paths, workload: str, kernel_regex: str, command: str, scale: float = 1.0,
+                   scale_note: str = "") -> dict:
     """Parse an ncu --csv metric list (dram__bytes_read.sum and
     dram__bytes_write.sum per launch) and store the mean read+write bytes per
     launch of the kernels matching kernel_regex for `workload`, tagged with
-    the current kernel-source hash."""
+    the current kernel-source hash.  `scale` converts a capture of a smaller
+    launch to the bench's launch (the ratio of the units both process, when
+    the traffic grows in proportion); `scale_note` says how."""
     import csv
     import re
     pat = re.compile(kernel_regex)
@@ -74,8 +77,11 @@ def record_traffic(csv_paths, workload: str, kernel_regex: str, command: str) ->
     if not per_launch:
         raise SystemExit(f"no launches of {kernel_regex} with DRAM metrics in {csv_paths}")
     rec = {"kernel_regex": kernel_regex, "launches": len(per_launch),
-           "bytes_per_launch": round(sum(per_launch.values()) / len(per_launch)),
+           "bytes_per_launch": round(scale * sum(per_launch.values()) / len(per_launch)),
            "kernel_source_sha256": kernel_source_hash(kernel_family(workload)), "command": command}
+    if scale != 1.0:
+        rec["scale"] = scale
+        rec["scale_note"] = scale_note
     data = {}
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
@@ -128,6 +134,9 @@ def parse():
                     help="store the mean DRAM bytes per roofline-kernel launch from an ncu --csv metric list "
                          "(dram__bytes_read.sum, dram__bytes_write.sum) for --workload, then exit")
     ap.add_argument("--traffic-command", default="", help="the ncu command that produced NCU_CSV (recorded)")
+    ap.add_argument("--traffic-scale", type=float, default=1.0,
+                    help="factor from the captured launch to the bench's launch (units processed)")
+    ap.add_argument("--traffic-scale-note", default="", help="how the factor was obtained (recorded)")
     ap.add_argument("--ref-step-seconds", type=float, default=0.0,
                     help="oracle time per reference-arm step (default: about 120 s over the whole run)")
     return ap.parse_args()
@@ -1153,7 +1162,8 @@ def main():
         # the roofline kernels: the persistent streaming decode GEMV, or the
         # int8 dense and 2:4 sparse forward GEMMs
         regex = r"gemv_stream_kernel" if wk.mode == "decode" else r"gemm_kernel<0|sp24_pair_kernel"
-        print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command)))
+        print(json.dumps(record_traffic(args.record_traffic, wk.name, regex, args.traffic_command,
+                                        args.traffic_scale, args.traffic_scale_note)))
         return
     if args.impl == "reference":
         run_reference(args, wk)

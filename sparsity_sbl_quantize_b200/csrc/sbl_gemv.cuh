@@ -432,8 +432,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         // dequantised, stored
         const float gam = ld_global_f32(P.gamma);
         const bool publish = (P.flags & kGvPublish) != 0;
+        // the warps with the fewest K slices (the highest-numbered: their first
+        // slice index is the largest) take the outputs first
         const int n_out = T * item_rows;
-        for (int o0 = warp * 32; o0 < n_out; o0 += kGvWarps * 32) {  // warp-uniform
+        for (int o0 = (kGvWarps - 1 - warp) * 32; o0 < n_out; o0 += kGvWarps * 32) {  // warp-uniform
             const int o = o0 + lane;
             const bool valid = o < n_out;
             const int t = valid ? o >> (4 + tl2) : 0, r = o - t * item_rows;
