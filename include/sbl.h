@@ -386,7 +386,7 @@ sbl_status sbl_linear_forward(const sbl_layer_desc *desc, const uint16_t *X, int
  * summary) from its 2-bit PK2 weights, exactly as sbl_forward with
  * SBL_FMT_PK2:
  *   Y[t,o] = fl32(fl32(sum_k W_eff[o,k] Xq[t,k]) * fl32(gamma * d[t])).
- * desc       the layer (in_features a multiple of 64, at most 14336);
+ * desc       the layer (in_features a multiple of 64, at most 13824);
  * pk2, gamma its packed weights (sbl_packed.pk2 and .gamma);
  * xq, d      its int8 activations [T, K] and token scales [T] (inputs), or,
  *            when input_is_previous_output is nonzero, unused: the input is
@@ -438,7 +438,7 @@ size_t sbl_forward_batch_workspace_bytes(const sbl_batch_layer *layers, int32_t 
  * sbl_forward (the weights are read before the wait on the previous kernel).
  * Two launches (one when every layer after the first is chained).
  * Errors: SBL_ERR_SHAPE for count, T or a descriptor out of range;
- * SBL_ERR_UNSUPPORTED for in_features not a multiple of 64 or above 14336;
+ * SBL_ERR_UNSUPPORTED for in_features not a multiple of 64 or above 13824;
  * SBL_ERR_INVALID_ARG for a null pointer a layer needs, a chained first
  * layer, or a chain whose shapes or output type do not match. */
 sbl_status sbl_forward_batch(const sbl_batch_layer *layers, int32_t count, int32_t T, void *workspace,

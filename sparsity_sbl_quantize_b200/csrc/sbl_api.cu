@@ -1021,7 +1021,7 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
 // ------------------------------------------------------ batched decode --
 static_assert(SBL_BATCH_MAX_LAYERS <= kGvMaxProblems, "the launch parameters hold every layer of a batch");
 static_assert(sizeof(GvArgs) <= 32000 && sizeof(GvPrepArgs) <= 32000, "kernel parameters are limited to 32764 bytes");
-constexpr int32_t kGvMaxK = 4 * kGvStageBytes / 16;  // 16-row items of K / 4 bytes per row fill a stage
+constexpr int32_t kGvMaxK = 4 * kGvStageBytes / 16 / kDecKUnit * kDecKUnit;  // 16-row items of K / 4 bytes per row fill a stage
 
 static bool batch_has_chain(const sbl_batch_layer *layers, int32_t count)
 {

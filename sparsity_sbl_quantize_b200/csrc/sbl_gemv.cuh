@@ -10,19 +10,19 @@
 // differs is how the weights reach the SMs:
 //
 //  * one CTA per SM runs for the whole batch; its work items are blocks of
-//    64, 32 or 16 rows of a layer (as many 16-row tiles as one 56 KB stage
+//    64, 32 or 16 rows of a layer (as many 16-row tiles as one 54 KB stage
 //    holds at that K), taken round-robin over the grid in batch order;
 //  * a producer warp streams each item's packed rows -- contiguous, since a
 //    PK2 row is exactly K / 4 bytes when K % 64 == 0 -- with ONE bulk copy
-//    (cp.async.bulk, evict-first in L2) into a ring of shared-memory stages,
+//    (cp.async.bulk, evict-first in L2) into a ring of four shared-memory stages,
 //    as far ahead as the ring allows and across layer boundaries: the
 //    weights never depend on the activations, so no launch gap or
 //    dependency stalls the stream;
 //  * sixteen consumer warps share an item: each owns one of its tiles and
 //    takes that tile's 128-weight K slices round-robin with the other warps
-//    of the tile (balanced for any K), frees the stage, and the warps meet in
-//    shared memory (exact int32 partials) where the item's T x rows outputs
-//    are summed and dequantised;
+//    of the tile (balanced for any K), frees the stage, and adds its exact
+//    int32 partials into the item's sums in shared memory (shared atomics),
+//    where the item's T x rows outputs are read, dequantised and stored;
 //  * an unchained layer reads its int8 activations in a prepared layout
 //    (every 16-byte group 4 x 4 transposed, written once per launch by a
 //    small kernel together with the per-token sums that remove the +1 code
@@ -50,13 +50,15 @@ namespace sbl {
 constexpr int kGvMaxProblems = 256;
 constexpr int kGvWarps = 16;                      // consumer warps
 constexpr int kGvThreads = 32 * (kGvWarps + 1);   // + the producer warp
-constexpr int kGvStageBytes = 56 * 1024;          // one item: 16 tiles x K/4 bytes per row
-constexpr int kGvStages = 3;
+constexpr int kGvStageBytes = 54 * 1024;          // one item: 16 tiles x K/4 bytes per row (2 tiles at K = 6912)
+constexpr int kGvStages = 4;
 constexpr int kGvSlice = 128;                     // weights of a row in one K slice of a unit
-constexpr int kGvPartStride = 20;                 // padded row count (16 rows) of a token's partials
+constexpr int kGvItemMaxRows = 64;
+constexpr int kGvPartStride = kGvItemMaxRows + 4;  // a token's row of item sums (padded: conflict-free adds)
 constexpr int kGvSyncWords = 32;                  // per layer: [0] items done, [1 + t] max |y_t| bits
-constexpr int kGvSmemBytes = kGvStages * kGvStageBytes + 2 * kGvWarps * kDecMaxTokens * kGvPartStride * 4 +
+constexpr int kGvSmemBytes = kGvStages * kGvStageBytes + 2 * kDecMaxTokens * kGvPartStride * 4 +
                              2 * kGvWarps * kDecMaxTokens * 4 + 2 * kGvStages * 8;
+static_assert(kGvSmemBytes + 256 <= 227 * 1024, "the ring, the sums and the barriers fit one SM's shared memory");
 
 enum : int32_t {
     kGvOutFp32 = 1,   // Y is fp32 (else bf16)
@@ -203,8 +205,8 @@ template <int NT>
 __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid_constant__ GvArgs args)
 {
     extern __shared__ __align__(128) uint8_t gv_smem[];
-    int32_t *part = reinterpret_cast<int32_t *>(gv_smem + kGvStages * kGvStageBytes);  // [2][warp][t][row of tile]
-    int32_t *csum = part + 2 * kGvWarps * kDecMaxTokens * kGvPartStride;                 // [2][warp][t]
+    int32_t *part = reinterpret_cast<int32_t *>(gv_smem + kGvStages * kGvStageBytes);  // [2][t][row of item]
+    int32_t *csum = part + 2 * kDecMaxTokens * kGvPartStride;                             // [2][warp][t]
     uint64_t *bars = reinterpret_cast<uint64_t *>(csum + 2 * kGvWarps * kDecMaxTokens);
     const uint32_t stage0 = smem_addr(gv_smem);
     auto full_bar = [&](int s) { return smem_addr(bars + s); };
@@ -224,6 +226,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         s_fail[0] = s_fail[1] = 0;
         fence_barrier_init();
     }
+    // the item sums start at zero; each finishing thread zeroes what it read
+    for (int i = threadIdx.x; i < 2 * kDecMaxTokens * kGvPartStride; i += blockDim.x) part[i] = 0;
     __syncthreads();
     // unchained batches have no waits between CTAs: the next kernel may start
     // launching (and streaming its own read-only data) right away
@@ -403,9 +407,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         if (lane == 0) mbar_arrive(empty_bar(stage));
         if (++stage == kGvStages) stage = 0, phase ^= 1u;
 
-        // partials: part[buf][warp][token][row of the warp's tile]; code sums
+        // partials added into the item's sums part[buf][token][row] (shared
+        // atomics; integer addition in any order is exact); code sums
         // (chained layers) csum[buf][warp][token]
-        int32_t *pw = part + (buf * kGvWarps + warp) * kDecMaxTokens * kGvPartStride;
+        int32_t *pb = part + buf * kDecMaxTokens * kGvPartStride + 16 * tile + g;
 #pragma unroll
         for (int b = 0; b < NT; ++b) {
             const int tA = 8 * b + 2 * tg;
@@ -415,10 +420,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 v[e] = acc[0][b][e] + (acc[1][b][e] >> 2) + (acc[2][b][e] >> 4) + (acc[3][b][e] >> 6);
-            pw[tA * kGvPartStride + g] = v[0];
-            pw[(tA + 1) * kGvPartStride + g] = v[1];
-            pw[tA * kGvPartStride + g + 8] = v[2];
-            pw[(tA + 1) * kGvPartStride + g + 8] = v[3];
+            if (tile_in && tA < T) {
+                atomicAdd(pb + tA * kGvPartStride, v[0]);
+                atomicAdd(pb + tA * kGvPartStride + 8, v[2]);
+            }
+            if (tile_in && tA + 1 < T) {
+                atomicAdd(pb + (tA + 1) * kGvPartStride, v[1]);
+                atomicAdd(pb + (tA + 1) * kGvPartStride + 8, v[3]);
+            }
             uint32_t s = cs[b];
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
@@ -427,9 +436,9 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
         gv_consumer_sync();
         if (s_fail[buf]) break;
 
-        // thread (t, r): the tile's warps' partials summed (wrapping int32
-        // arithmetic is exact when the result fits), the code sums removed,
-        // dequantised, stored
+        // thread (t, r): the item's sum (wrapping int32 arithmetic is exact
+        // when the result fits), the code sums removed, dequantised, stored;
+        // the sum is zeroed for the item after next
         const float gam = ld_global_f32(P.gamma);
         const bool publish = (P.flags & kGvPublish) != 0;
         // the warps with the fewest K slices (the highest-numbered: their first
@@ -439,8 +448,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
             const int o = o0 + lane;
             const bool valid = o < n_out;
             const int t = valid ? o >> (4 + tl2) : 0, r = o - t * item_rows;
-            const int tl = r >> 4, rr = r & 15;
             uint32_t absbits = 0u;
+            int32_t *ps = part + (buf * kDecMaxTokens + t) * kGvPartStride + r;
+            const uint32_t sum = valid ? static_cast<uint32_t>(*ps) : 0u;
+            if (valid) *ps = 0;
             if (valid && r < rows) {
                 float d_t;
                 uint32_t bias = 0u;
@@ -453,9 +464,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
                     d_t = ld_global_f32(P.d + t);
                     bias = static_cast<uint32_t>(__ldcg(P.colsum + t));
                 }
-                uint32_t s = 0u - bias;
-                for (int w = tl; w < kGvWarps; w += tiles)
-                    s += static_cast<uint32_t>(part[((buf * kGvWarps + w) * kDecMaxTokens + t) * kGvPartStride + rr]);
+                const uint32_t s = sum - bias;
                 const float y = __fmul_rn(__int2float_rn(static_cast<int32_t>(s)), __fmul_rn(gam, d_t));
                 const int64_t off = static_cast<int64_t>(t) * P.O + r0 + r;
                 if (P.flags & kGvOutFp32) {

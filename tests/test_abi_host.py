@@ -380,7 +380,7 @@ def test_batch_forward_validation_before_device(sbl):
     assert call([layer()], count=0) == 2 and call([layer()], count=257) == 2
     assert call([layer(K=250)]) == 2                       # invalid descriptor
     assert call([layer(K=272)]) == 4                       # K not a multiple of 64
-    assert call([layer(K=14400)]) == 4                     # K above the stage limit
+    assert call([layer(K=13888)]) == 4                     # K above the stage limit (13824)
     assert call([layer(pk2=None)]) == 1 and call([layer(xq=None)]) == 1
     assert call([layer(pk2=good + 8)]) == 3
     assert call([layer(chained=True)]) == 1                # a chain needs a previous layer
@@ -399,7 +399,7 @@ def test_batch_forward_validation_before_device(sbl):
     assert call(chain) == 5 and call(chain, ws=good, ws_bytes=nws - 1) == 5
     assert call(chain, ws=good + 16, ws_bytes=nws) == 3
     assert call(chain, ws=good, ws_bytes=nws) == 7         # valid: no sm_100 device here
-    big = [layer(), layer(O=64, K=14336)]
+    big = [layer(), layer(O=64, K=13824)]
     assert call(big, T=16) == 5
     nb = sbl.sbl_forward_batch_workspace_bytes(sbl.batch_array(big), 2, 16)
     assert call(big, T=16, ws=good, ws_bytes=nb) == 7
