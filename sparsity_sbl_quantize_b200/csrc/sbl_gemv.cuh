@@ -334,27 +334,46 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
             const uint2 zero_codes = make_uint2(0x55555555u, 0x55555555u);
             if (!chained) {
                 // the prepared activations: two 16-byte loads per slice and token
-                // block (L1 hits after the first item of a layer), no arithmetic
+                // block, no arithmetic.  Lanes of tokens t >= T read token 0's
+                // row (the same addresses, one request) and rows past the
+                // layer's last read the stage's other bytes: both only reach
+                // accumulator entries that are never stored, so the full
+                // slices need no selects; the ragged last slice (K % 128 ==
+                // 64) zeroes the lanes past K, whose products would land in
+                // stored entries.
                 const int8_t *xrow[NT];
-                bool tin[NT];
 #pragma unroll
                 for (int b = 0; b < NT; ++b) {
                     const int t = 8 * b + g;
-                    tin[b] = t < T;
-                    xrow[b] = P.xt + static_cast<int64_t>(tin[b] ? t : 0) * K + 32 * tg;
+                    xrow[b] = P.xt + static_cast<int64_t>(t < T ? t : 0) * K + 32 * tg;
                 }
-                for (int sl = sl0; sl < slices; sl += sl_step) {
+                const int full = K / kGvSlice;
+                int sl = sl0;
+                for (; sl < full; sl += sl_step) {
                     const int off = sl * kGvSlice;  // this slice's first weight
+                    const uint32_t bo = static_cast<uint32_t>(off / 4 + 8 * tg);
+                    const uint2 wa = ld_shared8(rowA + bo);
+                    const uint2 wb = ld_shared8(rowB + bo);
+                    uint4 xt[NT][2];
+#pragma unroll
+                    for (int b = 0; b < NT; ++b) {
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) xt[b][q] = ld_global16(xrow[b] + off + 16 * q);
+                    }
+                    gv_mma_slice<NT>(acc, wa, wb, xt);
+                }
+                if (sl < slices) {  // warp-uniform: this warp's share holds the ragged slice
+                    const int off = sl * kGvSlice;
                     const bool kin = off + 32 * tg < K;
                     const uint32_t bo = static_cast<uint32_t>(off / 4 + 8 * tg);
-                    const uint2 wa = (kin && inA) ? ld_shared8(rowA + bo) : zero_codes;
-                    const uint2 wb = (kin && inB) ? ld_shared8(rowB + bo) : zero_codes;
+                    const uint2 wa = kin ? ld_shared8(rowA + bo) : zero_codes;
+                    const uint2 wb = kin ? ld_shared8(rowB + bo) : zero_codes;
                     uint4 xt[NT][2];
 #pragma unroll
                     for (int b = 0; b < NT; ++b) {
 #pragma unroll
                         for (int q = 0; q < 2; ++q)
-                            xt[b][q] = (kin && tin[b]) ? ld_global16(xrow[b] + off + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
+                            xt[b][q] = kin ? ld_global16(xrow[b] + off + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
                     }
                     gv_mma_slice<NT>(acc, wa, wb, xt);
                 }
@@ -428,10 +447,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_stream_kernel(const __grid
                 atomicAdd(pb + (tA + 1) * kGvPartStride, v[1]);
                 atomicAdd(pb + (tA + 1) * kGvPartStride + 8, v[3]);
             }
-            uint32_t s = cs[b];
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            if (tg == 0) csum[(buf * kGvWarps + warp) * kDecMaxTokens + 8 * b + g] = static_cast<int32_t>(s);
+            if (chained) {
+                uint32_t s = cs[b];
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                if (tg == 0) csum[(buf * kGvWarps + warp) * kDecMaxTokens + 8 * b + g] = static_cast<int32_t>(s);
+            }
         }
         gv_consumer_sync();
         if (s_fail[buf]) break;
