@@ -150,17 +150,20 @@ static bool encode_kmajor(CUtensorMap *map, const void *base, CUtensorMapDataTyp
 
 // Output tensor map for the epilogue's TMA stores: rows x cols of bf16 or
 // fp32 with row stride ld elements; box = 32 rows x 128 bytes, 128-byte swizzle.
-static bool encode_output(CUtensorMap *map, void *base, bool fp32, int64_t rows, int64_t cols, int64_t ld)
+static bool encode_output(CUtensorMap *map, void *base, bool fp32, int64_t rows, int64_t cols, int64_t ld,
+                          bool rows64 = false)
 {
+    // box: 32 rows of 128 bytes, 128-byte swizzle; rows64: 32 rows of 64
+    // bytes, 64-byte swizzle (the bf16 output without the epilogue)
     const int eb = fp32 ? 4 : 2;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * eb)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), 32};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>((rows64 ? 64 : 128) / eb), 32};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                                 base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                rows64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -213,14 +216,16 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     CUtensorMap ta, tb, ty;
     if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
     if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, bn)) return SBL_ERR_CUDA;
-    if (!encode_output(&ty, args.out, args.out_fp32 != 0, M, N, args.ldo)) return SBL_ERR_CUDA;
+    const bool with_epi = KIND == kKindI8 && (args.relu2 || args.residual);
+    if (!encode_output(&ty, args.out, args.out_fp32 != 0, M, N, args.ldo, !args.out_fp32 && !with_epi))
+        return SBL_ERR_CUDA;
     args.M = M;
     args.N = N;
     args.K = K;
     args.k_blocks = static_cast<int32_t>((static_cast<int64_t>(K) * eb + kBKBytes - 1) / kBKBytes);
     args.err = di->err;
     if constexpr (KIND == kKindI8) {
-        if (args.relu2 || args.residual)
+        if (with_epi)
             return bn == 128 ? launch_gemm_bn<KIND, 128, true>(di, ta, tb, ty, args, stream)
                              : launch_gemm_bn<KIND, 256, true>(di, ta, tb, ty, args, stream);
     }

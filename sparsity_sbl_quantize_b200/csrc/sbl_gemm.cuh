@@ -261,8 +261,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = quarter * 32 + lane;
         const float g = args.gamma ? *args.gamma : 1.0f;
         const uint32_t buf = epi_base + static_cast<uint32_t>(warp - 2) * kEpiBufBytes;
-        constexpr int kColsPerChunk = 64;  // bf16: one 128-byte store; fp32: two
+        constexpr int kColsPerChunk = 64;  // bf16: two 64-byte stores (one 128-byte with the epilogue); fp32: two
         constexpr int kChunks = BN / kColsPerChunk / 2;  // per warp
+        uint32_t nstore = 0;  // bf16 blocks stored by this warp (staging half = nstore % 2)
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int tm, tn;
@@ -322,27 +323,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_before();
                 mbar_arrive(tempty_bar(acc));
+                // 32-column blocks (64-byte rows) staged in turn in the two
+                // halves of the warp's buffer: a block waits only for the store
+                // before last, so staging overlaps the previous store's read
 #pragma unroll
                 for (int jj = 0; jj < kChunks; ++jj) {
                     const int j = half * kChunks + jj;
-                    const int col = tn * BN + kColsPerChunk * j;
-                    if (col >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
-                    // the previous store from this buffer has finished reading it
-                    if (lane == 0) bulk_wait_group_read<0>();
-                    __syncwarp();
-                    // row `lane`: 8 chunks of 16 bytes, chunk c at position c ^ (lane % 8)
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t addr = buf + static_cast<uint32_t>(lane * 128 + ((c ^ (lane & 7)) * 16));
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[jj][4 * c]),
-                                     "r"(packed[jj][4 * c + 1]), "r"(packed[jj][4 * c + 2]), "r"(packed[jj][4 * c + 3])
-                                     : "memory");
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmY, buf, col, row0);
-                        bulk_commit_group();
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int col = tn * BN + kColsPerChunk * j + 32 * hh;
+                        if (col >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
+                        const uint32_t sbuf = buf + static_cast<uint32_t>((nstore & 1) * (kEpiBufBytes / 2));
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        // row `lane`: 4 chunks of 16 bytes, chunk c at position
+                        // c ^ ((lane / 2) % 4) (the 64-byte swizzle of the output map)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t addr = sbuf + static_cast<uint32_t>(lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16));
+                            const int w0 = 16 * hh + 4 * c;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[jj][w0]),
+                                         "r"(packed[jj][w0 + 1]), "r"(packed[jj][w0 + 2]), "r"(packed[jj][w0 + 3])
+                                         : "memory");
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmY, sbuf, col, row0);
+                            bulk_commit_group();
+                        }
+                        ++nstore;
                     }
                 }
                 continue;
