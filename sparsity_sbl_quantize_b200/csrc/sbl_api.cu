@@ -76,6 +76,10 @@ static sbl_status current_device(DeviceInfo **out)
                                  GemmCfg<256>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindI8, 128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindI8, 256, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindI8, 256, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -181,25 +185,32 @@ static int choose_bn(int32_t M, int32_t N, int num_sms)
     return 5 * rounds(128) <= 4 * rounds(256) ? 128 : 256;
 }
 
-template <int KIND, int BN, bool EPI>
+template <int KIND, int BN, bool EPI, bool PAIR = false>
 static sbl_status launch_gemm_bn(const DeviceInfo *di, const CUtensorMap &ta, const CUtensorMap &tb,
                                  const CUtensorMap &ty, GemmArgs args, cudaStream_t stream)
 {
-    args.tiles_m = static_cast<int32_t>((args.M + kBM - 1) / kBM);
+    constexpr int tile_m = PAIR ? 2 * kBM : kBM;
+    args.tiles_m = static_cast<int32_t>((args.M + tile_m - 1) / tile_m);
     args.tiles_n = static_cast<int32_t>((args.N + BN - 1) / BN);
     const int tiles = args.tiles_m * args.tiles_n;
+    const int units = PAIR ? di->num_sms / 2 : di->num_sms;  // CTAs, or CTA pairs
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles < di->num_sms ? tiles : di->num_sms));
+    cfg.gridDim = dim3(static_cast<unsigned>((PAIR ? 2 : 1) * (tiles < units ? tiles : units)));
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = GemmCfg<BN>::kSmemBytes;
+    cfg.dynamicSmemBytes = GemmCfg<BN, PAIR>::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, EPI>, ta, tb, ty, args) != cudaSuccess) return SBL_ERR_CUDA;
+    cfg.numAttrs = PAIR ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<KIND, BN, EPI, PAIR>, ta, tb, ty, args) != cudaSuccess)
+        return SBL_ERR_CUDA;
     return launch_status();
 }
 
@@ -213,9 +224,13 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
                                    : (KIND == kKindF16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int bn = choose_bn(M, N, di->num_sms);
+    // the int8 forward with 256-wide tiles runs on CTA pairs (256 x 256 per
+    // pair, each CTA loading 128 rows of B): a third fewer operand bytes per
+    // MMA, so more of them are in flight
+    const bool pair = KIND == kKindI8 && bn == 256 && M > kBM;
     CUtensorMap ta, tb, ty;
     if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
-    if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, bn)) return SBL_ERR_CUDA;
+    if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, pair ? bn / 2 : bn)) return SBL_ERR_CUDA;
     const bool with_epi = KIND == kKindI8 && (args.relu2 || args.residual);
     if (!encode_output(&ty, args.out, args.out_fp32 != 0, M, N, args.ldo, !args.out_fp32 && !with_epi))
         return SBL_ERR_CUDA;
@@ -225,6 +240,9 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     args.k_blocks = static_cast<int32_t>((static_cast<int64_t>(K) * eb + kBKBytes - 1) / kBKBytes);
     args.err = di->err;
     if constexpr (KIND == kKindI8) {
+        if (pair)
+            return with_epi ? launch_gemm_bn<KIND, 256, true, true>(di, ta, tb, ty, args, stream)
+                            : launch_gemm_bn<KIND, 256, false, true>(di, ta, tb, ty, args, stream);
         if (with_epi)
             return bn == 128 ? launch_gemm_bn<KIND, 128, true>(di, ta, tb, ty, args, stream)
                              : launch_gemm_bn<KIND, 256, true>(di, ta, tb, ty, args, stream);

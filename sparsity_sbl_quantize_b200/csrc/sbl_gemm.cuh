@@ -20,6 +20,13 @@
 // kernel is launched with programmatic dependent launch: its prologue
 // overlaps the previous kernel, and it waits for that kernel before touching
 // global memory.
+//
+// The int8 forward with 256-wide tiles runs the same roles on CTA pairs
+// (cta_group::2, clusters of two): 256 x 256 per pair, each CTA loading its
+// 128 A rows and 128 of the B rows, so a stage is 32 KiB and six are in
+// flight.  The single-CTA form moves 48 KiB per 128-byte K step and, at the
+// TMA latency measured on B200 (about 1.7 us per stage under load), four
+// stages keep the int8 tensor core busy only about 65% of the time.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,12 +50,15 @@ constexpr int kGroupM = 8;               // tile raster: groups of 8 row tiles
 constexpr int kEpiBufBytes = 32 * 128;
 constexpr int kEpiBytes = kEpiWarps * kEpiBufBytes;
 
-template <int BN>
+// PAIR: CTA pairs (cta_group::2) -- a tile is 256 A rows x BN, each CTA of
+// the pair holding its 128 A rows and half of the BN B rows per stage.
+template <int BN, bool PAIR = false>
 struct GemmCfg {
     static_assert(BN == 128 || BN == 256, "tile width");
-    static constexpr int kBBytes = BN * kBKBytes;
+    static constexpr int kBRows = PAIR ? BN / 2 : BN;  // B rows per CTA and stage
+    static constexpr int kBBytes = kBRows * kBKBytes;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = (192 * 1024) / kStageBytes;  // 4 (BN 256) or 6 (BN 128)
+    static constexpr int kStages = (192 * 1024) / kStageBytes;  // 4 (BN 256), 6 (BN 128 or a pair at 256)
     static constexpr int kNumAcc = kTmemCols / BN;              // 2 or 4 accumulators
     static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + 256;
 };
@@ -79,7 +89,7 @@ __device__ __forceinline__ float epilogue_op(float v, int32_t relu2, uint32_t re
     return v;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, int M = kBM>
 __device__ __forceinline__ constexpr uint32_t gemm_idesc()
 {
     // D format (bits 4-5), A/B formats (7-9, 10-12), K-major A and B (bits 15,
@@ -89,7 +99,7 @@ __device__ __forceinline__ constexpr uint32_t gemm_idesc()
     else if (KIND == kKindF16) d |= (1u << 4);                          // f32 <- f16 x f16
     else d |= (1u << 4) | (1u << 7) | (1u << 10);                       // f32 <- bf16 x bf16
     d |= static_cast<uint32_t>(BN >> 3) << 17;
-    d |= static_cast<uint32_t>(kBM >> 4) << 24;
+    d |= static_cast<uint32_t>(M >> 4) << 24;
     return d;
 }
 
@@ -104,16 +114,39 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
     tn = r / gm;
 }
 
+// D(tmem) (+)= A * B^T over a CTA pair (M = 256: 128 A rows from each CTA's
+// shared memory, B split the same way by rows), int8 -> int32; issued by the
+// even CTA.
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // EPI: the instantiation that applies the output epilogue (relu2 /
-// residual); the others compile without it.
-template <int KIND, int BN, bool EPI = false>
+// residual); the others compile without it.  PAIR: the CTA-pair form (int8
+// only): a cluster of two CTAs computes a 256 x BN tile with M = 256 MMAs
+// issued by the even CTA; each CTA loads its own 128 A rows and BN / 2 B rows
+// (so a stage is 32 KiB instead of 48 and six stages are in flight), the odd
+// CTA's loads complete on the even CTA's full barriers, the even CTA's
+// commits arrive on the barriers of both, each CTA drains its own 128 rows of
+// the accumulator and its epilogue warps arrive on the even CTA's
+// accumulator-free barriers.
+template <int KIND, int BN, bool EPI = false, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs args)
 {
-    using Cfg = GemmCfg<BN>;
+    static_assert(!PAIR || KIND == kKindI8, "CTA pairs run the int8 forward");
+    using Cfg = GemmCfg<BN, PAIR>;
     constexpr int kStages = Cfg::kStages;
     constexpr int kNumAcc = Cfg::kNumAcc;
+    constexpr int kTileM = PAIR ? 2 * kBM : kBM;  // A rows of a tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -132,6 +165,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = args.tiles_m * args.tiles_n;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // CTA of the pair
+    const bool leader = rank == 0;
+    // tiles are dealt to CTAs, or to pairs: unit g takes tiles g, g + units, ...
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     // ---------------------------------------------------------- prologue
     if (threadIdx.x == 0) {
@@ -141,7 +179,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < kNumAcc; ++a) {
             mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), kEpiWarps * 32);
+            // single CTA: every epilogue thread arrives; pair: one arrival per
+            // epilogue warp of both CTAs, on the even CTA's barrier
+            mbar_init(tempty_bar(a), PAIR ? 2 * kEpiWarps : kEpiWarps * 32);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -150,12 +190,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_prefetch_map(&tmY);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_addr(tmem_slot), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+            tmem_relinquish();
+        }
         tc_fence_before();
     }
     __syncthreads();
     tc_fence_after();
+    // both CTAs' barriers are initialised before either CTA signals the other
+    if constexpr (PAIR) cluster_sync_all();
     const uint32_t tmem_base = *tmem_slot;
     // the previous kernel's outputs (our A operand, gamma, scales) are ready
     // after this; our own dependents may start their prologue now
@@ -173,9 +220,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t issued_phase[kStages];
         for (int s = 0; s < kStages; ++s) issued_phase[s] = 0;
         constexpr int kElemsPerBlock = (KIND == kKindI8) ? 128 : 64;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        for (int tile = unit; ok && tile < num_tiles; tile += units) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+            const int arow = tm * kTileM + static_cast<int>(rank) * kBM;
+            const int brow = tn * BN + static_cast<int>(rank) * Cfg::kBRows;
             for (int kb = 0; kb < args.k_blocks; ++kb) {
                 const bool ready = mbar_wait(empty_bar(stage), phase ^ 1u, args.err, kErrGemmProducer);
                 if (!__all_sync(0xffffffffu, ready)) {
@@ -183,11 +232,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(full_bar(stage), Cfg::kStageBytes);
-                    tma_load_2d(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, tm * kBM,
-                                full_bar(stage));
-                    tma_load_2d(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, tn * BN,
-                                full_bar(stage));
+                    if constexpr (PAIR) {
+                        const uint32_t fb = map_shared_rank(full_bar(stage), 0);  // the even CTA's barrier
+                        if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * Cfg::kStageBytes);
+                        tma_load_2d_pair(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, arow, fb);
+                        tma_load_2d_pair(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, brow, fb);
+                    } else {
+                        mbar_arrive_expect_tx(full_bar(stage), Cfg::kStageBytes);
+                        tma_load_2d(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, arow, full_bar(stage));
+                        tma_load_2d(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, brow,
+                                    full_bar(stage));
+                    }
                 }
                 __syncwarp();
                 issued_mask |= 1u << stage;
@@ -195,19 +250,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (++stage == kStages) stage = 0, phase ^= 1u;
             }
         }
-        if (!ok) {
-            // let any load still in flight land before the CTA can exit
+        if (!ok && leader) {
+            // let any load still in flight land before the CTA can exit (a
+            // pair's loads all complete on the even CTA's barriers; the odd
+            // CTA stays alive through the closing cluster barrier)
             for (int s = 0; s < kStages; ++s)
                 if (issued_mask & (1u << s)) mbar_wait(full_bar(s), issued_phase[s], args.err, kErrGemmProducer);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 && leader) {
         // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = gemm_idesc<KIND, BN>();
+        constexpr uint32_t idesc = gemm_idesc<KIND, BN, kTileM>();
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         int local = 0;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+        for (int tile = unit; ok && tile < num_tiles; tile += units, ++local) {
             const int acc = local % kNumAcc;
             const uint32_t acc_phase = (local / kNumAcc) & 1;
             const bool free_acc = mbar_wait(tempty_bar(acc), acc_phase ^ 1u, args.err, kErrGemmMma);
@@ -231,27 +288,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int kk = 0; kk < kBKBytes / 32; ++kk) {
                         // +32 bytes along K = +2 in the 16-byte address field
                         const uint64_t step = static_cast<uint64_t>(2 * kk);
-                        if (KIND == kKindI8)
+                        if constexpr (PAIR)
+                            mma_i8_pair(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
+                        else if (KIND == kKindI8)
                             mma_i8(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
                         else
                             mma_f16(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
                     }
-                    tc_commit(empty_bar(stage));  // frees the stage once these MMAs finish
+                    // frees the stage (of both CTAs) once these MMAs finish
+                    if constexpr (PAIR)
+                        tc_commit_pair(empty_bar(stage), 0x3);
+                    else
+                        tc_commit(empty_bar(stage));
                 }
                 __syncwarp();
                 if (++stage == kStages) stage = 0, phase ^= 1u;
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(tfull_bar(acc));  // accumulator ready for the epilogue
+            if (lane == 0) {  // accumulator ready for the epilogue (of both CTAs)
+                if constexpr (PAIR)
+                    tc_commit_pair(tfull_bar(acc), 0x3);
+                else
+                    tc_commit(tfull_bar(acc));
+            }
             __syncwarp();
         }
         // every MMA issued above has completed before TMEM is released
-        if (lane == 0) tc_commit(drain_bar);
+        if (lane == 0) {
+            if constexpr (PAIR)
+                tc_commit_pair(drain_bar, 0x1);
+            else
+                tc_commit(drain_bar);
+        }
         __syncwarp();
         mbar_wait(drain_bar, 0, args.err, kErrGemmMma);
         __syncwarp();
-    } else {
+    } else if (warp >= 2) {
         // ---------------------------------------------------- epilogue (warps 2-9)
+        // this warp's share of accumulator a is in registers: hand it back
+        // (pair: lane 0 for the warp, on the even CTA's barrier)
+        auto release_accumulator = [&](int a) {
+            if constexpr (PAIR) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(a), 0));
+            } else {
+                mbar_arrive(tempty_bar(a));
+            }
+        };
         // Lane r of warp w drains TMEM row 32 (w % 4) + r over half of the
         // columns ((w - 2) / 4), scales it, and writes it as 128-byte rows
         // into a swizzled staging buffer that lane 0 stores with one TMA bulk
@@ -265,14 +348,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         constexpr int kChunks = BN / kColsPerChunk / 2;  // per warp
         uint32_t nstore = 0;  // bf16 blocks stored by this warp (staging half = nstore % 2)
         int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+        for (int tile = unit; tile < num_tiles; tile += units, ++local) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
             const int acc = local % kNumAcc;
             const uint32_t acc_phase = (local / kNumAcc) & 1;
-            const int m = tm * kBM + r;
+            const int m = tm * kTileM + static_cast<int>(rank) * kBM + r;
             const bool row_ok = m < args.M;
-            const int row0 = tm * kBM + quarter * 32;  // first row of this warp's block
+            const int row0 = m - lane;  // first row of this warp's block
             // the token scale is loaded while the MMAs of this tile still run
             const float d_m = (args.row_scale && row_ok) ? args.row_scale[m] : 0.0f;
             const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
@@ -322,7 +405,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(tempty_bar(acc));
+                release_accumulator(acc);
                 // 32-column blocks (64-byte rows) staged in turn in the two
                 // halves of the warp's buffer: a block waits only for the store
                 // before last, so staging overlaps the previous store's read
@@ -371,7 +454,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (jj == kChunks - 1) {
                     // all of this warp's share of the accumulator is in registers
                     tc_fence_before();
-                    mbar_arrive(tempty_bar(acc));
+                    release_accumulator(acc);
                 }
                 if (n0 >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
                 const int nparts = args.out_fp32 ? 2 : 1;  // 128-byte row blocks in this chunk
@@ -467,10 +550,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     __syncthreads();
+    // neither CTA of a pair leaves while the other may still read its shared
+    // memory or arrive on its barriers
+    if constexpr (PAIR) cluster_sync_all();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        if constexpr (PAIR)
+            tmem_dealloc_pair(tmem_base, kTmemCols);
+        else
+            tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
