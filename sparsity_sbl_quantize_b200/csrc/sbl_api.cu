@@ -80,6 +80,10 @@ static sbl_status current_device(DeviceInfo **out)
                                  GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindI8, 256, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindF16, 256, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<kKindBF16, 256, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Sp24PairCfg<224>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -224,10 +228,10 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
                                    : (KIND == kKindF16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int bn = choose_bn(M, N, di->num_sms);
-    // the int8 forward with 256-wide tiles runs on CTA pairs (256 x 256 per
-    // pair, each CTA loading 128 rows of B): a third fewer operand bytes per
-    // MMA, so more of them are in flight
-    const bool pair = KIND == kKindI8 && bn == 256 && M > kBM;
+    // 256-wide tiles run on CTA pairs (256 x 256 per pair, each CTA loading
+    // 128 rows of B): a third fewer operand bytes per MMA, so more of them are
+    // in flight
+    const bool pair = bn == 256 && M > kBM;
     CUtensorMap ta, tb, ty;
     if (!encode_kmajor(&ta, A, dt, eb, K, M, lda_bytes, kBM)) return SBL_ERR_CUDA;
     if (!encode_kmajor(&tb, B, dt, eb, K, N, ldb_bytes, pair ? bn / 2 : bn)) return SBL_ERR_CUDA;
@@ -247,6 +251,7 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
             return bn == 128 ? launch_gemm_bn<KIND, 128, true>(di, ta, tb, ty, args, stream)
                              : launch_gemm_bn<KIND, 256, true>(di, ta, tb, ty, args, stream);
     }
+    if (pair) return launch_gemm_bn<KIND, 256, false, true>(di, ta, tb, ty, args, stream);
     return bn == 128 ? launch_gemm_bn<KIND, 128, false>(di, ta, tb, ty, args, stream)
                      : launch_gemm_bn<KIND, 256, false>(di, ta, tb, ty, args, stream);
 }

@@ -21,7 +21,7 @@
 // overlaps the previous kernel, and it waits for that kernel before touching
 // global memory.
 //
-// The int8 forward with 256-wide tiles runs the same roles on CTA pairs
+// GEMMs with 256-wide tiles run the same roles on CTA pairs
 // (cta_group::2, clusters of two): 256 x 256 per pair, each CTA loading its
 // 128 A rows and 128 of the B rows, so a stage is 32 KiB and six are in
 // flight.  The single-CTA form moves 48 KiB per 128-byte K step and, at the
@@ -115,8 +115,8 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 }
 
 // D(tmem) (+)= A * B^T over a CTA pair (M = 256: 128 A rows from each CTA's
-// shared memory, B split the same way by rows), int8 -> int32; issued by the
-// even CTA.
+// shared memory, B split the same way by rows), int8 -> int32 or 16-bit
+// floats -> fp32; issued by the even CTA.
 __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate)
 {
@@ -128,9 +128,19 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // EPI: the instantiation that applies the output epilogue (relu2 /
-// residual); the others compile without it.  PAIR: the CTA-pair form (int8
-// only): a cluster of two CTAs computes a 256 x BN tile with M = 256 MMAs
+// residual); the others compile without it.  PAIR: the CTA-pair form: a cluster of two CTAs computes a 256 x BN tile with M = 256 MMAs
 // issued by the even CTA; each CTA loads its own 128 A rows and BN / 2 B rows
 // (so a stage is 32 KiB instead of 48 and six stages are in flight), the odd
 // CTA's loads complete on the even CTA's full barriers, the even CTA's
@@ -142,7 +152,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs args)
 {
-    static_assert(!PAIR || KIND == kKindI8, "CTA pairs run the int8 forward");
     using Cfg = GemmCfg<BN, PAIR>;
     constexpr int kStages = Cfg::kStages;
     constexpr int kNumAcc = Cfg::kNumAcc;
@@ -288,9 +297,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int kk = 0; kk < kBKBytes / 32; ++kk) {
                         // +32 bytes along K = +2 in the 16-byte address field
                         const uint64_t step = static_cast<uint64_t>(2 * kk);
-                        if constexpr (PAIR)
-                            mma_i8_pair(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
-                        else if (KIND == kKindI8)
+                        if constexpr (PAIR) {
+                            if constexpr (KIND == kKindI8)
+                                mma_i8_pair(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
+                            else
+                                mma_f16_pair(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
+                        } else if (KIND == kKindI8)
                             mma_i8(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
                         else
                             mma_f16(d_tmem, adesc + step, bdesc + step, idesc, (kb | kk) != 0);
