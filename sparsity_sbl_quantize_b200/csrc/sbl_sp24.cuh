@@ -268,13 +268,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t acc_phase = (local / kNumAcc) & 1;
             const int o0 = tm * 256 + static_cast<int>(rank) * kSpBM + quarter * 32;
             const int o = o0 + lane;
+            constexpr int kChunks = BN / 32;
+            constexpr int kMine = (kChunks + 1) / 2;  // chunks c = half, half + 2, ... (warp half 0 has the extra)
+            // the token scales of this warp's chunks are loaded while the
+            // tile's MMAs still run (one L2 round trip per tile, not per chunk)
+            float d_pre[kMine];
+#pragma unroll
+            for (int i = 0; i < kMine; ++i) {
+                const int t = tn * BN + 32 * (half + 2 * i) + lane;
+                d_pre[i] = (half + 2 * i < kChunks && t < args.T) ? args.d[t] : 0.0f;
+            }
             const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
             if (!__all_sync(0xffffffffu, ready)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(acc * BN);
-            constexpr int kChunks = BN / 32;
-            constexpr int kMine = (kChunks + 1) / 2;  // chunks c = half, half + 2, ... (warp half 0 has the extra)
             if (!args.out_fp32 && !EPI) {
                 // bf16: drain every chunk of this warp, converting it to 16
                 // packed words of the transposed block (lanes 2i and 2i+1 swap
@@ -288,7 +296,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (c >= kChunks) break;  // warp-uniform
                     const int t0 = tn * BN + 32 * c;
                     const int t = t0 + lane;
-                    const float sc = t < args.T ? __fmul_rn(g, args.d[t]) : 0.0f;
+                    const float sc = t < args.T ? __fmul_rn(g, d_pre[i]) : 0.0f;
                     const bool odd = lane & 1;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {  // 16 tokens at a time
@@ -352,7 +360,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = half; c < kChunks; c += 2) {
                 const int t0 = tn * BN + 32 * c;
                 const int t = t0 + lane;
-                const float sc = t < args.T ? __fmul_rn(g, args.d[t]) : 0.0f;
+                float dt = d_pre[0];
+#pragma unroll
+                for (int i = 1; i < kMine; ++i)
+                    if (c == half + 2 * i) dt = d_pre[i];
+                const float sc = t < args.T ? __fmul_rn(g, dt) : 0.0f;
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * c), v);
                 tmem_wait_ld();
