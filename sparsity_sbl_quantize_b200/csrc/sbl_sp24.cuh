@@ -290,38 +290,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // lane token j, the odd lane token j + 1), hand the
                 // accumulator back, and only then stage and store
                 uint32_t packed[kMine][16];
+                const bool odd = lane & 1;
+                // 16 tokens per step, step s = chunk s / 2, half s % 2; the
+                // next step's TMEM load is in flight while this one converts
+                // (registers va / vb in turn)
+                uint32_t va[16], vb[16];
+                tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(32 * half), va);
 #pragma unroll
-                for (int i = 0; i < kMine; ++i) {
+                for (int st = 0; st < 2 * kMine; ++st) {
+                    const int i = st >> 1, hh = st & 1;
                     const int c = half + 2 * i;
                     if (c >= kChunks) break;  // warp-uniform
+                    tmem_wait_ld();
+                    const int cn = half + 2 * ((st + 1) >> 1);
+                    if (st + 1 < 2 * kMine && cn < kChunks)
+                        tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(32 * cn + 16 * ((st + 1) & 1)), hh ? va : vb);
+                    const uint32_t(&v)[16] = hh ? vb : va;
                     const int t0 = tn * BN + 32 * c;
                     const int t = t0 + lane;
                     const float sc = t < args.T ? __fmul_rn(g, d_pre[i]) : 0.0f;
-                    const bool odd = lane & 1;
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {  // 16 tokens at a time
-                        uint32_t v[16];
-                        tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(32 * c + 16 * hh), v);
-                        tmem_wait_ld();
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        const int j = 16 * hh + jj;
+                        const float s0 = __shfl_sync(0xffffffffu, sc, j);
+                        const float s1 = __shfl_sync(0xffffffffu, sc, j + 1);
+                        const float y0 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[jj])), s0);
+                        const float y1 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[jj + 1])), s1);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? y0 : y1, 1);
+                        const __nv_bfloat162 b2 =
+                            odd ? __floats2bfloat162_rn(other, y1) : __floats2bfloat162_rn(y0, other);
+                        packed[i][j >> 1] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                    if (args.acc_out && o < args.O && t0 < args.T && o0 < args.O) {
 #pragma unroll
-                        for (int jj = 0; jj < 16; jj += 2) {
-                            const int j = 16 * hh + jj;
-                            const float s0 = __shfl_sync(0xffffffffu, sc, j);
-                            const float s1 = __shfl_sync(0xffffffffu, sc, j + 1);
-                            const float y0 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[jj])), s0);
-                            const float y1 = __fmul_rn(__int2float_rn(static_cast<int32_t>(v[jj + 1])), s1);
-                            const float other = __shfl_xor_sync(0xffffffffu, odd ? y0 : y1, 1);
-                            const __nv_bfloat162 b2 =
-                                odd ? __floats2bfloat162_rn(other, y1) : __floats2bfloat162_rn(y0, other);
-                            packed[i][j >> 1] = *reinterpret_cast<const uint32_t *>(&b2);
-                        }
-                        if (args.acc_out && o < args.O && t0 < args.T && o0 < args.O) {
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj)
-                                if (t0 + 16 * hh + jj < args.T)
-                                    args.acc_out[static_cast<int64_t>(t0 + 16 * hh + jj) * args.O + o] =
-                                        static_cast<int32_t>(v[jj]);
-                        }
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (t0 + 16 * hh + jj < args.T)
+                                args.acc_out[static_cast<int64_t>(t0 + 16 * hh + jj) * args.O + o] =
+                                    static_cast<int32_t>(v[jj]);
                     }
                 }
                 tc_fence_before();
