@@ -348,6 +348,28 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
                        int32_t T, const sbl_packed *w, sbl_format fmt,
                        void *Y, int32_t y_is_fp32, int32_t *acc_out, void *stream);
 
+#define SBL_GROUP_MAX 4
+
+/* Step 5 of the forward for `count` layers (1 <= count <= SBL_GROUP_MAX)
+ * that read the same activations (for example the gate and up projections of
+ * an MLP, or q, k and v): Y_i = the sbl_forward output of layer i with
+ * SBL_FMT_I8, bit for bit, computed by ONE launch whose tiles cover every
+ * layer's outputs (the launch's fixed cost is paid once, and the tile rounds
+ * are filled across layers).
+ * descs[i], w[i], Y[i]: layer i's descriptor, packed weights (w[i]->i8 and
+ * w[i]->gamma required) and output [T, out_features_i] (bf16 bits, or fp32
+ * when y_is_fp32); every layer has the same in_features K.  Xq [T, K], d [T]
+ * as for sbl_forward.  The arrays are host arrays read during the call; the
+ * buffers they point to are device memory owned by the caller.
+ * Errors: SBL_ERR_INVALID_ARG for a NULL array, entry or buffer or count out
+ * of range; SBL_ERR_SHAPE for a bad descriptor, T < 0 or differing
+ * in_features; SBL_ERR_ALIGNMENT for a buffer not 16-byte aligned.  T == 0
+ * enqueues nothing.  Launched like the SBL_FMT_I8 forward (programmatic
+ * dependent launch). */
+sbl_status sbl_forward_group(const sbl_layer_desc *const *descs, int32_t count, const int8_t *Xq,
+                             const float *d, int32_t T, const sbl_packed *const *w, void *const *Y,
+                             int32_t y_is_fp32, void *stream);
+
 /* Output epilogue fused into the forward (all members optional):
  *  relu2     non-zero: v = max(v, 0)^2 on the fp32 output (Squared ReLU of the
  *            BitNet b1.58 2B4T summary, "Squared ReLU Activation in the

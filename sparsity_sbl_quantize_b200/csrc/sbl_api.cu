@@ -82,6 +82,12 @@ static sbl_status current_device(DeviceInfo **out)
                                  GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindF16, 256, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_group_kernel<256, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_group_kernel<256, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_group_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_kernel<kKindBF16, 256, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmCfg<256, true>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(sp24_pair_kernel<224>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -254,6 +260,34 @@ static sbl_status launch_gemm(const DeviceInfo *di, const void *A, int64_t lda_b
     if (pair) return launch_gemm_bn<KIND, 256, false, true>(di, ta, tb, ty, args, stream);
     return bn == 128 ? launch_gemm_bn<KIND, 128, false>(di, ta, tb, ty, args, stream)
                      : launch_gemm_bn<KIND, 256, false>(di, ta, tb, ty, args, stream);
+}
+
+// One launch of grouped int8 products (p.grp and every map filled in).
+template <int BN, bool PAIR>
+static sbl_status launch_gemm_group(const DeviceInfo *di, GemmGroupParams &p, cudaStream_t stream)
+{
+    constexpr int tile_m = PAIR ? 2 * kBM : kBM;
+    p.args.tiles_m = static_cast<int32_t>((p.args.M + tile_m - 1) / tile_m);
+    p.args.tiles_n = p.grp.tn0[p.grp.count];
+    const int tiles = p.args.tiles_m * p.args.tiles_n;
+    const int units = PAIR ? di->num_sms / 2 : di->num_sms;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>((PAIR ? 2 : 1) * (tiles < units ? tiles : units)));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = GemmCfg<BN, PAIR>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = PAIR ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_group_kernel<BN, PAIR>, p) != cudaSuccess) return SBL_ERR_CUDA;
+    return launch_status();
 }
 
 // 3-D view of the SP24 metadata [O, row_bytes] for the sparse GEMM: dims
@@ -986,6 +1020,61 @@ sbl_status sbl_forward(const sbl_layer_desc *desc, const int8_t *Xq, const float
     return forward_impl(desc, Xq, d, T, w, fmt, Y, y_is_fp32, acc_out, nullptr, stream_p);
 }
 
+sbl_status sbl_forward_group(const sbl_layer_desc *const *descs, int32_t count, const int8_t *Xq,
+                             const float *d, int32_t T, const sbl_packed *const *w, void *const *Y,
+                             int32_t y_is_fp32, void *stream_p)
+{
+    if (!descs || !w || !Y || count < 1 || count > SBL_GROUP_MAX) return SBL_ERR_INVALID_ARG;
+    sbl_status st;
+    for (int32_t i = 0; i < count; ++i) {
+        if ((st = check_desc(descs[i])) != SBL_OK) return st;
+        if (descs[i]->in_features != descs[0]->in_features) return SBL_ERR_SHAPE;
+    }
+    if (T < 0) return SBL_ERR_SHAPE;
+    if (T == 0) return SBL_OK;
+    if (!Xq || !d) return SBL_ERR_INVALID_ARG;
+    if (!aligned16(Xq) || !aligned16(d)) return SBL_ERR_ALIGNMENT;
+    for (int32_t i = 0; i < count; ++i) {
+        if (!w[i] || !w[i]->i8 || !w[i]->gamma || !Y[i]) return SBL_ERR_INVALID_ARG;
+        if (!aligned16(w[i]->i8) || !aligned16(w[i]->gamma) || !aligned16(Y[i])) return SBL_ERR_ALIGNMENT;
+    }
+    DeviceInfo *di = nullptr;
+    if ((st = current_device(&di)) != SBL_OK) return st;
+    const int32_t K = descs[0]->in_features;
+    int64_t n_total = 0;
+    for (int32_t i = 0; i < count; ++i) n_total += descs[i]->out_features;
+    const int bn = choose_bn(T, static_cast<int32_t>(n_total), di->num_sms);
+    const bool pair = bn == 256 && T > kBM;
+    static GemmGroupParams p;  // 1.4 KB of kernel parameters, copied at launch
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    memset(&p, 0, sizeof(p));
+    if (!encode_kmajor(&p.a, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, T, K, kBM)) return SBL_ERR_CUDA;
+    int32_t tn = 0;
+    for (int32_t i = 0; i < count; ++i) {
+        const int32_t O = descs[i]->out_features;
+        if (!encode_kmajor(&p.b[i], w[i]->i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, O, K, pair ? bn / 2 : bn) ||
+            !encode_output(&p.y[i], Y[i], y_is_fp32 != 0, T, O, O, !y_is_fp32))
+            return SBL_ERR_CUDA;
+        p.grp.tn0[i] = tn;
+        p.grp.n[i] = O;
+        p.grp.gamma[i] = w[i]->gamma;
+        tn += (O + bn - 1) / bn;
+    }
+    p.grp.tn0[count] = tn;
+    p.grp.count = count;
+    p.args.M = T;
+    p.args.N = static_cast<int32_t>(n_total);
+    p.args.K = K;
+    p.args.k_blocks = (K + kBKBytes - 1) / kBKBytes;
+    p.args.out_fp32 = y_is_fp32 ? 1 : 0;
+    p.args.row_scale = d;
+    p.args.err = di->err;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_p);
+    if (pair) return launch_gemm_group<256, true>(di, p, stream);
+    return bn == 128 ? launch_gemm_group<128, false>(di, p, stream) : launch_gemm_group<256, false>(di, p, stream);
+}
+
 sbl_status sbl_forward_ex(const sbl_layer_desc *desc, const int8_t *Xq, const float *d, int32_t T,
                           const sbl_packed *w, sbl_format fmt, void *Y, int32_t y_is_fp32, int32_t *acc_out,
                           const sbl_epilogue *epi, void *stream_p)
@@ -1047,6 +1136,7 @@ sbl_format sbl_forward_format(const sbl_layer_desc *desc, int32_t tokens)
 }  // extern "C"
 
 // ------------------------------------------------------ batched decode --
+static_assert(SBL_GROUP_MAX == kGemmMaxGroups, "the launch parameters hold every map of a group");
 static_assert(SBL_BATCH_MAX_LAYERS <= kGvMaxProblems, "the launch parameters hold every layer of a batch");
 static_assert(sizeof(GvArgs) <= 32000 && sizeof(GvPrepArgs) <= 32000, "kernel parameters are limited to 32764 bytes");
 constexpr int32_t kGvMaxK = 4 * kGvStageBytes / 16 / kDecKUnit * kDecKUnit;  // 16-row items of K / 4 bytes per row fill a stage

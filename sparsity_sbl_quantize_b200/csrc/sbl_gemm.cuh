@@ -139,19 +139,45 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
-// EPI: the instantiation that applies the output epilogue (relu2 /
-// residual); the others compile without it.  PAIR: the CTA-pair form: a cluster of two CTAs computes a 256 x BN tile with M = 256 MMAs
-// issued by the even CTA; each CTA loads its own 128 A rows and BN / 2 B rows
-// (so a stage is 32 KiB instead of 48 and six stages are in flight), the odd
-// CTA's loads complete on the even CTA's full barriers, the even CTA's
-// commits arrive on the barriers of both, each CTA drains its own 128 rows of
-// the accumulator and its epilogue warps arrive on the even CTA's
-// accumulator-free barriers.
-template <int KIND, int BN, bool EPI = false, bool PAIR = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY, GemmArgs args)
+// Grouped GEMMs: up to kGemmMaxGroups products that share A (the same
+// activations, e.g. the gate and up projections) in one persistent grid.
+// Group i's BN-column tiles are the column tiles tn0[i] .. tn0[i + 1] - 1 of
+// the launch, with its own B and Y maps, width n[i] and gamma; the raster of
+// tile_coords runs over all of them, so every A tile is reused across groups.
+constexpr int kGemmMaxGroups = 4;
+struct GemmGroups {
+    int32_t count;
+    int32_t tn0[kGemmMaxGroups + 1];
+    int32_t n[kGemmMaxGroups];
+    const float *gamma[kGemmMaxGroups];
+};
+
+// The group of column tile tn and the tile's index inside it.
+__device__ __forceinline__ int group_of(const GemmGroups &grp, int tn, int &tn_local)
 {
+    int gi = 0;
+    while (gi + 1 < grp.count && tn >= grp.tn0[gi + 1]) ++gi;
+    tn_local = tn - grp.tn0[gi];
+    return gi;
+}
+
+// The kernel body.  tmB and tmY point at G maps (kernel parameters); G == 1
+// is the single product of `args` (grp unused), G > 1 the groups of grp
+// (plain epilogue only: no EPI, raw accumulators or keep bits).
+// EPI: the instantiation that applies the output epilogue (relu2 /
+// residual); the others compile without it.  PAIR: the CTA-pair form: a
+// cluster of two CTAs computes a 256 x BN tile with M = 256 MMAs issued by
+// the even CTA; each CTA loads its own 128 A rows and BN / 2 B rows (so a
+// stage is 32 KiB instead of 48 and six stages are in flight), the odd CTA's
+// loads complete on the even CTA's full barriers, the even CTA's commits
+// arrive on the barriers of both, each CTA drains its own 128 rows of the
+// accumulator and its epilogue warps arrive on the even CTA's
+// accumulator-free barriers.
+template <int KIND, int BN, bool EPI, bool PAIR, int G>
+__device__ __forceinline__ void gemm_body(const CUtensorMap *tmA, const CUtensorMap *tmB, const CUtensorMap *tmY,
+                                          const GemmArgs &args, const GemmGroups &grp)
+{
+    static_assert(G == 1 || !EPI, "grouped products take the plain epilogue");
     using Cfg = GemmCfg<BN, PAIR>;
     constexpr int kStages = Cfg::kStages;
     constexpr int kNumAcc = Cfg::kNumAcc;
@@ -194,9 +220,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
-        tma_prefetch_map(&tmA);
-        tma_prefetch_map(&tmB);
-        tma_prefetch_map(&tmY);
+        tma_prefetch_map(tmA);
+        for (int i = 0; i < (G > 1 ? grp.count : 1); ++i) {
+            tma_prefetch_map(tmB + i);
+            tma_prefetch_map(tmY + i);
+        }
     }
     if (warp == 1) {
         if constexpr (PAIR) {
@@ -232,8 +260,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int tile = unit; ok && tile < num_tiles; tile += units) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+            int tnl = tn;
+            const int gi = G > 1 ? group_of(grp, tn, tnl) : 0;
+            const CUtensorMap *mapB = tmB + gi;
             const int arow = tm * kTileM + static_cast<int>(rank) * kBM;
-            const int brow = tn * BN + static_cast<int>(rank) * Cfg::kBRows;
+            const int brow = tnl * BN + static_cast<int>(rank) * Cfg::kBRows;
             for (int kb = 0; kb < args.k_blocks; ++kb) {
                 const bool ready = mbar_wait(empty_bar(stage), phase ^ 1u, args.err, kErrGemmProducer);
                 if (!__all_sync(0xffffffffu, ready)) {
@@ -244,12 +275,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if constexpr (PAIR) {
                         const uint32_t fb = map_shared_rank(full_bar(stage), 0);  // the even CTA's barrier
                         if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * Cfg::kStageBytes);
-                        tma_load_2d_pair(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, arow, fb);
-                        tma_load_2d_pair(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, brow, fb);
+                        tma_load_2d_pair(a_base + stage * kABytes, tmA, kb * kElemsPerBlock, arow, fb);
+                        tma_load_2d_pair(b_base + stage * Cfg::kBBytes, mapB, kb * kElemsPerBlock, brow, fb);
                     } else {
                         mbar_arrive_expect_tx(full_bar(stage), Cfg::kStageBytes);
-                        tma_load_2d(a_base + stage * kABytes, &tmA, kb * kElemsPerBlock, arow, full_bar(stage));
-                        tma_load_2d(b_base + stage * Cfg::kBBytes, &tmB, kb * kElemsPerBlock, brow,
+                        tma_load_2d(a_base + stage * kABytes, tmA, kb * kElemsPerBlock, arow, full_bar(stage));
+                        tma_load_2d(b_base + stage * Cfg::kBBytes, mapB, kb * kElemsPerBlock, brow,
                                     full_bar(stage));
                     }
                 }
@@ -354,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int half = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;
-        const float g = args.gamma ? *args.gamma : 1.0f;
+        const float g1 = args.gamma ? *args.gamma : 1.0f;
         const uint32_t buf = epi_base + static_cast<uint32_t>(warp - 2) * kEpiBufBytes;
         constexpr int kColsPerChunk = 64;  // bf16: two 64-byte stores (one 128-byte with the epilogue); fp32: two
         constexpr int kChunks = BN / kColsPerChunk / 2;  // per warp
@@ -363,13 +394,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int tile = unit; tile < num_tiles; tile += units, ++local) {
             int tm, tn;
             tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+            // grouped: this tile's product (its map, width and gamma); tn is
+            // from here on the column tile inside it
+            const int gi = G > 1 ? group_of(grp, tn, tn) : 0;
+            const CUtensorMap *mapY = tmY + gi;
+            const int N = G > 1 ? grp.n[gi] : args.N;
             const int acc = local % kNumAcc;
             const uint32_t acc_phase = (local / kNumAcc) & 1;
             const int m = tm * kTileM + static_cast<int>(rank) * kBM + r;
             const bool row_ok = m < args.M;
             const int row0 = m - lane;  // first row of this warp's block
-            // the token scale is loaded while the MMAs of this tile still run
+            // the token scale (and a group's gamma) are loaded while the MMAs
+            // of this tile still run
             const float d_m = (args.row_scale && row_ok) ? args.row_scale[m] : 0.0f;
+            const float g = G > 1 ? *grp.gamma[gi] : g1;
             const bool ready = mbar_wait(tfull_bar(acc), acc_phase, args.err, kErrGemmEpilogue);
             if (!__all_sync(0xffffffffu, ready)) break;  // warp-uniform decision
             tc_fence_after();
@@ -407,7 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int n0 = tn * BN + kColsPerChunk * j;
                         for (int h = 0; h < 4; ++h) {
                             const int n = n0 + 16 * h;
-                            if (n >= args.N) break;
+                            if (n >= N) break;
                             uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + static_cast<int64_t>(m) * args.ldo + n);
                             const uint32_t *src = (h < 2) ? v0 + 16 * h : v1 + 16 * (h - 2);
 #pragma unroll
@@ -427,7 +465,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const int col = tn * BN + kColsPerChunk * j + 32 * hh;
-                        if (col >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
+                        if (col >= N || row0 >= args.M) continue;  // warp-uniform: block outside Y
                         const uint32_t sbuf = buf + static_cast<uint32_t>((nstore & 1) * (kEpiBufBytes / 2));
                         if (lane == 0) bulk_wait_group_read<1>();
                         __syncwarp();
@@ -444,7 +482,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(&tmY, sbuf, col, row0);
+                            tma_store_2d(mapY, sbuf, col, row0);
                             bulk_commit_group();
                         }
                         ++nstore;
@@ -468,11 +506,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_fence_before();
                     release_accumulator(acc);
                 }
-                if (n0 >= args.N || row0 >= args.M) continue;  // warp-uniform: block outside Y
+                if (n0 >= N || row0 >= args.M) continue;  // warp-uniform: block outside Y
                 const int nparts = args.out_fp32 ? 2 : 1;  // 128-byte row blocks in this chunk
                 for (int part = 0; part < nparts; ++part) {
                     const int col = args.out_fp32 ? n0 + 32 * part : n0;
-                    if (col >= args.N) break;  // warp-uniform
+                    if (col >= N) break;  // warp-uniform
                     uint32_t w[32];
                     const bool has_res = EPI && args.residual != nullptr && row_ok;
                     if (args.out_fp32) {
@@ -491,7 +529,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             if constexpr (EPI) {
                                 // the residual of columns col + 8q .. + 7, one 16-byte load per 8
                                 const int q = i >> 3;
-                                const uint4 r4 = (has_res && col + 8 * q < args.N)
+                                const uint4 r4 = (has_res && col + 8 * q < N)
                                                      ? *reinterpret_cast<const uint4 *>(args.residual + static_cast<int64_t>(m) * args.ldo + col + 8 * q)
                                                      : make_uint4(0u, 0u, 0u, 0u);
                                 const int e = i & 7;
@@ -513,7 +551,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             if constexpr (EPI) {
                                 // word i of the residual row holds columns col + 2i, col + 2i + 1
                                 const int q = i >> 2;
-                                const uint4 r4 = (has_res && col + 8 * q < args.N)
+                                const uint4 r4 = (has_res && col + 8 * q < N)
                                                      ? *reinterpret_cast<const uint4 *>(args.residual + static_cast<int64_t>(m) * args.ldo + col + 8 * q)
                                                      : make_uint4(0u, 0u, 0u, 0u);
                                 const int e = i & 3;
@@ -539,7 +577,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmY, buf, col, row0);
+                        tma_store_2d(mapY, buf, col, row0);
                         bulk_commit_group();
                     }
                 }
@@ -547,7 +585,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // raw accumulators for parity checks (direct stores)
                     for (int h = 0; h < 4; ++h) {
                         const int n = n0 + 16 * h;
-                        if (n >= args.N) break;
+                        if (n >= N) break;
                         uint4 *dst = reinterpret_cast<uint4 *>(args.acc_out + static_cast<int64_t>(m) * args.ldo + n);
                         const uint32_t *src = (h < 2) ? v0 + 16 * h : v1 + 16 * (h - 2);
 #pragma unroll
@@ -573,6 +611,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else
             tmem_dealloc(tmem_base, kTmemCols);
     }
+}
+
+template <int KIND, int BN, bool EPI = false, bool PAIR = false>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, GemmArgs args)
+{
+    gemm_body<KIND, BN, EPI, PAIR, 1>(&tmA, &tmB, &tmY, args, GemmGroups{});
+}
+
+// The products of one launch that share A (the int8 forward of several
+// layers on the same activations), every map and group in the parameters.
+struct GemmGroupParams {
+    CUtensorMap a;
+    CUtensorMap b[kGemmMaxGroups];
+    CUtensorMap y[kGemmMaxGroups];
+    GemmArgs args;
+    GemmGroups grp;
+};
+
+template <int BN, bool PAIR>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_group_kernel(const __grid_constant__ GemmGroupParams p)
+{
+    gemm_body<kKindI8, BN, false, PAIR, kGemmMaxGroups>(&p.a, p.b, p.y, p.args, p.grp);
 }
 
 }  // namespace sbl

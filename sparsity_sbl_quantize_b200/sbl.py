@@ -50,6 +50,8 @@ class sbl_pack_variant(ctypes.Structure):
     _fields_ = [("master_dtype", ctypes.c_int32), ("mask_source", ctypes.c_int32), ("order", ctypes.c_int32)]
 
 
+SBL_GROUP_MAX = 4  # layers of one sbl_forward_group launch
+
 SBL_MASTER_FP32, SBL_MASTER_BF16 = 0, 1
 SBL_MASK_FROM_MASTER, SBL_MASK_FROM_QUANTIZED = 0, 1
 SBL_QUANT_THEN_MASK, SBL_MASK_THEN_QUANT = 0, 1
@@ -108,6 +110,9 @@ _lib.sbl_quantize_act_rmsnorm.argtypes = [_P, _i32, _i32, _P, ctypes.c_float, _P
 _lib.sbl_forward.restype = ctypes.c_int
 _lib.sbl_forward.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, _P]
 _lib.sbl_backward_dual_ste.restype = ctypes.c_int
+_lib.sbl_forward_group.restype = ctypes.c_int
+_lib.sbl_forward_group.argtypes = [ctypes.POINTER(_D), _i32, _P, _P, _i32, ctypes.POINTER(_W), ctypes.POINTER(_P),
+                                   _i32, _P]
 _lib.sbl_backward_dual_ste.argtypes = [_D, _P, _P, _P, _i32, _W, _P, _i32, _P, _P, _sz, _P]
 _lib.sbl_forward_ex.restype = ctypes.c_int
 _lib.sbl_forward_ex.argtypes = [_D, _P, _P, _i32, _W, ctypes.c_int, _P, _i32, _P, ctypes.POINTER(sbl_epilogue), _P]
@@ -143,7 +148,8 @@ _lib.sbl_container_read.argtypes = [_P, _sz, ctypes.POINTER(sbl_host_buffers)]
 
 EXPORTED = ["sbl_status_string", "sbl_version", "sbl_packed_row_bytes", "sbl_workspace_bytes",
             "sbl_quantize_mask_pack", "sbl_quantize_mask_pack_stats", "sbl_quantize_mask_pack_noalloc", "sbl_quantize_act", "sbl_quantize_act_rmsnorm", "sbl_forward", "sbl_linear_forward",
-            "sbl_forward_ex", "sbl_forward_format", "sbl_forward_batch", "sbl_forward_batch_workspace_bytes",
+            "sbl_forward_ex", "sbl_forward_group", "sbl_forward_format", "sbl_forward_batch",
+            "sbl_forward_batch_workspace_bytes",
             "sbl_gamma_node_count", "sbl_gamma_partials", "sbl_gamma_combine", "sbl_quantize_mask_pack_shard",
             "sbl_backward_dual_ste", "sbl_backward_dual_ste_ex",
             "sbl_quantize_mask_pack_ex", "sbl_device_error", "sbl_selftest_wait_expiry", "sbl_container_bytes",
@@ -283,6 +289,18 @@ def sbl_forward(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, 
     cp = w.c()
     _check(_lib.sbl_forward(ctypes.byref(dsc), _ptr(Xq), _ptr(d), T, ctypes.byref(cp), fmt, _ptr(Y),
                             1 if y_is_fp32 else 0, _ptr(acc_out), _stream()), "sbl_forward")
+
+
+def sbl_forward_group(descs, Xq: torch.Tensor, d: torch.Tensor, T: int, ws, Ys, y_is_fp32: bool = False) -> None:
+    """The SBL_FMT_I8 forward of several layers on the same activations in
+    one launch: descs, ws (Packed) and Ys are equal-length sequences."""
+    n = len(descs)
+    cps = [w.c() for w in ws]
+    darr = (_D * n)(*[ctypes.pointer(x) for x in descs])
+    warr = (_W * n)(*[ctypes.pointer(c) for c in cps])
+    yarr = (_P * n)(*[_ptr(y) for y in Ys])
+    _check(_lib.sbl_forward_group(darr, n, _ptr(Xq), _ptr(d), T, warr, yarr, 1 if y_is_fp32 else 0, _stream()),
+           "sbl_forward_group")
 
 
 def sbl_forward_ex(dsc: sbl_layer_desc, Xq: torch.Tensor, d: torch.Tensor, T: int, w: Packed, fmt: int,

@@ -429,3 +429,36 @@ def test_sharding_calls_validate_before_device(sbl):
                 None) == 7
     assert _raw(sbl, "sbl_quantize_mask_pack_shard", ctypes.byref(d), None, sbl.SBL_FMT_I8, ctypes.byref(w),
                 None) == 1
+
+
+def test_group_forward_validation_before_device(sbl):
+    """sbl_forward_group: count, descriptors, shared in_features, null and
+    misaligned pointers are checked before the device lookup; a valid call on
+    a host without a GPU reports SBL_ERR_DEVICE."""
+    good = 0x10000
+    P = ctypes.c_void_p
+
+    def call(descs, ws, ys, T=64, xq=good, d=good, count=None):
+        n = len(descs)
+        darr = (ctypes.POINTER(sbl.sbl_layer_desc) * max(n, 1))(*[ctypes.pointer(x) for x in descs])
+        warr = (ctypes.POINTER(sbl.sbl_packed) * max(n, 1))(*[ctypes.pointer(w) for w in ws])
+        yarr = (P * max(n, 1))(*[P(y) if y else None for y in ys])
+        return _raw(sbl, "sbl_forward_group", darr, n if count is None else count, P(xq) if xq else None,
+                    P(d) if d else None, T, warr, yarr, 0, None)
+
+    w = sbl.sbl_packed(None, None, None, good, None, good)
+    d1, d2 = sbl.desc(4864, 896, 6, 8), sbl.desc(4864, 896, 6, 8)
+    assert _raw(sbl, "sbl_forward_group", None, 1, P(good), P(good), 64, None, None, 0, None) == 1
+    assert call([d1, d2], [w, w], [good, good], count=0) == 1
+    assert call([d1, d2], [w, w], [good, good], count=5) == 1
+    assert call([d1, sbl.desc(4864, 250, 6, 8)], [w, w], [good, good]) == 2      # invalid descriptor
+    assert call([d1, sbl.desc(4864, 1024, 6, 8)], [w, w], [good, good]) == 2     # in_features differ
+    assert call([d1, d2], [w, w], [good, good], T=-1) == 2
+    assert call([d1, d2], [w, w], [good, good], T=0) == 0                        # nothing to do
+    assert call([d1, d2], [w, w], [good, good], xq=None) == 1
+    assert call([d1, d2], [w, w], [good, None]) == 1
+    assert call([d1, d2], [w, sbl.sbl_packed(None, None, None, None, None, good)], [good, good]) == 1  # no I8
+    assert call([d1, d2], [w, w], [good, good + 8]) == 3
+    assert call([d1, d2], [w, sbl.sbl_packed(None, None, None, good + 4, None, good)], [good, good]) == 3
+    assert call([d1, d2], [w, w], [good, good], d=good + 4) == 3
+    assert call([d1, d2, d1, d2], [w] * 4, [good] * 4) == 7                      # valid: no sm_100 device here

@@ -191,3 +191,29 @@ def test_guard_bands_batched_decode_and_sharding():
         sbl.sbl_quantize_mask_pack_shard(ds, w[first:first + rows].contiguous(), sbl.SBL_FMT_I8 | sbl.SBL_FMT_PK2, p)
     g.check()
     assert sbl.sbl_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("T", [300, 100])  # on and off the CTA-pair path
+def test_guard_bands_grouped_forward(T):
+    """The grouped int8 forward writes only each layer's output: ragged
+    widths and a partial last token tile, bf16 and fp32."""
+    sbl = sbl_mod()
+    g = Guarded()
+    K = 1040
+    outs = (528, 48, 784)
+    descs, packs = [], []
+    for i, O in enumerate(outs):
+        d = sbl.desc(O, K, 6, 8)
+        p = _packed(sbl, g, d, sbl.SBL_FMT_I8)
+        ws = g.take((sbl.sbl_workspace_bytes(d, 0, sbl.SBL_OP_QUANTIZE_MASK_PACK),), torch.uint8)
+        sbl.sbl_quantize_mask_pack(d, torch.from_numpy(wl.master_weights(O, K, seed=20 + i)).cuda(),
+                                   sbl.SBL_FMT_I8, p, ws)
+        descs.append(d)
+        packs.append(p)
+    q, dv = g.take((T, K), torch.int8), g.take((T,), torch.float32)
+    sbl.sbl_quantize_act(bf16_dev(wl.activations(T, K, seed=3)), T, K, q, dv)
+    for fp32 in (False, True):
+        ys = [g.take((T, O), torch.float32 if fp32 else torch.bfloat16) for O in outs]
+        sbl.sbl_forward_group(descs, q, dv, T, packs, ys, y_is_fp32=fp32)
+    g.check()
+    assert sbl.sbl_device_error(clear=True) == 0
