@@ -193,14 +193,14 @@ def test_guard_bands_batched_decode_and_sharding():
     assert sbl.sbl_device_error(clear=True) == 0
 
 
-@pytest.mark.parametrize("T", [300, 100])  # on and off the CTA-pair path
-def test_guard_bands_grouped_forward(T):
+@pytest.mark.parametrize("T,outs", [(300, (528, 48, 784)), (100, (528, 48, 784)),
+                                    (1000, (4864, 4880, 48))])  # 128-wide tiles; 256-wide on CTA pairs
+def test_guard_bands_grouped_forward(T, outs):
     """The grouped int8 forward writes only each layer's output: ragged
     widths and a partial last token tile, bf16 and fp32."""
     sbl = sbl_mod()
     g = Guarded()
     K = 1040
-    outs = (528, 48, 784)
     descs, packs = [], []
     for i, O in enumerate(outs):
         d = sbl.desc(O, K, 6, 8)

@@ -30,6 +30,8 @@ def packed_layer(O, K, n, m, seed):
     (300, 512, (272, 1040, 48, 784), False), # ragged widths and tokens, four groups
     (100, 256, (512, 128), True),            # one CTA-row of tokens (no pairs), fp32
     (1, 64, (16,), False),                   # a single layer, a single token
+    (64, 256, (8192, 8192, 8192, 4864), False),  # 256-wide tiles on single CTAs (T <= 128)
+    (1000, 256, (4864, 4880, 48), True),     # CTA pairs with a partial last pair of row tiles, fp32
 ])
 def test_group_equals_one_launch_per_layer(T, K, outs, fp32):
     sbl = sbl_mod()
