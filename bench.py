@@ -180,7 +180,10 @@ def workload_config(wk, world: int) -> dict:
     return {"workload": wk.name, "tokens": wk.tokens if wk.mode == "decode" else wk.tokens[-1],
             "linears": [f"{l.name}:{l.d_in}->{l.d_out}" for l in wk.linears],
             "patterns": [f"{n}:{m}" for n, m in wk.patterns], "mode": wk.mode,
-            "parallelism": f"independent replicas x{world}"}
+            "parallelism": f"independent replicas x{world}",
+            # how the GPU arm keeps timed steps from reusing L2
+            "l2": ("inputs larger than L2 (rotating weight copies, > 4x L2)" if wk.mode == "decode"
+                   else "flushed between timed steps (512 MiB write outside the events)")}
 
 
 # Dense int8 tensor-core rate of one B200 SM per clock: 2 x the 8192 bf16
