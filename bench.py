@@ -385,7 +385,10 @@ class Runner:
         inputs = {}
         for li, lin in enumerate(wk.linears):
             w = wl.master_weights(lin.d_out, lin.d_in, seed=wk.seed, layer=li)
-            key = (lin.d_in, "shared" if lin.d_in == wk.linears[0].d_in else li)
+            # the decoder layer's dataflow: q / k / v read x, o the attention
+            # output, gate / up the normalised hidden state, down the MLP's
+            # activation (Linear.inp); an untagged linear reads its own input
+            key = lin.inp or f"#{li}"
             if key not in inputs:
                 x = wl.activations(T, lin.d_in, seed=wk.seed, layer=li, outlier_frac=wk.outlier_frac)
                 # one int8 copy per N:M pattern, so the patterns' passes can overlap

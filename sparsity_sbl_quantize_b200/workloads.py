@@ -64,6 +64,7 @@ class Linear:
     name: str
     d_in: int
     d_out: int
+    inp: str = ""  # the activation it reads: linears with the same name read one tensor ("": its own)
 
 
 @dataclass
@@ -87,14 +88,14 @@ WORKLOADS = {
         notes="one Sparse-BitLinear layer, T=64, K=256, O=128, 6:8, 1% outlier channels x20"),
     "qwen05b_mlp": Workload(
         "qwen05b_mlp", 2, [4096],
-        [Linear("gate", 896, 4864), Linear("up", 896, 4864), Linear("down", 4864, 896)],
+        [Linear("gate", 896, 4864, "x"), Linear("up", 896, 4864, "x"), Linear("down", 4864, 896, "act")],
         [(6, 8), (2, 4)], "forward",
         notes="Qwen2.5-0.5B MLP linears, T=4096, forward at 6:8 and 2:4"),
     "qwen15b_decoder": Workload(
         "qwen15b_decoder", 3, [8192],
-        [Linear("q", 1536, 1536), Linear("k", 1536, 256), Linear("v", 1536, 256),
-         Linear("o", 1536, 1536), Linear("gate", 1536, 8960), Linear("up", 1536, 8960),
-         Linear("down", 8960, 1536)],
+        [Linear("q", 1536, 1536, "x"), Linear("k", 1536, 256, "x"), Linear("v", 1536, 256, "x"),
+         Linear("o", 1536, 1536, "attn"), Linear("gate", 1536, 8960, "h"), Linear("up", 1536, 8960, "h"),
+         Linear("down", 8960, 1536, "act")],
         [(7, 8), (6, 8), (5, 8), (4, 8), (3, 8), (2, 8), (2, 4)], "forward",
         notes="Qwen2.5-1.5B decoder linears, T=8192, N:M sweep"),
     "bitnet2b_decode": Workload(
