@@ -1,7 +1,8 @@
 """Host-side logic of bench.py on the CPU: the DRAM-traffic records (ncu CSV
 parsing, kernel filter, unit conversion, invalidation when the kernel
-sources change), the clock-sample summary over the timed windows, and the
-algorithmic operation count the TOPS figures divide by."""
+sources change), the clock-sample summary over the timed windows, the
+algorithmic operation count the TOPS figures divide by, and which forward
+launches are grouped."""
 import datetime
 import json
 import os
@@ -196,3 +197,33 @@ def test_cpu_baseline_threads_split_outputs_disjointly():
                         patterns=[(6, 8)], mode="train")
     cb = bench.cpu_baselines(small, 0.4, 2)
     assert cb["cores"] == 2 and cb["single_thread"]["cores"] == 1 and cb["value"] > 0
+
+
+def _grouping(wk_name, sp24_layers=(), mode=None):
+    """bench.Runner.forward_groups on a stub runner: the workload's linears
+    with their inputs shared as the Runner shares them (Linear.inp)."""
+    import types
+    wk = wl.WORKLOADS[wk_name]
+    sbl = types.SimpleNamespace(SBL_FMT_I8=1, SBL_FMT_SP24=16, SBL_GROUP_MAX=4)
+    inputs, layers = {}, []
+    for li, lin in enumerate(wk.linears):
+        key = lin.inp or f"#{li}"
+        layers.append({"lin": lin, "inp": inputs.setdefault(key, {"name": key})})
+    pat = wk.patterns[0]
+    fmt = {(li, pat): (sbl.SBL_FMT_SP24 if lin.name in sp24_layers else sbl.SBL_FMT_I8)
+           for li, lin in enumerate(wk.linears)}
+    stub = types.SimpleNamespace(sbl=sbl, layers=layers, fwd_fmt=fmt,
+                                 wk=types.SimpleNamespace(mode=mode or wk.mode))
+    return [[wk.linears[li].name for li in g] for g in bench.Runner.forward_groups(stub, pat)]
+
+
+def test_forward_groups_follow_the_decoder_dataflow():
+    # q / k / v read x, o the attention output, gate / up the hidden state, down the activation
+    assert _grouping("qwen15b_decoder") == [["q", "k", "v"], ["o"], ["gate", "up"], ["down"]]
+    assert _grouping("qwen05b_mlp") == [["gate", "up"], ["down"]]
+    # a layer on the sparse operand breaks a group; the rest of the input's layers still group
+    assert _grouping("qwen15b_decoder", sp24_layers=("q",)) == [["q"], ["k", "v"], ["o"], ["gate", "up"], ["down"]]
+    assert _grouping("qwen15b_decoder", sp24_layers=("k",)) == [["q"], ["k"], ["v"], ["o"], ["gate", "up"], ["down"]]
+    # training runs each linear's backward right after its forward: never grouped
+    assert _grouping("qwen05b_mlp", mode="train") == [["gate"], ["up"], ["down"]]
+    assert _grouping("qwen3b_train") == [["up"], ["down"]]

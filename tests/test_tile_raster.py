@@ -1,4 +1,4 @@
-"""The persistent GEMM kernels' tile raster covers every output tile once.
+"""The persistent GEMM kernels' tile raster covers every output tile once (grouped launches included).
 
 The dense and the 2:4 sparse forward kernels walk tiles t = b, b + G,
 b + 2G, ... (b the CTA or CTA pair, G the grid) and map each t to a (row
@@ -44,3 +44,37 @@ def test_consecutive_tiles_share_a_column_tile_within_a_group():
         (m0, n0), (m1, n1) = tile_coords(t, tiles_m, tiles_n), tile_coords(t + 1, tiles_m, tiles_n)
         if (t + 1) % GROUP_M:          # inside a run of 8 row tiles
             assert n0 == n1 and m1 == m0 + 1
+
+
+def group_of(tn0, count, tn):
+    """The grouped launch's column tile -> (group, column tile inside it)."""
+    gi = 0
+    while gi + 1 < count and tn >= tn0[gi + 1]:
+        gi += 1
+    return gi, tn - tn0[gi]
+
+
+@pytest.mark.parametrize("widths,bn", [((4864, 4864), 256), ((1536, 256, 256), 256), ((272, 1040, 48, 784), 128),
+                                       ((16,), 128), ((8192, 8192, 8192, 4864), 256)])
+@pytest.mark.parametrize("tokens,pair", [(4096, True), (1000, True), (100, False), (1, False)])
+def test_grouped_raster_covers_every_output_tile_of_every_group_once(widths, bn, tokens, pair):
+    """sbl_forward_group: the launch's column tiles are the groups' tiles in
+    order (tn0 = prefix sums of ceil(width / BN)); every (group, row tile,
+    column tile) is visited exactly once by the grid-strided walk over CTAs
+    or CTA pairs, and no tile column lies past its group's width by a whole tile."""
+    tn0 = [0]
+    for w in widths:
+        tn0.append(tn0[-1] + -(-w // bn))
+    tile_m = 256 if pair else 128
+    tiles_m, tiles_n = -(-tokens // tile_m), tn0[-1]
+    num = tiles_m * tiles_n
+    units = min(num, 74 if pair else 148)
+    seen = []
+    for u in range(units):
+        for t in range(u, num, units):
+            tm, tn = tile_coords(t, tiles_m, tiles_n)
+            gi, tl = group_of(tn0, len(widths), tn)
+            assert tl * bn < widths[gi]          # the tile starts inside its group's columns
+            seen.append((gi, tm, tl))
+    expected = {(gi, tm, tl) for gi, w in enumerate(widths) for tm in range(tiles_m) for tl in range(-(-w // bn))}
+    assert len(seen) == len(expected) and set(seen) == expected
