@@ -578,25 +578,40 @@ class Runner:
 
     # end-to-end: host-resident inputs and outputs through the public API
     def setup_e2e(self):
+        """Pinned host copies of everything a step reads (master weights,
+        activations; output gradients when training) and room for everything
+        it returns (outputs; dX and dW when training)."""
         torch = self.torch
         self.h_w = [torch.from_numpy(L["w_host"]).pin_memory() for L in self.layers]
         self.h_x = [torch.from_numpy(inp["x_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
                     for inp in self.inputs]
         self.h_y = [torch.empty(L["y"][self.wk.patterns[0]].shape, dtype=torch.bfloat16).pin_memory()
                     for L in self.layers]
-        self.h2d = sum(t.numel() * t.element_size() for t in self.h_w + self.h_x) * len(self.wk.patterns)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.h_y) * len(self.wk.patterns)
+        ins, outs = self.h_w + self.h_x, list(self.h_y)
+        if self.wk.mode == "train":
+            self.h_dy = [L["dy"].cpu().pin_memory() for L in self.layers]
+            self.h_dx = [torch.empty(L["dx"].shape, dtype=L["dx"].dtype).pin_memory() for L in self.layers]
+            self.h_dw = [torch.empty(L["dw"].shape, dtype=L["dw"].dtype).pin_memory() for L in self.layers]
+            ins += self.h_dy
+            outs += self.h_dx + self.h_dw
+        self.h2d = sum(t.numel() * t.element_size() for t in ins) * len(self.wk.patterns)
+        self.d2h = sum(t.numel() * t.element_size() for t in outs) * len(self.wk.patterns)
 
     def step_e2e(self):
         """The same step through the public API from host memory: every pass
-        copies its weights and activations in and its outputs back, one
-        stream, in order (what a caller without device-resident data does)."""
+        copies its weights and activations (and, training, the output
+        gradients) in and its outputs (and dX, dW) back, one stream, in order
+        (what a caller without device-resident data does)."""
         sbl = self.sbl
+        train = self.wk.mode == "train"
         for (n, m) in self.wk.patterns:
             for L, hw in zip(self.layers, self.h_w):
                 L["w"].copy_(hw, non_blocking=True)
             for inp, hx in zip(self.inputs, self.h_x):
                 inp["x"].copy_(hx, non_blocking=True)
+            if train:
+                for L, hdy in zip(self.layers, self.h_dy):
+                    L["dy"].copy_(hdy, non_blocking=True)
             for li, L in enumerate(self.layers):
                 dsc, p = L["packed"][(n, m)]
                 if "stats" in L:
@@ -615,6 +630,11 @@ class Runner:
                 sbl.sbl_forward(dsc, inp["q"][(n, m)], inp["d"][(n, m)], self.T, p, self.fwd_fmt[(li, (n, m))],
                                 L["y"][(n, m)])
                 hy.copy_(L["y"][(n, m)], non_blocking=True)
+                if train:
+                    sbl.sbl_backward_dual_ste(dsc, L["dy"], inp["q"][(n, m)], inp["d"][(n, m)], self.T, p, L["dx"],
+                                              False, L["dw"], L["bws"])
+                    self.h_dx[li].copy_(L["dx"], non_blocking=True)
+                    self.h_dw[li].copy_(L["dw"], non_blocking=True)
         self.torch.cuda.current_stream().synchronize()
 
 
@@ -715,11 +735,14 @@ def run_ours(args, wk):
     g.replay()
     torch.cuda.synchronize()
     graph_out = {(li, pat): L["y"][pat].clone() for li, L in enumerate(r.layers) for pat in wk.patterns}
+    graph_grads = {li: (L["dx"].clone(), L["dw"].clone()) for li, L in enumerate(r.layers) if "dx" in L}
     # end to end: host buffers, copies inside the timed region
     r.setup_e2e()
     r.step_e2e()
     selfcheck = all(torch.equal(graph_out[(li, pat)], L["y"][pat])
                     for li, L in enumerate(r.layers) for pat in wk.patterns)
+    selfcheck = selfcheck and all(torch.equal(dx, r.layers[li]["dx"]) and torch.equal(dw, r.layers[li]["dw"])
+                                  for li, (dx, dw) in graph_grads.items())
     if not selfcheck:
         raise SystemExit("bench self-check failed: graph and single-stream outputs differ")
     if world > 1:
@@ -776,7 +799,7 @@ def run_ours(args, wk):
                            "launch (a grouped launch of the linears that share an input counts all their ops)",
         "clocks": clk,
         "device_error": err,
-        "selfcheck": "graph outputs bit-identical to the single-stream API path",
+        "selfcheck": "graph outputs (and dX, dW when training) bit-identical to the single-stream API path",
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
