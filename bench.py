@@ -1186,7 +1186,8 @@ def run_reference(args, wk):
     if rank != 0:
         return
     threads = cpu_threads(args.cpu_threads)
-    budget = args.ref_step_seconds or max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    # about two minutes for the whole run, at least half a second per sample
+    budget = args.ref_step_seconds or max(0.5, 120.0 / max(1, args.steps + args.warmup))
     res = []
     fn = cpu_baseline_decode if wk.mode == "decode" else cpu_baseline
     for i in range(args.warmup + args.steps):
