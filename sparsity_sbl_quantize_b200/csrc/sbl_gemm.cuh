@@ -21,12 +21,16 @@
 // overlaps the previous kernel, and it waits for that kernel before touching
 // global memory.
 //
-// GEMMs with 256-wide tiles run the same roles on CTA pairs
-// (cta_group::2, clusters of two): 256 x 256 per pair, each CTA loading its
-// 128 A rows and 128 of the B rows, so a stage is 32 KiB and six are in
-// flight.  The single-CTA form moves 48 KiB per 128-byte K step and, at the
-// TMA latency measured on B200 (about 1.7 us per stage under load), four
-// stages keep the int8 tensor core busy only about 65% of the time.
+// GEMMs with 256-wide tiles and more than 128 rows run the same roles on CTA
+// pairs (cta_group::2, clusters of two): 256 x 256 per pair, each CTA
+// loading its 128 A rows and 128 of the B rows, so a stage is 32 KiB and six
+// are in flight.  The single-CTA form moves 48 KiB per 128-byte K step and,
+// at the TMA latency measured on B200 (about 1.7 us per stage under load),
+// four stages keep the int8 tensor core busy only about 65% of the time.
+//
+// gemm_group_kernel runs up to four int8 products that share A (the linears
+// that read one input) in one launch, each with its own B and Y maps, width
+// and gamma; its column tiles are the groups' tiles in order.
 #pragma once
 
 #include <cuda_bf16.h>
