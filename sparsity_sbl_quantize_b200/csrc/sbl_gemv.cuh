@@ -50,7 +50,7 @@ namespace sbl {
 constexpr int kGvMaxProblems = 256;
 constexpr int kGvWarps = 16;                      // consumer warps
 constexpr int kGvThreads = 32 * (kGvWarps + 1);   // + the producer warp
-constexpr int kGvStageBytes = 54 * 1024;          // one item: 16 tiles x K/4 bytes per row (2 tiles at K = 6912)
+constexpr int kGvStageBytes = 54 * 1024;          // one item: 1, 2 or 4 tiles of 16 rows x K/4 bytes (2 at K = 6912)
 constexpr int kGvStages = 4;
 constexpr int kGvSlice = 128;                     // weights of a row in one K slice of a unit
 constexpr int kGvItemMaxRows = 64;
