@@ -78,3 +78,27 @@ def test_grouped_raster_covers_every_output_tile_of_every_group_once(widths, bn,
             seen.append((gi, tm, tl))
     expected = {(gi, tm, tl) for gi, w in enumerate(widths) for tm in range(tiles_m) for tl in range(-(-w // bn))}
     assert len(seen) == len(expected) and set(seen) == expected
+
+
+@pytest.mark.parametrize("M,N", [(4096, 4864), (1000, 9792), (16384, 2048), (300, 256)])
+def test_pair_tiles_split_rows_and_b_rows_between_the_two_ctas(M, N):
+    """CTA-pair form: tile (tm, tn) covers A rows [256 tm, 256 tm + 256) and B
+    rows [256 tn, 256 tn + 256); CTA rank r of the pair loads A rows
+    256 tm + 128 r .. + 127 and B rows 256 tn + 128 r .. + 127, and drains its
+    own 128 accumulator rows over all 256 columns.  Over the grid the A rows
+    and the output rows each come out exactly once per column tile."""
+    tiles_m, tiles_n = -(-M // 256), -(-N // 256)
+    a_rows, out_cells, b_rows = [], set(), []
+    for t in range(tiles_m * tiles_n):
+        tm, tn = tile_coords(t, tiles_m, tiles_n)
+        for r in (0, 1):
+            arow = tm * 256 + 128 * r
+            brow = tn * 256 + 128 * r
+            if tn == 0:
+                a_rows.extend(range(arow, arow + 128))
+            if tm == 0:
+                b_rows.extend(range(brow, brow + 128))
+            out_cells.add((arow, tn))      # 128 output rows x the tile's 256 columns
+    assert sorted(a_rows) == list(range(tiles_m * 256))
+    assert sorted(b_rows) == list(range(tiles_n * 256))
+    assert out_cells == {(tm * 256 + 128 * r, tn) for tm in range(tiles_m) for r in (0, 1) for tn in range(tiles_n)}
